@@ -1,0 +1,213 @@
+"""Python face of the CPU oracle (``dmel_oracle.c``): build it with gcc, load it with ctypes.
+
+TEST INFRASTRUCTURE ONLY. The test suite, the smoke check and the benchmark's CPU-baseline
+leg may use this module; the product package never imports it.
+
+Each function states the step it computes; the C file cites the passage each step follows
+("Inside Inkling: Audio Design", Part 1 · Modeling, and the readings listed there).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dmel_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle.so")
+
+HOP = 800
+WIN = 1600
+NBINS = 801
+NMEL = 80
+NLEV = 16
+LMIN = -7.0
+LMAX = 2.0
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (plain -O2, no fast-math) into oracle/_build/liboracle.so."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    if force or stale:
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+               "-std=c11", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        c_d, c_i64, c_int = ctypes.c_double, ctypes.c_int64, ctypes.c_int
+        vp = ctypes.c_void_p
+        L.oracle_threads.restype = c_int
+        L.oracle_frames_for_length.argtypes = [c_i64]
+        L.oracle_frames_for_length.restype = c_i64
+        L.oracle_window.argtypes = [vp]
+        L.oracle_hz_to_mel.argtypes = [c_d]
+        L.oracle_hz_to_mel.restype = c_d
+        L.oracle_mel_to_hz.argtypes = [c_d]
+        L.oracle_mel_to_hz.restype = c_d
+        L.oracle_filterbank.argtypes = [vp]
+        L.oracle_power.argtypes = [vp, vp]
+        L.oracle_mel.argtypes = [vp, vp]
+        L.oracle_log_clamp.argtypes = [c_d]
+        L.oracle_log_clamp.restype = c_d
+        L.oracle_quantise.argtypes = [c_d]
+        L.oracle_quantise.restype = c_int
+        L.oracle_frame_offsets.argtypes = [vp, c_int, vp]
+        L.oracle_frame_offsets.restype = c_int
+        L.oracle_codes.argtypes = [vp, vp, c_int, vp, vp, c_i64, vp, vp]
+        L.oracle_codes.restype = c_int
+        L.oracle_tails_out.argtypes = [vp, vp, c_int, vp, vp]
+        L.oracle_tails_out.restype = c_int
+        L.oracle_embed.argtypes = [vp, c_i64, vp, c_int, vp, c_d, vp]
+        L.oracle_embed.restype = c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def threads() -> int:
+    """OpenMP threads the oracle's frame loops use."""
+    return int(lib().oracle_threads())
+
+
+def frames_for_length(n: int) -> int:
+    """floor(n / 800): frames of an n-sample clip (-1 for n < 0)."""
+    return int(lib().oracle_frames_for_length(int(n)))
+
+
+def window() -> np.ndarray:
+    """Periodic Hann window of 1600 points."""
+    w = np.zeros(WIN, np.float64)
+    lib().oracle_window(_ptr(w))
+    return w
+
+
+def hz_to_mel(f: float) -> float:
+    return float(lib().oracle_hz_to_mel(float(f)))
+
+
+def mel_to_hz(m: float) -> float:
+    return float(lib().oracle_mel_to_hz(float(m)))
+
+
+def filterbank() -> np.ndarray:
+    """[80, 801] HTK triangular filterbank evaluated at 10 Hz bin spacing."""
+    fb = np.zeros((NMEL, NBINS), np.float64)
+    lib().oracle_filterbank(_ptr(fb))
+    return fb
+
+
+def power(frame: np.ndarray) -> np.ndarray:
+    """|DFT(window * frame)|^2 for bins 0..800 of one raw 1600-sample frame (naive DFT)."""
+    fr = np.ascontiguousarray(frame, np.float64)
+    assert fr.shape == (WIN,)
+    P = np.zeros(NBINS, np.float64)
+    lib().oracle_power(_ptr(fr), _ptr(P))
+    return P
+
+
+def mel(frame: np.ndarray) -> np.ndarray:
+    """80 mel energies of one raw 1600-sample frame."""
+    fr = np.ascontiguousarray(frame, np.float64)
+    assert fr.shape == (WIN,)
+    M = np.zeros(NMEL, np.float64)
+    lib().oracle_mel(_ptr(fr), _ptr(M))
+    return M
+
+
+def log_clamp(M: float) -> float:
+    """min(max(log10(max(M, 1e-10)), -7), 2)."""
+    return float(lib().oracle_log_clamp(float(M)))
+
+
+def quantise(lhat: float) -> int:
+    """min(15, floor((lhat + 7) * 16 / 9))."""
+    return int(lib().oracle_quantise(float(lhat)))
+
+
+def frame_offsets(sample_offsets: np.ndarray) -> np.ndarray:
+    so = np.ascontiguousarray(sample_offsets, np.int64)
+    n = so.shape[0] - 1
+    fo = np.zeros(n + 1, np.int64)
+    rc = lib().oracle_frame_offsets(_ptr(so), n, _ptr(fo))
+    if rc != 0:
+        raise ValueError("bad sample offsets")
+    return fo
+
+
+def codes(wav: np.ndarray, sample_offsets: np.ndarray, tails: np.ndarray | None = None,
+          frame_ids: np.ndarray | None = None, want_lhat: bool = True):
+    """dMel codes [n, 80] (uint8) and clamped log-mel values [n, 80] (float64) for all frames
+    (frame_ids None) or for the listed global frame indices."""
+    w = np.ascontiguousarray(wav, np.float32)
+    so = np.ascontiguousarray(sample_offsets, np.int64)
+    n_clips = so.shape[0] - 1
+    t = None if tails is None else np.ascontiguousarray(tails, np.float32)
+    if t is not None:
+        assert t.shape == (n_clips, HOP)
+    if frame_ids is None:
+        n = int(frame_offsets(so)[-1])
+        ids = None
+    else:
+        ids = np.ascontiguousarray(frame_ids, np.int64)
+        n = ids.shape[0]
+    c = np.zeros((n, NMEL), np.uint8)
+    lh = np.zeros((n, NMEL), np.float64) if want_lhat else None
+    rc = lib().oracle_codes(_ptr(w), _ptr(so), n_clips, _ptr(t), _ptr(ids), n, _ptr(c), _ptr(lh))
+    if rc != 0:
+        raise ValueError("oracle_codes: bad offsets or frame index")
+    return (c, lh) if want_lhat else c
+
+
+def tails_out(wav: np.ndarray, sample_offsets: np.ndarray, tails: np.ndarray | None = None) -> np.ndarray:
+    """Carried tail after each clip: the 800 samples ending at sample 800 * F."""
+    w = np.ascontiguousarray(wav, np.float32)
+    so = np.ascontiguousarray(sample_offsets, np.int64)
+    n_clips = so.shape[0] - 1
+    t = None if tails is None else np.ascontiguousarray(tails, np.float32)
+    out = np.zeros((n_clips, HOP), np.float32)
+    rc = lib().oracle_tails_out(_ptr(w), _ptr(so), n_clips, _ptr(t), _ptr(out))
+    if rc != 0:
+        raise ValueError("bad sample offsets")
+    return out
+
+
+def embed(codes_: np.ndarray, table: np.ndarray, rms_weight: np.ndarray | None = None,
+          eps: float = 1e-6) -> np.ndarray:
+    """Sum of rows 16 b + c_b of `table` (converted exactly to float64) per frame, then the
+    optional RMSNorm with weight `rms_weight`; float64 [n_frames, dim]."""
+    c = np.ascontiguousarray(codes_, np.uint8)
+    assert c.ndim == 2 and c.shape[1] == NMEL
+    T = np.ascontiguousarray(table, np.float64)
+    assert T.shape[0] == NMEL * NLEV
+    dim = T.shape[1]
+    g = None if rms_weight is None else np.ascontiguousarray(rms_weight, np.float64)
+    out = np.zeros((c.shape[0], dim), np.float64)
+    rc = lib().oracle_embed(_ptr(c), c.shape[0], _ptr(T), dim, _ptr(g), float(eps), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_embed: code out of range")
+    return out
+
+
+def boundary_distance(lhat: np.ndarray) -> np.ndarray:
+    """Distance of each clamped log-mel value to the nearest of the 15 inner level boundaries
+    -7 + 9k/16, k = 1..15 (used by the agreement rule for codes)."""
+    k = np.arange(1, NLEV, dtype=np.float64)
+    bnd = LMIN + (LMAX - LMIN) * k / NLEV
+    return np.min(np.abs(lhat[..., None] - bnd), axis=-1)

@@ -1,0 +1,337 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself.
+
+Sources of truth used here: the constants printed in "Inside Inkling: Audio Design"
+(Part 1 · Modeling), library routines that compute the same textbook objects (scipy's periodic
+Hann window, numpy's FFT, the HTK filterbanks of transformers and torchaudio, torch's RMSNorm),
+closed forms (a bin-centred tone under a Hann window, Parseval, the one-level gain shift) and
+brute force on tiny tables.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from encoder_free_audio_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_constants.json")
+
+
+def _frame_of(x, t):
+    """Raw samples of frame t of a clip under the causal framing (zeros before the clip)."""
+    idx = np.arange(800 * (t - 1), 800 * (t + 1))
+    out = np.zeros(1600, np.float64)
+    ok = idx >= 0
+    out[ok] = x[idx[ok]]
+    return out
+
+
+# ---------------------------------------------------------------- page constants (golden)
+
+def test_page_constants(oracle_mod):
+    g = json.load(open(GOLDEN))
+    o = oracle_mod
+    assert g["sample_rate_hz"] // g["hop_samples"] == g["tokens_per_second"]
+    assert o.HOP == g["hop_samples"] and o.WIN == g["window_samples"]
+    assert o.NMEL == g["n_mel_bins"] and o.NLEV == g["mel_vocab_size"]
+    assert o.NMEL * o.NLEV == g["table_rows"]
+    assert round(g["table_rows"] * g["table_dim"] / 1e6, 1) == g["table_weights_rounded_millions"]
+    # 20 frames per second of audio, 24k frames for a 20-minute clip
+    for sec in (1, 2, 10, 30, 60):
+        assert o.frames_for_length(g["sample_rate_hz"] * sec) == g["tokens_per_second"] * sec
+    assert o.frames_for_length(g["max_clip_minutes"] * 60 * g["sample_rate_hz"]) == g["tokens_for_max_clip"]
+    # the clamp ends
+    assert o.log_clamp(0.0) == g["dmel_min_value"]
+    assert o.log_clamp(1e30) == g["dmel_max_value"]
+
+
+def test_frame_count_edges(oracle_mod):
+    o = oracle_mod
+    assert [o.frames_for_length(n) for n in (0, 1, 799, 800, 801, 1599, 1600)] == [0, 0, 0, 1, 1, 1, 2]
+    assert o.frames_for_length(-1) == -1
+    fo = o.frame_offsets(np.array([0, 799, 2399, 2399, 4000]))
+    assert fo.tolist() == [0, 0, 2, 2, 4]
+    with pytest.raises(ValueError):
+        o.frame_offsets(np.array([0, 900, 800]))
+    with pytest.raises(ValueError):
+        o.frame_offsets(np.array([5, 900]))
+
+
+# ---------------------------------------------------------------- window and DFT
+
+def test_window_is_scipy_periodic_hann(oracle_mod):
+    from scipy.signal import get_window
+    w = oracle_mod.window()
+    ref = get_window("hann", 1600, fftbins=True)
+    np.testing.assert_allclose(w, ref, rtol=0, atol=1e-15)
+    assert abs(w.sum() - 800.0) < 1e-9
+    assert abs((w * w).sum() - 600.0) < 1e-9
+
+
+def test_power_matches_numpy_rfft(oracle_mod):
+    from scipy.signal import get_window
+    r = np.random.default_rng(3)
+    w = get_window("hann", 1600, fftbins=True)
+    for scale in (1e-4, 0.3, 1.0):
+        fr = r.uniform(-scale, scale, 1600)
+        ref = np.abs(np.fft.rfft(w * fr)) ** 2
+        P = oracle_mod.power(fr)
+        assert P.shape == (801,)
+        np.testing.assert_allclose(P, ref, rtol=1e-9, atol=1e-11 * ref.max())
+
+
+@pytest.mark.parametrize("k0,A,phi", [(2, 1.0, 0.0), (100, 0.5, 1.1), (437, 0.25, -2.0), (798, 0.9, 3.0)])
+def test_closed_form_tone(oracle_mod, k0, A, phi):
+    """A cos(2 pi k0 n / 1600 + phi) under a periodic Hann window: P_k0 = (400 A)^2,
+    P_{k0 +- 1} = (200 A)^2, every other bin zero, for any phase."""
+    n = np.arange(1600)
+    P = oracle_mod.power(A * np.cos(2 * np.pi * k0 * n / 1600 + phi))
+    peak = (400 * A) ** 2
+    assert abs(P[k0] - peak) < 1e-9 * peak
+    assert abs(P[k0 - 1] - (200 * A) ** 2) < 1e-9 * peak
+    assert abs(P[k0 + 1] - (200 * A) ** 2) < 1e-9 * peak
+    rest = np.delete(P, [k0 - 1, k0, k0 + 1])
+    assert rest.max() < 1e-12 * peak
+
+
+def test_parseval(oracle_mod):
+    r = np.random.default_rng(4)
+    w = oracle_mod.window()
+    for _ in range(3):
+        fr = r.standard_normal(1600)
+        P = oracle_mod.power(fr)
+        lhs = P[0] + 2 * P[1:800].sum() + P[800]
+        rhs = 1600 * np.sum((w * fr) ** 2)
+        assert abs(lhs - rhs) < 1e-10 * rhs
+
+
+# ---------------------------------------------------------------- mel filterbank
+
+def test_htk_mel_scale_textbook(oracle_mod):
+    # the HTK scale puts 1000 Hz at (very nearly) 1000 mel
+    assert abs(oracle_mod.hz_to_mel(1000.0) - 1000.0) < 0.05
+    for f in (0.0, 123.4, 1000.0, 8000.0):
+        assert abs(oracle_mod.mel_to_hz(oracle_mod.hz_to_mel(f)) - f) < 1e-9
+
+
+def test_filterbank_matches_transformers_htk(oracle_mod):
+    from transformers.audio_utils import mel_filter_bank
+    ref = mel_filter_bank(num_frequency_bins=801, num_mel_filters=80, min_frequency=0.0, max_frequency=8000.0,
+                          sampling_rate=16000, norm=None, mel_scale="htk")
+    fb = oracle_mod.filterbank()
+    assert ref.shape == (801, 80)
+    np.testing.assert_allclose(fb, ref.T, rtol=0, atol=1e-12)
+
+
+def test_filterbank_matches_torchaudio_htk(oracle_mod):
+    import torchaudio.functional as AF
+    ref = AF.melscale_fbanks(n_freqs=801, f_min=0.0, f_max=8000.0, n_mels=80, sample_rate=16000, norm=None,
+                             mel_scale="htk").double().numpy()
+    np.testing.assert_allclose(oracle_mod.filterbank(), ref.T, rtol=0, atol=2e-5)
+
+
+def test_filterbank_partition_of_unity(oracle_mod):
+    """Adjacent triangles share their points, so between the peak of the first filter and the
+    peak of the last one the 80 weights at every bin add up to 1."""
+    fb = oracle_mod.filterbank()
+    pk_first = np.argmax(fb[0])
+    pk_last = np.argmax(fb[79])
+    s = fb[:, pk_first + 1:pk_last].sum(axis=0)  # bins strictly between the two peaks
+    np.testing.assert_allclose(s, 1.0, atol=1e-12)
+    assert (fb >= 0).all() and fb.max() <= 1.0 + 1e-12
+    assert (fb.sum(axis=1) > 0).all()  # no empty filter at 10 Hz bin spacing
+
+
+def test_tone_lights_expected_mel_bin(oracle_mod):
+    """A bin-centred tone at the peak bin of filter b (taken from the transformers filterbank)
+    gives its largest mel energy in channel b, for every channel wider than the Hann main lobe."""
+    from transformers.audio_utils import mel_filter_bank
+    ref = mel_filter_bank(num_frequency_bins=801, num_mel_filters=80, min_frequency=0.0, max_frequency=8000.0,
+                          sampling_rate=16000, norm=None, mel_scale="htk")
+    n = np.arange(1600)
+    for b in range(10, 80):
+        k = int(np.argmax(ref[:, b]))
+        M = oracle_mod.mel(0.5 * np.cos(2 * np.pi * k * n / 1600))
+        assert int(np.argmax(M)) == b, (b, k)
+
+
+# ---------------------------------------------------------------- log, clamp, quantise
+
+def test_quantiser_levels(oracle_mod):
+    o = oracle_mod
+    for k in range(16):
+        lo = -7.0 + 9.0 * k / 16
+        hi = -7.0 + 9.0 * (k + 1) / 16
+        assert o.quantise(lo + 1e-9) == k
+        assert o.quantise(0.5 * (lo + hi)) == k
+        if k < 15:
+            assert o.quantise(hi - 1e-9) == k
+    assert o.quantise(-7.0) == 0
+    assert o.quantise(2.0) == 15
+    assert o.log_clamp(0.0) == -7.0
+    assert o.log_clamp(float("nan")) == -7.0
+    assert o.log_clamp(float("inf")) == 2.0
+    assert o.log_clamp(-5.0) == -7.0
+    assert abs(o.log_clamp(1e-3) - (-3.0)) < 1e-15
+    assert o.log_clamp(1e5) == 2.0
+
+
+def test_silence_codes_zero(oracle_mod):
+    wav = np.zeros(16000, np.float32)
+    c, lh = oracle_mod.codes(wav, np.array([0, 16000]))
+    assert c.shape == (20, 80)
+    assert (c == 0).all() and (lh == -7.0).all()
+
+
+def test_full_scale_noise_reaches_top_level(oracle_mod):
+    r = np.random.default_rng(5)
+    wav = np.where(r.random(16000 * 4) < 0.5, -1.0, 1.0).astype(np.float32)
+    c = oracle_mod.codes(wav, np.array([0, wav.size]), want_lhat=False)
+    assert (c[1:] == 15).mean() >= 0.99  # frame 0 is half zeros
+    n = np.arange(1600 * 4)
+    tone = np.cos(2 * np.pi * 100 * n / 1600).astype(np.float32)  # 1 kHz, bin-centred, full scale
+    c2 = oracle_mod.codes(tone, np.array([0, tone.size]), want_lhat=False)
+    fb = oracle_mod.filterbank()
+    b = int(np.argmax(fb[:, 100]))
+    assert (c2[1:, b] == 15).all()
+
+
+def test_gain_shift_is_one_level(oracle_mod):
+    """x -> x * 10^(9/32) multiplies every energy by 10^(9/16), i.e. adds 0.5625 (one level) to L."""
+    wav, off = synth.one_clip_2s()
+    g = 10.0 ** (9.0 / 32.0)
+    c0, l0 = oracle_mod.codes(wav, off)
+    c1, l1 = oracle_mod.codes((wav.astype(np.float64) * g).astype(np.float32), off)
+    inner = (l0 > -7.0 + 1e-6) & (l0 < 2.0 - 0.5625 - 1e-6)
+    assert inner.sum() > 500
+    # fp32 rounding of the scaled input perturbs L by ~1e-7
+    assert np.max(np.abs((l1 - l0)[inner] - 0.5625)) < 1e-5
+    safe = inner & (oracle_mod.boundary_distance(l0) > 1e-4)
+    assert (c1[safe].astype(int) - c0[safe].astype(int) == 1).all()
+
+
+def test_nonfinite_samples_give_valid_codes(oracle_mod):
+    wav = np.zeros(8000, np.float32)
+    wav[1000] = np.nan
+    wav[5000] = np.inf
+    c = oracle_mod.codes(wav, np.array([0, 8000]), want_lhat=False)
+    assert c.shape == (10, 80) and c.max() <= 15
+
+
+# ---------------------------------------------------------------- framing: streaming and ragged
+
+def test_streaming_equals_offline(oracle_mod):
+    wav, off = synth.one_clip_2s()
+    full = oracle_mod.codes(wav, off, want_lhat=False)
+    tail = np.zeros((1, 800), np.float32)
+    got = []
+    for k in range(40):
+        piece = wav[800 * k:800 * (k + 1)]
+        got.append(oracle_mod.codes(piece, np.array([0, 800]), tails=tail, want_lhat=False))
+        tail = oracle_mod.tails_out(piece, np.array([0, 800]), tails=tail)
+    np.testing.assert_array_equal(np.concatenate(got), full)
+
+
+def test_tail_out_rules(oracle_mod):
+    x = np.arange(2000, dtype=np.float32)
+    t_in = -np.ones((1, 800), np.float32)
+    out = oracle_mod.tails_out(x, np.array([0, 2000]), tails=t_in)
+    np.testing.assert_array_equal(out[0], x[800:1600])  # F = 2: samples [800, 1600)
+    out0 = oracle_mod.tails_out(x[:500], np.array([0, 500]), tails=t_in)
+    np.testing.assert_array_equal(out0[0], t_in[0])  # F = 0: tail passes through
+
+
+def test_ragged_equals_per_clip(oracle_mod):
+    r = np.random.default_rng(6)
+    lengths = [800, 0, 2399, 799, 5000, 1600]
+    off = synth.offsets_from_lengths(lengths)
+    wav = r.uniform(-0.5, 0.5, int(off[-1])).astype(np.float32)
+    allc = oracle_mod.codes(wav, off, want_lhat=False)
+    fo = oracle_mod.frame_offsets(off)
+    for c, n in enumerate(lengths):
+        one = oracle_mod.codes(wav[off[c]:off[c + 1]], np.array([0, n]), want_lhat=False)
+        np.testing.assert_array_equal(allc[fo[c]:fo[c + 1]], one)
+
+
+def test_frame_subset_equals_full_run(oracle_mod):
+    wav, off = synth.one_clip_2s()
+    full = oracle_mod.codes(wav, off, want_lhat=False)
+    ids = np.array([39, 0, 17, 17, 5])
+    np.testing.assert_array_equal(oracle_mod.codes(wav, off, frame_ids=ids, want_lhat=False), full[ids])
+    with pytest.raises(ValueError):
+        oracle_mod.codes(wav, off, frame_ids=np.array([40]))
+
+
+def test_frame_alignment_closed_form(oracle_mod):
+    """Frame t of a clip sees samples [800 (t - 1), 800 (t + 1)): a clip that is silent except
+    for a bin-centred tone in [800 t0, 800 t0 + 800) lights frames t0 and t0 + 1 only."""
+    x = np.zeros(8000, np.float32)
+    t0 = 4
+    n = np.arange(800)
+    x[800 * t0:800 * t0 + 800] = np.cos(2 * np.pi * 100 * n / 1600)
+    c = oracle_mod.codes(x, np.array([0, 8000]), want_lhat=False)
+    lit = np.where(c.max(axis=1) > 0)[0].tolist()
+    assert lit == [t0, t0 + 1]
+    # and the oracle's frame equals a direct slice under the same rule
+    P = oracle_mod.power(_frame_of(x.astype(np.float64), t0))
+    assert P.max() > 1e3
+
+
+# ---------------------------------------------------------------- embedding and RMSNorm
+
+def test_embed_bruteforce_tiny_integer_table(oracle_mod):
+    r = np.random.default_rng(7)
+    dim = 8
+    T = r.integers(-8, 9, size=(1280, dim)).astype(np.float64)
+    codes = r.integers(0, 16, size=(5, 80)).astype(np.uint8)
+    got = oracle_mod.embed(codes, T)
+    for f in range(5):
+        for j in range(dim):
+            s = 0
+            for b in range(80):
+                s += int(T[16 * b + int(codes[f, b]), j])
+            assert got[f, j] == s
+    # a row layout 16 * c + b (transposed) would give a different answer
+    alt = np.array([[sum(T[16 * int(codes[f, b]) % 1280 + b, j] for b in range(80)) for j in range(dim)]
+                    for f in range(5)])
+    assert not np.array_equal(alt, got)
+
+
+def test_embed_order_invariance(oracle_mod):
+    """The sum does not depend on which bin is added first: permuting bins together with the
+    table's 16-row blocks leaves every frame vector unchanged."""
+    r = np.random.default_rng(8)
+    T = r.normal(0, 0.02, (1280, 16))
+    codes = r.integers(0, 16, size=(7, 80)).astype(np.uint8)
+    perm = r.permutation(80)
+    Tp = T.reshape(80, 16, 16)[perm].reshape(1280, 16)
+    a = oracle_mod.embed(codes, T)
+    b = oracle_mod.embed(codes[:, perm], Tp)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_closed_form(oracle_mod):
+    c = 0.0125
+    T = np.full((1280, 24), c)
+    g = np.linspace(0.5, 1.5, 24)
+    codes = np.random.default_rng(9).integers(0, 16, size=(3, 80)).astype(np.uint8)
+    y = oracle_mod.embed(codes, T, g, eps=1e-6)
+    x = 80 * c
+    np.testing.assert_allclose(y, np.broadcast_to(g * x / np.sqrt(x * x + 1e-6), y.shape), rtol=1e-14)
+
+
+def test_rmsnorm_matches_torch(oracle_mod):
+    import torch
+    r = np.random.default_rng(10)
+    T = r.normal(0, 0.02, (1280, 64))
+    g = r.normal(1, 0.1, 64)
+    codes = r.integers(0, 16, size=(6, 80)).astype(np.uint8)
+    x = oracle_mod.embed(codes, T)
+    y = oracle_mod.embed(codes, T, g, eps=1e-6)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x), (64,), torch.from_numpy(g), eps=1e-6).numpy()
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=0)
+
+
+def test_embed_rejects_bad_code(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.embed(np.full((1, 80), 16, np.uint8), np.zeros((1280, 8)))
