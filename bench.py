@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Benchmark of the dMel front end on B200: dMel tokens/s (waveform to 6144-d bf16 vector) and
+the fraction of the HBM roofline.
+
+Workload: 64 clips x 10 s of 16 kHz fp32 audio (pink noise + chirps, 10% silent clips, 5%
+clipped), 12,800 frames, bf16 table 1280 x 6144 ~ N(0, 0.02), RMSNorm on (eps 1e-6), bf16 out.
+A step is one dmel_forward over the whole batch with inputs resident in HBM; L2 is flushed
+(256 MB write) between timed steps and each step is timed with its own CUDA events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank runs its own copy of the batch on its own GPU (replicas,
+no collective on the data path); the step time is the max over ranks. --impl reference times
+the CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dMel tokens/sec (waveform to 6144-d bf16 embed); % of HBM roofline"
+WORKLOAD = ("batch64_10s: 64 clips x 10 s of 16 kHz mono fp32 (pink noise + linear chirp, 10% silent, "
+            "5% clipped), 12,800 frames, bf16 table 1280x6144 N(0,0.02), RMSNorm on (eps 1e-6, w~N(1,0.1)), "
+            "bf16 out")
+DIM = 6144
+# algorithmic HBM bytes per frame of the whole path (bf16 out): 800 new fp32 samples in,
+# 6144 bf16 out
+PATH_BYTES_PER_FRAME = 800 * 4 + DIM * 2
+# embedding stage (the dominant kernels): codes in (80 B), bf16 vector out
+EMBED_BYTES_PER_FRAME = 80 + DIM * 2
+# the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144
+ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of one GPU while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(wav, off, table64, g64, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands (codes + embedding + RMSNorm, fp64) on a bounded random sample of
+    the workload's frames, on this host's cores."""
+    from oracle import oracle
+    oracle.build()
+    fo = oracle.frame_offsets(off)
+    F = int(fo[-1])
+    rng = np.random.default_rng(77)
+
+    def run(n):
+        ids = np.sort(rng.choice(F, n, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        c = oracle.codes(wav, off, frame_ids=ids, want_lhat=False)
+        oracle.embed(c, table64, g64, 1e-6)
+        return time.perf_counter() - t0
+
+    n0 = 64
+    t0 = run(n0)
+    n = int(min(F, max(n0, n0 * budget_s / max(t0, 1e-6))))
+    t = run(n)
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} random frames of the {F}-frame workload (codes + embedding + RMSNorm, fp64)"}
+
+
+def load_workload():
+    from encoder_free_audio_b200 import synth
+    wav, off = synth.batch64_10s()
+    table = synth.table()
+    g = synth.rms_weight()
+    return wav, off, table, g
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import oracle
+    import torch
+    wav, off, table, g = load_workload()
+    tb = torch.from_numpy(table).to(torch.bfloat16).float().numpy().astype(np.float64)
+    gb = torch.from_numpy(g).to(torch.bfloat16).float().numpy().astype(np.float64)
+    oracle.build()
+    F = int(oracle.frame_offsets(off)[-1])
+    rng = np.random.default_rng(78)
+    per_step = 128
+    times = []
+    for i in range(args.warmup + args.steps):
+        ids = np.sort(rng.choice(F, per_step, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        c = oracle.codes(wav, off, frame_ids=ids, want_lhat=False)
+        oracle.embed(c, tb, gb, 1e-6)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = per_step * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "step": f"{per_step} random frames of the workload per step"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": f"{per_step} random frames per step, {args.steps} timed steps"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from encoder_free_audio_b200 import build, dmel
+    from encoder_free_audio_b200.frontend import FrontEnd
+    build.build()
+
+    wav, off, table, g = load_workload()
+    T = torch.from_numpy(table).to(torch.bfloat16).to(dev)
+    G = torch.from_numpy(g).to(torch.bfloat16).to(dev)
+    fe = FrontEnd(T, G, 1e-6, torch.bfloat16)
+    plan = fe.plan(off)
+    F = plan.n_frames
+    wav_d = torch.from_numpy(wav).to(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------- device-resident timed region
+    for _ in range(args.warmup):
+        flush.zero_()
+        fe.forward(wav_d, plan)
+    barrier()
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches = 0
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        fe.forward(wav_d, plan)
+        evs[i][1].record(stream)
+        launches += dmel.dmel_last_launch_count()
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(step_ms))
+
+    # ---------------------------------------------------------- stage breakdown (same kernels)
+    # dmel_codes and dmel_embed called separately, each bracketed by events on the stream the
+    # kernels run on: the embedding stage is the dominant one.
+    ws = plan.workspace
+    codes_ms, embed_ms = [], []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        dmel.dmel_codes(wav_d, plan.sample_offsets, plan.frame_offsets, F, plan.codes)
+        e1.record(stream)
+        dmel.dmel_embed(plan.codes, T, plan.out, rms_weight=G, eps=1e-6, workspace=ws)
+        e2.record(stream)
+        e2.synchronize()
+        if i >= args.warmup:
+            codes_ms.append(e0.elapsed_time(e1))
+            embed_ms.append(e1.elapsed_time(e2))
+    clocks = sampler.stop()
+
+    # ---------------------------------------------------------- end to end from host memory
+    wav_h = torch.from_numpy(wav).pin_memory()
+    codes_h = torch.empty((F, 80), dtype=torch.uint8).pin_memory()
+    for _ in range(args.warmup):
+        fe.forward_host(wav_h, plan, codes_h)
+    barrier()
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_evs[i][0].record(stream)
+        fe.forward_host(wav_h, plan, codes_h)
+        e2e_evs[i][1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
+    err_bits = dmel.dmel_get_device_error(clear=True)
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
+    pk = peaks()
+    value = world * F * args.steps / (total_ms / 1e3)
+    emb_avg_s = statistics.mean(embed_ms) / 1e3
+    emb_achieved = EMBED_BYTES_PER_FRAME * F / emb_avg_s / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "frames_per_gpu": F, "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)",
+                   "compute": "fp64 transform, bf16 x bf16 -> fp32 tensor-core sum, bf16 out"},
+        "hbm_roofline_frac": PATH_BYTES_PER_FRAME * value / world / (pk["hbm_gbs"] * 1e9),
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
+        "e2e": {"value": world * F * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(wav.nbytes), "d2h_bytes_per_step": int(F * 80)},
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "achieved": emb_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": emb_achieved / pk["hbm_gbs"], "traffic": None,
+                     "kernel": "dmel_embed stage (embed_tc_kernel + rms_rescale_kernel)",
+                     "peak_source": pk["source"]},
+        "roofline_tensor": {"achieved": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12,
+                            "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                            "frac": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12 / pk["bf16_tflops_sustained"],
+                            "note": "one-hot product flops 2*1280*6144 per frame, sustained bf16 peak"},
+        "stages_ms": {"codes": statistics.mean(codes_ms), "embed": statistics.mean(embed_ms)},
+        "device_error_bits": err_bits,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        tb = T.float().cpu().numpy().astype(np.float64)
+        gb = G.float().cpu().numpy().astype(np.float64)
+        line["cpu_baseline"] = cpu_baseline(wav, off, tb, gb)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,212 @@
+// C ABI of the dMel front end: argument checks, workspace layout and dispatch to the kernels.
+#include <cstring>
+#include <mutex>
+
+#include "dmel.h"
+#include "common.cuh"
+#include "dmel_debug.h"
+#include "internal.h"
+
+namespace dmel {
+namespace {
+
+__device__ uint32_t d_error_word;
+
+thread_local int t_last_launches = 0;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int major = 0;
+  uint32_t *err = nullptr;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[256];
+
+// Per-device facts, looked up once: SM count, compute capability, address of the error word.
+cudaError_t device_info(DeviceInfo *out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo &d = g_dev[dev];
+  if (!d.ready) {
+    if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return e;
+    void *p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, d_error_word)) != cudaSuccess) return e;
+    d.err = static_cast<uint32_t *>(p);
+    d.ready = true;
+  }
+  *out = d;
+  return cudaSuccess;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool dtype_ok(dmel_dtype t) { return t == DMEL_F32 || t == DMEL_BF16; }
+
+// Checks of the embedding arguments; check_codes = false when the codes buffer is the
+// library's own (dmel_forward without codes_out).
+dmel_status check_embed_args(const uint8_t *codes, bool check_codes, int64_t n_frames, const void *table,
+                             dmel_dtype table_dtype, int D, const void *rms_weight, float eps, const void *out,
+                             dmel_dtype out_dtype) {
+  if (n_frames < 0 || D <= 0 || D % 8 != 0) return DMEL_ERR_INVALID_ARG;
+  if (!dtype_ok(table_dtype) || !dtype_ok(out_dtype)) return DMEL_ERR_INVALID_ARG;
+  if (n_frames == 0) return DMEL_OK;
+  if (!table || !out) return DMEL_ERR_INVALID_ARG;
+  if (check_codes && (codes == nullptr || !aligned(codes, 16))) return DMEL_ERR_INVALID_ARG;
+  if (rms_weight && !(eps > 0.0f)) return DMEL_ERR_INVALID_ARG;
+  // 16-byte vector access of rows: table, weight and output bases 16-byte aligned; codes rows
+  // (80 bytes) read as 16-byte vectors by the tensor-core path.
+  if (!aligned(table, 16) || !aligned(out, 16) || (rms_weight && !aligned(rms_weight, 16)))
+    return DMEL_ERR_INVALID_ARG;
+  if (!embed_uses_tensor_cores(table_dtype, D) && D > 16384) return DMEL_ERR_INVALID_ARG;
+  return DMEL_OK;
+}
+
+dmel_status check_codes_args(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                             int n_clips, int64_t n_frames, const uint8_t *codes) {
+  if (n_clips < 0 || n_frames < 0) return DMEL_ERR_INVALID_ARG;
+  if (n_clips == 0 && n_frames > 0) return DMEL_ERR_INVALID_ARG;
+  if (n_clips == 0) return DMEL_OK;
+  if (!sample_offsets || !frame_offsets) return DMEL_ERR_INVALID_ARG;
+  if (n_frames > 0 && (!wav || !codes)) return DMEL_ERR_INVALID_ARG;
+  return DMEL_OK;
+}
+
+dmel_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DMEL_OK : DMEL_ERR_CUDA; }
+
+}  // namespace
+}  // namespace dmel
+
+using namespace dmel;
+
+extern "C" {
+
+int64_t dmel_frames_for_length(int64_t n_samples) { return n_samples < 0 ? -1 : n_samples / kHop; }
+
+dmel_status dmel_frame_offsets(const int64_t *h_sample_offsets, int n_clips, int64_t *h_frame_offsets) {
+  if (!h_sample_offsets || !h_frame_offsets || n_clips < 0) return DMEL_ERR_INVALID_ARG;
+  if (h_sample_offsets[0] != 0) return DMEL_ERR_INVALID_ARG;
+  int64_t acc = 0;
+  for (int c = 0; c < n_clips; ++c)
+    if (h_sample_offsets[c + 1] < h_sample_offsets[c]) return DMEL_ERR_INVALID_ARG;
+  h_frame_offsets[0] = 0;
+  for (int c = 0; c < n_clips; ++c) {
+    acc += dmel_frames_for_length(h_sample_offsets[c + 1] - h_sample_offsets[c]);
+    h_frame_offsets[c + 1] = acc;
+  }
+  return DMEL_OK;
+}
+
+size_t dmel_workspace_size(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm,
+                           int with_codes_out) {
+  if (n_frames <= 0 || embed_dim <= 0) return 0;
+  size_t bytes = 0;
+  if (!with_codes_out) bytes += round_up((size_t)n_frames * kMel, 256);
+  bytes += round_up(embed_workspace_bytes(n_frames, embed_dim, table_dtype, with_rmsnorm), 256);
+  return bytes;
+}
+
+dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                       int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes, dmel_stream_t stream) {
+  t_last_launches = 0;
+  dmel_status st = check_codes_args(wav, sample_offsets, frame_offsets, n_clips, n_frames, codes);
+  if (st != DMEL_OK || n_clips == 0) return st;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  cudaError_t e = launch_codes(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, codes, d.err,
+                               d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
+dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
+                       const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
+                       size_t workspace_bytes, dmel_stream_t stream) {
+  t_last_launches = 0;
+  dmel_status st =
+      check_embed_args(codes, true, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype);
+  if (st != DMEL_OK || n_frames == 0) return st;
+  const size_t need = embed_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  cudaError_t e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype,
+                               workspace, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
+dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                         int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                         dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                         dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
+                         dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (n_clips < 0 || n_frames < 0 || (n_clips == 0 && n_frames > 0)) return DMEL_ERR_INVALID_ARG;
+  if (!sample_offsets && n_clips > 0) return DMEL_ERR_INVALID_ARG;
+  if (!frame_offsets && n_clips > 0) return DMEL_ERR_INVALID_ARG;
+  if (n_frames > 0 && !wav) return DMEL_ERR_INVALID_ARG;
+  dmel_status st = check_embed_args(codes_out, codes_out != nullptr, n_frames, table, table_dtype, embed_dim,
+                                    rms_weight, eps, out, out_dtype);
+  if (st != DMEL_OK) return st;
+  if (n_clips == 0) return DMEL_OK;
+  const size_t need = dmel_workspace_size(n_frames, embed_dim, table_dtype, rms_weight != nullptr, codes_out != nullptr);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  uint8_t *codes = codes_out;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  if (!codes && n_frames > 0) {
+    codes = ws;
+    ws += round_up((size_t)n_frames * kMel, 256);
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = launch_codes(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, codes, d.err,
+                               d.sms, s, &launches);
+  if (e == cudaSuccess)
+    e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype, ws, d.err, d.sms,
+                     s, &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
+dmel_status dmel_get_device_error(uint32_t *h_bits, int clear) {
+  if (!h_bits) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DMEL_ERR_CUDA;
+  if (cudaMemcpy(h_bits, d.err, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (clear && cudaMemset(d.err, 0, sizeof(uint32_t)) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (clear && cudaDeviceSynchronize() != cudaSuccess) return DMEL_ERR_CUDA;
+  return DMEL_OK;
+}
+
+const char *dmel_status_string(dmel_status status) {
+  switch (status) {
+    case DMEL_OK: return "DMEL_OK";
+    case DMEL_ERR_INVALID_ARG: return "DMEL_ERR_INVALID_ARG: argument out of contract";
+    case DMEL_ERR_UNSUPPORTED: return "DMEL_ERR_UNSUPPORTED: request not supported on this device";
+    case DMEL_ERR_CUDA: return "DMEL_ERR_CUDA: a CUDA call or kernel launch failed";
+  }
+  return "DMEL_ERR_UNKNOWN";
+}
+
+int dmel_last_launch_count(void) { return t_last_launches; }
+
+void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {
+  emulate_codes_frame_host(frame1600, codes80, lhat80);
+}
+
+}  // extern "C"

@@ -1,0 +1,537 @@
+// dMel embedding: x_j = sum_b T[16 b + c_b, j] over the 80 channels of a frame, optional
+// RMSNorm y_j = g_j x_j / sqrt(mean_j x_j^2 + eps) ("Inside Inkling: Audio Design",
+// Part 1 · Modeling: each (bin, level) pair owns one row, a frame's 80 rows are summed,
+// optional RMSNorm).
+//
+// Tensor-core path (bf16 table, D % 256 == 0). The row sum is the product
+// onehot(codes) [frames x 1280] . T [1280 x D]: a dense contraction with K = 1280, run as a
+// tcgen05 GEMM with fp32 accumulators in TMEM.
+//   tile 128 frames x 256 columns, K in 20 blocks of 64 (4 channels x 16 levels);
+//   warp 0      TMA loads of the table block [64 rows x 256 cols] (4 boxes of 64 x 64, 128B
+//               swizzle, L2 evict-last: the 15.7 MB table stays in L2);
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators) and issues the MMAs;
+//   warps 2-5   write the one-hot A block [128 frames x 64] in the 128B-swizzled K-major layout
+//               straight from the codes (one frame row per thread);
+//   warps 6-9   epilogue: TMEM -> registers -> output (streaming stores); with RMSNorm they store
+//               x and the frame's sum of squares over the 256 columns, and a second kernel
+//               scales each row once all 24 partial sums are known.
+// CUDA-core path (any other request): one block per frame, 80-row gather-sum in fp32.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dmel {
+namespace {
+
+// ---------------------------------------------------------------- element helpers
+
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
+  __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+  __stcs(reinterpret_cast<float4 *>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]);
+  u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]);
+  u.w = pack_bf16x2(v[6], v[7]);
+  __stcs(reinterpret_cast<uint4 *>(p), u);
+}
+
+__device__ __forceinline__ void load8_out(const float *p, float (&v)[8]) {
+  const float4 a = __ldcs(reinterpret_cast<const float4 *>(p));
+  const float4 b = __ldcs(reinterpret_cast<const float4 *>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8_out(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 u = __ldcs(reinterpret_cast<const uint4 *>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// ---------------------------------------------------------------- CUDA-core path
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtMaxDim = 16384;
+
+template <typename TT, typename OT>
+__global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t *__restrict__ codes, int64_t F,
+                                                                  const TT *__restrict__ table, int D,
+                                                                  const TT *__restrict__ g, float eps,
+                                                                  OT *__restrict__ out, uint32_t *err) {
+  extern __shared__ __align__(16) float xs[];  // [D] when RMSNorm is on
+  __shared__ int rows[kMel];
+  __shared__ float red[kSimtThreads / 32];
+  const int nv = D / 8;
+  for (int64_t f = blockIdx.x; f < F; f += gridDim.x) {
+    if (threadIdx.x < kMel) {
+      int c = codes[f * kMel + threadIdx.x];
+      if (c > 15) {
+        record_error(err, DMEL_DEVERR_CODE_RANGE);
+        c &= 15;
+      }
+      rows[threadIdx.x] = kLev * threadIdx.x + c;
+    }
+    __syncthreads();
+    float ss = 0.0f;
+    for (int v = threadIdx.x; v < nv; v += kSimtThreads) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int b = 0; b < kMel; ++b) {
+        float t[8];
+        load8(table + (size_t)rows[b] * D + 8 * v, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += t[i];
+      }
+      if (g) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          xs[8 * v + i] = acc[i];
+          ss += acc[i] * acc[i];
+        }
+      } else {
+        store8(out + f * D + 8 * v, acc);
+      }
+    }
+    if (g) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+      __syncthreads();
+      float tot = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kSimtThreads / 32; ++w) tot += red[w];
+      const float inv = 1.0f / sqrtf(tot / (float)D + eps);
+      for (int v = threadIdx.x; v < nv; v += kSimtThreads) {
+        float gv[8], y[8];
+        load8(g + 8 * v, gv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = gv[i] * (xs[8 * v + i] * inv);
+        store8(out + f * D + 8 * v, y);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------- RMSNorm row scaling
+
+// One warp per frame: ss = sum of the n_ct partial sums of squares, then
+// out_j <- g_j * (out_j / sqrt(ss / D + eps)) in place.
+template <typename OT>
+__global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, int64_t F, int D,
+                                                          const __nv_bfloat16 *__restrict__ g,
+                                                          const float *__restrict__ partials, int n_ct, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t f = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < F; f += warps) {
+    float ss = 0.0f;
+    for (int c = lane; c < n_ct; c += 32) ss += partials[(int64_t)c * F + f];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float inv = 1.0f / sqrtf(ss / (float)D + eps);
+    OT *row = out + f * D;
+    for (int v = lane; v < D / 8; v += 32) {
+      float x[8], gv[8], y[8];
+      load8_out(row + 8 * v, x);
+      load8(g + 8 * v, gv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) y[i] = gv[i] * (x[i] * inv);
+      store8(row + 8 * v, y);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- tensor-core path
+
+namespace tc {
+constexpr int BM = 128;                       // frames per tile (TMEM lanes)
+constexpr int BN = 256;                       // table columns per tile
+constexpr int BK = 64;                        // K per pipeline stage: 4 channels x 16 levels
+constexpr int STAGES = 4;
+constexpr int KBLOCKS = kRows / BK;           // 20
+constexpr int A_STAGE = BM * BK * 2;          // 16 KB one-hot block
+constexpr int B_BOX = BK * 64 * 2;            // 8 KB: 64 K-rows x 64 columns
+constexpr int B_STAGE = BK * BN * 2;          // 32 KB table block
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_BAR = OFF_B + STAGES * B_STAGE;
+constexpr int N_BARS = 4 * STAGES + 5;
+constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack for the 1024-B swizzle atoms
+constexpr int THREADS = 320;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+}  // namespace tc
+
+template <typename OT, bool kRms>
+__global__ void __launch_bounds__(tc::THREADS, 1)
+    embed_tc_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
+                    OT *__restrict__ out, float *__restrict__ partials, uint32_t *err) {
+  using namespace tc;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_a = [&](int s) { return bar0 + 8u * s; };
+  auto full_b = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (3 * STAGES + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (3 * STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (3 * STAGES + 4);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+
+  const int n_tiles_n = D / BN;
+  const int64_t n_tiles = ((F + BM - 1) / BM) * n_tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_a(s), 128);
+      mbar_init(full_b(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 128);
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer: table blocks
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pending = 0;          // stages with a load issued
+      uint32_t pending_phase = 0;    // phase bit of that load, per stage
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        const int n0 = (int)(t % n_tiles_n) * BN;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_b(stage), B_STAGE);
+          const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i) tma_load_2d(dst + i * B_BOX, &tmap, n0 + 64 * i, kb * BK, full_b(stage), pol);
+          pending |= 1u << stage;
+          pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // every load issued must land before the block may exit
+      for (int s = 0; s < STAGES; ++s)
+        if (pending & (1u << s)) mbar_wait(full_b(s), (pending_phase >> s) & 1u, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+        const uint32_t acc = it & 1, acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(tempty(acc), acc_phase ^ 1u, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          if (!mbar_wait(full_a(stage), phase, err) || !mbar_wait(full_b(stage), phase, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(smem + OFF_A + stage * A_STAGE);
+          const uint32_t b0 = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // A: K-major, 128B swizzle, 8-row groups 1024 B apart; K advances 32 B per step.
+            const uint64_t adesc = smem_desc(a0 + 32u * k, 16u, 1024u, kSwizzle128B);
+            // B: MN-major, 128B swizzle; 64-column boxes 8 KB apart (LBO), 8-row K groups
+            // 1024 B apart (SBO); K advances 16 rows = 2 KB per step.
+            const uint64_t bdesc = smem_desc(b0 + 2048u * k, (uint32_t)B_BOX, 1024u, kSwizzle128B);
+            tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull(acc));
+      }
+      tc_commit(done_bar);
+      mbar_wait(done_bar, 0, err);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ one-hot A producers (row r per thread)
+    const int r = threadIdx.x - 64;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+      const int64_t f = (t / n_tiles_n) * BM + r;
+      uint32_t cw[20];
+      const bool valid = f < F;
+      if (valid) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + f * kMel);
+#pragma unroll
+        for (int q = 0; q < 5; ++q) {
+          const uint4 u = __ldg(src + q);
+          cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+        }
+        uint32_t bad = 0;
+#pragma unroll
+        for (int q = 0; q < 20; ++q) bad |= cw[q] & 0xF0F0F0F0u;
+        if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 20; ++q) cw[q] = 0;
+      }
+      const uint32_t row_off = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+#pragma unroll
+      for (int kb = 0; kb < KBLOCKS; ++kb) {
+        if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
+        uint8_t *rowp = smem + OFF_A + stage * A_STAGE + row_off;
+        const uint32_t w = cw[kb];  // codes of channels 4 kb .. 4 kb + 3
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          // 16-byte chunk ch holds levels 8 (ch & 1) .. +7 of channel 4 kb + (ch >> 1)
+          const uint32_t c = (w >> (8 * (ch >> 1))) & 15u;
+          const bool hit = valid && ((c >> 3) == (uint32_t)(ch & 1));
+          const uint32_t e = c & 7u;
+          const uint32_t one = (e & 1u) ? 0x3F800000u : 0x00003F80u;  // bf16 1.0 in the low or high half
+          uint4 v;
+          v.x = (hit && (e >> 1) == 0) ? one : 0u;
+          v.y = (hit && (e >> 1) == 1) ? one : 0u;
+          v.z = (hit && (e >> 1) == 2) ? one : 0u;
+          v.w = (hit && (e >> 1) == 3) ? one : 0u;
+          *reinterpret_cast<uint4 *>(rowp + ((ch ^ (r & 7)) << 4)) = v;  // 128B swizzle
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(full_a(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (TMEM lanes 32 (warp % 4) ..)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    bool ok = true;
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
+      const uint32_t acc = it & 1, acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(tfull(acc), acc_phase, err)) { ok = false; break; }
+      tc_fence_after();
+      const int64_t f = (t / n_tiles_n) * BM + r;
+      const int nt = (int)(t % n_tiles_n);
+      const bool valid = f < F;
+      OT *orow = out + (valid ? f : 0) * (int64_t)D + nt * BN;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+      float ss = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v0[16], v1[16];
+        tmem_ld16(tbase + c * 32, v0);
+        tmem_ld16(tbase + c * 32 + 16, v1);
+        tmem_wait_ld();
+        if (valid) {
+          float x[8];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t u = h < 2 ? v0[8 * h + i] : v1[8 * (h - 2) + i];
+              x[i] = __uint_as_float(u);
+              if (kRms) ss += x[i] * x[i];
+            }
+            store8(orow + c * 32 + 8 * h, x);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty(acc));
+      if (kRms && valid) partials[(int64_t)nt * F + f] = ss;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+template <typename K>
+cudaError_t set_smem_attr_once(K kernel, int bytes, bool *flags) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (flags[dev & 255]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) flags[dev & 255] = true;
+  return e;
+}
+
+template <typename OT, bool kRms>
+cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, float *partials,
+                      uint32_t *err, int num_sms, cudaStream_t stream) {
+  static bool attr[256] = {false};
+  cudaError_t e = set_smem_attr_once(embed_tc_kernel<OT, kRms>, tc::SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)kRows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)tc::BK};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(table), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * (D / tc::BN);
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  embed_tc_kernel<OT, kRms><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, partials, err);
+  return cudaGetLastError();
+}
+
+template <typename TT, typename OT>
+cudaError_t launch_simt(const uint8_t *codes, int64_t F, const TT *table, int D, const TT *g, float eps, OT *out,
+                        uint32_t *err, int num_sms, cudaStream_t stream) {
+  const int smem = g ? D * (int)sizeof(float) : 0;
+  static bool attr[256] = {false};
+  cudaError_t e = set_smem_attr_once(embed_simt_kernel<TT, OT>, kSimtMaxDim * (int)sizeof(float), attr);
+  if (e != cudaSuccess) return e;
+  const int64_t cap = (int64_t)num_sms * 8;
+  const int grid = (int)(F < cap ? F : cap);
+  embed_simt_kernel<TT, OT><<<grid, kSimtThreads, smem, stream>>>(codes, F, table, D, g, eps, out, err);
+  return cudaGetLastError();
+}
+
+template <typename OT>
+cudaError_t launch_rescale(OT *out, int64_t F, int D, const __nv_bfloat16 *g, const float *partials, float eps,
+                           int num_sms, cudaStream_t stream) {
+  const int64_t blocks_needed = (F + 7) / 8;
+  const int64_t cap = (int64_t)num_sms * 8;
+  const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
+  rms_rescale_kernel<OT><<<grid, 256, 0, stream>>>(out, F, D, g, partials, D / tc::BN, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
+  return table_dtype == DMEL_BF16 && embed_dim > 0 && embed_dim % tc::BN == 0;
+}
+
+size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
+  if (!with_rmsnorm || !embed_uses_tensor_cores(table_dtype, embed_dim) || n_frames <= 0) return 0;
+  return (size_t)n_frames * (size_t)(embed_dim / tc::BN) * sizeof(float);
+}
+
+cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,
+                         const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
+                         uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
+  if (F <= 0) return cudaSuccess;
+  cudaError_t e;
+  if (embed_uses_tensor_cores(table_dtype, D)) {
+    const auto *T = static_cast<const __nv_bfloat16 *>(table);
+    const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
+    float *partials = static_cast<float *>(workspace);
+    if (out_dtype == DMEL_BF16) {
+      auto *o = static_cast<__nv_bfloat16 *>(out);
+      e = g ? launch_tc<__nv_bfloat16, true>(codes, F, T, D, o, partials, err, num_sms, stream)
+            : launch_tc<__nv_bfloat16, false>(codes, F, T, D, o, nullptr, err, num_sms, stream);
+      if (e == cudaSuccess) ++*launches;
+      if (e == cudaSuccess && g) {
+        e = launch_rescale(o, F, D, g, partials, eps, num_sms, stream);
+        if (e == cudaSuccess) ++*launches;
+      }
+    } else {
+      auto *o = static_cast<float *>(out);
+      e = g ? launch_tc<float, true>(codes, F, T, D, o, partials, err, num_sms, stream)
+            : launch_tc<float, false>(codes, F, T, D, o, nullptr, err, num_sms, stream);
+      if (e == cudaSuccess) ++*launches;
+      if (e == cudaSuccess && g) {
+        e = launch_rescale(o, F, D, g, partials, eps, num_sms, stream);
+        if (e == cudaSuccess) ++*launches;
+      }
+    }
+    return e;
+  }
+  if (table_dtype == DMEL_BF16) {
+    const auto *T = static_cast<const __nv_bfloat16 *>(table);
+    const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
+    e = out_dtype == DMEL_BF16
+            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), err, num_sms, stream)
+            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), err, num_sms, stream);
+  } else {
+    const auto *T = static_cast<const float *>(table);
+    const auto *g = static_cast<const float *>(rms_weight);
+    e = out_dtype == DMEL_BF16
+            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), err, num_sms, stream)
+            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), err, num_sms, stream);
+  }
+  if (e == cudaSuccess) ++*launches;
+  return e;
+}
+
+}  // namespace dmel

@@ -1,0 +1,30 @@
+// Host-side interface between the library's translation units (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "dmel.h"
+
+namespace dmel {
+
+// Codes of n_frames frames (and the carried tails when tails_out != nullptr) on `stream`.
+// Adds the number of kernels launched to *launches.
+cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *foff, int n_clips, int64_t n_frames,
+                         const float *tails, float *tails_out, uint8_t *codes, uint32_t *err, int num_sms,
+                         cudaStream_t stream, int *launches);
+
+// Whether the tensor-core embedding path takes this request.
+bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim);
+
+// Scratch bytes the embedding needs (RMSNorm partial sums of the tensor-core path).
+size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm);
+
+// Embedding of n_frames codes; workspace holds embed_workspace_bytes(...) bytes.
+cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                         int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
+                         void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
+
+void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
+
+}  // namespace dmel

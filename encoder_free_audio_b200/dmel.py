@@ -1,0 +1,187 @@
+"""Python binding of the dMel C ABI (include/dmel.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and passes device pointers of
+torch tensors (plus the current CUDA stream) straight through; all computation runs in the
+CUDA kernels of libdmel.so. The library must have been built (``encoder_free_audio_b200.build``);
+importing this module without it raises, so nothing can silently fall back to another path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_build", "libdmel.so")
+
+DMEL_OK = 0
+DMEL_ERR_INVALID_ARG = 1
+DMEL_ERR_UNSUPPORTED = 2
+DMEL_ERR_CUDA = 3
+DMEL_F32 = 0
+DMEL_BF16 = 1
+DMEL_DEVERR_CODE_RANGE = 0x1
+DMEL_DEVERR_WAIT_TIMEOUT = 0x2
+DMEL_DEVERR_OFFSETS = 0x4
+
+HOP = 800
+WIN = 1600
+N_MEL = 80
+N_LEVELS = 16
+TABLE_ROWS = 1280
+MODEL_DIM = 6144
+
+
+class DmelError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib().dmel_status_string(status).decode()}")
+
+
+_L = None
+
+
+def _lib():
+    global _L
+    if _L is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdmel.so is not built ({LIB_PATH}); run encoder_free_audio_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        L.dmel_frames_for_length.argtypes = [i64]
+        L.dmel_frames_for_length.restype = i64
+        L.dmel_frame_offsets.argtypes = [vp, i32, vp]
+        L.dmel_frame_offsets.restype = i32
+        L.dmel_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+        L.dmel_workspace_size.restype = sz
+        L.dmel_codes.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, vp]
+        L.dmel_codes.restype = i32
+        L.dmel_embed.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, sz, vp]
+        L.dmel_embed.restype = i32
+        L.dmel_forward.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, vp,
+                                   sz, vp]
+        L.dmel_forward.restype = i32
+        L.dmel_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        L.dmel_get_device_error.restype = i32
+        L.dmel_status_string.argtypes = [i32]
+        L.dmel_status_string.restype = ctypes.c_char_p
+        L.dmel_last_launch_count.argtypes = []
+        L.dmel_last_launch_count.restype = i32
+        L.dmel_debug_codes_frame_host.argtypes = [vp, vp, vp]
+        L.dmel_debug_codes_frame_host.restype = None
+        _L = L
+    return _L
+
+
+def library():
+    """The loaded ctypes library (for symbol checks)."""
+    return _lib()
+
+
+# ---------------------------------------------------------------------------------- helpers
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float32:
+        return DMEL_F32
+    if t.dtype == torch.bfloat16:
+        return DMEL_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check(rc: int, where: str):
+    if rc != DMEL_OK:
+        raise DmelError(rc, where)
+
+
+# ---------------------------------------------------------------------------------- entry points
+
+def dmel_frames_for_length(n_samples: int) -> int:
+    return int(_lib().dmel_frames_for_length(int(n_samples)))
+
+
+def dmel_frame_offsets(sample_offsets) -> np.ndarray:
+    """Host int64 frame offsets [n_clips + 1] of host sample offsets."""
+    so = np.ascontiguousarray(np.asarray(sample_offsets, dtype=np.int64))
+    fo = np.zeros_like(so)
+    rc = _lib().dmel_frame_offsets(so.ctypes.data_as(ctypes.c_void_p), so.shape[0] - 1,
+                                   fo.ctypes.data_as(ctypes.c_void_p))
+    _check(rc, "dmel_frame_offsets")
+    return fo
+
+
+def dmel_workspace_size(n_frames: int, embed_dim: int, table_dtype: int, with_rmsnorm: bool,
+                        with_codes_out: bool) -> int:
+    return int(_lib().dmel_workspace_size(int(n_frames), int(embed_dim), int(table_dtype), int(bool(with_rmsnorm)),
+                                          int(bool(with_codes_out))))
+
+
+def dmel_codes(wav, sample_offsets, frame_offsets, n_frames: int, codes, tails=None, tails_out=None, stream=None):
+    """dmel_codes on torch CUDA tensors: wav fp32, offsets int64 [n_clips + 1], codes uint8
+    [n_frames, 80], tails / tails_out fp32 [n_clips, 800] or None."""
+    n_clips = sample_offsets.shape[0] - 1
+    rc = _lib().dmel_codes(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames), _ptr(tails),
+                           _ptr(tails_out), _ptr(codes), _stream(stream))
+    _check(rc, "dmel_codes")
+
+
+def dmel_embed(codes, table, out, rms_weight=None, eps: float = 1e-6, workspace=None, stream=None):
+    """dmel_embed on torch CUDA tensors: codes uint8 [F, 80], table [1280, D] fp32/bf16,
+    out [F, D] fp32/bf16, rms_weight [D] in the table's dtype or None, workspace uint8 or None."""
+    n = codes.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_embed(_ptr(codes), n, _ptr(table), _dtype_code(table), table.shape[1], _ptr(rms_weight),
+                           float(eps), _ptr(out), _dtype_code(out), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_embed")
+
+
+def dmel_forward(wav, sample_offsets, frame_offsets, n_frames: int, table, out, rms_weight=None, eps: float = 1e-6,
+                 tails=None, tails_out=None, codes_out=None, workspace=None, stream=None):
+    """dmel_forward on torch CUDA tensors (see dmel_codes and dmel_embed for the arguments)."""
+    n_clips = sample_offsets.shape[0] - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_forward(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames),
+                             _ptr(tails), _ptr(tails_out), _ptr(table), _dtype_code(table), table.shape[1],
+                             _ptr(rms_weight), float(eps), _ptr(out), _dtype_code(out), _ptr(codes_out),
+                             _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_forward")
+
+
+def dmel_get_device_error(clear: bool = True) -> int:
+    bits = ctypes.c_uint32(0)
+    rc = _lib().dmel_get_device_error(ctypes.byref(bits), int(clear))
+    _check(rc, "dmel_get_device_error")
+    return int(bits.value)
+
+
+def dmel_status_string(status: int) -> str:
+    return _lib().dmel_status_string(int(status)).decode()
+
+
+def dmel_last_launch_count() -> int:
+    return int(_lib().dmel_last_launch_count())
+
+
+def dmel_debug_codes_frame_host(frame1600: np.ndarray):
+    """Host emulation of the codes kernel's per-frame arithmetic (diagnostic, see dmel_debug.h)."""
+    fr = np.ascontiguousarray(frame1600, np.float32)
+    assert fr.shape == (WIN,)
+    codes = np.zeros(N_MEL, np.uint8)
+    lhat = np.zeros(N_MEL, np.float64)
+    _lib().dmel_debug_codes_frame_host(fr.ctypes.data_as(ctypes.c_void_p), codes.ctypes.data_as(ctypes.c_void_p),
+                                       lhat.ctypes.data_as(ctypes.c_void_p))
+    return codes, lhat

@@ -1,0 +1,82 @@
+"""Convenience layer over the C ABI for callers that hold torch tensors.
+
+``FrontEnd`` keeps the embedding table and RMSNorm weight on the device and runs
+``dmel_forward`` on batches of clips. ``plan()`` sizes the per-batch buffers (device offsets,
+frame offsets, output, workspace) once, so repeated calls allocate nothing new.
+``forward_host()`` is the end-to-end call: pinned host waveforms in, codes back on the host,
+frame vectors left on the device for the model that consumes them.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import dmel
+
+
+@dataclass
+class Plan:
+    sample_offsets_host: np.ndarray
+    frame_offsets_host: np.ndarray
+    sample_offsets: torch.Tensor   # device int64 [n_clips + 1]
+    frame_offsets: torch.Tensor    # device int64 [n_clips + 1]
+    n_samples: int
+    n_frames: int
+    out: torch.Tensor              # device [n_frames, D]
+    codes: torch.Tensor            # device uint8 [n_frames, 80]
+    workspace: torch.Tensor | None
+    wav: torch.Tensor              # device fp32 [n_samples] (input staging for forward_host)
+
+    @property
+    def n_clips(self) -> int:
+        return self.sample_offsets_host.shape[0] - 1
+
+
+class FrontEnd:
+    def __init__(self, table: torch.Tensor, rms_weight: torch.Tensor | None = None, eps: float = 1e-6,
+                 out_dtype: torch.dtype = torch.bfloat16):
+        assert table.is_cuda and table.dim() == 2 and table.shape[0] == dmel.TABLE_ROWS
+        self.table = table.contiguous()
+        self.rms_weight = None if rms_weight is None else rms_weight.to(table.dtype).contiguous()
+        self.eps = float(eps)
+        self.out_dtype = out_dtype
+        self.dim = int(table.shape[1])
+
+    def plan(self, sample_offsets_host) -> Plan:
+        so = np.ascontiguousarray(np.asarray(sample_offsets_host, np.int64))
+        fo = dmel.dmel_frame_offsets(so)
+        dev = self.table.device
+        F = int(fo[-1])
+        ws_bytes = dmel.dmel_workspace_size(F, self.dim, dmel._dtype_code(self.table), self.rms_weight is not None,
+                                            True)
+        return Plan(
+            sample_offsets_host=so,
+            frame_offsets_host=fo,
+            sample_offsets=torch.from_numpy(so).to(dev),
+            frame_offsets=torch.from_numpy(fo).to(dev),
+            n_samples=int(so[-1]),
+            n_frames=F,
+            out=torch.empty((F, self.dim), dtype=self.out_dtype, device=dev),
+            codes=torch.empty((F, dmel.N_MEL), dtype=torch.uint8, device=dev),
+            workspace=torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None,
+            wav=torch.empty(int(so[-1]), dtype=torch.float32, device=dev),
+        )
+
+    def forward(self, wav: torch.Tensor, plan: Plan, tails=None, tails_out=None, stream=None) -> torch.Tensor:
+        """Frame vectors of device waveforms `wav` (fp32 [n_samples]) into plan.out; codes into
+        plan.codes."""
+        dmel.dmel_forward(wav, plan.sample_offsets, plan.frame_offsets, plan.n_frames, self.table, plan.out,
+                          rms_weight=self.rms_weight, eps=self.eps, tails=tails, tails_out=tails_out,
+                          codes_out=plan.codes, workspace=plan.workspace, stream=stream)
+        return plan.out
+
+    def forward_host(self, wav_host: torch.Tensor, plan: Plan, codes_host: torch.Tensor, stream=None):
+        """End to end from host memory: copies the pinned fp32 waveforms to the device, runs the
+        front end, copies the codes (uint8 [n_frames, 80], pinned) back. All on one stream,
+        asynchronous; the caller synchronises."""
+        plan.wav.copy_(wav_host, non_blocking=True)
+        self.forward(plan.wav, plan, stream=stream)
+        codes_host.copy_(plan.codes, non_blocking=True)
+        return plan.out

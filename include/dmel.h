@@ -1,0 +1,154 @@
+/*
+ * dmel.h — C ABI of the dMel audio front end on NVIDIA B200 (sm_100a).
+ *
+ * The front end turns 16 kHz mono waveforms into one D-dimensional vector per 50 ms frame
+ * ("Inside Inkling: Audio Design", Part 1 · Modeling): 1600-sample windows at an 800-sample
+ * hop, power spectrum, 80 mel channels, log, clamp to [-7, 2], 16 levels per channel, then the
+ * sum of the 80 table rows 16*b + c_b of a 1280 x D embedding table with an optional RMSNorm.
+ * The readings of what the pages leave open (causal framing, periodic Hann window, 1600-point
+ * DFT, HTK mel triangles, log10 with a 1e-10 floor, 16 equal levels, row layout) are stated at
+ * each entry point below.
+ *
+ * Conventions for every call
+ *   - Pointers named h_* are host memory; every other array pointer is device memory of the
+ *     current CUDA device. The caller allocates and owns all of them; the library keeps no
+ *     pointer after a call returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *     never synchronise, except that the first call on each device uploads constant tables
+ *     (window, twiddles, mel weights) with a blocking copy; make that first call before any
+ *     stream capture.
+ *   - Arguments are checked on the host before anything is launched; a bad argument returns
+ *     DMEL_ERR_INVALID_ARG and launches nothing. A failed launch returns DMEL_ERR_CUDA.
+ *     Device-side faults are never used as error reports: kernels that find bad data (a code
+ *     above 15, an offset that does not match) record it in a device error word that
+ *     dmel_get_device_error() reads, and carry on with a clamped value.
+ *   - n_clips == 0 or n_frames == 0 is a valid call that does nothing.
+ *   - No entry point allocates device memory. Scratch space comes from the caller's workspace;
+ *     dmel_workspace_size() says how much.
+ */
+#ifndef DMEL_H
+#define DMEL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *dmel_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  DMEL_OK = 0,
+  DMEL_ERR_INVALID_ARG = 1, /* a pointer, size, offset or flag is out of contract */
+  DMEL_ERR_UNSUPPORTED = 2, /* valid request that this build does not run (e.g. no sm_100 device) */
+  DMEL_ERR_CUDA = 3         /* a CUDA runtime call or kernel launch failed */
+} dmel_status;
+
+typedef enum { DMEL_F32 = 0, DMEL_BF16 = 1 } dmel_dtype;
+
+#define DMEL_SAMPLE_RATE 16000
+#define DMEL_HOP 800        /* 50 ms: 20 frames per second */
+#define DMEL_WIN 1600       /* 100 ms window, also the DFT size */
+#define DMEL_N_BINS 801     /* one-sided DFT bins, 10 Hz apart */
+#define DMEL_N_MEL 80       /* mel channels */
+#define DMEL_N_LEVELS 16    /* quantisation levels per channel */
+#define DMEL_TABLE_ROWS 1280 /* 80 x 16 */
+#define DMEL_MODEL_DIM 6144 /* embedding width of the released model */
+
+/* Device error word bits (see dmel_get_device_error). */
+#define DMEL_DEVERR_CODE_RANGE 0x1u  /* a code above 15 reached an embedding kernel (used code & 15) */
+#define DMEL_DEVERR_WAIT_TIMEOUT 0x2u /* a pipeline wait inside a kernel gave up (results invalid) */
+#define DMEL_DEVERR_OFFSETS 0x4u     /* device frame offsets disagree with the sample offsets */
+
+/* Frames of one clip of n_samples samples: floor(n_samples / 800) (20 per second of audio;
+ * "Inside Inkling: Audio Design", Part 1 · Modeling). Host only, pure. Returns -1 for
+ * n_samples < 0. */
+int64_t dmel_frames_for_length(int64_t n_samples);
+
+/* Host exclusive scan of frame counts: h_frame_offsets[0] = 0,
+ * h_frame_offsets[c+1] = h_frame_offsets[c] + dmel_frames_for_length(len_c), where
+ * len_c = h_sample_offsets[c+1] - h_sample_offsets[c]. Both arrays have n_clips + 1 entries.
+ * This is the per-item frame count the serving renderer reports as "audio_tokens"
+ * ("Inside Inkling: Audio Design", Part 3 · Inference). Errors: DMEL_ERR_INVALID_ARG when a
+ * pointer is NULL, n_clips < 0, h_sample_offsets[0] != 0 or the offsets decrease. */
+dmel_status dmel_frame_offsets(const int64_t *h_sample_offsets, int n_clips, int64_t *h_frame_offsets);
+
+/* Bytes of device workspace that dmel_embed / dmel_forward need for this request (0 when none).
+ * with_codes_out: nonzero when the caller passes its own codes buffer to dmel_forward.
+ * with_rmsnorm: nonzero when rms_weight will be non-NULL. */
+size_t dmel_workspace_size(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm,
+                           int with_codes_out);
+
+/* dMel codes of every frame of a batch of clips.
+ *
+ * wav             fp32 samples of all clips, concatenated with no padding [sample_offsets[n_clips]]
+ * sample_offsets  int64 [n_clips + 1], device copy of the host offsets (start 0, non-decreasing)
+ * frame_offsets   int64 [n_clips + 1], device copy of dmel_frame_offsets() of the same offsets
+ * n_clips         number of clips (>= 0)
+ * n_frames        h_frame_offsets[n_clips] (host value, so no device read is needed to size the grid)
+ * tails           NULL, or fp32 [n_clips x 800]: the 800 samples that came before each clip
+ *                 (streaming); NULL means zeros
+ * tails_out       NULL, or fp32 [n_clips x 800]: receives the 800 samples that end at sample
+ *                 800*F of each clip (F its frame count), or the tail in when F == 0. May equal
+ *                 `tails` (it is written after every frame has been read).
+ * codes           uint8 [n_frames x 80], row-major, receives c_b in 0..15 per frame and channel
+ *
+ * Per frame t of a clip x (causal framing, "Inside Inkling: Audio Design", Part 1 · Modeling:
+ * hop 800, window 1600): s[n] = x[800 (t-1) + n], n < 1600, samples before the clip from the
+ * tail; P_k = |sum_n w[n] s[n] e^{-2 pi i k n/1600}|^2 with w the periodic Hann window;
+ * M_b = sum_k H_b(10 k Hz) P_k with 80 HTK mel triangles on 0..8000 Hz;
+ * L = min(max(log10(max(M_b, 1e-10)), -7), 2); c_b = min(15, floor((L + 7) * 16 / 9)).
+ * The transform runs in fp64. Errors: DMEL_ERR_INVALID_ARG for NULL required pointers,
+ * n_clips < 0 or n_frames < 0. */
+dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                       int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes, dmel_stream_t stream);
+
+/* Embedding of dMel codes ("Inside Inkling: Audio Design", Part 1 · Modeling: each
+ * (channel, level) pair owns one row; a frame's 80 rows are summed; optional RMSNorm).
+ *
+ * codes        uint8 [n_frames x 80], values 0..15 (a larger value is used as value & 15 and
+ *              flagged in the device error word)
+ * table        [1280 x embed_dim] row-major, fp32 or bf16 (table_dtype); row of channel b and
+ *              level c is 16 b + c
+ * embed_dim    D, a positive multiple of 8 (6144 for the model). bf16 tables with D a multiple
+ *              of 256 run on the tensor cores (tcgen05); other requests run on the CUDA cores,
+ *              which take D <= 16384.
+ * rms_weight   NULL (no RMSNorm) or [embed_dim] in table_dtype: y_j = g_j x_j / sqrt(mean x^2 + eps)
+ * eps          RMSNorm epsilon (> 0 when rms_weight is given; the model uses 1e-6)
+ * out          [n_frames x embed_dim] in out_dtype (fp32, or bf16 rounded to nearest even)
+ * workspace    device scratch of at least dmel_workspace_size(n_frames, embed_dim, table_dtype,
+ *              rms_weight != NULL, 1) bytes, 256-byte aligned (may be NULL when that size is 0)
+ * Sums accumulate in fp32. */
+dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
+                       const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
+                       size_t workspace_bytes, dmel_stream_t stream);
+
+/* dmel_codes followed by dmel_embed on the same stream: waveforms to frame vectors.
+ * Arguments are those of the two calls; codes_out is NULL (codes kept in the workspace) or
+ * uint8 [n_frames x 80] to receive the codes as well. workspace must hold
+ * dmel_workspace_size(n_frames, embed_dim, table_dtype, rms_weight != NULL, codes_out != NULL)
+ * bytes. */
+dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                         int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                         dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                         dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
+                         dmel_stream_t stream);
+
+/* Reads (and, when clear != 0, clears) the device error word of the current device. This call
+ * synchronises the device. *h_bits receives DMEL_DEVERR_* bits (0 = no error). */
+dmel_status dmel_get_device_error(uint32_t *h_bits, int clear);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *dmel_status_string(dmel_status status);
+
+/* Number of kernel launches the last successful call on this host thread issued (for launch
+ * accounting in benchmarks; 0 after a call that launched nothing). */
+int dmel_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMEL_H */

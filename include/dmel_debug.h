@@ -1,0 +1,25 @@
+/*
+ * dmel_debug.h — diagnostics of the dMel library. Not part of the front end's data path: no
+ * entry point of dmel.h calls these.
+ */
+#ifndef DMEL_DEBUG_H
+#define DMEL_DEBUG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Runs, on the host, the same per-frame step functions the codes kernel runs on the device
+ * (25 x 32 split of the 800-point complex DFT, real-signal split, sparse mel sums, log10,
+ * clamp, quantise), lane after lane, for one already-framed block of 1600 samples
+ * (frame1600 = x[800 (t-1) .. 800 (t+1))). Writes 80 codes and, when lhat80 != NULL, the 80
+ * clamped log10 mel energies. Lets the kernel's arithmetic be checked without a GPU. */
+void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMEL_DEBUG_H */

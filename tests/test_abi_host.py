@@ -1,0 +1,144 @@
+"""CPU tests of the C ABI: the library loads, exports what the headers declare, and its host
+logic (frame counts, offsets, workspace sizing, argument checks) behaves without a GPU.
+Also checks the codes kernel's per-frame arithmetic, run lane by lane on the host through
+dmel_debug_codes_frame_host, against the oracle."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from encoder_free_audio_b200 import build, dmel, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return dmel.library()
+
+
+def _declared(header):
+    txt = open(os.path.join(ROOT, "include", header)).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(dmel_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared("dmel.h") + _declared("dmel_debug.h")
+    assert "dmel_forward" in names and "dmel_codes" in names and "dmel_embed" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_frame_counts(lib):
+    assert [dmel.dmel_frames_for_length(n) for n in (0, 799, 800, 32000, 160000, 19_200_000)] == [0, 0, 1, 40, 200,
+                                                                                                 24000]
+    assert dmel.dmel_frames_for_length(-5) == -1
+
+
+def test_frame_offsets_host(lib, oracle_mod):
+    so = synth.offsets_from_lengths([800, 0, 2399, 799, 5000, 1600, 16000 * 30])
+    np.testing.assert_array_equal(dmel.dmel_frame_offsets(so), oracle_mod.frame_offsets(so))
+    with pytest.raises(dmel.DmelError):
+        dmel.dmel_frame_offsets(np.array([0, 10, 5]))
+    with pytest.raises(dmel.DmelError):
+        dmel.dmel_frame_offsets(np.array([3, 10]))
+
+
+def test_workspace_size(lib):
+    F = 12800
+    assert dmel.dmel_workspace_size(0, 6144, dmel.DMEL_BF16, True, False) == 0
+    with_codes = dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True)
+    assert with_codes == F * 24 * 4  # partial sums of squares, one per frame and 256-column tile
+    assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, False) == with_codes + F * 80
+    assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, False, True) == 0
+    assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_F32, True, True) == 0  # CUDA-core path
+
+
+def test_argument_checks_return_invalid_arg_without_gpu(lib):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: every call below fails its host checks first
+    # negative sizes
+    assert lib.dmel_codes(fake, fake, fake, -1, 0, None, None, fake, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert lib.dmel_codes(fake, fake, fake, 1, -1, None, None, fake, None) == dmel.DMEL_ERR_INVALID_ARG
+    # frames without clips, missing offsets, missing codes
+    assert lib.dmel_codes(fake, fake, fake, 0, 5, None, None, fake, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert lib.dmel_codes(fake, None, fake, 2, 5, None, None, fake, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert lib.dmel_codes(fake, fake, fake, 2, 5, None, None, None, None) == dmel.DMEL_ERR_INVALID_ARG
+    # zero clips is a no-op
+    assert lib.dmel_codes(None, None, None, 0, 0, None, None, None, None) == dmel.DMEL_OK
+    E = lib.dmel_embed
+    # embed_dim not a multiple of 8, bad dtype, missing pointers, misaligned output, eps <= 0
+    assert E(fake, 4, fake, 1, 6100, None, 1e-6, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert E(fake, 4, fake, 7, 6144, None, 1e-6, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert E(None, 4, fake, 1, 6144, None, 1e-6, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert E(fake, 4, None, 1, 6144, None, 1e-6, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert E(fake, 4, fake, 1, 6144, None, 1e-6, vp((1 << 20) + 2), 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert E(fake, 4, fake, 1, 6144, fake, 0.0, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    # RMSNorm on the tensor-core path without the workspace it needs
+    assert E(fake, 4, fake, 1, 6144, fake, 1e-6, fake, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    # CUDA-core path is limited to D <= 16384
+    assert E(fake, 4, fake, 0, 16392, None, 1e-6, fake, 0, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    # zero frames is a no-op
+    assert E(None, 0, None, 1, 6144, None, 1e-6, None, 1, None, 0, None) == dmel.DMEL_OK
+    Fw = lib.dmel_forward
+    assert Fw(fake, fake, fake, 1, 4, None, None, fake, 1, 6144, fake, 1e-6, fake, 1, None, None, 0,
+              None) == dmel.DMEL_ERR_INVALID_ARG  # no workspace for codes + partial sums
+    assert Fw(None, None, None, 0, 0, None, None, fake, 1, 6144, None, 1e-6, fake, 1, None, None, 0,
+              None) == dmel.DMEL_OK
+    bits = ctypes.c_uint32(0)
+    assert lib.dmel_get_device_error(None, 0) == dmel.DMEL_ERR_INVALID_ARG
+    del bits
+
+
+def test_status_strings(lib):
+    for s in range(4):
+        assert dmel.dmel_status_string(s).startswith("DMEL_")
+    assert dmel.dmel_status_string(99) == "DMEL_ERR_UNKNOWN"
+
+
+def _frames(wav, off, ids, oracle_mod):
+    """Raw 1600-sample frames of the listed global frames under the causal framing."""
+    fo = oracle_mod.frame_offsets(off)
+    out = np.zeros((len(ids), 1600), np.float32)
+    for i, g in enumerate(ids):
+        c = int(np.searchsorted(fo, g, side="right") - 1)
+        t = g - fo[c]
+        for n in range(1600):
+            j = 800 * (t - 1) + n
+            out[i, n] = wav[off[c] + j] if j >= 0 else 0.0
+    return out
+
+
+def _compare_codes(gc, gl, oc, ol, oracle_mod):
+    dist = oracle_mod.boundary_distance(ol)
+    mism = gc != oc
+    assert not (mism & (dist > 1e-4)).any(), "code mismatch away from a level boundary"
+    inner = (ol > -7.0) & (ol < 2.0)
+    np.testing.assert_allclose(gl[inner], ol[inner], rtol=0, atol=1e-9)
+
+
+def test_kernel_arithmetic_on_host_matches_oracle(lib, oracle_mod):
+    wav, off = synth.one_clip_2s()
+    ids = np.arange(40)
+    frames = _frames(wav, off, ids, oracle_mod)
+    oc, ol = oracle_mod.codes(wav, off)
+    for i in range(40):
+        gc, gl = dmel.dmel_debug_codes_frame_host(frames[i])
+        _compare_codes(gc, gl, oc[i], ol[i], oracle_mod)
+
+
+def test_kernel_arithmetic_on_host_tones_and_noise(lib, oracle_mod):
+    r = np.random.default_rng(11)
+    n = np.arange(1600)
+    cases = [np.zeros(1600), np.cos(2 * np.pi * 100 * n / 1600), 0.3 * np.cos(2 * np.pi * 3.37 * n / 1600 + 1.0),
+             r.uniform(-1, 1, 1600), 1e-5 * r.standard_normal(1600),
+             synth.harmonic_tone(1600, 123.4, 0.4, 10, 0.3)]
+    for x in cases:
+        fr = x.astype(np.float32)
+        gc, gl = dmel.dmel_debug_codes_frame_host(fr)
+        oc, ol = oracle_mod.codes(fr, np.array([0, 1600]), tails=None, frame_ids=np.array([1]))
+        _compare_codes(gc, gl, oc[0], ol[0], oracle_mod)

@@ -1,0 +1,283 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs. Codes must match except within 1e-4 of a level boundary (flips are counted and
+printed); embeddings within 1e-5 (fp32 output) or 1e-2 (bf16 output) of max(|o_j|, rms(o))."""
+import numpy as np
+import pytest
+import torch
+
+from encoder_free_audio_b200 import build, dmel, synth
+from encoder_free_audio_b200.frontend import FrontEnd
+from helpers import bf16_table, compare_codes, compare_embed
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    dmel.library()
+    dmel.dmel_get_device_error(clear=True)
+    yield
+    assert dmel.dmel_get_device_error(clear=True) == 0
+
+
+@pytest.fixture(scope="module")
+def table_bf16():
+    t, t64 = bf16_table(synth.table())
+    return t.to(DEV), t64
+
+
+@pytest.fixture(scope="module")
+def rmsw_bf16():
+    g = torch.from_numpy(synth.rms_weight()).to(torch.bfloat16)
+    return g.to(DEV), g.float().numpy().astype(np.float64)
+
+
+def _codes_gpu(wav, off, tails=None, want_tails=False):
+    fo = dmel.dmel_frame_offsets(off)
+    F = int(fo[-1])
+    w = torch.from_numpy(wav).to(DEV)
+    so_d = torch.from_numpy(off).to(DEV)
+    fo_d = torch.from_numpy(fo).to(DEV)
+    codes = torch.empty((F, 80), dtype=torch.uint8, device=DEV)
+    t_in = None if tails is None else torch.from_numpy(tails).to(DEV)
+    t_out = torch.full((off.shape[0] - 1, 800), -5.0, device=DEV) if want_tails else None
+    dmel.dmel_codes(w, so_d, fo_d, F, codes, tails=t_in, tails_out=t_out)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), (None if t_out is None else t_out.cpu().numpy())
+
+
+# ------------------------------------------------------------------------- codes
+
+def test_codes_one_clip_2s(oracle_mod):
+    wav, off = synth.one_clip_2s()
+    g, tails = _codes_gpu(wav, off, want_tails=True)
+    oc, ol = oracle_mod.codes(wav, off)
+    flips, _ = compare_codes(g, oc, ol)
+    print(f"one_clip_2s: 40 frames, flips {flips}")
+    np.testing.assert_array_equal(tails, oracle_mod.tails_out(wav, off))
+
+
+def test_codes_edge_lengths_and_tails(oracle_mod):
+    r = np.random.default_rng(21)
+    lengths = [0, 1, 799, 800, 801, 1599, 1600, 2400, 5 * 800 + 13, 0, 3200]
+    off = synth.offsets_from_lengths(lengths)
+    wav = r.uniform(-0.7, 0.7, int(off[-1])).astype(np.float32)
+    tails = r.uniform(-0.5, 0.5, (len(lengths), 800)).astype(np.float32)
+    g, t_out = _codes_gpu(wav, off, tails=tails, want_tails=True)
+    oc, ol = oracle_mod.codes(wav, off, tails=tails)
+    compare_codes(g, oc, ol)
+    np.testing.assert_array_equal(t_out, oracle_mod.tails_out(wav, off, tails))
+
+
+def test_codes_silence_and_full_scale(oracle_mod):
+    r = np.random.default_rng(22)
+    off = synth.offsets_from_lengths([16000, 16000])
+    wav = np.concatenate([np.zeros(16000), np.where(r.random(16000) < 0.5, -1.0, 1.0)]).astype(np.float32)
+    g, _ = _codes_gpu(wav, off)
+    assert (g[:20] == 0).all()
+    oc, ol = oracle_mod.codes(wav, off)
+    compare_codes(g, oc, ol)
+
+
+def test_codes_nonfinite_samples_stay_in_range():
+    wav = np.zeros(8000, np.float32)
+    wav[1234] = np.nan
+    wav[4321] = np.inf
+    g, _ = _codes_gpu(wav, np.array([0, 8000]))
+    assert g.shape == (10, 80) and g.max() <= 15
+
+
+def test_codes_no_frames_is_noop():
+    wav = np.zeros(500, np.float32)
+    off = np.array([0, 500], np.int64)
+    g, _ = _codes_gpu(wav, off)
+    assert g.shape == (0, 80)
+
+
+# ------------------------------------------------------------------------- embedding
+
+@pytest.mark.parametrize("dim", [8, 24, 1000, 256, 512])
+@pytest.mark.parametrize("tdt", ["f32", "bf16"])
+def test_embed_small_integer_tables_exact(dim, tdt, oracle_mod):
+    """Tables of small integers: every partial sum is exact in fp32, so the CUDA-core path and
+    the tensor-core path (bf16, D % 256 == 0) must give the oracle's sums bit for bit."""
+    r = np.random.default_rng(30 + dim)
+    T = r.integers(-6, 7, size=(1280, dim)).astype(np.float32)
+    F = 300  # 2 full tiles of 128 frames and a ragged tail of 44
+    codes = synth.random_codes(31, F)
+    tt = torch.from_numpy(T).to(DEV)
+    if tdt == "bf16":
+        tt = tt.to(torch.bfloat16)
+    out = torch.empty((F, dim), dtype=torch.float32, device=DEV)
+    dmel.dmel_embed(torch.from_numpy(codes).to(DEV), tt, out)
+    torch.cuda.synchronize()
+    ref = oracle_mod.embed(codes, T.astype(np.float64))
+    np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("out_dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rms", [False, True])
+def test_embed_tensor_core_model_dim(out_dt, rms, table_bf16, rmsw_bf16, oracle_mod):
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    F = 1000
+    codes = synth.random_codes(41, F)
+    out = torch.empty((F, 6144), dtype=out_dt, device=DEV)
+    ws_n = dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, rms, True)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=DEV)
+    dmel.dmel_embed(torch.from_numpy(codes).to(DEV), T, out, rms_weight=g if rms else None, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle_mod.embed(codes, T64, g64 if rms else None, 1e-6)
+    worst = compare_embed(out.float().cpu().numpy(), ref, 1e-5 if out_dt == torch.float32 else 1e-2)
+    print(f"tensor-core embed out={out_dt} rms={rms}: worst {worst:.2e}")
+
+
+def test_embed_fp32_table_rmsnorm(oracle_mod):
+    T = synth.table(seed=9, dim=512)
+    gw = synth.rms_weight(seed=10, dim=512)
+    F = 77
+    codes = synth.random_codes(42, F)
+    out = torch.empty((F, 512), dtype=torch.float32, device=DEV)
+    dmel.dmel_embed(torch.from_numpy(codes).to(DEV), torch.from_numpy(T).to(DEV), out,
+                    rms_weight=torch.from_numpy(gw).to(DEV), eps=1e-6)
+    torch.cuda.synchronize()
+    ref = oracle_mod.embed(codes, T.astype(np.float64), gw.astype(np.float64), 1e-6)
+    compare_embed(out.cpu().numpy(), ref, 1e-5)
+
+
+def test_embed_out_of_range_codes_are_flagged(table_bf16):
+    T, _ = table_bf16
+    codes = torch.zeros((130, 80), dtype=torch.uint8, device=DEV)
+    codes[129, 5] = 200
+    out = torch.empty((130, 6144), dtype=torch.bfloat16, device=DEV)
+    dmel.dmel_embed(codes, T, out)
+    assert dmel.dmel_get_device_error(clear=True) & dmel.DMEL_DEVERR_CODE_RANGE
+    assert torch.isfinite(out.float()).all()
+
+
+# ------------------------------------------------------------------------- full path, workloads
+
+def _forward(wav, off, table, rmsw, out_dtype, tails=None):
+    fe = FrontEnd(table, rmsw, 1e-6, out_dtype)
+    plan = fe.plan(off)
+    w = torch.from_numpy(wav).to(DEV)
+    t_in = None if tails is None else torch.from_numpy(tails).to(DEV)
+    fe.forward(w, plan, tails=t_in)
+    torch.cuda.synchronize()
+    return plan
+
+
+def _check_forward(wav, off, plan, T64, g64, rtol, oracle_mod, frame_ids=None, embed_ids=None, label=""):
+    gc = plan.codes.cpu().numpy()
+    if frame_ids is None:
+        oc, ol = oracle_mod.codes(wav, off)
+        gsel = gc
+    else:
+        oc, ol = oracle_mod.codes(wav, off, frame_ids=frame_ids)
+        gsel = gc[frame_ids]
+    flips, flipped = compare_codes(gsel, oc, ol)
+    ids = np.arange(gsel.shape[0]) if embed_ids is None else embed_ids
+    ids = ids[~flipped[ids]]
+    rows = ids if frame_ids is None else frame_ids[ids]
+    ref = oracle_mod.embed(oc[ids], T64, g64, 1e-6)
+    worst = compare_embed(plan.out[torch.from_numpy(rows).to(DEV)].float().cpu().numpy(), ref, rtol)
+    print(f"{label}: frames {plan.n_frames}, code cells checked {gsel.size}, flips {flips}, "
+          f"embeddings checked {len(ids)}, worst {worst:.2e}")
+
+
+def test_forward_one_clip_2s_fp32(oracle_mod):
+    wav, off = synth.one_clip_2s()
+    T = synth.table()
+    plan = _forward(wav, off, torch.from_numpy(T).to(DEV), None, torch.float32)
+    _check_forward(wav, off, plan, T.astype(np.float64), None, 1e-5, oracle_mod, label="one_clip_2s")
+
+
+def test_forward_batch64_10s(table_bf16, rmsw_bf16, oracle_mod):
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    wav, off = synth.batch64_10s()
+    plan = _forward(wav, off, T, g, torch.bfloat16)
+    assert plan.n_frames == 12800
+    r = np.random.default_rng(51)
+    emb = np.sort(r.choice(12800, 1536, replace=False))
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, embed_ids=emb, label="batch64_10s")
+
+
+def test_forward_long_20min(table_bf16, rmsw_bf16, oracle_mod):
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    wav, off = synth.long_20min()
+    plan = _forward(wav, off, T, g, torch.bfloat16)
+    assert plan.n_frames == 24000
+    r = np.random.default_rng(52)
+    emb = np.sort(r.choice(24000, 1024, replace=False))
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, embed_ids=emb, label="long_20min")
+
+
+def test_forward_ragged1024(table_bf16, rmsw_bf16, oracle_mod):
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    wav, off = synth.ragged1024()
+    plan = _forward(wav, off, T, g, torch.bfloat16)
+    fo = plan.frame_offsets_host
+    r = np.random.default_rng(53)
+    clips = r.choice(1024, 24, replace=False)
+    ids = [np.arange(fo[c], fo[c + 1]) for c in clips]
+    rest = r.choice(plan.n_frames, int(0.01 * plan.n_frames), replace=False)
+    frame_ids = np.unique(np.concatenate(ids + [rest, [0, plan.n_frames - 1]])).astype(np.int64)
+    emb = np.sort(r.choice(frame_ids.shape[0], 768, replace=False))
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, frame_ids=frame_ids, embed_ids=emb,
+                   label="ragged1024 (sampled)")
+
+
+def test_streaming_4096_matches_offline_and_oracle(table_bf16, rmsw_bf16, oracle_mod):
+    """4096 streams, 800 new samples per call plus the carried tail. Every call's codes and
+    vectors equal those of one offline call on the concatenated stream (bit for bit), and
+    sampled calls match the oracle."""
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    S = synth.Streams4096()
+    n_calls = 1000
+    check_calls = {0, 1, 2, 500, 999}
+    fe = FrontEnd(T, g, 1e-6, torch.bfloat16)
+    plan = fe.plan(synth.offsets_from_lengths([800] * S.n))
+    tails = torch.zeros((S.n, 800), device=DEV)
+    prev = None
+    offline_streams = np.arange(0, S.n, 512)
+    offline_wav = [[] for _ in offline_streams]
+    offline_out = [[] for _ in offline_streams]
+    for k in range(n_calls):
+        x = S.call(k)
+        for i, s in enumerate(offline_streams):
+            if k < 40:
+                offline_wav[i].append(x[s])
+        fe.forward(torch.from_numpy(x).to(DEV).reshape(-1), plan, tails=tails, tails_out=tails)
+        if k < 40:
+            o = plan.out[torch.from_numpy(offline_streams).to(DEV)].cpu()
+            for i in range(len(offline_streams)):
+                offline_out[i].append(o[i])
+        if k in check_calls:
+            torch.cuda.synchronize()
+            tail_in = prev if prev is not None else np.zeros((S.n, 800), np.float32)
+            oc, ol = oracle_mod.codes(x.reshape(-1), plan.sample_offsets_host, tails=tail_in)
+            flips, flipped = compare_codes(plan.codes.cpu().numpy(), oc, ol)
+            ids = np.arange(0, S.n, 37)
+            ids = ids[~flipped[ids]]
+            ref = oracle_mod.embed(oc[ids], T64, g64, 1e-6)
+            worst = compare_embed(plan.out[torch.from_numpy(ids).to(DEV)].float().cpu().numpy(), ref, 1e-2)
+            print(f"stream call {k}: flips {flips}, worst {worst:.2e}")
+        prev = x
+    torch.cuda.synchronize()
+    # streaming equals offline: 40 calls of selected streams against one call on their samples
+    fe2 = FrontEnd(T, g, 1e-6, torch.bfloat16)
+    for i in range(len(offline_streams)):
+        wav = np.concatenate(offline_wav[i])
+        p2 = fe2.plan(np.array([0, wav.size]))
+        fe2.forward(torch.from_numpy(wav).to(DEV), p2)
+        torch.cuda.synchronize()
+        got = torch.stack(offline_out[i]).to(DEV)
+        assert torch.equal(got, p2.out), f"stream {offline_streams[i]}: streaming differs from offline"
