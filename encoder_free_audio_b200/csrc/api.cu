@@ -182,6 +182,27 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
   return from_cuda(e);
 }
 
+dmel_status dmel_embed_noalloc(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                               int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
+                               dmel_stream_t stream) {
+  t_last_launches = 0;
+  dmel_status st =
+      check_embed_args(codes, true, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype);
+  if (st != DMEL_OK || n_frames == 0) return st;
+  const size_t need = embed_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
+  if (need > kNoAllocScratchBytes) return DMEL_ERR_TOO_LARGE;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  void *scratch = nullptr;
+  if (need > 0 && noalloc_scratch(&scratch) != cudaSuccess) return DMEL_ERR_CUDA;
+  int launches = 0;
+  cudaError_t e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype,
+                               scratch, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
 dmel_status dmel_get_device_error(uint32_t *h_bits, int clear) {
   if (!h_bits) return DMEL_ERR_INVALID_ARG;
   DeviceInfo d;
@@ -199,6 +220,7 @@ const char *dmel_status_string(dmel_status status) {
     case DMEL_ERR_INVALID_ARG: return "DMEL_ERR_INVALID_ARG: argument out of contract";
     case DMEL_ERR_UNSUPPORTED: return "DMEL_ERR_UNSUPPORTED: request not supported on this device";
     case DMEL_ERR_CUDA: return "DMEL_ERR_CUDA: a CUDA call or kernel launch failed";
+    case DMEL_ERR_TOO_LARGE: return "DMEL_ERR_TOO_LARGE: request needs more than the fixed 4 MiB scratch";
   }
   return "DMEL_ERR_UNKNOWN";
 }

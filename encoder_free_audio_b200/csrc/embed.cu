@@ -478,6 +478,36 @@ cudaError_t launch_rescale(OT *out, int64_t F, int D, const __nv_bfloat16 *g, co
 
 }  // namespace
 
+// ---------------------------------------------------------------- allocation-free variant
+
+// Fixed scratch for dmel_embed_noalloc: the RMSNorm partial sums of the tensor-core path live
+// here instead of in a caller workspace. Every device that loads the library holds these
+// 4 MiB until the process exits; all calls share them.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[256] = {nullptr};
+}  // namespace
+
+cudaError_t noalloc_scratch(void **ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    // The array's name is only a host-side stand-in; its device address must be looked up,
+    // once per device, with that device current.
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
 bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
   return table_dtype == DMEL_BF16 && embed_dim > 0 && embed_dim % tc::BN == 0;
 }

@@ -25,6 +25,12 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *tab
                          int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
                          void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
 
+// Size of the fixed device scratch used by dmel_embed_noalloc.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+
+// Device address of that scratch on the current device (looked up once per device).
+cudaError_t noalloc_scratch(void **ptr);
+
 void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
 
 }  // namespace dmel

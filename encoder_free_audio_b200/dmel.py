@@ -19,6 +19,7 @@ DMEL_OK = 0
 DMEL_ERR_INVALID_ARG = 1
 DMEL_ERR_UNSUPPORTED = 2
 DMEL_ERR_CUDA = 3
+DMEL_ERR_TOO_LARGE = 4
 DMEL_F32 = 0
 DMEL_BF16 = 1
 DMEL_DEVERR_CODE_RANGE = 0x1
@@ -62,6 +63,8 @@ def _lib():
         L.dmel_forward.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, vp,
                                    sz, vp]
         L.dmel_forward.restype = i32
+        L.dmel_embed_noalloc.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp]
+        L.dmel_embed_noalloc.restype = i32
         L.dmel_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         L.dmel_get_device_error.restype = i32
         L.dmel_status_string.argtypes = [i32]
@@ -147,6 +150,15 @@ def dmel_embed(codes, table, out, rms_weight=None, eps: float = 1e-6, workspace=
     rc = _lib().dmel_embed(_ptr(codes), n, _ptr(table), _dtype_code(table), table.shape[1], _ptr(rms_weight),
                            float(eps), _ptr(out), _dtype_code(out), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dmel_embed")
+
+
+def dmel_embed_noalloc(codes, table, out, rms_weight=None, eps: float = 1e-6, stream=None):
+    """dmel_embed_noalloc on torch CUDA tensors: dmel_embed without a workspace, for callers
+    that cannot allocate (the library's fixed 4 MiB scratch is used instead)."""
+    n = codes.shape[0]
+    rc = _lib().dmel_embed_noalloc(_ptr(codes), n, _ptr(table), _dtype_code(table), table.shape[1],
+                                   _ptr(rms_weight), float(eps), _ptr(out), _dtype_code(out), _stream(stream))
+    _check(rc, "dmel_embed_noalloc")
 
 
 def dmel_forward(wav, sample_offsets, frame_offsets, n_frames: int, table, out, rms_weight=None, eps: float = 1e-6,

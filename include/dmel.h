@@ -43,7 +43,8 @@ typedef enum {
   DMEL_OK = 0,
   DMEL_ERR_INVALID_ARG = 1, /* a pointer, size, offset or flag is out of contract */
   DMEL_ERR_UNSUPPORTED = 2, /* valid request that this build does not run (e.g. no sm_100 device) */
-  DMEL_ERR_CUDA = 3         /* a CUDA runtime call or kernel launch failed */
+  DMEL_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  DMEL_ERR_TOO_LARGE = 4    /* dmel_embed_noalloc: the request needs more than its fixed scratch */
 } dmel_status;
 
 typedef enum { DMEL_F32 = 0, DMEL_BF16 = 1 } dmel_dtype;
@@ -124,6 +125,31 @@ dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const in
 dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
                        const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
                        size_t workspace_bytes, dmel_stream_t stream);
+
+/* dmel_embed for callers that cannot allocate device memory: the paper has no counterpart of
+ * this entry point; it exists for integration only.
+ *
+ * Some callers have no way to provide a workspace: a real-time audio callback or a serving
+ * step being captured into a CUDA graph may not call cudaMalloc (it can synchronise the device
+ * and is not allowed during stream capture), and some host frameworks own all device memory
+ * and hand a library nothing but input and output pointers. This variant takes the same
+ * arguments as dmel_embed minus the workspace and allocates nothing: the scratch it needs (the
+ * RMSNorm partial sums of the tensor-core path) is a fixed 4 MiB array inside the library,
+ * which every device that loads the library holds until the process exits.
+ *
+ * Limit: with rms_weight != NULL and a bf16 table whose embed_dim is a multiple of 256, the
+ * request needs n_frames * (embed_dim / 256) * 4 bytes of scratch (43,690 frames at
+ * embed_dim 6144); a larger request returns DMEL_ERR_TOO_LARGE and launches nothing. Other
+ * requests need no scratch and have no extra limit.
+ *
+ * The first call on each device looks up the scratch's device address (and uploads nothing
+ * else); make that first call before any stream capture. All calls share the one scratch
+ * array, which keeps the last call's contents (every value a call reads it writes first):
+ * calls that overlap on the GPU, e.g. on two streams at once, race on it and must be ordered
+ * by the caller. */
+dmel_status dmel_embed_noalloc(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                               int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
+                               dmel_stream_t stream);
 
 /* dmel_codes followed by dmel_embed on the same stream: waveforms to frame vectors.
  * Arguments are those of the two calls; codes_out is NULL (codes kept in the workspace) or

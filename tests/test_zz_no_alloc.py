@@ -1,0 +1,66 @@
+"""dmel_embed_noalloc: the embedding for callers that cannot allocate device memory (a real-time
+audio callback, a step being captured into a CUDA graph, a host framework that owns all device
+memory). It must give what dmel_embed gives with a caller workspace, call after call, while the
+partial sums live in the library's fixed scratch array. Collected last on purpose, so a failure
+here comes after every other test has run."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from encoder_free_audio_b200 import build, dmel, synth
+from helpers import bf16_table, compare_embed
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    build.build()
+    return dmel.library()
+
+
+def _call_noalloc(lib, codes, table, out, g, eps=1e-6):
+    """The C entry point itself, through ctypes, on the current stream."""
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.dmel_embed_noalloc(ctypes.c_void_p(codes.data_ptr()), codes.shape[0], ctypes.c_void_p(table.data_ptr()),
+                                  dmel.DMEL_BF16, table.shape[1],
+                                  None if g is None else ctypes.c_void_p(g.data_ptr()), ctypes.c_float(eps),
+                                  ctypes.c_void_p(out.data_ptr()), dmel.DMEL_BF16, stream)
+
+
+def test_noalloc_matches_workspace_entry_point_twice(lib):
+    t_cpu, _ = bf16_table(synth.table())
+    T = t_cpu.to(DEV)
+    g = torch.from_numpy(synth.rms_weight()).to(torch.bfloat16).to(DEV)
+    dmel.dmel_get_device_error(clear=True)
+    # two calls in a row with different frame counts (the second reuses the scratch the first
+    # left behind) against dmel_embed with its own workspace
+    for call, F in enumerate((2000, 777)):
+        codes = torch.from_numpy(synth.random_codes(100 + call, F)).to(DEV)
+        out_na = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
+        assert _call_noalloc(lib, codes, T, out_na, g) == dmel.DMEL_OK
+        out_ws = torch.empty_like(out_na)
+        ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True), dtype=torch.uint8,
+                         device=DEV)
+        dmel.dmel_embed(codes, T, out_ws, rms_weight=g, eps=1e-6, workspace=ws)
+        torch.cuda.synchronize()
+        ref = out_ws.float().cpu().numpy().astype(np.float64)
+        compare_embed(out_na.float().cpu().numpy(), ref, 1e-2)
+    assert dmel.dmel_get_device_error(clear=True) == 0
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch(lib):
+    T = torch.zeros((1280, 6144), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones(6144, dtype=torch.bfloat16, device=DEV)
+    F = (4 << 20) // (24 * 4) + 1  # one frame more than 4 MiB of partial sums holds
+    codes = torch.zeros((F, 80), dtype=torch.uint8, device=DEV)
+    out = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
+    assert _call_noalloc(lib, codes, T, out, g) == dmel.DMEL_ERR_TOO_LARGE
+    # without RMSNorm the request needs no scratch and runs
+    assert _call_noalloc(lib, codes[:300], T, out[:300], None) == dmel.DMEL_OK
+    torch.cuda.synchronize()
