@@ -8,13 +8,19 @@
 // agree with an exact evaluation everywhere except within ~1e-12 of a level boundary.
 //
 // Real DFT of 1600 points through one complex DFT of 800 points, z_m = u_{2m} + i u_{2m+1}
-// (u = windowed samples), 800 = 25 x 32:
-//   A  lane l (0..31) takes z_{32 j + l}, j = 0..24, does a 25-point DFT in registers (5 x 5),
-//      multiplies output k1 by W_800^{l k1} and writes Y[k1][l];
-//   C  lane k1 (0..24) takes Y[k1][0..31], does a 32-point DFT (radix 2) and writes
-//      Z[k1 + 25 k2];
-//   D  X_k = (Z_k + conj Z_{800-k}) / 2 + W_1600^k (Z_k - conj Z_{800-k}) / (2 i), P_k = |X_k|^2;
-//   E  lane l sums the sparse mel triangles assigned to it, then log10, clamp, quantise.
+// (u = windowed samples). 800 = 25 x 32 with m = 32 j + l and k = k1 + 25 k2:
+//   A   lane l (0..31): 25-point DFT over j of z_{32 j + l} (5 x 5, in registers), output k1
+//       times W_800^{l k1} -> row k1, column l of the warp's 25 x 32 buffer;
+//   C1  the 32-point DFTs over l of each row, as 4 x 8 (l = l0 + 4 l1, k2 = k2a + 8 k2b):
+//       100 in-place 8-point DFTs over l1, times W_32^{l0 k2a};
+//   C2  200 in-place 4-point DFTs over l0; Z[k1 + 25 (k2a + 8 k2b)] ends in row k1, column
+//       k2b + 4 k2a;
+//   D   X_k = (Z_k + conj Z_{800-k}) / 2 + W_1600^k (Z_k - conj Z_{800-k}) / (2 i),
+//       P_k = |X_k|^2, each lane owning the pairs (k, 800 - k) it reads;
+//   E   lane l sums the sparse mel triangles assigned to it, then log10, clamp, quantise.
+// Every root of unity comes from one fp64 table of W_1600^k, k = 0..800 (W_800 = W_1600^2,
+// W_32 = W_1600^50, W_25 = W_1600^64, W^{1600 - k} = conj W^k). The buffer is swizzled so the
+// column accesses of A, C1 and C2 are free of shared-memory bank conflicts.
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -26,17 +32,28 @@
 namespace dmel {
 namespace {
 
-constexpr int kYStride = 33;                 // padded row of Y[25][33] (bank spread)
-constexpr int kYElems = 25 * kYStride;       // 825 complex values; P[801] reuses this space
-constexpr int kZElems = 800;
-constexpr int kWarpSmemBytes = (kYElems + kZElems) * 16;  // 26,000 B per warp
-constexpr int kWarpsPerBlock = 4;
+#ifndef DMEL_CODES_WARPS
+#define DMEL_CODES_WARPS 12
+#endif
+constexpr int kWarpsPerBlock = DMEL_CODES_WARPS;
 constexpr int kMaxFiltPerLane = 8;
-constexpr int kMelNnzMax = 2048;
+constexpr int kMelNnzMax = 1600;
+constexpr int kPairsPerLane = 13;  // ceil(401 / 32) pairs (k, 800 - k) per lane in step D
+
+// Shared memory of one block: the constant tables once, then one 800-element complex buffer
+// per warp (Y, then Z in place, then P in place).
+constexpr int kSmW = 0;                                    // double2 [801]: W_1600^k
+constexpr int kSmMelW = 801 * 16;                          // double [kMelNnzMax]
+constexpr int kSmMelK0 = kSmMelW + kMelNnzMax * 8;         // int [80]
+constexpr int kSmMelN = kSmMelK0 + kMel * 4;               // int [80]
+constexpr int kSmMelOff = kSmMelN + kMel * 4;              // int [80]
+constexpr int kSmLaneFilt = kSmMelOff + kMel * 4;          // signed char [32 * 8]
+constexpr int kSmTables = (kSmLaneFilt + 32 * kMaxFiltPerLane + 127) / 128 * 128;
+constexpr int kWarpBufBytes = 800 * 16;
+constexpr int kSmemBytes = kSmTables + kWarpsPerBlock * kWarpBufBytes;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // Constant tables, filled once per device from host-computed fp64 values.
-__device__ double d_win[kWin];
-__device__ double2 d_w800[800];
 __device__ double2 d_w1600[kBins];
 __device__ double d_melw[kMelNnzMax];
 __device__ int d_mel_k0[kMel];
@@ -45,9 +62,7 @@ __device__ int d_mel_off[kMel];
 __device__ signed char d_lane_filt[32 * kMaxFiltPerLane];
 
 struct Tables {
-  const double *win;
-  const double2 *w800;
-  const double2 *w1600;
+  const double2 *w;  // W_1600^k = exp(-2 pi i k / 1600), k = 0..800
   const double *melw;
   const int *mel_k0;
   const int *mel_n;
@@ -55,11 +70,36 @@ struct Tables {
   const signed char *lane_filt;
 };
 
+// W_1600^idx for idx in [0, 1600).
+__host__ __device__ inline double2 tw(const Tables &T, int idx) {
+  if (idx <= 800) return T.w[idx];
+  const double2 v = T.w[1600 - idx];
+  return make_double2(v.x, -v.y);
+}
+
 __host__ __device__ inline void cmul(double &re, double &im, double wr, double wi) {
   const double r = re * wr - im * wi;
   const double i = re * wi + im * wr;
   re = r;
   im = i;
+}
+
+// Periodic Hann window w[n] = 0.5 - 0.5 cos(2 pi n / 1600), the cosine being Re W_1600^n.
+__host__ __device__ inline double hann(const Tables &T, int n) { return 0.5 - 0.5 * tw(T, n).x; }
+
+// Element (row k1, column c) of a warp's 25 x 32 buffer. The three low bits of the column are
+// permuted (bits 3..4 of the column and bit 0 of the row feed in), so that eight lanes of A
+// (one row, eight columns), C1 (two rows, columns l0 + 4 l1) and C2 (one row, columns
+// l0 + 4 k2a) touch eight different 16-byte bank groups.
+__host__ __device__ inline int slot(int k1, int c) {
+  const int low = ((c & 3) ^ ((c >> 3) & 3)) | ((((c >> 2) ^ k1) & 1) << 2);
+  return k1 * 32 + (c & 24) + low;
+}
+
+// Where Z_k sits after step C2: row k % 25, column k2b + 4 k2a with k2 = k / 25.
+__host__ __device__ inline int zslot(int k) {
+  const int k1 = k % 25, k2 = k / 25;
+  return slot(k1, (k2 >> 3) + 4 * (k2 & 7));
 }
 
 // 5-point DFT X_k = sum_n x_n W_5^{nk}, W_5 = exp(-2 pi i / 5), of x0..x4 (in place).
@@ -90,6 +130,60 @@ __host__ __device__ inline void dft5(double &r0, double &i0, double &r1, double 
   i3 = bi + vr;
 }
 
+// 8-point DFT X_k = sum_n x_n W_8^{nk} (in place, natural order in and out): radix-2
+// decimation in time on the bit-reversed input order.
+__host__ __device__ inline void dft8(double (&r)[8], double (&i)[8]) {
+  const double h = 0.70710678118654752440;  // cos(pi / 4)
+  double ar[8], ai[8];
+  const int br[8] = {0, 4, 2, 6, 1, 5, 3, 7};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    ar[q] = r[br[q]];
+    ai[q] = i[br[q]];
+  }
+  // span 1: W_2^0
+#pragma unroll
+  for (int q = 0; q < 8; q += 2) {
+    const double xr = ar[q + 1], xi = ai[q + 1];
+    ar[q + 1] = ar[q] - xr;
+    ai[q + 1] = ai[q] - xi;
+    ar[q] += xr;
+    ai[q] += xi;
+  }
+  // span 2: W_4^0 = 1, W_4^1 = -i
+#pragma unroll
+  for (int q = 0; q < 8; q += 4) {
+    double xr = ar[q + 2], xi = ai[q + 2];
+    ar[q + 2] = ar[q] - xr;
+    ai[q + 2] = ai[q] - xi;
+    ar[q] += xr;
+    ai[q] += xi;
+    xr = ai[q + 3];  // (-i) x = (x.im, -x.re)
+    xi = -ar[q + 3];
+    ar[q + 3] = ar[q + 1] - xr;
+    ai[q + 3] = ai[q + 1] - xi;
+    ar[q + 1] += xr;
+    ai[q + 1] += xi;
+  }
+  // span 4: W_8^0 = 1, W_8^1 = h (1 - i), W_8^2 = -i, W_8^3 = -h (1 + i)
+  {
+    double xr, xi;
+    xr = ar[4]; xi = ai[4];
+    ar[4] = ar[0] - xr; ai[4] = ai[0] - xi; ar[0] += xr; ai[0] += xi;
+    xr = h * (ar[5] + ai[5]); xi = h * (ai[5] - ar[5]);
+    ar[5] = ar[1] - xr; ai[5] = ai[1] - xi; ar[1] += xr; ai[1] += xi;
+    xr = ai[6]; xi = -ar[6];
+    ar[6] = ar[2] - xr; ai[6] = ai[2] - xi; ar[2] += xr; ai[2] += xi;
+    xr = h * (ai[7] - ar[7]); xi = -h * (ar[7] + ai[7]);
+    ar[7] = ar[3] - xr; ai[7] = ai[3] - xi; ar[3] += xr; ai[3] += xi;
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    r[q] = ar[q];
+    i[q] = ai[q];
+  }
+}
+
 // Raw sample n (0..1599) of frame t of a clip: x[800 (t - 1) + n], with samples before the clip
 // taken from the carried tail (tail points one past its last sample) or zero.
 struct ClipSampler {
@@ -109,31 +203,27 @@ struct FrameSampler {
   __host__ __device__ double operator()(int n) const { return (double)frame[n]; }
 };
 
-__host__ __device__ inline int bitrev5(int k) {
-  return ((k & 1) << 4) | ((k & 2) << 2) | (k & 4) | ((k & 8) >> 2) | ((k & 16) >> 4);
-}
-
 // Step A for lane l. sample(n) returns raw frame sample n (0..1599) as double.
 template <class SampleFn>
-__host__ __device__ inline void step_a(int l, SampleFn sample, const Tables &T, double2 *Y) {
+__host__ __device__ inline void step_a(int l, SampleFn sample, const Tables &T, double2 *B) {
   double ar[25], ai[25];
 #pragma unroll
   for (int j = 0; j < 25; ++j) {
     const int n0 = 64 * j + 2 * l;
-    ar[j] = T.win[n0] * sample(n0);
-    ai[j] = T.win[n0 + 1] * sample(n0 + 1);
+    ar[j] = hann(T, n0) * sample(n0);
+    ai[j] = hann(T, n0 + 1) * sample(n0 + 1);
   }
   // 25 = 5 x 5, j = j1 + 5 j2: inner DFTs over j2, result for (j1, ka) stored at j1 + 5 ka
 #pragma unroll
   for (int j1 = 0; j1 < 5; ++j1)
     dft5(ar[j1], ai[j1], ar[j1 + 5], ai[j1 + 5], ar[j1 + 10], ai[j1 + 10], ar[j1 + 15], ai[j1 + 15], ar[j1 + 20],
          ai[j1 + 20]);
-  // twiddle W_25^{j1 ka} = W_800^{32 j1 ka}
+  // twiddle W_25^{j1 ka} = W_1600^{64 j1 ka}
 #pragma unroll
   for (int j1 = 1; j1 < 5; ++j1)
 #pragma unroll
     for (int ka = 1; ka < 5; ++ka) {
-      const double2 w = T.w800[(32 * j1 * ka) % 800];
+      const double2 w = tw(T, 64 * j1 * ka);
       cmul(ar[j1 + 5 * ka], ai[j1 + 5 * ka], w.x, w.y);
     }
   // outer DFTs over j1 for each ka (inputs at 5 ka + j1), output k1 = ka + 5 kb
@@ -151,65 +241,92 @@ __host__ __device__ inline void step_a(int l, SampleFn sample, const Tables &T, 
       const int k1 = ka + 5 * kb;
       double yr = r[kb], yi = i[kb];
       if (l * k1 != 0) {
-        const double2 w = T.w800[(l * k1) % 800];  // W_800^{l k1}
+        const double2 w = tw(T, (2 * l * k1) % 1600);  // W_800^{l k1}
         cmul(yr, yi, w.x, w.y);
       }
-      Y[k1 * kYStride + l] = make_double2(yr, yi);
+      B[slot(k1, l)] = make_double2(yr, yi);
     }
   }
 }
 
-// Step C for lane k1 < 25: 32-point DFT over l of Y[k1][l], written to Z[k1 + 25 k2].
-__host__ __device__ inline void step_c(int k1, const Tables &T, const double2 *Y, double2 *Z) {
-  double re[32], im[32];
+// Step C1, unit u = 4 k1 + l0 (0..99): 8-point DFT over l1 of row k1, columns l0 + 4 l1, times
+// W_32^{l0 k2a}, written back to the same columns (output k2a in column l0 + 4 k2a).
+__host__ __device__ inline void step_c1(int u, const Tables &T, double2 *B) {
+  const int k1 = u >> 2, l0 = u & 3;
+  double r[8], i[8];
 #pragma unroll
-  for (int l = 0; l < 32; ++l) {
-    const double2 y = Y[k1 * kYStride + l];
-    re[l] = y.x;
-    im[l] = y.y;
+  for (int l1 = 0; l1 < 8; ++l1) {
+    const double2 v = B[slot(k1, l0 + 4 * l1)];
+    r[l1] = v.x;
+    i[l1] = v.y;
   }
-  // radix-2 decimation in frequency; output k lands at position bitrev5(k)
+  dft8(r, i);
 #pragma unroll
-  for (int span = 16; span >= 1; span >>= 1) {
-#pragma unroll
-    for (int start = 0; start < 32; start += 2 * span) {
-#pragma unroll
-      for (int i = 0; i < span; ++i) {
-        const int a = start + i, b = a + span;
-        const double tr = re[a] - re[b], ti = im[a] - im[b];
-        re[a] += re[b];
-        im[a] += im[b];
-        const int m = i * (16 / span);  // W_{2 span}^i = W_32^m = W_800^{25 m}
-        if (m == 0) {
-          re[b] = tr;
-          im[b] = ti;
-        } else {
-          const double2 w = T.w800[25 * m];
-          re[b] = tr * w.x - ti * w.y;
-          im[b] = tr * w.y + ti * w.x;
-        }
-      }
+  for (int k2a = 0; k2a < 8; ++k2a) {
+    double xr = r[k2a], xi = i[k2a];
+    if (l0 * k2a != 0) {
+      const double2 w = tw(T, 50 * l0 * k2a);  // W_32^{l0 k2a}
+      cmul(xr, xi, w.x, w.y);
     }
-  }
-#pragma unroll
-  for (int k2 = 0; k2 < 32; ++k2) {
-    const int p = bitrev5(k2);
-    Z[k1 + 25 * k2] = make_double2(re[p], im[p]);
+    B[slot(k1, l0 + 4 * k2a)] = make_double2(xr, xi);
   }
 }
 
-// Step D for lane l: power of bins k = l, l + 32, ... <= 800.
-__host__ __device__ inline void step_d(int l, const Tables &T, const double2 *Z, double *P) {
-  for (int k = l; k <= 800; k += 32) {
-    const double2 a = Z[k % 800];
-    const double2 b = Z[(800 - k) % 800];
-    const double er = 0.5 * (a.x + b.x), ei = 0.5 * (a.y - b.y);  // (Z_k + conj Z_{800-k}) / 2
-    const double dr = a.x - b.x, di = a.y + b.y;                    // Z_k - conj Z_{800-k}
-    const double or_ = 0.5 * di, oi = -0.5 * dr;                    // / (2 i)
-    const double2 w = T.w1600[k];
-    const double xr = er + (or_ * w.x - oi * w.y);
-    const double xi = ei + (or_ * w.y + oi * w.x);
-    P[k] = xr * xr + xi * xi;
+// Step C2, unit u = 8 k1 + k2a (0..199): 4-point DFT over l0 of row k1, columns l0 + 4 k2a;
+// output k2b goes to column k2b + 4 k2a.
+__host__ __device__ inline void step_c2(int u, double2 *B) {
+  const int k1 = u >> 3, k2a = u & 7;
+  double2 x[4];
+#pragma unroll
+  for (int l0 = 0; l0 < 4; ++l0) x[l0] = B[slot(k1, l0 + 4 * k2a)];
+  // X_k2b = sum_l0 x_l0 W_4^{l0 k2b}, W_4 = -i
+  const double s02r = x[0].x + x[2].x, s02i = x[0].y + x[2].y;
+  const double d02r = x[0].x - x[2].x, d02i = x[0].y - x[2].y;
+  const double s13r = x[1].x + x[3].x, s13i = x[1].y + x[3].y;
+  const double d13r = x[1].x - x[3].x, d13i = x[1].y - x[3].y;
+  B[slot(k1, 0 + 4 * k2a)] = make_double2(s02r + s13r, s02i + s13i);
+  B[slot(k1, 1 + 4 * k2a)] = make_double2(d02r + d13i, d02i - d13r);  // d02 - i d13
+  B[slot(k1, 2 + 4 * k2a)] = make_double2(s02r - s13r, s02i - s13i);
+  B[slot(k1, 3 + 4 * k2a)] = make_double2(d02r - d13i, d02i + d13r);  // d02 + i d13
+}
+
+// Step D, first half for lane l: read Z_k and Z_{800 - k} of the lane's pairs k = l + 32 q
+// (k <= 400) into registers.
+struct PairRegs {
+  double2 a[kPairsPerLane], b[kPairsPerLane];
+};
+
+__host__ __device__ inline void step_d_load(int l, const double2 *B, PairRegs &R) {
+#pragma unroll
+  for (int q = 0; q < kPairsPerLane; ++q) {
+    const int k = l + 32 * q;
+    if (k <= 400) {
+      R.a[q] = B[zslot(k)];
+      R.b[q] = B[zslot((800 - k) % 800)];
+    }
+  }
+}
+
+// |X_k|^2 of the real 1600-point DFT from a = Z_k and b = Z_{800-k}.
+__host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, double2 b) {
+  const double er = 0.5 * (a.x + b.x), ei = 0.5 * (a.y - b.y);  // (Z_k + conj Z_{800-k}) / 2
+  const double dr = a.x - b.x, di = a.y + b.y;                    // Z_k - conj Z_{800-k}
+  const double or_ = 0.5 * di, oi = -0.5 * dr;                    // / (2 i)
+  const double2 w = tw(T, k);
+  const double xr = er + (or_ * w.x - oi * w.y);
+  const double xi = ei + (or_ * w.y + oi * w.x);
+  return xr * xr + xi * xi;
+}
+
+// Step D, second half: P_k and P_{800 - k} in natural order over the buffer (as doubles).
+__host__ __device__ inline void step_d_store(int l, const Tables &T, const PairRegs &R, double *P) {
+#pragma unroll
+  for (int q = 0; q < kPairsPerLane; ++q) {
+    const int k = l + 32 * q;
+    if (k <= 400) {
+      P[k] = power_bin(T, k, R.a[q], R.b[q]);
+      if (k != 400) P[800 - k] = power_bin(T, 800 - k, R.b[q], R.a[q]);
+    }
   }
 }
 
@@ -219,8 +336,18 @@ __host__ __device__ inline void step_e(int l, const Tables &T, const double *P, 
     const int b = T.lane_filt[l * kMaxFiltPerLane + s];
     if (b < 0) break;
     const int k0 = T.mel_k0[b], n = T.mel_n[b], off = T.mel_off[b];
-    double acc = 0.0;
-    for (int i = 0; i < n; ++i) acc += T.melw[off + i] * P[k0 + i];
+    const double *w = T.melw + off;
+    const double *p = P + k0;
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;  // four independent chains
+    int i = 0;
+    for (; i + 4 <= n; i += 4) {
+      a0 += w[i] * p[i];
+      a1 += w[i + 1] * p[i + 1];
+      a2 += w[i + 2] * p[i + 2];
+      a3 += w[i + 3] * p[i + 3];
+    }
+    for (; i < n; ++i) a0 += w[i] * p[i];
+    const double acc = (a0 + a1) + (a2 + a3);
     double L = log10(fmax(acc, 1e-10));  // fmax drops a NaN energy
     L = fmin(fmax(L, -7.0), 2.0);
     int c = (int)floor((L + 7.0) * 16.0 / 9.0);
@@ -233,24 +360,17 @@ __host__ __device__ inline void step_e(int l, const Tables &T, const double *P, 
 // ---------------------------------------------------------------- host tables
 
 struct HostTables {
-  std::vector<double> win, melw;
-  std::vector<double2> w800, w1600;
+  std::vector<double> melw;
+  std::vector<double2> w;
   int k0[kMel], n[kMel], off[kMel];
   signed char lane_filt[32 * kMaxFiltPerLane];
-  Tables view() const {
-    return Tables{win.data(), w800.data(), w1600.data(), melw.data(), k0, n, off, lane_filt};
-  }
+  Tables view() const { return Tables{w.data(), melw.data(), k0, n, off, lane_filt}; }
 };
 
 void build_host_tables(HostTables &H) {
   const double two_pi = 6.283185307179586476925286766559;
-  H.win.resize(kWin);
-  for (int i = 0; i < kWin; ++i) H.win[i] = 0.5 - 0.5 * std::cos(two_pi * i / kWin);
-  H.w800.resize(800);
-  for (int j = 0; j < 800; ++j) H.w800[j] = make_double2(std::cos(two_pi * j / 800), -std::sin(two_pi * j / 800));
-  H.w1600.resize(kBins);
-  for (int k = 0; k < kBins; ++k)
-    H.w1600[k] = make_double2(std::cos(two_pi * k / 1600), -std::sin(two_pi * k / 1600));
+  H.w.resize(kBins);
+  for (int k = 0; k < kBins; ++k) H.w[k] = make_double2(std::cos(two_pi * k / 1600), -std::sin(two_pi * k / 1600));
   // HTK mel points: 82 points equally spaced in mel on [0, 8000] Hz
   const double mel_top = 2595.0 * std::log10(1.0 + 8000.0 / 700.0);
   double fp[kMel + 2];
@@ -307,9 +427,8 @@ cudaError_t ensure_device_tables() {
   std::lock_guard<std::mutex> lock(g_upload_mu);
   if (g_uploaded[dev]) return cudaSuccess;
   const HostTables &H = host_tables();
-  if ((e = cudaMemcpyToSymbol(d_win, H.win.data(), sizeof(double) * kWin)) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_w800, H.w800.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_w1600, H.w1600.data(), sizeof(double2) * kBins)) != cudaSuccess) return e;
+  if (H.melw.size() > (size_t)kMelNnzMax) return cudaErrorInvalidValue;
+  if ((e = cudaMemcpyToSymbol(d_w1600, H.w.data(), sizeof(double2) * kBins)) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_melw, H.melw.data(), sizeof(double) * H.melw.size())) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_mel_k0, H.k0, sizeof(H.k0))) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_mel_n, H.n, sizeof(H.n))) != cudaSuccess) return e;
@@ -323,18 +442,40 @@ cudaError_t ensure_device_tables() {
 
 // ---------------------------------------------------------------- kernels
 
-__global__ void __launch_bounds__(kWarpsPerBlock * 32) codes_kernel_entry(const float *__restrict__ wav,
-                                                                          const int64_t *__restrict__ soff,
-                                                                          const int64_t *__restrict__ foff, int n_clips,
-                                                                          int64_t n_frames,
-                                                                          const float *__restrict__ tails,
-                                                                          uint8_t *__restrict__ codes, uint32_t *err) {
+__global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(const float *__restrict__ wav,
+                                                                             const int64_t *__restrict__ soff,
+                                                                             const int64_t *__restrict__ foff,
+                                                                             int n_clips, int64_t n_frames,
+                                                                             const float *__restrict__ tails,
+                                                                             uint8_t *__restrict__ codes,
+                                                                             uint32_t *err) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  double2 *Y = reinterpret_cast<double2 *>(smem + warp * kWarpSmemBytes);
-  double2 *Z = Y + kYElems;
-  double *P = reinterpret_cast<double *>(Y);  // Y is dead once step C has run
-  const Tables T{d_win, d_w800, d_w1600, d_melw, d_mel_k0, d_mel_n, d_mel_off, d_lane_filt};
+
+  // constant tables: global -> shared once per block
+  {
+    double2 *w = reinterpret_cast<double2 *>(smem + kSmW);
+    double *melw = reinterpret_cast<double *>(smem + kSmMelW);
+    int *k0 = reinterpret_cast<int *>(smem + kSmMelK0);
+    int *nn = reinterpret_cast<int *>(smem + kSmMelN);
+    int *off = reinterpret_cast<int *>(smem + kSmMelOff);
+    signed char *lf = reinterpret_cast<signed char *>(smem + kSmLaneFilt);
+    for (int i = threadIdx.x; i < kBins; i += blockDim.x) w[i] = d_w1600[i];
+    for (int i = threadIdx.x; i < kMelNnzMax; i += blockDim.x) melw[i] = d_melw[i];
+    for (int i = threadIdx.x; i < kMel; i += blockDim.x) {
+      k0[i] = d_mel_k0[i];
+      nn[i] = d_mel_n[i];
+      off[i] = d_mel_off[i];
+    }
+    for (int i = threadIdx.x; i < 32 * kMaxFiltPerLane; i += blockDim.x) lf[i] = d_lane_filt[i];
+  }
+  __syncthreads();
+  const Tables T{reinterpret_cast<const double2 *>(smem + kSmW), reinterpret_cast<const double *>(smem + kSmMelW),
+                 reinterpret_cast<const int *>(smem + kSmMelK0), reinterpret_cast<const int *>(smem + kSmMelN),
+                 reinterpret_cast<const int *>(smem + kSmMelOff),
+                 reinterpret_cast<const signed char *>(smem + kSmLaneFilt)};
+  double2 *B = reinterpret_cast<double2 *>(smem + kSmTables + warp * kWarpBufBytes);
+  double *P = reinterpret_cast<double *>(B);
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int64_t gw = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
@@ -363,11 +504,20 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) codes_kernel_entry(const 
     }
     const ClipSampler sample{wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr,
                              (int64_t)kHop * (t - 1)};
-    step_a(lane, sample, T, Y);
+    step_a(lane, sample, T, B);
     __syncwarp();
-    if (lane < 25) step_c(lane, T, Y, Z);
+#pragma unroll 1
+    for (int u = lane; u < 100; u += 32) step_c1(u, T, B);
     __syncwarp();
-    step_d(lane, T, Z, P);
+#pragma unroll 1
+    for (int u = lane; u < 200; u += 32) step_c2(u, B);
+    __syncwarp();
+    {
+      PairRegs R;
+      step_d_load(lane, B, R);
+      __syncwarp();  // every Z value is in registers before P overwrites the buffer
+      step_d_store(lane, T, R, P);
+    }
     __syncwarp();
     step_e(lane, T, P, crow, nullptr);
     __syncwarp();
@@ -410,16 +560,14 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if (!attr_set[dev & 255]) {
-    e = cudaFuncSetAttribute(codes_kernel_entry, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kWarpSmemBytes * kWarpsPerBlock);
+    e = cudaFuncSetAttribute(codes_kernel_entry, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set[dev & 255] = true;
   }
   if (n_frames > 0) {
     int64_t blocks = (n_frames + kWarpsPerBlock - 1) / kWarpsPerBlock;
-    const int64_t cap = (int64_t)num_sms * 2;
-    if (blocks > cap) blocks = cap;
-    codes_kernel_entry<<<(unsigned)blocks, kWarpsPerBlock * 32, kWarpSmemBytes * kWarpsPerBlock, stream>>>(
+    if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM
+    codes_kernel_entry<<<(unsigned)blocks, kWarpsPerBlock * 32, kSmemBytes, stream>>>(
         wav, soff, foff, n_clips, n_frames, tails, codes, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
@@ -435,18 +583,22 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
   return cudaSuccess;
 }
 
-// Host emulation of the per-frame arithmetic of codes_kernel_entry (the same step functions,
-// lanes run one after another). Diagnostic only: no entry point of the front end calls it.
+// Host emulation of the per-frame arithmetic of codes_kernel_entry (the same step functions;
+// the lanes and units of each step run one after another, and a step's loads all complete
+// before its stores where the kernel separates them with __syncwarp). Diagnostic only: no
+// entry point of the front end calls it.
 void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {
   const HostTables &H = host_tables();
   const Tables T = H.view();
-  std::vector<double2> Yb(kYElems), Zb(kZElems);
-  std::vector<double> Pb(kBins);
+  std::vector<double2> B(800);
+  std::vector<PairRegs> R(32);
   const FrameSampler sample{frame1600};
-  for (int l = 0; l < 32; ++l) step_a(l, sample, T, Yb.data());
-  for (int l = 0; l < 25; ++l) step_c(l, T, Yb.data(), Zb.data());
-  for (int l = 0; l < 32; ++l) step_d(l, T, Zb.data(), Pb.data());
-  for (int l = 0; l < 32; ++l) step_e(l, T, Pb.data(), codes80, lhat80);
+  for (int l = 0; l < 32; ++l) step_a(l, sample, T, B.data());
+  for (int u = 0; u < 100; ++u) step_c1(u, T, B.data());
+  for (int u = 0; u < 200; ++u) step_c2(u, B.data());
+  for (int l = 0; l < 32; ++l) step_d_load(l, B.data(), R[l]);
+  for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<double *>(B.data()));
+  for (int l = 0; l < 32; ++l) step_e(l, T, reinterpret_cast<const double *>(B.data()), codes80, lhat80);
 }
 
 }  // namespace dmel

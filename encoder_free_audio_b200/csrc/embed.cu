@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t 
 
 // One warp per frame: ss = sum of the n_ct partial sums of squares, then
 // out_j <- g_j * (out_j / sqrt(ss / D + eps)) in place.
+constexpr int tc_bm = 128;  // frames per tile of the tensor-core kernel (partials layout)
 template <typename OT>
 __global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, int64_t F, int D,
                                                           const __nv_bfloat16 *__restrict__ g,
@@ -156,7 +157,8 @@ __global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, 
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t f = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < F; f += warps) {
     float ss = 0.0f;
-    for (int c = lane; c < n_ct; c += 32) ss += partials[(int64_t)c * F + f];
+    const float *col = partials + (f / tc_bm) * n_ct * tc_bm + (f % tc_bm);  // [frame tile][column tile][row]
+    for (int c = lane; c < n_ct; c += 32) ss += col[(int64_t)c * tc_bm];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.0f / sqrtf(ss / (float)D + eps);
@@ -187,17 +189,66 @@ constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_BAR = OFF_B + STAGES * B_STAGE;
 constexpr int N_BARS = 4 * STAGES + 5;
-constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
+constexpr int OFF_G = OFF_BAR + 256;          // 256 fp32 RMSNorm weights of the block's columns
+constexpr int SMEM_USED = OFF_G + BN * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack for the 1024-B swizzle atoms
 constexpr int THREADS = 320;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace tc
 
-template <typename OT, bool kRms>
+// Epilogue variants of the tensor-core kernel.
+enum TcMode : int {
+  kPlain = 0,     // no RMSNorm: store x
+  kPartials = 1,  // store x and each row's sum of squares over the tile (rms_rescale_kernel follows)
+  kFused = 2      // groups of D/256 blocks exchange the row sums and store the normalised rows
+};
+
+__device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Barrier of the 128 epilogue threads that also ANDs a flag across them, so every epilogue
+// thread takes the same branch after a bounded wait.
+__device__ __forceinline__ bool epi_barrier_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Tile i of this block's schedule: (frame tile m, column tile nt). kPlain / kPartials walk all
+// tiles with stride gridDim.x; kFused gives each block a fixed column tile (blockIdx % P) and
+// makes each group of P consecutive blocks walk the same frame tiles.
+template <int kMode>
+__device__ __forceinline__ bool tile_at(int64_t i, int64_t n_m_tiles, int P, int64_t &m, int &nt) {
+  if (kMode == kFused) {
+    const int64_t G = gridDim.x / P;
+    m = blockIdx.x / P + i * G;
+    nt = blockIdx.x % P;
+    return m < n_m_tiles;
+  }
+  const int64_t t = blockIdx.x + i * (int64_t)gridDim.x;
+  m = t / P;
+  nt = (int)(t % P);
+  return m < n_m_tiles;
+}
+
+template <typename OT, int kMode>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     embed_tc_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
-                    OT *__restrict__ out, float *__restrict__ partials, uint32_t *err) {
+                    OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                    const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,9 +262,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   auto tempty = [&](int a) { return bar0 + 8u * (3 * STAGES + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (3 * STAGES + 4);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+  float *gsm = reinterpret_cast<float *>(smem + OFF_G);  // RMSNorm weight of this block's columns
 
-  const int n_tiles_n = D / BN;
-  const int64_t n_tiles = ((F + BM - 1) / BM) * n_tiles_n;
+  const int P = D / BN;  // column tiles per row
+  const int64_t n_m_tiles = (F + BM - 1) / BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -227,6 +279,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     }
     mbar_init(done_bar, 1);
     mbar_fence_init();
+  }
+  if (kMode == kFused && threadIdx.x < BN) {
+    const int nt = blockIdx.x % P;
+    gsm[threadIdx.x] = __bfloat162float(gw[nt * BN + threadIdx.x]);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
@@ -244,17 +300,19 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       const uint64_t pol = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t pending = 0;          // stages with a load issued
-      uint32_t pending_phase = 0;    // phase bit of that load, per stage
+      uint32_t pending = 0;        // stages with a load issued
+      uint32_t pending_phase = 0;  // phase bit of that load, per stage
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-        const int n0 = (int)(t % n_tiles_n) * BN;
+      int64_t m;
+      int nt;
+      for (int64_t i = 0; ok && tile_at<kMode>(i, n_m_tiles, P, m, nt); ++i) {
+        const int n0 = nt * BN;
         for (int kb = 0; kb < KBLOCKS; ++kb) {
           if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
           mbar_arrive_expect_tx(full_b(stage), B_STAGE);
           const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
 #pragma unroll
-          for (int i = 0; i < BN / 64; ++i) tma_load_2d(dst + i * B_BOX, &tmap, n0 + 64 * i, kb * BK, full_b(stage), pol);
+          for (int q = 0; q < BN / 64; ++q) tma_load_2d(dst + q * B_BOX, &tmap, n0 + 64 * q, kb * BK, full_b(stage), pol);
           pending |= 1u << stage;
           pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -271,9 +329,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
-      for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-        const uint32_t acc = it & 1, acc_phase = (it >> 1) & 1;
+      int64_t m;
+      int nt;
+      for (int64_t i = 0; ok && tile_at<kMode>(i, n_m_tiles, P, m, nt); ++i) {
+        const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
         if (!mbar_wait(tempty(acc), acc_phase ^ 1u, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -306,8 +365,10 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
-      const int64_t f = (t / n_tiles_n) * BM + r;
+    int64_t m;
+    int nt;
+    for (int64_t i = 0; ok && tile_at<kMode>(i, n_m_tiles, P, m, nt); ++i) {
+      const int64_t f = m * BM + r;
       uint32_t cw[20];
       const bool valid = f < F;
       if (valid) {
@@ -355,17 +416,61 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     bool ok = true;
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++it) {
-      const uint32_t acc = it & 1, acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(tfull(acc), acc_phase, err)) { ok = false; break; }
+    int64_t m;
+    int nt;
+    for (int64_t i = 0; ok && tile_at<kMode>(i, n_m_tiles, P, m, nt); ++i) {
+      const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
+      if (!epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
       tc_fence_after();
-      const int64_t f = (t / n_tiles_n) * BM + r;
-      const int nt = (int)(t % n_tiles_n);
+      const int64_t f = m * BM + r;
       const bool valid = f < F;
       OT *orow = out + (valid ? f : 0) * (int64_t)D + nt * BN;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
-      float ss = 0.0f;
+      float scale = 1.0f;
+      if (kMode != kPlain) {
+        // the row's sum of squares over this tile's 256 columns
+        float ss = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tbase + c * 32, v0);
+          tmem_ld16(tbase + c * 32 + 16, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float a = __uint_as_float(v0[q]), b = __uint_as_float(v1[q]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+        float *slot = partials + ((m * P + nt) * BM);
+        if (kMode == kPartials) {
+          slot[r] = ss;
+        } else {
+          // publish this tile's row sums, wait until the group's P column tiles have all
+          // published theirs (bounded), then add them in a fixed order
+          __stcg(slot + r, ss);
+          __threadfence();
+          epi_barrier();
+          if (r == 0) {
+            atomicAdd(counters + m, 1);
+            uint32_t polls = 0;
+            while (ld_acquire(counters + m) < P) {
+              if (++polls > kMaxPolls) {
+                record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+                break;
+              }
+              __nanosleep(32);
+            }
+          }
+          epi_barrier();
+          __threadfence();
+          const float *col = partials + m * P * BM + r;
+          float tot = 0.0f;
+          for (int q = 0; q < P; ++q) tot += __ldcg(col + q * BM);
+          scale = 1.0f / sqrtf(tot / (float)D + eps);
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v0[16], v1[16];
@@ -373,14 +478,14 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         tmem_ld16(tbase + c * 32 + 16, v1);
         tmem_wait_ld();
         if (valid) {
-          float x[8];
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
+            float x[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t u = h < 2 ? v0[8 * h + i] : v1[8 * (h - 2) + i];
-              x[i] = __uint_as_float(u);
-              if (kRms) ss += x[i] * x[i];
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t u = h < 2 ? v0[8 * h + q] : v1[8 * (h - 2) + q];
+              x[q] = __uint_as_float(u);
+              if (kMode == kFused) x[q] = gsm[c * 32 + 8 * h + q] * (x[q] * scale);
             }
             store8(orow + c * 32 + 8 * h, x);
           }
@@ -388,7 +493,6 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       }
       tc_fence_before();
       mbar_arrive(tempty(acc));
-      if (kRms && valid) partials[(int64_t)nt * F + f] = ss;
     }
   }
 
@@ -430,26 +534,76 @@ cudaError_t set_smem_attr_once(K kernel, int bytes, bool *flags) {
   return e;
 }
 
-template <typename OT, bool kRms>
-cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, float *partials,
-                      uint32_t *err, int num_sms, cudaStream_t stream) {
-  static bool attr[256] = {false};
-  cudaError_t e = set_smem_attr_once(embed_tc_kernel<OT, kRms>, tc::SMEM_BYTES, attr);
-  if (e != cudaSuccess) return e;
+bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D) {
   EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return cudaErrorNotSupported;
-  CUtensorMap tmap;
+  if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)kRows};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)tc::BK};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(table), dims, strides, box,
+  CUresult r = enc(tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(table), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * (D / tc::BN);
-  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  embed_tc_kernel<OT, kRms><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, partials, err);
+  return r == CUDA_SUCCESS;
+}
+
+// Scratch of the tensor-core path with RMSNorm: row sums of squares [frame tile][column tile][128]
+// and one arrival counter per frame tile.
+struct TcScratch {
+  float *partials;
+  int *counters;
+};
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t tc_scratch_bytes(int64_t F, int D) {
+  const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
+  return round256(m_tiles * (size_t)(D / tc::BN) * tc::BM * sizeof(float)) + round256(m_tiles * sizeof(int));
+}
+
+TcScratch tc_scratch(void *ws, int64_t F, int D) {
+  const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
+  uint8_t *p = static_cast<uint8_t *>(ws);
+  TcScratch s;
+  s.partials = reinterpret_cast<float *>(p);
+  s.counters = reinterpret_cast<int *>(p + round256(m_tiles * (size_t)(D / tc::BN) * tc::BM * sizeof(float)));
+  return s;
+}
+
+// Whether the fused RMSNorm schedule can run: every block of a group of D/256 blocks must be
+// resident at once (cooperative launch, one block per SM).
+bool fused_possible(int D, int num_sms, int *grid) {
+  static int coop[256] = {0};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (coop[dev & 255] == 0) {
+    int v = 0;
+    coop[dev & 255] = (cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && v) ? 1 : 2;
+  }
+  const int P = D / tc::BN;
+  const int G = num_sms / P;
+  *grid = G * P;
+  return coop[dev & 255] == 1 && G >= 1;
+}
+
+template <typename OT, int kMode>
+cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+                      const __nv_bfloat16 *g, float eps, uint32_t *err, int grid, cudaStream_t stream) {
+  static bool attr[256] = {false};
+  cudaError_t e = set_smem_attr_once(embed_tc_kernel<OT, kMode>, tc::SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmap;
+  if (!make_table_map(&tmap, table, D)) return cudaErrorInvalidValue;
+  if (kMode == kFused) {
+    const int64_t m_tiles = (F + tc::BM - 1) / tc::BM;
+    if ((e = cudaMemsetAsync(sc.counters, 0, (size_t)m_tiles * sizeof(int), stream)) != cudaSuccess) return e;
+    void *args[] = {&tmap, (void *)&codes, (void *)&F, (void *)&D, (void *)&out, (void *)&sc.partials,
+                    (void *)&sc.counters, (void *)&g, (void *)&eps, (void *)&err};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(embed_tc_kernel<OT, kMode>), dim3(grid),
+                                       dim3(tc::THREADS), args, tc::SMEM_BYTES, stream);
+  }
+  embed_tc_kernel<OT, kMode><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, sc.partials,
+                                                                             sc.counters, g, eps, err);
   return cudaGetLastError();
 }
 
@@ -474,6 +628,36 @@ cudaError_t launch_rescale(OT *out, int64_t F, int D, const __nv_bfloat16 *g, co
   const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
   rms_rescale_kernel<OT><<<grid, 256, 0, stream>>>(out, F, D, g, partials, D / tc::BN, eps);
   return cudaGetLastError();
+}
+
+// Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
+// partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel.
+template <typename OT>
+cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, const __nv_bfloat16 *g,
+                   float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
+  const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * (D / tc::BN);
+  const int plain_grid = (int)(tiles < num_sms ? tiles : num_sms);
+  cudaError_t e;
+  if (!g) {
+    e = launch_tc<OT, kPlain>(codes, F, T, D, out, TcScratch{nullptr, nullptr}, nullptr, eps, err, plain_grid, stream);
+    if (e == cudaSuccess) ++*launches;
+    return e;
+  }
+  const TcScratch sc = tc_scratch(workspace, F, D);
+  int fgrid = 0;
+  if (fused_possible(D, num_sms, &fgrid)) {
+    e = launch_tc<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, fgrid, stream);
+    if (e == cudaSuccess) ++*launches;
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    (void)cudaGetLastError();  // clear the refused launch; fall through to the two-kernel form
+  }
+  e = launch_tc<OT, kPartials>(codes, F, T, D, out, sc, g, eps, err, plain_grid, stream);
+  if (e == cudaSuccess) ++*launches;
+  if (e == cudaSuccess) {
+    e = launch_rescale(out, F, D, g, sc.partials, eps, num_sms, stream);
+    if (e == cudaSuccess) ++*launches;
+  }
+  return e;
 }
 
 }  // namespace
@@ -514,7 +698,7 @@ bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
 
 size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
   if (!with_rmsnorm || !embed_uses_tensor_cores(table_dtype, embed_dim) || n_frames <= 0) return 0;
-  return (size_t)n_frames * (size_t)(embed_dim / tc::BN) * sizeof(float);
+  return tc_scratch_bytes(n_frames, embed_dim);
 }
 
 cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,
@@ -525,27 +709,10 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dme
   if (embed_uses_tensor_cores(table_dtype, D)) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);
     const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
-    float *partials = static_cast<float *>(workspace);
-    if (out_dtype == DMEL_BF16) {
-      auto *o = static_cast<__nv_bfloat16 *>(out);
-      e = g ? launch_tc<__nv_bfloat16, true>(codes, F, T, D, o, partials, err, num_sms, stream)
-            : launch_tc<__nv_bfloat16, false>(codes, F, T, D, o, nullptr, err, num_sms, stream);
-      if (e == cudaSuccess) ++*launches;
-      if (e == cudaSuccess && g) {
-        e = launch_rescale(o, F, D, g, partials, eps, num_sms, stream);
-        if (e == cudaSuccess) ++*launches;
-      }
-    } else {
-      auto *o = static_cast<float *>(out);
-      e = g ? launch_tc<float, true>(codes, F, T, D, o, partials, err, num_sms, stream)
-            : launch_tc<float, false>(codes, F, T, D, o, nullptr, err, num_sms, stream);
-      if (e == cudaSuccess) ++*launches;
-      if (e == cudaSuccess && g) {
-        e = launch_rescale(o, F, D, g, partials, eps, num_sms, stream);
-        if (e == cudaSuccess) ++*launches;
-      }
-    }
-    return e;
+    if (out_dtype == DMEL_BF16)
+      return run_tc(codes, F, T, D, static_cast<__nv_bfloat16 *>(out), g, eps, workspace, err, num_sms, stream,
+                    launches);
+    return run_tc(codes, F, T, D, static_cast<float *>(out), g, eps, workspace, err, num_sms, stream, launches);
   }
   if (table_dtype == DMEL_BF16) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);

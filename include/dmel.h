@@ -138,9 +138,10 @@ dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table
  * which every device that loads the library holds until the process exits.
  *
  * Limit: with rms_weight != NULL and a bf16 table whose embed_dim is a multiple of 256, the
- * request needs n_frames * (embed_dim / 256) * 4 bytes of scratch (43,690 frames at
- * embed_dim 6144); a larger request returns DMEL_ERR_TOO_LARGE and launches nothing. Other
- * requests need no scratch and have no extra limit.
+ * request needs the scratch dmel_workspace_size(n_frames, embed_dim, DMEL_BF16, 1, 1) reports,
+ * about n_frames * (embed_dim / 256) * 4 bytes (up to 43,648 frames at embed_dim 6144); a
+ * larger request returns DMEL_ERR_TOO_LARGE and launches nothing. Other requests need no
+ * scratch and have no extra limit.
  *
  * The first call on each device looks up the scratch's device address (and uploads nothing
  * else); make that first call before any stream capture. All calls share the one scratch

@@ -52,7 +52,11 @@ def test_workspace_size(lib):
     F = 12800
     assert dmel.dmel_workspace_size(0, 6144, dmel.DMEL_BF16, True, False) == 0
     with_codes = dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True)
-    assert with_codes == F * 24 * 4  # partial sums of squares, one per frame and 256-column tile
+    # row sums of squares [frame tiles of 128][24 column tiles][128] fp32 + one counter per frame
+    # tile, each region rounded to 256 bytes
+    tiles = (F + 127) // 128
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert with_codes == r256(tiles * 24 * 128 * 4) + r256(tiles * 4)
     assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, False) == with_codes + F * 80
     assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, False, True) == 0
     assert dmel.dmel_workspace_size(F, 6144, dmel.DMEL_F32, True, True) == 0  # CUDA-core path

@@ -136,6 +136,22 @@ def test_embed_tensor_core_model_dim(out_dt, rms, table_bf16, rmsw_bf16, oracle_
     print(f"tensor-core embed out={out_dt} rms={rms}: worst {worst:.2e}")
 
 
+@pytest.mark.parametrize("dim", [256, 768, 2048])
+def test_embed_tensor_core_rmsnorm_widths(dim, oracle_mod):
+    """Fused RMSNorm with groups of dim / 256 column tiles (1, 3 and 8 blocks per group) and a
+    ragged last frame tile."""
+    T, T64 = bf16_table(synth.table(seed=12, dim=dim))
+    gw = torch.from_numpy(synth.rms_weight(seed=13, dim=dim)).to(torch.bfloat16)
+    F = 700
+    codes = synth.random_codes(43, F)
+    out = torch.empty((F, dim), dtype=torch.float32, device=DEV)
+    ws = torch.empty(dmel.dmel_workspace_size(F, dim, dmel.DMEL_BF16, True, True), dtype=torch.uint8, device=DEV)
+    dmel.dmel_embed(torch.from_numpy(codes).to(DEV), T.to(DEV), out, rms_weight=gw.to(DEV), eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    ref = oracle_mod.embed(codes, T64, gw.float().numpy().astype(np.float64), 1e-6)
+    compare_embed(out.cpu().numpy(), ref, 1e-5)
+
+
 def test_embed_fp32_table_rmsnorm(oracle_mod):
     T = synth.table(seed=9, dim=512)
     gw = synth.rms_weight(seed=10, dim=512)
