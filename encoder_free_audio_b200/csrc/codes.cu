@@ -4,8 +4,10 @@
 // readings of what the pages leave open, stated in include/dmel.h).
 //
 // One warp computes one frame; a warp walks a contiguous run of frames so that consecutive
-// frames share half their samples through L1. The transform runs in fp64 so that the codes
-// agree with an exact evaluation everywhere except within ~1e-12 of a level boundary.
+// frames share half their samples through L1. The DFT runs in fp64, so the power spectrum is
+// exact to ~1e-15 relative even in bins ~120 dB below the frame's peak; the mel sums, log10,
+// clamp and quantiser then run in fp32, which moves the log-mel value by ~1e-7 at most, far
+// inside the 1e-4 band around a level boundary where either neighbouring code is accepted.
 //
 // Real DFT of 1600 points through one complex DFT of 800 points, z_m = u_{2m} + i u_{2m+1}
 // (u = windowed samples). 800 = 25 x 32 with m = 32 j + l and k = k1 + 25 k2:
@@ -16,8 +18,12 @@
 //   C2  200 in-place 4-point DFTs over l0; Z[k1 + 25 (k2a + 8 k2b)] ends in row k1, column
 //       k2b + 4 k2a;
 //   D   X_k = (Z_k + conj Z_{800-k}) / 2 + W_1600^k (Z_k - conj Z_{800-k}) / (2 i),
-//       P_k = |X_k|^2, each lane owning the pairs (k, 800 - k) it reads;
-//   E   lane l sums the sparse mel triangles assigned to it, then log10, clamp, quantise.
+//       P_k = |X_k|^2; lane l of round r reads Z at row r, column l and its partner
+//       Z_{800-k} at row 25 - r, column 31 - l (both bank-conflict free);
+//   E   the 1571 non-zero mel weights, as one list sorted by channel, are cut into 32 equal
+//       chunks; lane l sums its chunk into per-channel partials, then 80 channel sums, log10,
+//       clamp, quantise (fp32).
+// Each frame's 1600 samples are first copied into the warp's buffer with coalesced loads.
 // Every root of unity comes from one fp64 table of W_1600^k, k = 0..800 (W_800 = W_1600^2,
 // W_32 = W_1600^50, W_25 = W_1600^64, W^{1600 - k} = conj W^k). The buffer is swizzled so the
 // column accesses of A, C1 and C2 are free of shared-memory bank conflicts.
@@ -36,38 +42,48 @@ namespace {
 #define DMEL_CODES_WARPS 12
 #endif
 constexpr int kWarpsPerBlock = DMEL_CODES_WARPS;
-constexpr int kMaxFiltPerLane = 8;
 constexpr int kMelNnzMax = 1600;
-constexpr int kPairsPerLane = 13;  // ceil(401 / 32) pairs (k, 800 - k) per lane in step D
+constexpr int kMaxSegs = 128;      // channel segments of the 32 mel chunks (<= 80 + 31)
 
 // Shared memory of one block: the constant tables once, then one 800-element complex buffer
-// per warp (Y, then Z in place, then P in place).
+// per warp (Y, then Z in place, then P in place; the mel partials follow P).
 constexpr int kSmW = 0;                                    // double2 [801]: W_1600^k
-constexpr int kSmMelW = 801 * 16;                          // double [kMelNnzMax]
-constexpr int kSmMelK0 = kSmMelW + kMelNnzMax * 8;         // int [80]
-constexpr int kSmMelN = kSmMelK0 + kMel * 4;               // int [80]
-constexpr int kSmMelOff = kSmMelN + kMel * 4;              // int [80]
-constexpr int kSmLaneFilt = kSmMelOff + kMel * 4;          // signed char [32 * 8]
-constexpr int kSmTables = (kSmLaneFilt + 32 * kMaxFiltPerLane + 127) / 128 * 128;
+constexpr int kSmHann = kSmW + 801 * 16;                   // double2 [800]: (w[2m], w[2m+1])
+constexpr int kSmTwA = kSmHann + 800 * 16;                 // double2 [25 * 32]: W_800^{l k1}
+constexpr int kSmMelW = kSmTwA + 800 * 16;                 // float [kMelNnzMax]: weights
+constexpr int kSmMelK = kSmMelW + kMelNnzMax * 4;          // short [kMelNnzMax]: bin of each weight
+constexpr int kSmMelB = kSmMelK + kMelNnzMax * 2;          // uchar [kMelNnzMax]: channel of each weight
+constexpr int kSmChunk = kSmMelB + kMelNnzMax;             // int [33]: chunk bounds per lane
+constexpr int kSmSegFirst = kSmChunk + 36 * 4;             // int [32]: first segment of each lane
+constexpr int kSmChanSeg = kSmSegFirst + 32 * 4;           // int [81]: segment range per channel
+constexpr int kSmTables = (kSmChanSeg + 84 * 4 + 127) / 128 * 128;
 constexpr int kWarpBufBytes = 800 * 16;
+constexpr int kPartOffset = 3216;                          // mel partials (floats) after P[801]
 constexpr int kSmemBytes = kSmTables + kWarpsPerBlock * kWarpBufBytes;
+static_assert(kPartOffset + kMaxSegs * 4 <= kWarpBufBytes, "mel partials fit behind P");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // Constant tables, filled once per device from host-computed fp64 values.
 __device__ double2 d_w1600[kBins];
-__device__ double d_melw[kMelNnzMax];
-__device__ int d_mel_k0[kMel];
-__device__ int d_mel_n[kMel];
-__device__ int d_mel_off[kMel];
-__device__ signed char d_lane_filt[32 * kMaxFiltPerLane];
+__device__ double2 d_hann2[800];
+__device__ double2 d_twa[800];
+__device__ float d_melw[kMelNnzMax];
+__device__ short d_melk[kMelNnzMax];
+__device__ unsigned char d_melb[kMelNnzMax];
+__device__ int d_chunk[33];
+__device__ int d_segfirst[32];
+__device__ int d_chanseg[81];
 
 struct Tables {
-  const double2 *w;  // W_1600^k = exp(-2 pi i k / 1600), k = 0..800
-  const double *melw;
-  const int *mel_k0;
-  const int *mel_n;
-  const int *mel_off;
-  const signed char *lane_filt;
+  const double2 *w;      // W_1600^k = exp(-2 pi i k / 1600), k = 0..800
+  const double2 *hann2;  // periodic Hann pairs (w[2m], w[2m+1]), m = 0..799
+  const double2 *twa;    // W_800^{l k1} at [k1 * 32 + l]
+  const float *melw;     // non-zero mel weights (fp32), sorted by channel then bin
+  const short *melk;     // their bins
+  const unsigned char *melb;  // their channels
+  const int *chunk;      // lane l sums entries [chunk[l], chunk[l + 1])
+  const int *segfirst;   // first partial-sum slot of lane l
+  const int *chanseg;    // channel b adds the partials [chanseg[b], chanseg[b + 1])
 };
 
 // W_1600^idx for idx in [0, 1600).
@@ -83,9 +99,6 @@ __host__ __device__ inline void cmul(double &re, double &im, double wr, double w
   re = r;
   im = i;
 }
-
-// Periodic Hann window w[n] = 0.5 - 0.5 cos(2 pi n / 1600), the cosine being Re W_1600^n.
-__host__ __device__ inline double hann(const Tables &T, int n) { return 0.5 - 0.5 * tw(T, n).x; }
 
 // Element (row k1, column c) of a warp's 25 x 32 buffer. The three low bits of the column are
 // permuted (bits 3..4 of the column and bit 0 of the row feed in), so that eight lanes of A
@@ -184,35 +197,38 @@ __host__ __device__ inline void dft8(double (&r)[8], double (&i)[8]) {
   }
 }
 
-// Raw sample n (0..1599) of frame t of a clip: x[800 (t - 1) + n], with samples before the clip
-// taken from the carried tail (tail points one past its last sample) or zero.
-struct ClipSampler {
-  const float *base;
-  const float *tail;
-  int64_t start;
-  __host__ __device__ double operator()(int n) const {
-    const int64_t i = start + n;
-    if (i >= 0) return (double)base[i];
-    return tail ? (double)tail[i] : 0.0;
+// Copies the 1600 raw samples of frame t of a clip, x[800 (t - 1) + n], into S[n] with
+// coalesced loads (lane l takes n = l + 32 i). Samples before the clip come from the carried
+// tail (tail points one past its last sample) or are zero.
+__device__ inline void stage_frame(int l, const float *base, const float *tail, int64_t start, float *S) {
+  if (start >= 0) {
+    const float *src = base + start;
+#pragma unroll 10
+    for (int n = l; n < 1600; n += 32) S[n] = __ldg(src + n);
+  } else {
+#pragma unroll 10
+    for (int n = l; n < 1600; n += 32) {
+      const int64_t i = start + n;
+      S[n] = i >= 0 ? __ldg(base + i) : (tail ? __ldg(tail + i) : 0.0f);
+    }
   }
-};
+}
 
-// Sample n of one already-framed 1600-sample buffer.
-struct FrameSampler {
-  const float *frame;
-  __host__ __device__ double operator()(int n) const { return (double)frame[n]; }
-};
-
-// Step A for lane l. sample(n) returns raw frame sample n (0..1599) as double.
-template <class SampleFn>
-__host__ __device__ inline void step_a(int l, SampleFn sample, const Tables &T, double2 *B) {
-  double ar[25], ai[25];
+// Step A, first half for lane l: windowed z_{32 j + l} = (w s)[64 j + 2 l] + i (w s)[64 j + 2 l + 1]
+// for j = 0..24 from the staged samples S (read before the buffer is overwritten).
+__host__ __device__ inline void step_a_load(int l, const float *S, const Tables &T, double (&ar)[25],
+                                            double (&ai)[25]) {
 #pragma unroll
   for (int j = 0; j < 25; ++j) {
-    const int n0 = 64 * j + 2 * l;
-    ar[j] = hann(T, n0) * sample(n0);
-    ai[j] = hann(T, n0 + 1) * sample(n0 + 1);
+    const float2 x = *reinterpret_cast<const float2 *>(S + 64 * j + 2 * l);
+    const double2 w = T.hann2[32 * j + l];  // periodic Hann at 64 j + 2 l and the next sample
+    ar[j] = w.x * (double)x.x;
+    ai[j] = w.y * (double)x.y;
   }
+}
+
+// Step A, second half: 25-point DFT over j, twiddle W_800^{l k1}, store to row k1, column l.
+__host__ __device__ inline void step_a_dft(int l, const Tables &T, double (&ar)[25], double (&ai)[25], double2 *B) {
   // 25 = 5 x 5, j = j1 + 5 j2: inner DFTs over j2, result for (j1, ka) stored at j1 + 5 ka
 #pragma unroll
   for (int j1 = 0; j1 < 5; ++j1)
@@ -240,8 +256,8 @@ __host__ __device__ inline void step_a(int l, SampleFn sample, const Tables &T, 
     for (int kb = 0; kb < 5; ++kb) {
       const int k1 = ka + 5 * kb;
       double yr = r[kb], yi = i[kb];
-      if (l * k1 != 0) {
-        const double2 w = tw(T, (2 * l * k1) % 1600);  // W_800^{l k1}
+      if (k1 != 0) {
+        const double2 w = T.twa[k1 * 32 + l];  // W_800^{l k1}
         cmul(yr, yi, w.x, w.y);
       }
       B[slot(k1, l)] = make_double2(yr, yi);
@@ -290,20 +306,25 @@ __host__ __device__ inline void step_c2(int u, double2 *B) {
   B[slot(k1, 3 + 4 * k2a)] = make_double2(d02r - d13i, d02i + d13r);  // d02 + i d13
 }
 
-// Step D, first half for lane l: read Z_k and Z_{800 - k} of the lane's pairs k = l + 32 q
-// (k <= 400) into registers.
+// Step D, first half for lane l: pairs (k, 800 - k). Round r = 1..12 takes Z at row r, column
+// l (k = r + 25 k2 with k2 = (l >> 2) + 8 (l & 3)) and its partner Z_{800-k} at row 25 - r,
+// column 31 - l; round 0 takes row 0 (k = 25 k2, k2 <= 16; the partner is Z_{800-k} in row 0).
 struct PairRegs {
-  double2 a[kPairsPerLane], b[kPairsPerLane];
+  double2 a[13], b[13];
 };
 
+__host__ __device__ inline int dk2(int l) { return (l >> 2) + 8 * (l & 3); }
+
 __host__ __device__ inline void step_d_load(int l, const double2 *B, PairRegs &R) {
+  const int k2 = dk2(l);
+  if (k2 <= 16) {
+    R.a[0] = B[slot(0, l)];
+    R.b[0] = B[zslot((800 - 25 * k2) % 800)];
+  }
 #pragma unroll
-  for (int q = 0; q < kPairsPerLane; ++q) {
-    const int k = l + 32 * q;
-    if (k <= 400) {
-      R.a[q] = B[zslot(k)];
-      R.b[q] = B[zslot((800 - k) % 800)];
-    }
+  for (int r = 1; r <= 12; ++r) {
+    R.a[r] = B[slot(r, l)];
+    R.b[r] = B[slot(25 - r, 31 - l)];
   }
 }
 
@@ -318,95 +339,119 @@ __host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, d
   return xr * xr + xi * xi;
 }
 
-// Step D, second half: P_k and P_{800 - k} in natural order over the buffer (as doubles).
-__host__ __device__ inline void step_d_store(int l, const Tables &T, const PairRegs &R, double *P) {
+// Step D, second half: P_k and P_{800 - k} (fp32) in natural order over the buffer.
+__host__ __device__ inline void step_d_store(int l, const Tables &T, const PairRegs &R, float *P) {
+  const int k2 = dk2(l);
+  if (k2 <= 16) {
+    const int k = 25 * k2;
+    P[k] = (float)power_bin(T, k, R.a[0], R.b[0]);
+    if (k != 400) P[800 - k] = (float)power_bin(T, 800 - k, R.b[0], R.a[0]);
+  }
 #pragma unroll
-  for (int q = 0; q < kPairsPerLane; ++q) {
-    const int k = l + 32 * q;
-    if (k <= 400) {
-      P[k] = power_bin(T, k, R.a[q], R.b[q]);
-      if (k != 400) P[800 - k] = power_bin(T, 800 - k, R.b[q], R.a[q]);
-    }
+  for (int r = 1; r <= 12; ++r) {
+    const int k = r + 25 * k2;
+    P[k] = (float)power_bin(T, k, R.a[r], R.b[r]);
+    P[800 - k] = (float)power_bin(T, 800 - k, R.b[r], R.a[r]);
   }
 }
 
-// Step E for lane l: mel channels assigned to this lane -> clamped log10 and level.
-__host__ __device__ inline void step_e(int l, const Tables &T, const double *P, uint8_t *codes_row, double *lhat_row) {
-  for (int s = 0; s < kMaxFiltPerLane; ++s) {
-    const int b = T.lane_filt[l * kMaxFiltPerLane + s];
-    if (b < 0) break;
-    const int k0 = T.mel_k0[b], n = T.mel_n[b], off = T.mel_off[b];
-    const double *w = T.melw + off;
-    const double *p = P + k0;
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;  // four independent chains
-    int i = 0;
-    for (; i + 4 <= n; i += 4) {
-      a0 += w[i] * p[i];
-      a1 += w[i + 1] * p[i + 1];
-      a2 += w[i + 2] * p[i + 2];
-      a3 += w[i + 3] * p[i + 3];
+// Step E, first half for lane l: the entries [chunk[l], chunk[l + 1]) of the weight list,
+// summed per channel into the partial-sum slots segfirst[l], segfirst[l] + 1, ...
+__host__ __device__ inline void step_e_chunk(int l, const Tables &T, const float *P, float *part) {
+  const int e0 = T.chunk[l], e1 = T.chunk[l + 1];
+  int seg = T.segfirst[l];
+  int cur = T.melb[e0];
+  float acc = 0.0f;
+#pragma unroll 4
+  for (int e = e0; e < e1; ++e) {
+    const float v = T.melw[e] * P[T.melk[e]];
+    const int b = T.melb[e];
+    if (b != cur) {
+      part[seg++] = acc;
+      acc = 0.0f;
+      cur = b;
     }
-    for (; i < n; ++i) a0 += w[i] * p[i];
-    const double acc = (a0 + a1) + (a2 + a3);
-    double L = log10(fmax(acc, 1e-10));  // fmax drops a NaN energy
-    L = fmin(fmax(L, -7.0), 2.0);
-    int c = (int)floor((L + 7.0) * 16.0 / 9.0);
+    acc += v;
+  }
+  part[seg] = acc;
+}
+
+// Step E, second half: channel b = lane, lane + 32, lane + 64 adds its partials, then log10,
+// clamp and quantise.
+__host__ __device__ inline void step_e_codes(int l, const Tables &T, const float *part, uint8_t *codes_row,
+                                             double *lhat_row) {
+  for (int b = l; b < kMel; b += 32) {
+    float m = 0.0f;
+    for (int q = T.chanseg[b]; q < T.chanseg[b + 1]; ++q) m += part[q];
+    float L = log10f(fmaxf(m, 1e-10f));  // fmaxf drops a NaN energy
+    L = fminf(fmaxf(L, -7.0f), 2.0f);
+    int c = (int)floorf((L + 7.0f) * 16.0f / 9.0f);
     c = c > 15 ? 15 : (c < 0 ? 0 : c);
     codes_row[b] = (uint8_t)c;
-    if (lhat_row) lhat_row[b] = L;
+    if (lhat_row) lhat_row[b] = (double)L;
   }
 }
 
 // ---------------------------------------------------------------- host tables
 
 struct HostTables {
-  std::vector<double> melw;
-  std::vector<double2> w;
-  int k0[kMel], n[kMel], off[kMel];
-  signed char lane_filt[32 * kMaxFiltPerLane];
-  Tables view() const { return Tables{w.data(), melw.data(), k0, n, off, lane_filt}; }
+  std::vector<double2> w, hann2, twa;
+  std::vector<float> melw;
+  std::vector<short> melk;
+  std::vector<unsigned char> melb;
+  int chunk[33], segfirst[32], chanseg[81];
+  Tables view() const {
+    return Tables{w.data(), hann2.data(), twa.data(), melw.data(), melk.data(), melb.data(), chunk, segfirst, chanseg};
+  }
 };
 
 void build_host_tables(HostTables &H) {
   const double two_pi = 6.283185307179586476925286766559;
   H.w.resize(kBins);
   for (int k = 0; k < kBins; ++k) H.w[k] = make_double2(std::cos(two_pi * k / 1600), -std::sin(two_pi * k / 1600));
-  // HTK mel points: 82 points equally spaced in mel on [0, 8000] Hz
+  H.hann2.resize(800);
+  for (int m = 0; m < 800; ++m)
+    H.hann2[m] = make_double2(0.5 - 0.5 * std::cos(two_pi * (2 * m) / 1600), 0.5 - 0.5 * std::cos(two_pi * (2 * m + 1) / 1600));
+  H.twa.resize(800);
+  for (int k1 = 0; k1 < 25; ++k1)
+    for (int l = 0; l < 32; ++l) {
+      const int j = (l * k1) % 800;
+      H.twa[k1 * 32 + l] = make_double2(std::cos(two_pi * j / 800), -std::sin(two_pi * j / 800));
+    }
+  // HTK mel points: 82 points equally spaced in mel on [0, 8000] Hz; non-zero triangle weights
+  // listed channel by channel, bins ascending
   const double mel_top = 2595.0 * std::log10(1.0 + 8000.0 / 700.0);
   double fp[kMel + 2];
   for (int i = 0; i < kMel + 2; ++i) fp[i] = 700.0 * (std::pow(10.0, (mel_top * i / (kMel + 1)) / 2595.0) - 1.0);
   H.melw.clear();
-  for (int b = 0; b < kMel; ++b) {
-    H.off[b] = (int)H.melw.size();
-    H.k0[b] = -1;
-    H.n[b] = 0;
+  H.melk.clear();
+  H.melb.clear();
+  for (int b = 0; b < kMel; ++b)
     for (int k = 0; k < kBins; ++k) {
       const double f = 10.0 * k;
       const double up = (f - fp[b]) / (fp[b + 1] - fp[b]);
       const double down = (fp[b + 2] - f) / (fp[b + 2] - fp[b + 1]);
       const double h = up < down ? up : down;
       if (h > 0.0) {
-        if (H.k0[b] < 0) H.k0[b] = k;
-        H.melw.push_back(h);
-        ++H.n[b];
+        H.melw.push_back((float)h);
+        H.melk.push_back((short)k);
+        H.melb.push_back((unsigned char)b);
       }
     }
+  const int nnz = (int)H.melw.size();
+  for (int l = 0; l <= 32; ++l) H.chunk[l] = (int)((int64_t)l * nnz / 32);
+  // partial-sum slots: one per maximal run of one channel inside a chunk, numbered lane by lane
+  int seg = 0;
+  for (int b = 0; b <= kMel; ++b) H.chanseg[b] = -1;
+  for (int l = 0; l < 32; ++l) {
+    H.segfirst[l] = seg;
+    for (int e = H.chunk[l]; e < H.chunk[l + 1]; ++e) {
+      if (e > H.chunk[l] && H.melb[e] != H.melb[e - 1]) ++seg;
+      if (H.chanseg[H.melb[e]] < 0) H.chanseg[H.melb[e]] = seg;
+    }
+    ++seg;
   }
-  // longest-first assignment of channels to lanes, balancing summed triangle widths
-  int load[32] = {0}, cnt[32] = {0};
-  std::memset(H.lane_filt, -1, sizeof(H.lane_filt));
-  int order[kMel];
-  for (int b = 0; b < kMel; ++b) order[b] = b;
-  for (int a = 0; a < kMel; ++a)
-    for (int c = a + 1; c < kMel; ++c)
-      if (H.n[order[c]] > H.n[order[a]]) std::swap(order[a], order[c]);
-  for (int a = 0; a < kMel; ++a) {
-    int best = 0;
-    for (int l = 1; l < 32; ++l)
-      if (cnt[l] < kMaxFiltPerLane && (load[l] < load[best] || cnt[best] >= kMaxFiltPerLane)) best = l;
-    H.lane_filt[best * kMaxFiltPerLane + cnt[best]++] = (signed char)order[a];
-    load[best] += H.n[order[a]];
-  }
+  H.chanseg[kMel] = seg;
 }
 
 const HostTables &host_tables() {
@@ -427,13 +472,16 @@ cudaError_t ensure_device_tables() {
   std::lock_guard<std::mutex> lock(g_upload_mu);
   if (g_uploaded[dev]) return cudaSuccess;
   const HostTables &H = host_tables();
-  if (H.melw.size() > (size_t)kMelNnzMax) return cudaErrorInvalidValue;
+  if (H.melw.size() > (size_t)kMelNnzMax || H.chanseg[kMel] > kMaxSegs) return cudaErrorInvalidValue;
   if ((e = cudaMemcpyToSymbol(d_w1600, H.w.data(), sizeof(double2) * kBins)) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_melw, H.melw.data(), sizeof(double) * H.melw.size())) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_mel_k0, H.k0, sizeof(H.k0))) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_mel_n, H.n, sizeof(H.n))) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_mel_off, H.off, sizeof(H.off))) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_lane_filt, H.lane_filt, sizeof(H.lane_filt))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_hann2, H.hann2.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_twa, H.twa.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_melw, H.melw.data(), sizeof(float) * H.melw.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_melk, H.melk.data(), sizeof(short) * H.melk.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_melb, H.melb.data(), H.melb.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_chunk, H.chunk, sizeof(H.chunk))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_segfirst, H.segfirst, sizeof(H.segfirst))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_chanseg, H.chanseg, sizeof(H.chanseg))) != cudaSuccess) return e;
   g_uploaded[dev] = true;
   return cudaSuccess;
 }
@@ -455,27 +503,38 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
   // constant tables: global -> shared once per block
   {
     double2 *w = reinterpret_cast<double2 *>(smem + kSmW);
-    double *melw = reinterpret_cast<double *>(smem + kSmMelW);
-    int *k0 = reinterpret_cast<int *>(smem + kSmMelK0);
-    int *nn = reinterpret_cast<int *>(smem + kSmMelN);
-    int *off = reinterpret_cast<int *>(smem + kSmMelOff);
-    signed char *lf = reinterpret_cast<signed char *>(smem + kSmLaneFilt);
+    double2 *h2 = reinterpret_cast<double2 *>(smem + kSmHann);
+    double2 *ta = reinterpret_cast<double2 *>(smem + kSmTwA);
+    float *mw = reinterpret_cast<float *>(smem + kSmMelW);
+    short *mk = reinterpret_cast<short *>(smem + kSmMelK);
+    unsigned char *mb = reinterpret_cast<unsigned char *>(smem + kSmMelB);
+    int *ch = reinterpret_cast<int *>(smem + kSmChunk);
+    int *sf = reinterpret_cast<int *>(smem + kSmSegFirst);
+    int *cs = reinterpret_cast<int *>(smem + kSmChanSeg);
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) w[i] = d_w1600[i];
-    for (int i = threadIdx.x; i < kMelNnzMax; i += blockDim.x) melw[i] = d_melw[i];
-    for (int i = threadIdx.x; i < kMel; i += blockDim.x) {
-      k0[i] = d_mel_k0[i];
-      nn[i] = d_mel_n[i];
-      off[i] = d_mel_off[i];
+    for (int i = threadIdx.x; i < 800; i += blockDim.x) {
+      h2[i] = d_hann2[i];
+      ta[i] = d_twa[i];
     }
-    for (int i = threadIdx.x; i < 32 * kMaxFiltPerLane; i += blockDim.x) lf[i] = d_lane_filt[i];
+    for (int i = threadIdx.x; i < kMelNnzMax; i += blockDim.x) {
+      mw[i] = d_melw[i];
+      mk[i] = d_melk[i];
+      mb[i] = d_melb[i];
+    }
+    for (int i = threadIdx.x; i < 33; i += blockDim.x) ch[i] = d_chunk[i];
+    for (int i = threadIdx.x; i < 32; i += blockDim.x) sf[i] = d_segfirst[i];
+    for (int i = threadIdx.x; i < 81; i += blockDim.x) cs[i] = d_chanseg[i];
   }
   __syncthreads();
-  const Tables T{reinterpret_cast<const double2 *>(smem + kSmW), reinterpret_cast<const double *>(smem + kSmMelW),
-                 reinterpret_cast<const int *>(smem + kSmMelK0), reinterpret_cast<const int *>(smem + kSmMelN),
-                 reinterpret_cast<const int *>(smem + kSmMelOff),
-                 reinterpret_cast<const signed char *>(smem + kSmLaneFilt)};
+  const Tables T{reinterpret_cast<const double2 *>(smem + kSmW), reinterpret_cast<const double2 *>(smem + kSmHann),
+                 reinterpret_cast<const double2 *>(smem + kSmTwA), reinterpret_cast<const float *>(smem + kSmMelW),
+                 reinterpret_cast<const short *>(smem + kSmMelK),
+                 reinterpret_cast<const unsigned char *>(smem + kSmMelB), reinterpret_cast<const int *>(smem + kSmChunk),
+                 reinterpret_cast<const int *>(smem + kSmSegFirst), reinterpret_cast<const int *>(smem + kSmChanSeg)};
   double2 *B = reinterpret_cast<double2 *>(smem + kSmTables + warp * kWarpBufBytes);
-  double *P = reinterpret_cast<double *>(B);
+  float *P = reinterpret_cast<float *>(B);  // P (fp32) over the buffer after step D
+  float *S = reinterpret_cast<float *>(B);  // the frame's raw samples before step A
+  float *part = reinterpret_cast<float *>(smem + kSmTables + warp * kWarpBufBytes + kPartOffset);
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int64_t gw = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
@@ -502,9 +561,18 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
       for (int b = lane; b < kMel; b += 32) crow[b] = 0;
       continue;
     }
-    const ClipSampler sample{wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr,
-                             (int64_t)kHop * (t - 1)};
-    step_a(lane, sample, T, B);
+    // the next frame of this clip needs samples [800 (t + 1), 800 (t + 2)): start them into L1
+    if (g + 1 < g1 && (int64_t)kHop * (t + 2) <= len && lane < 25)
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(wav + soff[clip] + (int64_t)kHop * (t + 1) + 32 * lane));
+    stage_frame(lane, wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr, (int64_t)kHop * (t - 1),
+                S);
+    __syncwarp();
+    {
+      double ar[25], ai[25];
+      step_a_load(lane, S, T, ar, ai);
+      __syncwarp();  // every lane has its samples before the DFT outputs overwrite them
+      step_a_dft(lane, T, ar, ai, B);
+    }
     __syncwarp();
 #pragma unroll 1
     for (int u = lane; u < 100; u += 32) step_c1(u, T, B);
@@ -519,7 +587,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
       step_d_store(lane, T, R, P);
     }
     __syncwarp();
-    step_e(lane, T, P, crow, nullptr);
+    step_e_chunk(lane, T, P, part);
+    __syncwarp();
+    step_e_codes(lane, T, part, crow, nullptr);
     __syncwarp();
   }
 }
@@ -592,13 +662,20 @@ void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *
   const Tables T = H.view();
   std::vector<double2> B(800);
   std::vector<PairRegs> R(32);
-  const FrameSampler sample{frame1600};
-  for (int l = 0; l < 32; ++l) step_a(l, sample, T, B.data());
+  std::vector<float> part(kMaxSegs);
+  std::vector<double> arb(32 * 25), aib(32 * 25);
+  for (int l = 0; l < 32; ++l)
+    step_a_load(l, frame1600, T, *reinterpret_cast<double(*)[25]>(&arb[25 * l]),
+                *reinterpret_cast<double(*)[25]>(&aib[25 * l]));
+  for (int l = 0; l < 32; ++l)
+    step_a_dft(l, T, *reinterpret_cast<double(*)[25]>(&arb[25 * l]), *reinterpret_cast<double(*)[25]>(&aib[25 * l]),
+               B.data());
   for (int u = 0; u < 100; ++u) step_c1(u, T, B.data());
   for (int u = 0; u < 200; ++u) step_c2(u, B.data());
   for (int l = 0; l < 32; ++l) step_d_load(l, B.data(), R[l]);
-  for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<double *>(B.data()));
-  for (int l = 0; l < 32; ++l) step_e(l, T, reinterpret_cast<const double *>(B.data()), codes80, lhat80);
+  for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<float *>(B.data()));
+  for (int l = 0; l < 32; ++l) step_e_chunk(l, T, reinterpret_cast<const float *>(B.data()), part.data());
+  for (int l = 0; l < 32; ++l) step_e_codes(l, T, part.data(), codes80, lhat80);
 }
 
 }  // namespace dmel

@@ -101,8 +101,9 @@ size_t dmel_workspace_size(int64_t n_frames, int embed_dim, dmel_dtype table_dty
  * tail; P_k = |sum_n w[n] s[n] e^{-2 pi i k n/1600}|^2 with w the periodic Hann window;
  * M_b = sum_k H_b(10 k Hz) P_k with 80 HTK mel triangles on 0..8000 Hz;
  * L = min(max(log10(max(M_b, 1e-10)), -7), 2); c_b = min(15, floor((L + 7) * 16 / 9)).
- * The transform runs in fp64. Errors: DMEL_ERR_INVALID_ARG for NULL required pointers,
- * n_clips < 0 or n_frames < 0. */
+ * The DFT runs in fp64; the mel sums, log10, clamp and quantiser run in fp32 (they move L by
+ * ~1e-7 at most). Errors: DMEL_ERR_INVALID_ARG for NULL required pointers, n_clips < 0 or
+ * n_frames < 0. */
 dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
                        int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes, dmel_stream_t stream);
 

@@ -122,7 +122,8 @@ def _compare_codes(gc, gl, oc, ol, oracle_mod):
     mism = gc != oc
     assert not (mism & (dist > 1e-4)).any(), "code mismatch away from a level boundary"
     inner = (ol > -7.0) & (ol < 2.0)
-    np.testing.assert_allclose(gl[inner], ol[inner], rtol=0, atol=1e-9)
+    # the DFT runs in fp64, the mel sums and log10 in fp32: ~1e-7 in L
+    np.testing.assert_allclose(gl[inner], ol[inner], rtol=0, atol=2e-6)
 
 
 def test_kernel_arithmetic_on_host_matches_oracle(lib, oracle_mod):
