@@ -19,6 +19,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -504,6 +506,324 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- tensor-core path, CTA pairs
+
+// A cluster of two CTAs computes a 256-frame x 256-column tile with tcgen05.mma.cta_group::2:
+// each CTA writes the one-hot rows of its own 128 frames and loads half of the table block
+// (128 columns), the even CTA issues the MMAs for both, and each CTA's TMEM receives its 128
+// rows x 256 columns. Per SM this halves the table traffic from L2 and the operand bytes the
+// tensor core reads from shared memory, compared with the one-CTA tile.
+namespace tc2 {
+constexpr int BM = 128;                      // frames per CTA
+constexpr int BN = 256;                      // columns per pair tile
+constexpr int BNH = 128;                     // columns loaded by each CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
+constexpr int KBLOCKS = kRows / BK;
+constexpr int A_STAGE = BM * BK * 2;         // 16 KB
+constexpr int B_BOX = BK * 64 * 2;           // 8 KB
+constexpr int B_STAGE = BK * BNH * 2;        // 16 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_BAR = OFF_B + STAGES * B_STAGE;
+constexpr int N_BARS = 3 * STAGES + 5;
+constexpr int OFF_G = OFF_BAR + 256;
+constexpr int SMEM_USED = OFF_G + BN * 4;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+constexpr int THREADS = 320;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+static_assert(N_BARS * 8 + 16 <= 256, "barrier area");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+}  // namespace tc2
+
+// Pair tile i of this cluster: (pair frame tile mp, column tile nt). kPlain / kPartials walk all
+// pair tiles with stride = number of clusters; kFused gives each cluster a fixed column tile
+// and makes each group of P clusters walk the same pair frame tiles.
+template <int kMode>
+__device__ __forceinline__ bool pair_tile_at(int64_t i, int64_t n_pm, int P, int64_t &mp, int &nt) {
+  const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  if (kMode == kFused) {
+    const int64_t G = ncl / P;
+    mp = cid / P + i * G;
+    nt = (int)(cid % P);
+    return mp < n_pm;
+  }
+  const int64_t t = cid + i * ncl;
+  mp = t / P;
+  nt = (int)(t % P);
+  return mp < n_pm;
+}
+
+template <typename OT, int kMode>
+__global__ void __launch_bounds__(tc2::THREADS, 1)
+    embed_tc2_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
+                     OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                     const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
+  using namespace tc2;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_a = [&](int s) { return bar0 + 8u * s; };
+  auto full_b = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (3 * STAGES + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (3 * STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (3 * STAGES + 4);
+  auto in_leader = [&](uint32_t local_bar) { return mapa_shared(local_bar, 0); };
+  auto in_peer = [&](uint32_t local_bar) { return mapa_shared(local_bar, 1); };
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+  float *gsm = reinterpret_cast<float *>(smem + OFF_G);
+
+  const int P = D / BN;
+  const int64_t n_m_tiles = (F + BM - 1) / BM;      // 128-frame tiles with at least one frame
+  const int64_t n_pm = (F + 2 * BM - 1) / (2 * BM);  // 256-frame pair tiles
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_a(s), 8);  // 4 producer warps of each CTA (used in the even CTA)
+      mbar_init(full_b(s), 1);  // the leader's expect-tx for both halves
+      mbar_init(empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 8);  // 4 epilogue warps of each CTA (used in the even CTA)
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (kMode == kFused && threadIdx.x < BN) {
+    const int nt = (int)((blockIdx.x >> 1) % P);
+    gsm[threadIdx.x] = __bfloat162float(gw[nt * BN + threadIdx.x]);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap);
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer: this CTA's half of the table block
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pending = 0, pending_phase = 0;
+      bool ok = true;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; ok && pair_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+        const int n0 = nt * BN + (int)rank * BNH;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
+          const uint32_t fb = in_leader(full_b(stage));
+          if (leader) mbar_arrive_expect_tx(full_b(stage), 2 * B_STAGE);  // both CTAs' halves
+          const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int q = 0; q < BNH / 64; ++q) tma_load_2d_pair(dst + q * B_BOX, &tmap, n0 + 64 * q, kb * BK, fb, pol);
+          pending |= 1u << stage;
+          pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // the leader's MMA thread consumes every load; the leader waits for the last ones below
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (pending & (1u << s)) mbar_wait(full_b(s), (pending_phase >> s) & 1u, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (even CTA only)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; ok && pair_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+        const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
+        if (!mbar_wait(tempty(acc), acc_phase ^ 1u, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          if (!mbar_wait(full_a(stage), phase, err) || !mbar_wait(full_b(stage), phase, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(smem + OFF_A + stage * A_STAGE);
+          const uint32_t b0 = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t adesc = smem_desc(a0 + 32u * k, 16u, 1024u, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(b0 + 2048u * k, (uint32_t)B_BOX, 1024u, kSwizzle128B);
+            tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(empty(stage));
+          tc_commit_pair(in_peer(empty(stage)));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull(acc));
+        tc_commit_pair(in_peer(tfull(acc)));
+      }
+      tc_commit_pair(done_bar);
+      mbar_wait(done_bar, 0, err);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ one-hot A producers (row r per thread)
+    const int r = threadIdx.x - 64;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int64_t mp;
+    int nt;
+    for (int64_t i = 0; ok && pair_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      const int64_t f = (2 * mp + rank) * BM + r;
+      uint32_t cw[20];
+      const bool valid = f < F;
+      if (valid) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + f * kMel);
+#pragma unroll
+        for (int q = 0; q < 5; ++q) {
+          const uint4 u = __ldg(src + q);
+          cw[4 * q] = u.x; cw[4 * q + 1] = u.y; cw[4 * q + 2] = u.z; cw[4 * q + 3] = u.w;
+        }
+        uint32_t bad = 0;
+#pragma unroll
+        for (int q = 0; q < 20; ++q) bad |= cw[q] & 0xF0F0F0F0u;
+        if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 20; ++q) cw[q] = 0;
+      }
+      const uint32_t row_off = (uint32_t)(r >> 3) * 1024u + (uint32_t)(r & 7) * 128u;
+#pragma unroll
+      for (int kb = 0; kb < KBLOCKS; ++kb) {
+        if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
+        uint8_t *rowp = smem + OFF_A + stage * A_STAGE + row_off;
+        const uint32_t w = cw[kb];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t c = (w >> (8 * (ch >> 1))) & 15u;
+          const bool hit = valid && ((c >> 3) == (uint32_t)(ch & 1));
+          const uint32_t e = c & 7u;
+          const uint32_t one = (e & 1u) ? 0x3F800000u : 0x00003F80u;
+          uint4 v;
+          v.x = (hit && (e >> 1) == 0) ? one : 0u;
+          v.y = (hit && (e >> 1) == 1) ? one : 0u;
+          v.z = (hit && (e >> 1) == 2) ? one : 0u;
+          v.w = (hit && (e >> 1) == 3) ? one : 0u;
+          *reinterpret_cast<uint4 *>(rowp + ((ch ^ (r & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(in_leader(full_a(stage)));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (this CTA's 128 rows)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    bool ok = true;
+    int64_t mp;
+    int nt;
+    for (int64_t i = 0; ok && pair_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
+      if (!epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
+      tc_fence_after();
+      const int64_t m = 2 * mp + rank;
+      const int64_t f = m * BM + r;
+      const bool valid = f < F;
+      const bool live = m < n_m_tiles;  // the pair's second half may hold no frame at all
+      OT *orow = out + (valid ? f : 0) * (int64_t)D + nt * BN;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
+      float scale = 1.0f;
+      if (kMode != kPlain && live) {
+        float ss = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tbase + c * 32, v0);
+          tmem_ld16(tbase + c * 32 + 16, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float a = __uint_as_float(v0[q]), b = __uint_as_float(v1[q]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+        float *slot = partials + ((m * P + nt) * BM);
+        if (kMode == kPartials) {
+          slot[r] = ss;
+        } else {
+          __stcg(slot + r, ss);
+          __threadfence();
+          epi_barrier();
+          if (r == 0) {
+            atomicAdd(counters + m, 1);
+            uint32_t polls = 0;
+            while (ld_acquire(counters + m) < P) {
+              if (++polls > kMaxPolls) {
+                record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+                break;
+              }
+              __nanosleep(32);
+            }
+          }
+          epi_barrier();
+          __threadfence();
+          const float *col = partials + m * P * BM + r;
+          float tot = 0.0f;
+          for (int q = 0; q < P; ++q) tot += __ldcg(col + q * BM);
+          scale = 1.0f / sqrtf(tot / (float)D + eps);
+        }
+      }
+      if (live) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tbase + c * 32, v0);
+          tmem_ld16(tbase + c * 32 + 16, v1);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              float x[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint32_t u = h < 2 ? v0[8 * h + q] : v1[8 * (h - 2) + q];
+                x[q] = __uint_as_float(u);
+                if (kMode == kFused) x[q] = gsm[c * 32 + 8 * h + q] * (x[q] * scale);
+              }
+              store8(orow + c * 32 + 8 * h, x);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(in_leader(tempty(acc)));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();  // every MMA into either CTA's TMEM has completed (the leader waited above)
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -630,20 +950,92 @@ cudaError_t launch_rescale(OT *out, int64_t F, int D, const __nv_bfloat16 *g, co
   return cudaGetLastError();
 }
 
+// CTA-pair launch (clusters of 2); cooperative when the fused schedule needs every group
+// co-resident. Returns cudaErrorNotSupported when the pairs cannot all be resident at once.
+template <typename OT, int kMode>
+cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+                       const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
+  static bool attr[256] = {false};
+  cudaError_t e = set_smem_attr_once(embed_tc2_kernel<OT, kMode>, tc2::SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmap;
+  if (!make_table_map(&tmap, table, D)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(tc2::THREADS);
+  cfg.dynamicSmemBytes = tc2::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeCooperative;
+  at[1].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int resident = 0;
+  if (cudaOccupancyMaxActiveClusters(&resident, embed_tc2_kernel<OT, kMode>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
+  }
+  if (kMode == kFused) {
+    if (resident < clusters) return cudaErrorNotSupported;
+    cfg.numAttrs = 2;
+    const int64_t m_tiles = (F + tc2::BM - 1) / tc2::BM;
+    if ((e = cudaMemsetAsync(sc.counters, 0, (size_t)m_tiles * sizeof(int), stream)) != cudaSuccess) return e;
+  } else if (resident < 1) {
+    return cudaErrorNotSupported;
+  }
+  return cudaLaunchKernelEx(&cfg, embed_tc2_kernel<OT, kMode>, tmap, codes, F, D, out, sc.partials, sc.counters, g, eps,
+                            err);
+}
+
+// One-CTA tiles instead of CTA pairs when the environment sets DMEL_EMBED_TILE=single (read
+// once per process; for comparisons and tests).
+bool pairs_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("DMEL_EMBED_TILE");
+    return !(v && strcmp(v, "single") == 0);
+  }();
+  return on;
+}
+
 // Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
-// partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel.
+// partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel. CTA pairs
+// first; one-CTA tiles when pairs are switched off or cannot launch.
 template <typename OT>
 cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, const __nv_bfloat16 *g,
                    float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
-  const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * (D / tc::BN);
+  const int P = D / tc::BN;
+  const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * P;
   const int plain_grid = (int)(tiles < num_sms ? tiles : num_sms);
+  const int64_t pair_tiles = ((F + 2 * tc2::BM - 1) / (2 * tc2::BM)) * P;
+  const int max_clusters = num_sms / 2;
+  const int plain_clusters = (int)(pair_tiles < max_clusters ? pair_tiles : max_clusters);
+  const TcScratch sc = g ? tc_scratch(workspace, F, D) : TcScratch{nullptr, nullptr};
   cudaError_t e;
   if (!g) {
-    e = launch_tc<OT, kPlain>(codes, F, T, D, out, TcScratch{nullptr, nullptr}, nullptr, eps, err, plain_grid, stream);
+    if (pairs_enabled()) {
+      e = launch_tc2<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, plain_clusters, stream);
+      if (e == cudaSuccess) {
+        ++*launches;
+        return e;
+      }
+      (void)cudaGetLastError();  // pairs refused: one-CTA tiles below
+    }
+    e = launch_tc<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, plain_grid, stream);
     if (e == cudaSuccess) ++*launches;
     return e;
   }
-  const TcScratch sc = tc_scratch(workspace, F, D);
+  if (pairs_enabled() && max_clusters / P >= 1) {
+    e = launch_tc2<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, (max_clusters / P) * P, stream);
+    if (e == cudaSuccess) {
+      ++*launches;
+      return e;
+    }
+    (void)cudaGetLastError();  // pairs refused (co-residency or launch attributes): one-CTA tiles below
+  }
   int fgrid = 0;
   if (fused_possible(D, num_sms, &fgrid)) {
     e = launch_tc<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, fgrid, stream);
