@@ -41,6 +41,9 @@ PATH_BYTES_PER_FRAME = 800 * 4 + DIM * 2
 EMBED_BYTES_PER_FRAME = 80 + DIM * 2
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
+# DRAM bytes (read + write) of one launch of the dominant kernel on this workload, from the ncu
+# capture summarised in profiles/ (None when the kernel changed since the capture)
+EMBED_TRAFFIC_PER_LAUNCH = None
 
 
 def peaks():
@@ -135,6 +138,32 @@ def cpu_baseline(wav, off, table64, g64, budget_s: float = 12.0) -> dict:
             "sample": f"{n} random frames of the {F}-frame workload (codes + embedding + RMSNorm, fp64)"}
 
 
+def streaming_latency(torch, dev, T, G, FrontEnd, dmel, warmup: int, calls: int = 200) -> dict:
+    """Streaming shape: 4096 streams, each call brings 800 new samples per stream plus the
+    carried 800-sample tail (one frame per stream). Per-call device time with CUDA events."""
+    from encoder_free_audio_b200 import synth
+    S = synth.Streams4096()
+    fe = FrontEnd(T, G, 1e-6, torch.bfloat16)
+    plan = fe.plan(synth.offsets_from_lengths([800] * S.n))
+    xs = [torch.from_numpy(S.call(k)).to(dev).reshape(-1) for k in range(8)]
+    tails = torch.zeros((S.n, 800), device=dev)
+    for k in range(warmup):
+        fe.forward(xs[k % 8], plan, tails=tails, tails_out=tails)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+    st = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    for k in range(calls):
+        evs[k][0].record(st)
+        fe.forward(xs[k % 8], plan, tails=tails, tails_out=tails)
+        evs[k][1].record(st)
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    return {"workload": "streams4096: 4096 streams x (800 new + 800 carried samples) per call, bf16, RMSNorm",
+            "frames_per_call": S.n, "calls": calls, "p50_us": 1e3 * ms[len(ms) // 2],
+            "p99_us": 1e3 * ms[min(len(ms) - 1, int(0.99 * len(ms)))],
+            "tokens_per_s": S.n * calls / (sum(ms) / 1e3), "launches_per_call": dmel.dmel_last_launch_count()}
+
+
 def load_workload():
     from encoder_free_audio_b200 import synth
     wav, off = synth.batch64_10s()
@@ -193,7 +222,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    from encoder_free_audio_b200 import build, dmel
+    from encoder_free_audio_b200 import build, dmel, replicas
     from encoder_free_audio_b200.frontend import FrontEnd
     build.build()
 
@@ -214,11 +243,7 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return replicas.max_over_ranks(x, world, dev)
 
     # ---------------------------------------------------------- device-resident timed region
     for _ in range(args.warmup):
@@ -278,6 +303,8 @@ def run_ours(args):
         e2e_evs[i][1].record(stream)
     barrier()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
+    # ---------------------------------------------------------- streaming shape (context line)
+    stream_line = streaming_latency(torch, dev, T, G, FrontEnd, dmel, args.warmup)
     err_bits = dmel.dmel_get_device_error(clear=True)
 
     if rank != 0:
@@ -287,7 +314,7 @@ def run_ours(args):
         return 0
 
     pk = peaks()
-    value = world * F * args.steps / (total_ms / 1e3)
+    value = replicas.job_throughput([F * args.steps] * world, total_ms / 1e3)
     emb_avg_s = statistics.mean(embed_ms) / 1e3
     emb_achieved = EMBED_BYTES_PER_FRAME * F / emb_avg_s / 1e9
     line = {
@@ -312,14 +339,15 @@ def run_ours(args):
                 "h2d_bytes_per_step": int(wav.nbytes), "d2h_bytes_per_step": int(F * 80)},
         "gpu_launches": launches,
         "roofline": {"bound": "hbm", "achieved": emb_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": emb_achieved / pk["hbm_gbs"], "traffic": None,
-                     "kernel": "dmel_embed stage (embed_tc_kernel + rms_rescale_kernel)",
+                     "frac": emb_achieved / pk["hbm_gbs"], "traffic": EMBED_TRAFFIC_PER_LAUNCH,
+                     "kernel": "embed_tc2_kernel (fused RMSNorm, CTA pairs), timed as the dmel_embed call",
                      "peak_source": pk["source"]},
         "roofline_tensor": {"achieved": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12,
                             "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                             "frac": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12 / pk["bf16_tflops_sustained"],
                             "note": "one-hot product flops 2*1280*6144 per frame, sustained bf16 peak"},
         "stages_ms": {"codes": statistics.mean(codes_ms), "embed": statistics.mean(embed_ms)},
+        "streaming": stream_line,
         "device_error_bits": err_bits,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -906,6 +906,8 @@ bool fused_possible(int D, int num_sms, int *grid) {
   return coop[dev & 255] == 1 && G >= 1;
 }
 
+bool cooperative_enabled();
+
 template <typename OT, int kMode>
 cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
                       const __nv_bfloat16 *g, float eps, uint32_t *err, int grid, cudaStream_t stream) {
@@ -917,10 +919,12 @@ cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
   if (kMode == kFused) {
     const int64_t m_tiles = (F + tc::BM - 1) / tc::BM;
     if ((e = cudaMemsetAsync(sc.counters, 0, (size_t)m_tiles * sizeof(int), stream)) != cudaSuccess) return e;
-    void *args[] = {&tmap, (void *)&codes, (void *)&F, (void *)&D, (void *)&out, (void *)&sc.partials,
-                    (void *)&sc.counters, (void *)&g, (void *)&eps, (void *)&err};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(embed_tc_kernel<OT, kMode>), dim3(grid),
-                                       dim3(tc::THREADS), args, tc::SMEM_BYTES, stream);
+    if (cooperative_enabled()) {
+      void *args[] = {&tmap, (void *)&codes, (void *)&F, (void *)&D, (void *)&out, (void *)&sc.partials,
+                      (void *)&sc.counters, (void *)&g, (void *)&eps, (void *)&err};
+      return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(embed_tc_kernel<OT, kMode>), dim3(grid),
+                                         dim3(tc::THREADS), args, tc::SMEM_BYTES, stream);
+    }
   }
   embed_tc_kernel<OT, kMode><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, sc.partials,
                                                                              sc.counters, g, eps, err);
@@ -981,7 +985,7 @@ cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tab
   }
   if (kMode == kFused) {
     if (resident < clusters) return cudaErrorNotSupported;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = cooperative_enabled() ? 2 : 1;
     const int64_t m_tiles = (F + tc2::BM - 1) / tc2::BM;
     if ((e = cudaMemsetAsync(sc.counters, 0, (size_t)m_tiles * sizeof(int), stream)) != cudaSuccess) return e;
   } else if (resident < 1) {
@@ -989,6 +993,19 @@ cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tab
   }
   return cudaLaunchKernelEx(&cfg, embed_tc2_kernel<OT, kMode>, tmap, codes, F, D, out, sc.partials, sc.counters, g, eps,
                             err);
+}
+
+// Fused kernels are launched cooperatively, which guarantees that every block of a group is
+// resident while the group exchanges row sums. DMEL_COOPERATIVE=0 (read once per process)
+// launches the same kernel and grid without that attribute, which profilers that cannot replay
+// cooperative cluster launches need; the bounded waits then report DMEL_DEVERR_WAIT_TIMEOUT
+// rather than stall if other work keeps some blocks off the GPU.
+bool cooperative_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("DMEL_COOPERATIVE");
+    return !(v && strcmp(v, "0") == 0);
+  }();
+  return on;
 }
 
 // One-CTA tiles instead of CTA pairs when the environment sets DMEL_EMBED_TILE=single (read

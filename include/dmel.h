@@ -25,6 +25,10 @@
  *   - n_clips == 0 or n_frames == 0 is a valid call that does nothing.
  *   - No entry point allocates device memory. Scratch space comes from the caller's workspace;
  *     dmel_workspace_size() says how much.
+ *   - Environment (read once per process): DMEL_EMBED_TILE=single runs the tensor-core
+ *     embedding on one-CTA tiles instead of CTA pairs; DMEL_COOPERATIVE=0 launches the fused
+ *     RMSNorm kernels without the cooperative attribute (for profilers that cannot replay
+ *     cooperative cluster launches). Both exist for comparison and measurement.
  */
 #ifndef DMEL_H
 #define DMEL_H
