@@ -206,11 +206,11 @@ __device__ inline void stage_frame(int l, const float *base, const float *tail, 
 #pragma unroll 10
     for (int n = l; n < 1600; n += 32) S[n] = __ldg(src + n);
   } else {
-#pragma unroll 10
-    for (int n = l; n < 1600; n += 32) {
-      const int64_t i = start + n;
-      S[n] = i >= 0 ? __ldg(base + i) : (tail ? __ldg(tail + i) : 0.0f);
-    }
+    // first frame of a clip (start = -800): the carried tail (or zeros), then the new samples
+#pragma unroll 5
+    for (int n = l; n < 800; n += 32) S[n] = tail ? __ldg(tail + (n - 800)) : 0.0f;
+#pragma unroll 5
+    for (int n = 800 + l; n < 1600; n += 32) S[n] = __ldg(base + (n - 800));
   }
 }
 
@@ -543,11 +543,26 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
   const int64_t g1 = g0 + chunk < n_frames ? g0 + chunk : n_frames;
   if (g0 >= g1) return;
 
-  // last clip with foff[clip] <= g0
+  // last clip with foff[clip] <= g0: a 32-way search, each lane probing one point per round
   int lo = 0, hi = n_clips - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (foff[mid] <= g0) lo = mid; else hi = mid - 1;
+  while (hi - lo > 31) {
+    const int64_t span = hi - lo;
+    const int probe = lo + (int)((span * (lane + 1)) / 33);
+    const unsigned le = __ballot_sync(0xffffffffu, foff[probe] <= g0);
+    if (le == 0) {
+      hi = lo + (int)((span * 1) / 33) - 1;
+    } else {
+      const int top = 31 - __clz(le);  // last probe with foff <= g0 (foff is non-decreasing)
+      const int nlo = lo + (int)((span * (top + 1)) / 33);
+      const int nhi = top == 31 ? hi : lo + (int)((span * (top + 2)) / 33) - 1;
+      lo = nlo;
+      hi = nhi;
+    }
+  }
+  {
+    const int probe = lo + lane;
+    const unsigned le = __ballot_sync(0xffffffffu, probe <= hi && foff[probe] <= g0);
+    lo = lo + (31 - __clz(le));
   }
   int clip = lo;
 
@@ -594,28 +609,30 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
   }
 }
 
-__global__ void tails_kernel_entry(const float *__restrict__ wav, const int64_t *__restrict__ soff,
-                                   const int64_t *__restrict__ foff, int n_clips, const float *tails,
-                                   float *tails_out, uint32_t *err) {
-  const int64_t total = (int64_t)n_clips * kHop;
-  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int c = (int)(idx / kHop);
-    const int n = (int)(idx % kHop);
+// Carried tails: one block per clip row (800 floats); the source is the last 800 consumed
+// samples of the clip, or the tail in when the clip has no frame.
+__global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restrict__ wav,
+                                                          const int64_t *__restrict__ soff,
+                                                          const int64_t *__restrict__ foff, int n_clips,
+                                                          const float *tails, float *tails_out, uint32_t *err) {
+  for (int c = blockIdx.x; c < n_clips; c += gridDim.x) {
     const int64_t F = foff[c + 1] - foff[c];
     const int64_t len = soff[c + 1] - soff[c];
-    float v;
-    if (F >= 1) {
-      if ((int64_t)kHop * F <= len) {
-        v = wav[soff[c] + (int64_t)kHop * (F - 1) + n];
-      } else {
-        record_error(err, DMEL_DEVERR_OFFSETS);
-        v = 0.0f;
-      }
-    } else {
-      v = tails ? tails[idx] : 0.0f;
+    float *dst = tails_out + (int64_t)c * kHop;
+    if (F >= 1 && (int64_t)kHop * F > len) {
+      if (threadIdx.x == 0) record_error(err, DMEL_DEVERR_OFFSETS);
+      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = 0.0f;
+      continue;
     }
-    tails_out[idx] = v;
+    const float *src = F >= 1 ? wav + soff[c] + (int64_t)kHop * (F - 1) : (tails ? tails + (int64_t)c * kHop : nullptr);
+    if (!src) {
+      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = 0.0f;
+    } else if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      for (int n = threadIdx.x; n < kHop / 4; n += blockDim.x)
+        reinterpret_cast<float4 *>(dst)[n] = reinterpret_cast<const float4 *>(src)[n];
+    } else {
+      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = src[n];
+    }
   }
 }
 
@@ -643,9 +660,8 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
     ++*launches;
   }
   if (tails_out && n_clips > 0) {
-    const int64_t total = (int64_t)n_clips * kHop;
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    int64_t blocks = n_clips;
+    if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
     tails_kernel_entry<<<(unsigned)blocks, 256, 0, stream>>>(wav, soff, foff, n_clips, tails, tails_out, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;

@@ -17,6 +17,19 @@ from . import dmel
 
 
 @dataclass
+class ChunkPlan:
+    """A run of whole clips [clip0, clip1) of a batch, with offsets rebased to the run."""
+    clip0: int
+    clip1: int
+    sample0: int
+    sample1: int
+    frame0: int
+    frame1: int
+    sample_offsets: torch.Tensor  # device int64, rebased to 0
+    frame_offsets: torch.Tensor   # device int64, rebased to 0
+
+
+@dataclass
 class Plan:
     sample_offsets_host: np.ndarray
     frame_offsets_host: np.ndarray
@@ -28,6 +41,7 @@ class Plan:
     codes: torch.Tensor            # device uint8 [n_frames, 80]
     workspace: torch.Tensor | None
     wav: torch.Tensor              # device fp32 [n_samples] (input staging for forward_host)
+    chunks: list                   # ChunkPlan runs used by forward_host to overlap copies and compute
 
     @property
     def n_clips(self) -> int:
@@ -44,13 +58,29 @@ class FrontEnd:
         self.out_dtype = out_dtype
         self.dim = int(table.shape[1])
 
-    def plan(self, sample_offsets_host) -> Plan:
+    def plan(self, sample_offsets_host, chunks: int = 4) -> Plan:
+        """Buffers for batches with these clip boundaries; `chunks` runs of whole clips (balanced
+        by frames) for the pipelined host path."""
         so = np.ascontiguousarray(np.asarray(sample_offsets_host, np.int64))
         fo = dmel.dmel_frame_offsets(so)
         dev = self.table.device
         F = int(fo[-1])
+        n_clips = so.shape[0] - 1
         ws_bytes = dmel.dmel_workspace_size(F, self.dim, dmel._dtype_code(self.table), self.rms_weight is not None,
                                             True)
+        runs = []
+        k = max(1, min(int(chunks), n_clips))
+        bounds = [0]
+        for i in range(1, k):
+            c = int(np.searchsorted(fo, F * i // k, side="left"))
+            bounds.append(min(max(c, bounds[-1]), n_clips))
+        bounds.append(n_clips)
+        for c0, c1 in zip(bounds[:-1], bounds[1:]):
+            if c1 <= c0:
+                continue
+            runs.append(ChunkPlan(c0, c1, int(so[c0]), int(so[c1]), int(fo[c0]), int(fo[c1]),
+                                  torch.from_numpy(so[c0:c1 + 1] - so[c0]).to(dev),
+                                  torch.from_numpy(fo[c0:c1 + 1] - fo[c0]).to(dev)))
         return Plan(
             sample_offsets_host=so,
             frame_offsets_host=fo,
@@ -62,6 +92,7 @@ class FrontEnd:
             codes=torch.empty((F, dmel.N_MEL), dtype=torch.uint8, device=dev),
             workspace=torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None,
             wav=torch.empty(int(so[-1]), dtype=torch.float32, device=dev),
+            chunks=runs,
         )
 
     def forward(self, wav: torch.Tensor, plan: Plan, tails=None, tails_out=None, stream=None) -> torch.Tensor:
@@ -72,11 +103,33 @@ class FrontEnd:
                           codes_out=plan.codes, workspace=plan.workspace, stream=stream)
         return plan.out
 
-    def forward_host(self, wav_host: torch.Tensor, plan: Plan, codes_host: torch.Tensor, stream=None):
+    def forward_host(self, wav_host: torch.Tensor, plan: Plan, codes_host: torch.Tensor, copy_stream=None):
         """End to end from host memory: copies the pinned fp32 waveforms to the device, runs the
-        front end, copies the codes (uint8 [n_frames, 80], pinned) back. All on one stream,
-        asynchronous; the caller synchronises."""
-        plan.wav.copy_(wav_host, non_blocking=True)
-        self.forward(plan.wav, plan, stream=stream)
-        codes_host.copy_(plan.codes, non_blocking=True)
+        front end, copies the codes (uint8 [n_frames, 80], pinned) back; the frame vectors stay
+        in plan.out. The batch goes in plan.chunks runs of whole clips: the host-to-device copy
+        of run i + 1 (on `copy_stream`) overlaps the kernels of run i (on the current stream).
+        Asynchronous; the caller synchronises the current stream."""
+        compute = torch.cuda.current_stream()
+        copy = copy_stream if copy_stream is not None else self._copy_stream()
+        copy.wait_stream(compute)  # the buffers are free once earlier work on them is done
+        ready = []
+        for r in plan.chunks:
+            with torch.cuda.stream(copy):
+                plan.wav[r.sample0:r.sample1].copy_(wav_host[r.sample0:r.sample1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(copy)
+            ready.append(ev)
+        for r, ev in zip(plan.chunks, ready):
+            compute.wait_event(ev)
+            if r.frame1 > r.frame0:
+                dmel.dmel_forward(plan.wav[r.sample0:r.sample1], r.sample_offsets, r.frame_offsets,
+                                  r.frame1 - r.frame0, self.table, plan.out[r.frame0:r.frame1],
+                                  rms_weight=self.rms_weight, eps=self.eps, codes_out=plan.codes[r.frame0:r.frame1],
+                                  workspace=plan.workspace, stream=compute)
+                codes_host[r.frame0:r.frame1].copy_(plan.codes[r.frame0:r.frame1], non_blocking=True)
         return plan.out
+
+    def _copy_stream(self):
+        if getattr(self, "_copy", None) is None or self._copy.device != self.table.device:
+            self._copy = torch.cuda.Stream(device=self.table.device)
+        return self._copy

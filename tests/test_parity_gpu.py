@@ -223,6 +223,24 @@ def test_forward_batch64_10s(table_bf16, rmsw_bf16, oracle_mod):
     _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, embed_ids=emb, label="batch64_10s")
 
 
+def test_forward_host_pipelined_equals_single_call(table_bf16, rmsw_bf16):
+    """The host path (copies of run i + 1 overlapping the kernels of run i) gives the same
+    vectors and codes, bit for bit, as one device-side call on the whole batch."""
+    T, _ = table_bf16
+    g, _ = rmsw_bf16
+    wav, off = synth.ragged1024(n_clips=40)
+    fe = FrontEnd(T, g, 1e-6, torch.bfloat16)
+    one = fe.plan(off)
+    fe.forward(torch.from_numpy(wav).to(DEV), one)
+    for chunks in (1, 3, 7):
+        p = fe.plan(off, chunks=chunks)
+        codes_h = torch.empty((p.n_frames, 80), dtype=torch.uint8).pin_memory()
+        fe.forward_host(torch.from_numpy(wav).pin_memory(), p, codes_h)
+        torch.cuda.synchronize()
+        assert torch.equal(p.out, one.out), chunks
+        assert torch.equal(codes_h, one.codes.cpu()), chunks
+
+
 def test_forward_long_20min(table_bf16, rmsw_bf16, oracle_mod):
     T, T64 = table_bf16
     g, g64 = rmsw_bf16
