@@ -227,6 +227,16 @@ const char *dmel_status_string(dmel_status status) {
 
 int dmel_last_launch_count(void) { return t_last_launches; }
 
+dmel_status dmel_debug_wait_timeout(uint32_t polls, uint32_t *h_bits) {
+  if (!h_bits || polls == 0) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int returned = 0;
+  if (run_wait_timeout_selftest(polls, d.err, &returned) != cudaSuccess || returned != 1) return DMEL_ERR_CUDA;
+  return dmel_get_device_error(h_bits, 1);
+}
+
 void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {
   emulate_codes_frame_host(frame1600, codes80, lhat80);
 }

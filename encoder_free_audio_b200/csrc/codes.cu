@@ -54,8 +54,8 @@ constexpr int kSmMelW = kSmTwA + 800 * 16;                 // float [kMelNnzMax]
 constexpr int kSmMelK = kSmMelW + kMelNnzMax * 4;          // short [kMelNnzMax]: bin of each weight
 constexpr int kSmMelB = kSmMelK + kMelNnzMax * 2;          // uchar [kMelNnzMax]: channel of each weight
 constexpr int kSmChunk = kSmMelB + kMelNnzMax;             // int [33]: chunk bounds per lane
-constexpr int kSmSegFirst = kSmChunk + 36 * 4;             // int [32]: first segment of each lane
-constexpr int kSmChanSeg = kSmSegFirst + 32 * 4;           // int [81]: segment range per channel
+constexpr int kSmSegFirst = kSmChunk + 36 * 4;             // int [33]: first segment of each lane
+constexpr int kSmChanSeg = kSmSegFirst + 36 * 4;           // int [81]: segment range per channel
 constexpr int kSmTables = (kSmChanSeg + 84 * 4 + 127) / 128 * 128;
 constexpr int kWarpBufBytes = 800 * 16;
 constexpr int kPartOffset = 3216;                          // mel partials (floats) after P[801]
@@ -71,7 +71,7 @@ __device__ float d_melw[kMelNnzMax];
 __device__ short d_melk[kMelNnzMax];
 __device__ unsigned char d_melb[kMelNnzMax];
 __device__ int d_chunk[33];
-__device__ int d_segfirst[32];
+__device__ int d_segfirst[33];
 __device__ int d_chanseg[81];
 
 struct Tables {
@@ -82,7 +82,7 @@ struct Tables {
   const short *melk;     // their bins
   const unsigned char *melb;  // their channels
   const int *chunk;      // lane l sums entries [chunk[l], chunk[l + 1])
-  const int *segfirst;   // first partial-sum slot of lane l
+  const int *segfirst;   // lane l owns the partial-sum slots [segfirst[l], segfirst[l + 1])
   const int *chanseg;    // channel b adds the partials [chanseg[b], chanseg[b + 1])
 };
 
@@ -266,16 +266,20 @@ __host__ __device__ inline void step_a_dft(int l, const Tables &T, double (&ar)[
 }
 
 // Step C1, unit u = 4 k1 + l0 (0..99): 8-point DFT over l1 of row k1, columns l0 + 4 l1, times
-// W_32^{l0 k2a}, written back to the same columns (output k2a in column l0 + 4 k2a).
-__host__ __device__ inline void step_c1(int u, const Tables &T, double2 *B) {
+// W_32^{l0 k2a}, written back to the same columns (output k2a in column l0 + 4 k2a). Units own
+// disjoint columns, so a lane loads two units before storing either (the loads overlap).
+__host__ __device__ inline void c1_load(int u, const double2 *B, double (&r)[8], double (&i)[8]) {
   const int k1 = u >> 2, l0 = u & 3;
-  double r[8], i[8];
 #pragma unroll
   for (int l1 = 0; l1 < 8; ++l1) {
     const double2 v = B[slot(k1, l0 + 4 * l1)];
     r[l1] = v.x;
     i[l1] = v.y;
   }
+}
+
+__host__ __device__ inline void c1_finish(int u, const Tables &T, double (&r)[8], double (&i)[8], double2 *B) {
+  const int k1 = u >> 2, l0 = u & 3;
   dft8(r, i);
 #pragma unroll
   for (int k2a = 0; k2a < 8; ++k2a) {
@@ -288,22 +292,49 @@ __host__ __device__ inline void step_c1(int u, const Tables &T, double2 *B) {
   }
 }
 
-// Step C2, unit u = 8 k1 + k2a (0..199): 4-point DFT over l0 of row k1, columns l0 + 4 k2a;
-// output k2b goes to column k2b + 4 k2a.
-__host__ __device__ inline void step_c2(int u, double2 *B) {
-  const int k1 = u >> 3, k2a = u & 7;
-  double2 x[4];
+// All C1 units of lane l: u = l, l + 32, l + 64 (and l + 96 for l < 4), two at a time.
+__host__ __device__ inline void step_c1_lane(int l, const Tables &T, double2 *B) {
 #pragma unroll
-  for (int l0 = 0; l0 < 4; ++l0) x[l0] = B[slot(k1, l0 + 4 * k2a)];
-  // X_k2b = sum_l0 x_l0 W_4^{l0 k2b}, W_4 = -i
-  const double s02r = x[0].x + x[2].x, s02i = x[0].y + x[2].y;
-  const double d02r = x[0].x - x[2].x, d02i = x[0].y - x[2].y;
-  const double s13r = x[1].x + x[3].x, s13i = x[1].y + x[3].y;
-  const double d13r = x[1].x - x[3].x, d13i = x[1].y - x[3].y;
-  B[slot(k1, 0 + 4 * k2a)] = make_double2(s02r + s13r, s02i + s13i);
-  B[slot(k1, 1 + 4 * k2a)] = make_double2(d02r + d13i, d02i - d13r);  // d02 - i d13
-  B[slot(k1, 2 + 4 * k2a)] = make_double2(s02r - s13r, s02i - s13i);
-  B[slot(k1, 3 + 4 * k2a)] = make_double2(d02r - d13i, d02i + d13r);  // d02 + i d13
+  for (int q = 0; q < 4; q += 2) {
+    const int u0 = l + 32 * q, u1 = l + 32 * (q + 1);
+    double r0[8], i0[8], r1[8], i1[8];
+    const bool has1 = u1 < 100;
+    c1_load(u0, B, r0, i0);
+    if (has1) c1_load(u1, B, r1, i1);
+    c1_finish(u0, T, r0, i0, B);
+    if (has1) c1_finish(u1, T, r1, i1, B);
+  }
+}
+
+// Step C2, unit u = 8 k1 + k2a (0..199): 4-point DFT over l0 of row k1, columns l0 + 4 k2a;
+// output k2b goes to column k2b + 4 k2a. A lane loads all its (up to 7) units first.
+__host__ __device__ inline void step_c2_lane(int l, double2 *B) {
+  double2 x[7][4];
+#pragma unroll
+  for (int q = 0; q < 7; ++q) {
+    const int u = l + 32 * q;
+    if (u < 200) {
+      const int k1 = u >> 3, k2a = u & 7;
+#pragma unroll
+      for (int l0 = 0; l0 < 4; ++l0) x[q][l0] = B[slot(k1, l0 + 4 * k2a)];
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 7; ++q) {
+    const int u = l + 32 * q;
+    if (u < 200) {
+      const int k1 = u >> 3, k2a = u & 7;
+      // X_k2b = sum_l0 x_l0 W_4^{l0 k2b}, W_4 = -i
+      const double s02r = x[q][0].x + x[q][2].x, s02i = x[q][0].y + x[q][2].y;
+      const double d02r = x[q][0].x - x[q][2].x, d02i = x[q][0].y - x[q][2].y;
+      const double s13r = x[q][1].x + x[q][3].x, s13i = x[q][1].y + x[q][3].y;
+      const double d13r = x[q][1].x - x[q][3].x, d13i = x[q][1].y - x[q][3].y;
+      B[slot(k1, 0 + 4 * k2a)] = make_double2(s02r + s13r, s02i + s13i);
+      B[slot(k1, 1 + 4 * k2a)] = make_double2(d02r + d13i, d02i - d13r);  // d02 - i d13
+      B[slot(k1, 2 + 4 * k2a)] = make_double2(s02r - s13r, s02i - s13i);
+      B[slot(k1, 3 + 4 * k2a)] = make_double2(d02r - d13i, d02i + d13r);  // d02 + i d13
+    }
+  }
 }
 
 // Step D, first half for lane l: pairs (k, 800 - k). Round r = 1..12 takes Z at row r, column
@@ -356,7 +387,8 @@ __host__ __device__ inline void step_d_store(int l, const Tables &T, const PairR
 }
 
 // Step E, first half for lane l: the entries [chunk[l], chunk[l + 1]) of the weight list,
-// summed per channel into the partial-sum slots segfirst[l], segfirst[l] + 1, ...
+// summed per channel into the partial-sum slots segfirst[l], segfirst[l] + 1, ... Every lane
+// walks the same number of entries (within one), so the loop does not diverge.
 __host__ __device__ inline void step_e_chunk(int l, const Tables &T, const float *P, float *part) {
   const int e0 = T.chunk[l], e1 = T.chunk[l + 1];
   int seg = T.segfirst[l];
@@ -399,7 +431,7 @@ struct HostTables {
   std::vector<float> melw;
   std::vector<short> melk;
   std::vector<unsigned char> melb;
-  int chunk[33], segfirst[32], chanseg[81];
+  int chunk[33], segfirst[33], chanseg[81];
   Tables view() const {
     return Tables{w.data(), hann2.data(), twa.data(), melw.data(), melk.data(), melb.data(), chunk, segfirst, chanseg};
   }
@@ -451,6 +483,7 @@ void build_host_tables(HostTables &H) {
     }
     ++seg;
   }
+  H.segfirst[32] = seg;
   H.chanseg[kMel] = seg;
 }
 
@@ -522,7 +555,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
       mb[i] = d_melb[i];
     }
     for (int i = threadIdx.x; i < 33; i += blockDim.x) ch[i] = d_chunk[i];
-    for (int i = threadIdx.x; i < 32; i += blockDim.x) sf[i] = d_segfirst[i];
+    for (int i = threadIdx.x; i < 33; i += blockDim.x) sf[i] = d_segfirst[i];
     for (int i = threadIdx.x; i < 81; i += blockDim.x) cs[i] = d_chanseg[i];
   }
   __syncthreads();
@@ -589,11 +622,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
       step_a_dft(lane, T, ar, ai, B);
     }
     __syncwarp();
-#pragma unroll 1
-    for (int u = lane; u < 100; u += 32) step_c1(u, T, B);
+    step_c1_lane(lane, T, B);
     __syncwarp();
-#pragma unroll 1
-    for (int u = lane; u < 200; u += 32) step_c2(u, B);
+    step_c2_lane(lane, B);
     __syncwarp();
     {
       PairRegs R;
@@ -686,8 +717,8 @@ void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *
   for (int l = 0; l < 32; ++l)
     step_a_dft(l, T, *reinterpret_cast<double(*)[25]>(&arb[25 * l]), *reinterpret_cast<double(*)[25]>(&aib[25 * l]),
                B.data());
-  for (int u = 0; u < 100; ++u) step_c1(u, T, B.data());
-  for (int u = 0; u < 200; ++u) step_c2(u, B.data());
+  for (int l = 0; l < 32; ++l) step_c1_lane(l, T, B.data());
+  for (int l = 0; l < 32; ++l) step_c2_lane(l, B.data());
   for (int l = 0; l < 32; ++l) step_d_load(l, B.data(), R[l]);
   for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<float *>(B.data()));
   for (int l = 0; l < 32; ++l) step_e_chunk(l, T, reinterpret_cast<const float *>(B.data()), part.data());

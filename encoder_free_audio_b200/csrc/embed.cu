@@ -1101,6 +1101,36 @@ cudaError_t noalloc_scratch(void **ptr) {
   return cudaSuccess;
 }
 
+// ---------------------------------------------------------------- bounded-wait self test
+
+// One thread waits on an mbarrier whose phase can never complete (count 2, one arrival) with
+// the given poll limit: the wait must give up, record DMEL_DEVERR_WAIT_TIMEOUT and return.
+__global__ void wait_timeout_kernel(uint32_t polls, uint32_t *err, int *returned) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_addr(&bar);
+  mbar_init(b, 2);
+  mbar_fence_init();
+  mbar_arrive(b);
+  bool done = false;
+  for (uint32_t i = 0; i < polls && !done; ++i) done = mbar_try_wait(b, 0);
+  if (!done) record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+  *returned = 1;
+}
+
+__device__ int g_selftest_returned;
+
+cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned) {
+  void *d = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&d, g_selftest_returned);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemset(d, 0, sizeof(int))) != cudaSuccess) return e;
+  wait_timeout_kernel<<<1, 1>>>(polls, err, static_cast<int *>(d));
+  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(h_returned, d, sizeof(int), cudaMemcpyDeviceToHost);
+  return e;
+}
+
 bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
   return table_dtype == DMEL_BF16 && embed_dim > 0 && embed_dim % tc::BN == 0;
 }

@@ -31,6 +31,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 // Device address of that scratch on the current device (looked up once per device).
 cudaError_t noalloc_scratch(void **ptr);
 
+// Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
+cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);
+
 void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
 
 }  // namespace dmel

@@ -71,6 +71,8 @@ def _lib():
         L.dmel_status_string.restype = ctypes.c_char_p
         L.dmel_last_launch_count.argtypes = []
         L.dmel_last_launch_count.restype = i32
+        L.dmel_debug_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32)]
+        L.dmel_debug_wait_timeout.restype = i32
         L.dmel_debug_codes_frame_host.argtypes = [vp, vp, vp]
         L.dmel_debug_codes_frame_host.restype = None
         _L = L
@@ -197,3 +199,11 @@ def dmel_debug_codes_frame_host(frame1600: np.ndarray):
     _lib().dmel_debug_codes_frame_host(fr.ctypes.data_as(ctypes.c_void_p), codes.ctypes.data_as(ctypes.c_void_p),
                                        lhat.ctypes.data_as(ctypes.c_void_p))
     return codes, lhat
+
+
+def dmel_debug_wait_timeout(polls: int = 1 << 16) -> int:
+    """Runs the bounded-wait self test (see dmel_debug.h); returns the device error bits."""
+    bits = ctypes.c_uint32(0)
+    rc = _lib().dmel_debug_wait_timeout(int(polls), ctypes.byref(bits))
+    _check(rc, "dmel_debug_wait_timeout")
+    return int(bits.value)

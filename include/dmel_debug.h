@@ -7,6 +7,8 @@
 
 #include <stdint.h>
 
+#include "dmel.h"
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -17,6 +19,13 @@ extern "C" {
  * (frame1600 = x[800 (t-1) .. 800 (t+1))). Writes 80 codes and, when lhat80 != NULL, the 80
  * clamped log10 mel energies. Lets the kernel's arithmetic be checked without a GPU. */
 void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
+
+/* Failure-detection self test: launches one thread that waits, with a limit of `polls`
+ * mbarrier polls, on a barrier phase that can never complete (two arrivals expected, one
+ * made). The wait must give up and the kernel return; the call synchronises, then reads and
+ * clears the device error word into *h_bits (DMEL_DEVERR_WAIT_TIMEOUT expected). Nothing
+ * faults or hangs: the context stays usable. */
+dmel_status dmel_debug_wait_timeout(uint32_t polls, uint32_t *h_bits);
 
 #ifdef __cplusplus
 }
