@@ -66,6 +66,25 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
   __stcs(reinterpret_cast<uint4 *>(p), u);
 }
 
+// 16 bytes of output values: 4 fp32 (x[0..3]) or 8 bf16 (x[0..7], round to nearest even).
+template <typename OT>
+__device__ __forceinline__ uint4 pack16(const float (&x)[8]);
+template <>
+__device__ __forceinline__ uint4 pack16<float>(const float (&x)[8]) {
+  return make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+}
+template <>
+__device__ __forceinline__ uint4 pack16<__nv_bfloat16>(const float (&x)[8]) {
+  return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                    pack_bf16x2(x[6], x[7]));
+}
+
+// Streaming (evict-first) 16-byte store.
+template <typename OT>
+__device__ __forceinline__ void st_stream16(OT *p, uint4 w) {
+  __stcs(reinterpret_cast<uint4 *>(p), w);
+}
+
 __device__ __forceinline__ void load8_out(const float *p, float (&v)[8]) {
   const float4 a = __ldcs(reinterpret_cast<const float4 *>(p));
   const float4 b = __ldcs(reinterpret_cast<const float4 *>(p) + 1);
@@ -824,6 +843,496 @@ __global__ void __launch_bounds__(tc2::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- 2:4-sparse one-hot product
+
+// Each bin's 16 one-hot columns hold a single 1, so every group of four consecutive table rows
+// has at most one non-zero in A: A is 2:4 sparse and tcgen05.mma.sp halves the tensor work.
+// Per bin and frame with level c: A keeps two values out of each group of four rows (group
+// c >> 2 keeps rows (0, 1) or (2, 3) of the group, whichever holds c; the other groups keep
+// (0, 1) with zeros), so the 16 logical columns become 8 stored bf16 (16 bytes) with the 1 at
+// position 2 (c >> 2) + (c & 1), and 16 bits of metadata (a nibble of two 2-bit row positions
+// per group). The metadata lives in TMEM, one 32-bit column per MMA (logical K = 32, two bins).
+// Tiles are 256 frames x 176 columns: two fp32 accumulators at TMEM columns 0 and 256 leave
+// columns 496..511 for a four-stage metadata ring. With RMSNorm, groups of ceil(D / 176)
+// clusters (35 at D = 6144, two groups on 148 SMs) own fixed column slices and walk the same
+// frame tiles together; each row's sum of squares
+// over a slice is published into a buffer pre-filled with a sentinel and the other slices'
+// sums are read as they appear (all clusters are co-resident under the cooperative launch).
+// An mbarrier wait in the thread that issues tcgen05.mma stalls that thread behind its queued
+// MMAs and leaves the tensor pipe idle for a few hundred cycles per wait, so a separate warp does
+// every wait and hands each stage to the MMA warp through named barriers, running up to three
+// stages ahead (a wait that times out is recorded and the waiter stops waiting but keeps
+// handing over stages, so the kernel finishes).
+// Each commit signals the barrier in both CTAs at once. Eight epilogue warps (two
+// per TMEM lane quarter, 96 columns each) stage their rows in shared memory and write whole
+// 64-byte (bf16) or 128-byte (fp32) row pieces, 8 or 4 rows per warp instruction.
+namespace sp {
+constexpr int BM = 128;                 // frames per CTA
+constexpr int BN = 192;                 // columns per pair tile
+constexpr int BNH = 96;                 // columns used from each CTA's half of the table block
+constexpr int BKL = 128;                // table rows (logical K) per stage: 8 bins
+constexpr int KBLOCKS = kRows / BKL;    // 10
+constexpr int STAGES_A = 3;             // A + metadata slots in TMEM
+constexpr int STAGES_B = 7;             // table blocks in shared memory
+constexpr int B_BOX_COLS = 32;          // 64-byte rows, 64-byte swizzle
+constexpr int B_BOXES = BNH / B_BOX_COLS;
+constexpr int B_BOX = B_BOX_COLS * BKL * 2;  // 32 columns x 128 rows: 8 KB
+constexpr int B_STAGE = B_BOXES * B_BOX;     // exactly the 96 columns used
+constexpr int OFF_B = 0;
+constexpr int OFF_BAR = OFF_B + STAGES_B * B_STAGE;
+constexpr int N_BARS = 2 * STAGES_A + 2 * STAGES_B + 5;
+constexpr int BN_EPI = BN;              // columns the epilogue walks
+constexpr int EPI_WARPS = 8;            // two per TMEM lane quarter
+constexpr int EPI_COLS = BN / 2;        // columns per epilogue warp
+constexpr int EPI_CHUNK = 32;           // columns staged at a time
+constexpr int OFF_G = OFF_BAR + 256;    // RMSNorm weights of the cluster's column slice
+constexpr int OFF_EPI = OFF_G + BN_EPI * 4;  // row sums [2][128] and scales [128]
+constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;  // staging: 8 warps x 32 rows x up to 128 bytes
+constexpr int SMEM_USED = OFF_STG + EPI_WARPS * 32 * 128;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+constexpr int WAITER_WARP = 6 + EPI_WARPS;  // warps: 0 TMA, 1 MMA, 2..5 A, 6..13 epilogue, 14 waits
+constexpr int THREADS = 32 * (WAITER_WARP + 1);
+// TMEM columns: accumulators [0, 192) and [256, 448); A slots (32 columns: 64 stored bf16 per
+// row) at 192, 224, 448; metadata slots (4 columns) at 480, 484, 488.
+constexpr uint32_t ACC_STRIDE = 256;
+__host__ __device__ constexpr uint32_t a_col(int s) { return s == 0 ? 192u : s == 1 ? 224u : 448u; }
+constexpr uint32_t META_COL = 480;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t kSentinel = 0xFFFFFFFFu;  // a NaN no arithmetic produces: "not yet published"
+static_assert(KBLOCKS * BKL == kRows, "stages cover the table");
+static_assert(BN % 64 == 0 && BN <= 192, "accumulator columns end where the A slots start");
+static_assert(STAGES_A == 3 && META_COL >= 448 + 32 && META_COL + 4 * STAGES_A <= TMEM_COLS, "TMEM map");
+static_assert(N_BARS * 8 + 16 <= 256, "barrier area");
+static_assert(B_BOXES * B_BOX_COLS == BNH && B_STAGE % 1024 == 0 && STAGES_B <= 32, "table stages");
+static_assert(OFF_STG % 128 == 0, "staging rows are 128-byte aligned");
+static_assert(EPI_COLS % EPI_CHUNK == 0 && EPI_CHUNK == 32, "epilogue slices");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+}  // namespace sp
+
+// Named barrier 1 over the sparse kernel's 8 epilogue warps; the _and form returns whether v held
+// in every thread. Named barrier 2 joins the waiter warp and the MMA warp once per stage.
+__device__ __forceinline__ void sp_epi_barrier() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ bool sp_epi_barrier_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
+}
+// Stage handoff between the waiter warp and the MMA warp: named barriers 2..4 ("stage j is
+// ready", waiter arrives, MMA warp syncs) and 5..7 ("stage j was issued", MMA warp arrives,
+// waiter syncs), j = stage mod 3. The waiter announces stage s + 3 only after the MMA warp
+// acknowledged stage s, so it runs at most three stages ahead and never arrives twice on a
+// barrier the MMA warp has not yet consumed.
+__device__ __forceinline__ void sp_ready_arrive(int j) { asm volatile("bar.arrive %0, 64;" ::"r"(2 + j) : "memory"); }
+__device__ __forceinline__ void sp_ready_sync(int j) { asm volatile("bar.sync %0, 64;" ::"r"(2 + j) : "memory"); }
+__device__ __forceinline__ void sp_issued_arrive(int j) { asm volatile("bar.arrive %0, 64;" ::"r"(5 + j) : "memory"); }
+__device__ __forceinline__ void sp_issued_sync(int j) { asm volatile("bar.sync %0, 64;" ::"r"(5 + j) : "memory"); }
+
+__device__ __forceinline__ void st_relaxed_f32(float *p, float v) {
+  asm volatile("st.relaxed.gpu.global.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const float *p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Number of column tiles of the sparse kernel (the last one may be partial).
+__host__ __device__ constexpr int sp_col_tiles(int D) { return (D + sp::BN - 1) / sp::BN; }
+
+// Tile i of this cluster: pair frame tile mp, column tile nt. Without RMSNorm the clusters walk
+// one global order (frame tile major); with it, groups of P clusters own fixed column slices
+// and walk the same frame tiles.
+template <int kMode>
+__device__ __forceinline__ bool sp_tile_at(int64_t i, int64_t n_pm, int P, int64_t &mp, int &nt) {
+  const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  if (kMode == kFused) {
+    mp = cid / P + i * (ncl / P);
+    nt = (int)(cid % P);
+    return mp < n_pm;
+  }
+  const int64_t t = cid + i * ncl;
+  mp = t / P;
+  nt = (int)(t % P);
+  return mp < n_pm;
+}
+
+// Metadata of one bin at level c: groups keep rows (0, 1) (nibble 0x4) except group c >> 2,
+// which keeps (2, 3) (nibble 0xE) when c & 3 is 2 or 3.
+__device__ __forceinline__ uint32_t sp_meta_field(uint32_t c) {
+  return 0x4444u | ((c & 2u) ? (0xAu << (4u * (c >> 2))) : 0u);
+}
+
+template <typename OT, int kMode>
+__global__ void __launch_bounds__(sp::THREADS, 1)
+    embed_sp_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
+                    OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                    const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
+  using namespace sp;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_a = [&](int s) { return bar0 + 8u * s; };
+  auto empty_a = [&](int s) { return bar0 + 8u * (STAGES_A + s); };
+  auto full_b = [&](int s) { return bar0 + 8u * (2 * STAGES_A + s); };
+  auto empty_b = [&](int s) { return bar0 + 8u * (2 * STAGES_A + STAGES_B + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * STAGES_A + 2 * STAGES_B + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * STAGES_A + 2 * STAGES_B + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES_A + 2 * STAGES_B + 4);
+  auto in_leader = [&](uint32_t local_bar) { return mapa_shared(local_bar, 0); };
+  auto in_peer = [&](uint32_t local_bar) { return mapa_shared(local_bar, 1); };
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+  float *gsm = reinterpret_cast<float *>(smem + OFF_G);
+
+  const int P = sp_col_tiles(D);
+  const int64_t n_m_tiles = (F + BM - 1) / BM;      // 128-frame tiles with at least one frame
+  const int64_t n_pm = (F + 2 * BM - 1) / (2 * BM);  // 256-frame pair tiles
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES_A; ++s) {
+      mbar_init(full_a(s), 8);  // 4 producer warps of each CTA (used in the even CTA)
+      mbar_init(empty_a(s), 1);
+    }
+    for (int s = 0; s < STAGES_B; ++s) {
+      mbar_init(full_b(s), 1);  // the leader's expect-tx for both halves
+      mbar_init(empty_b(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 2 * EPI_WARPS);  // epilogue warps of both CTAs (used in the even CTA)
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (kMode == kFused && threadIdx.x < BN_EPI) {
+    const int c = (int)((blockIdx.x >> 1) % P) * BN + threadIdx.x;
+    gsm[threadIdx.x] = c < D ? __bfloat162float(gw[c]) : 0.0f;
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmap);
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer: this CTA's half of the table block
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t pending = 0, pending_phase = 0;
+      bool ok = true;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+        const int n0 = nt * BN + (int)rank * BNH;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          if (!mbar_wait(empty_b(stage), phase ^ 1u, err)) { ok = false; break; }
+          const uint32_t fb = in_leader(full_b(stage));
+          if (leader) mbar_arrive_expect_tx(full_b(stage), 2 * B_STAGE);  // both CTAs' halves
+          const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int q = 0; q < B_BOXES; ++q)
+            tma_load_2d_pair(dst + q * B_BOX, &tmap, n0 + B_BOX_COLS * q, kb * BKL, fb, pol);
+          pending |= 1u << stage;
+          pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES_B) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (leader)
+        for (int s = 0; s < STAGES_B; ++s)
+          if (pending & (1u << s)) mbar_wait(full_b(s), (pending_phase >> s) & 1u, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA warp (even CTA only): lane 0 issues
+    // Stage by stage the waiter warp reports (named barrier 2) that the accumulator, A slot and
+    // table block are ready; this warp itself never waits on an mbarrier while MMAs are queued.
+    if (leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, 1) | kIdescSparse;
+      int sa = 0, sb = 0;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+        const uint32_t acc = i & 1;
+        const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
+        for (int kb = 0; kb < KBLOCKS; ++kb) {
+          sp_ready_sync(sa);  // A slot sa cycles with the stage index mod 3
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t b0 = smem_addr(smem + OFF_B + sb * B_STAGE);
+            const uint32_t a0 = tmem_base + a_col(sa);
+#pragma unroll
+            for (int k = 0; k < BKL / 32; ++k) {
+              // MN-major, 64-byte swizzle: atoms of 32 columns x 8 rows (512 bytes), boxes of 32
+              // columns B_BOX apart; 32 table rows (2048 bytes) per MMA
+              const uint64_t bdesc = smem_desc(b0 + 2048u * k, (uint32_t)B_BOX, 512u, kSwizzle64B);
+              const uint32_t mcol = META_COL + 4u * sa + k;
+              tc_mma_sp_pair_ts(d_tmem, a0 + 8u * k, bdesc, idesc | (mcol & 1u), tmem_base + (mcol & ~1u),
+                                (kb | k) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_both(empty_a(sa), 3);
+            tc_commit_pair_both(empty_b(sb), 3);
+            if (kb == KBLOCKS - 1) tc_commit_pair_both(tfull(acc), 3);
+          }
+          __syncwarp();
+          sp_issued_arrive(sa);
+          if (++sa == STAGES_A) sa = 0;
+          if (++sb == STAGES_B) sb = 0;
+        }
+      }
+      if (lane == 0) {
+        tc_commit_pair(done_bar);
+        mbar_wait(done_bar, 0, err);
+      }
+    }
+  } else if (warp == WAITER_WARP) {
+    // ------------------------------------------------ waits for the MMA warp (even CTA only)
+    if (leader) {
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0;
+      bool ok = true;  // after a timed-out wait: no more waiting, stages still handed over
+      int64_t n = 0;   // stages announced
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+        const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
+        for (int kb = 0; kb < KBLOCKS; ++kb, ++n) {
+          if (n >= STAGES_A) sp_issued_sync(sa);  // stage n - 3 (same slot) was issued
+          if (lane == 0 && ok) {
+            if (kb == 0) ok = mbar_wait(tempty(acc), acc_phase ^ 1u, err);
+            ok = ok && mbar_wait(full_a(sa), pa, err) && mbar_wait(full_b(sb), pb, err);
+          }
+          __syncwarp();
+          sp_ready_arrive(sa);
+          if (++sa == STAGES_A) { sa = 0; pa ^= 1u; }
+          if (++sb == STAGES_B) { sb = 0; pb ^= 1u; }
+        }
+      }
+      // consume the acknowledgements of the last stages (at most three), oldest first
+      for (int64_t q = n > STAGES_A ? n - STAGES_A : 0; q < n; ++q) sp_issued_sync((int)(q % STAGES_A));
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // ------------------------------------------------ compressed one-hot A + metadata into TMEM
+    // Warp w may only touch TMEM lanes 32 (w % 4) .. + 31, so it owns those rows (row r in lane r).
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    // Metadata lane order within the warp: lane t holds rows (t & 7) + 16 (t >> 4) (low half)
+    // and that + 8 (high half) of this warp's 32 rows, for bin (t >> 3) & 1 of the MMA's two.
+    const int src_lo = (lane & 7) + 16 * (lane >> 4);
+    const int src_hi = src_lo + 8;
+    const uint32_t half_shift = 16u * ((lane >> 3) & 1);
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    int64_t mp;
+    int nt;
+    // this row's codes, loaded one tile ahead so a tile boundary does not wait on L2
+    auto load_codes = [&](int64_t mp_, uint4 (&u)[5]) {
+      const int64_t f_ = (2 * mp_ + rank) * BM + r;
+      if (f_ < F) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(codes + f_ * kMel);
+#pragma unroll
+        for (int q = 0; q < 5; ++q) u[q] = __ldg(src + q);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 5; ++q) u[q] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    uint4 next[5];
+    if (sp_tile_at<kMode>(0, n_pm, P, mp, nt)) load_codes(mp, next);
+    for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      const int64_t f = (2 * mp + rank) * BM + r;
+      const bool valid = f < F;
+      uint32_t cw[20];
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        cw[4 * q] = next[q].x; cw[4 * q + 1] = next[q].y; cw[4 * q + 2] = next[q].z; cw[4 * q + 3] = next[q].w;
+      }
+      {
+        int64_t mp2;
+        int nt2;
+        if (sp_tile_at<kMode>(i + 1, n_pm, P, mp2, nt2)) load_codes(mp2, next);
+      }
+      if (valid) {
+        uint32_t bad = 0;
+#pragma unroll
+        for (int q = 0; q < 20; ++q) bad |= cw[q] & 0xF0F0F0F0u;
+        if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
+      }
+      const uint32_t one_mask = valid ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+      for (int kb = 0; kb < KBLOCKS; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(empty_a(stage), phase ^ 1u, err))) { ok = false; break; }
+        const uint32_t wlo = cw[2 * kb], whi = cw[2 * kb + 1];
+        // bin j of the stage: stored bf16 8j .. 8j + 7 = columns 4j .. 4j + 3, the 1 in column
+        // 4j + (c >> 2), low half when c is even
+        uint32_t av[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t c = ((j < 4 ? wlo : whi) >> (8 * (j & 3))) & 15u;
+          const uint32_t one = ((c & 1u) ? 0x3F800000u : 0x00003F80u) & one_mask;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) av[4 * j + g] = (c >> 2) == (uint32_t)g ? one : 0u;
+        }
+        tmem_st32(lane_base + a_col(stage), av);
+        uint32_t m[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w = k < 2 ? wlo : whi;
+          const uint32_t c0 = (w >> (16 * (k & 1))) & 15u, c1 = (w >> (16 * (k & 1) + 8)) & 15u;
+          const uint32_t pk = sp_meta_field(c0) | (sp_meta_field(c1) << 16);
+          const uint32_t lo = __shfl_sync(0xffffffffu, pk, src_lo), hi = __shfl_sync(0xffffffffu, pk, src_hi);
+          m[k] = ((lo >> half_shift) & 0xFFFFu) | (((hi >> half_shift) & 0xFFFFu) << 16);
+        }
+        tmem_st4(lane_base + META_COL + 4u * stage, m[0], m[1], m[2], m[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(in_leader(full_a(stage)));
+        if (++stage == STAGES_A) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp >= 6 && warp < 6 + EPI_WARPS) {
+    // ------------------------------------------------ epilogue: 32 rows x 96 columns per warp
+    const int quad = warp & 3;
+    const int half = (warp - 6) >> 2;  // columns [96 half, 96 half + 96) of the tile
+    const int r = quad * 32 + lane;
+    const int cb = half * EPI_COLS;
+    float *ssp = reinterpret_cast<float *>(smem + OFF_EPI);  // [2][128] row sums of the halves
+    float *scl = ssp + 2 * BM;                               // [128] row scales
+    // staging slab of this warp: 32 rows of NP 16-byte pieces (a 32-column chunk), pieces
+    // swizzled so both the row-wise writes and the piece-wise reads are free of bank conflicts
+    constexpr int NP = 2 * (int)sizeof(OT);  // 4 (bf16) or 8 (fp32)
+    constexpr int RB = 16 * NP;
+    uint8_t *slab = smem + OFF_STG + (warp - 6) * 32 * 128;
+    auto piece = [](int q, int j) {
+      return NP == 8 ? (j ^ (q & 7)) : (j ^ ((q >> 1) & 3));
+    };
+    bool ok = true;
+    int64_t mp;
+    int nt;
+    for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
+      if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
+      tc_fence_after();
+      const int64_t m = 2 * mp + rank;
+      const bool live = m < n_m_tiles;  // uniform over the CTA: the pair's second half may hold no frame
+      const int n0 = nt * BN;
+      const int ncols = D - n0 < BN ? D - n0 : BN;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + cb;
+      float scale = 1.0f;
+      if (kMode == kFused && live) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int c = 0; c < EPI_COLS; c += 32) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tbase + c, v0);
+          tmem_ld16(tbase + c + 16, v1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float a = __uint_as_float(v0[q]), b = __uint_as_float(v1[q]);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+          }
+        }
+        ssp[half * BM + r] = ss;
+        sp_epi_barrier();
+        if (half == 0) {
+          // columns past D are zero in the accumulator (the table loads fill them with zeros)
+          st_relaxed_f32(partials + (m * P + nt) * BM + r, ssp[r] + ssp[BM + r]);
+          // the other slices' sums: 32 independent loads per sweep (one L2 round trip), swept
+          // again until none is the sentinel; added in slice order
+          const float *col = partials + m * P * BM + r;
+          float tot = 0.0f;
+          uint32_t polls = 0;
+          for (int q0 = 0; q0 < P; q0 += 32) {
+            uint32_t u[32];
+            for (;;) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) u[j] = q0 + j < P ? ld_relaxed_u32(col + (q0 + j) * BM) : 0u;
+              bool ready = true;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ready &= u[j] != kSentinel;
+              if (ready) break;
+              if (++polls > kMaxPolls) {
+                record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) u[j] = u[j] == kSentinel ? 0u : u[j];
+                break;
+              }
+              __nanosleep(32);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) tot += __uint_as_float(u[j]);
+          }
+          scl[r] = 1.0f / sqrtf(tot / (float)D + eps);
+        }
+        sp_epi_barrier();
+        scale = scl[r];
+      }
+      if (live) {
+        // rows of this warp: frames m * BM + 32 quad + q, q = 0..31
+        const int64_t f_warp = m * BM + quad * 32;
+#pragma unroll 1
+        for (int c0 = cb; c0 < cb + EPI_COLS && c0 < ncols; c0 += EPI_CHUNK) {
+          uint32_t v[2][16];
+          tmem_ld16(tbase + (c0 - cb), v[0]);
+          tmem_ld16(tbase + (c0 - cb) + 16, v[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < NP; ++h) {  // 16-byte piece h of this thread's row
+            constexpr int E = 16 / (int)sizeof(OT);
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+              const int cc = h * E + e;
+              x[e] = __uint_as_float(v[cc >> 4][cc & 15]);
+              if (kMode == kFused) x[e] = gsm[c0 + cc] * (x[e] * scale);
+            }
+            *reinterpret_cast<uint4 *>(slab + lane * RB + (piece(lane, h) << 4)) = pack16<OT>(x);
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < NP; ++it) {  // 32 / NP rows per instruction
+            const int q = it * (32 / NP) + lane / NP, j = lane % NP;
+            const uint4 w = *reinterpret_cast<const uint4 *>(slab + q * RB + (piece(q, j) << 4));
+            const int col = c0 + j * (16 / (int)sizeof(OT));
+            if (f_warp + q < F && col < ncols)
+              st_stream16(out + (f_warp + q) * (int64_t)D + n0 + col, w);
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(in_leader(tempty(acc)));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();  // every MMA into either CTA's TMEM has completed (the leader waited above)
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -854,15 +1363,18 @@ cudaError_t set_smem_attr_once(K kernel, int bytes, bool *flags) {
   return e;
 }
 
-bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D) {
+// Tensor map of the bf16 table [1280 x D]: boxes of box_cols columns x box_rows rows, with the
+// swizzle whose span is one box row (64 columns: 128 bytes; 32 columns: 64 bytes).
+bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D, int box_rows = tc::BK, int box_cols = 64) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)kRows};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)tc::BK};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(table), dims, strides, box,
-                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -876,17 +1388,23 @@ struct TcScratch {
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
+// Partial sums are laid out [frame tile][column tile][128]; the sparse kernel's 240-column tiles
+// are the most numerous, so the region is sized for them and the 256-column kernels use a prefix.
+size_t tc_partials_bytes(int64_t F, int D) {
+  const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
+  return round256(m_tiles * (size_t)sp_col_tiles(D) * tc::BM * sizeof(float));
+}
+
 size_t tc_scratch_bytes(int64_t F, int D) {
   const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
-  return round256(m_tiles * (size_t)(D / tc::BN) * tc::BM * sizeof(float)) + round256(m_tiles * sizeof(int));
+  return tc_partials_bytes(F, D) + round256(m_tiles * sizeof(int));
 }
 
 TcScratch tc_scratch(void *ws, int64_t F, int D) {
-  const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
   uint8_t *p = static_cast<uint8_t *>(ws);
   TcScratch s;
   s.partials = reinterpret_cast<float *>(p);
-  s.counters = reinterpret_cast<int *>(p + round256(m_tiles * (size_t)(D / tc::BN) * tc::BM * sizeof(float)));
+  s.counters = reinterpret_cast<int *>(p + tc_partials_bytes(F, D));
   return s;
 }
 
@@ -995,6 +1513,48 @@ cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tab
                             err);
 }
 
+// Sparse CTA-pair launch; same contract as launch_tc2. With RMSNorm every cluster must be
+// resident (tiles of one frame tile wait for each other).
+template <typename OT, int kMode>
+cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+                      const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
+  static bool attr[256] = {false};
+  cudaError_t e = set_smem_attr_once(embed_sp_kernel<OT, kMode>, sp::SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  CUtensorMap tmap;
+  if (!make_table_map(&tmap, table, D, sp::BKL, sp::B_BOX_COLS)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(sp::THREADS);
+  cfg.dynamicSmemBytes = sp::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeCooperative;
+  at[1].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int resident = 0;
+  if (cudaOccupancyMaxActiveClusters(&resident, embed_sp_kernel<OT, kMode>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
+  }
+  if (kMode == kFused) {
+    if (resident < clusters) return cudaErrorNotSupported;
+    cfg.numAttrs = cooperative_enabled() ? 2 : 1;
+    const int64_t m_tiles = (F + sp::BM - 1) / sp::BM;
+    const size_t bytes = (size_t)m_tiles * sp_col_tiles(D) * sp::BM * sizeof(float);
+    if ((e = cudaMemsetAsync(sc.partials, 0xFF, bytes, stream)) != cudaSuccess) return e;  // all sentinel
+  } else if (resident < 1) {
+    return cudaErrorNotSupported;
+  }
+  return cudaLaunchKernelEx(&cfg, embed_sp_kernel<OT, kMode>, tmap, codes, F, D, out, sc.partials, sc.counters, g, eps,
+                            err);
+}
+
 // Fused kernels are launched cooperatively, which guarantees that every block of a group is
 // resident while the group exchanges row sums. DMEL_COOPERATIVE=0 (read once per process)
 // launches the same kernel and grid without that attribute, which profilers that cannot replay
@@ -1018,6 +1578,16 @@ bool pairs_enabled() {
   return on;
 }
 
+// The 2:4-sparse product unless the environment sets DMEL_EMBED_MMA=dense (read once per
+// process; for comparisons and tests).
+bool sparse_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("DMEL_EMBED_MMA");
+    return !(v && strcmp(v, "dense") == 0);
+  }();
+  return on;
+}
+
 // Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
 // partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel. CTA pairs
 // first; one-CTA tiles when pairs are switched off or cannot launch.
@@ -1032,6 +1602,18 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
   const int plain_clusters = (int)(pair_tiles < max_clusters ? pair_tiles : max_clusters);
   const TcScratch sc = g ? tc_scratch(workspace, F, D) : TcScratch{nullptr, nullptr};
   cudaError_t e;
+  const int Psp = sp_col_tiles(D);
+  if (pairs_enabled() && sparse_enabled() && max_clusters >= Psp) {
+    const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
+    const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
+    e = g ? launch_sp<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, (max_clusters / Psp) * Psp, stream)
+          : launch_sp<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, sp_clusters, stream);
+    if (e == cudaSuccess) {
+      ++*launches;
+      return e;
+    }
+    (void)cudaGetLastError();  // sparse pairs refused: dense kernels below
+  }
   if (!g) {
     if (pairs_enabled()) {
       e = launch_tc2<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, plain_clusters, stream);

@@ -138,8 +138,9 @@ def test_embed_tensor_core_model_dim(out_dt, rms, table_bf16, rmsw_bf16, oracle_
 
 @pytest.mark.parametrize("dim", [256, 768, 2048])
 def test_embed_tensor_core_rmsnorm_widths(dim, oracle_mod):
-    """Fused RMSNorm with groups of dim / 256 column tiles (1, 3 and 8 blocks per group) and a
-    ragged last frame tile."""
+    """Fused RMSNorm where a frame tile's row sums come from several column tiles (sparse
+    kernel: 192-column tiles, so 256 = 192 + 64, 768 = 4 x 192, 2048 = 10 x 192 + 128, partial
+    last tiles included; dense kernels: 1, 3 and 8 tiles of 256) and a ragged last frame tile."""
     T, T64 = bf16_table(synth.table(seed=12, dim=dim))
     gw = torch.from_numpy(synth.rms_weight(seed=13, dim=dim)).to(torch.bfloat16)
     F = 700

@@ -1,6 +1,7 @@
-"""The one-CTA tensor-core tiles (DMEL_EMBED_TILE=single) against the oracle: the embedding
-parity tests run again in a fresh process with CTA pairs switched off, so both tile shapes of
-the tcgen05 kernel stay covered."""
+"""The other tensor-core kernels against the oracle: the embedding parity tests run again in a
+fresh process with the 2:4-sparse product switched off (DMEL_EMBED_MMA=dense: dense CTA-pair
+tiles) and with CTA pairs switched off (DMEL_EMBED_TILE=single: dense one-CTA tiles), so every
+tile shape of the tcgen05 path stays covered."""
 import os
 import subprocess
 import sys
@@ -12,9 +13,17 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_embedding_parity_with_single_cta_tiles():
-    env = dict(os.environ, DMEL_EMBED_TILE="single")
+def _run_embed_parity(**env_overrides):
+    env = dict(os.environ, **env_overrides)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_parity_gpu.py"), "-k", "embed or batch64"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+def test_embedding_parity_with_dense_pair_tiles():
+    _run_embed_parity(DMEL_EMBED_MMA="dense")
+
+
+def test_embedding_parity_with_single_cta_tiles():
+    _run_embed_parity(DMEL_EMBED_TILE="single")
