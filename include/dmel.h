@@ -25,10 +25,11 @@
  *   - n_clips == 0 or n_frames == 0 is a valid call that does nothing.
  *   - No entry point allocates device memory. Scratch space comes from the caller's workspace;
  *     dmel_workspace_size() says how much.
- *   - Environment (read once per process): DMEL_EMBED_TILE=single runs the tensor-core
- *     embedding on one-CTA tiles instead of CTA pairs; DMEL_COOPERATIVE=0 launches the fused
+ *   - Environment (read once per process): DMEL_EMBED_MMA=dense runs the tensor-core embedding
+ *     as a dense one-hot product instead of the 2:4-sparse one; DMEL_EMBED_TILE=single runs it
+ *     dense on one-CTA tiles instead of CTA pairs; DMEL_COOPERATIVE=0 launches the fused
  *     RMSNorm kernels without the cooperative attribute (for profilers that cannot replay
- *     cooperative cluster launches). Both exist for comparison and measurement.
+ *     cooperative cluster launches). All exist for comparison and measurement.
  */
 #ifndef DMEL_H
 #define DMEL_H
@@ -144,7 +145,7 @@ dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table
  *
  * Limit: with rms_weight != NULL and a bf16 table whose embed_dim is a multiple of 256, the
  * request needs the scratch dmel_workspace_size(n_frames, embed_dim, DMEL_BF16, 1, 1) reports,
- * about n_frames * (embed_dim / 256) * 4 bytes (up to 43,648 frames at embed_dim 6144); a
+ * about n_frames * ceil(embed_dim / 192) * 4 bytes (up to 32,640 frames at embed_dim 6144); a
  * larger request returns DMEL_ERR_TOO_LARGE and launches nothing. Other requests need no
  * scratch and have no extra limit.
  *

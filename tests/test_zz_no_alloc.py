@@ -57,7 +57,15 @@ def test_noalloc_matches_workspace_entry_point_twice(lib):
 def test_noalloc_rejects_requests_beyond_its_scratch(lib):
     T = torch.zeros((1280, 6144), dtype=torch.bfloat16, device=DEV)
     g = torch.ones(6144, dtype=torch.bfloat16, device=DEV)
-    F = (4 << 20) // (24 * 4) + 1  # one frame more than 4 MiB of partial sums holds
+    # the smallest frame count whose scratch (what dmel_workspace_size reports) exceeds 4 MiB
+    F = 1
+    while dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True) <= (4 << 20):
+        F *= 2
+    lo, hi = F // 2, F
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if dmel.dmel_workspace_size(mid, 6144, dmel.DMEL_BF16, True, True) <= (4 << 20) else (lo, mid)
+    F = hi
     codes = torch.zeros((F, 80), dtype=torch.uint8, device=DEV)
     out = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
     assert _call_noalloc(lib, codes, T, out, g) == dmel.DMEL_ERR_TOO_LARGE
