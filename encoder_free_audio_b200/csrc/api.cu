@@ -127,13 +127,16 @@ dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const in
   return from_cuda(e);
 }
 
-dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
-                       const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
-                       size_t workspace_bytes, dmel_stream_t stream) {
+dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                            int embed_dim, const void *rms_weight, float eps, void *out, const int64_t *out_rows,
+                            int64_t out_n_rows, dmel_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                            dmel_stream_t stream) {
   t_last_launches = 0;
   dmel_status st =
       check_embed_args(codes, true, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype);
-  if (st != DMEL_OK || n_frames == 0) return st;
+  if (st != DMEL_OK) return st;
+  if (out_rows && (out_n_rows <= 0 || !aligned(out_rows, 8))) return DMEL_ERR_INVALID_ARG;
+  if (n_frames == 0) return DMEL_OK;
   const size_t need = embed_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DMEL_ERR_INVALID_ARG;
   DeviceInfo d;
@@ -141,18 +144,27 @@ dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table
   if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
   int launches = 0;
   cudaError_t e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype,
-                               workspace, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+                               workspace, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches, out_rows,
+                               out_n_rows);
   t_last_launches = launches;
   return from_cuda(e);
 }
 
-dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
-                         int64_t n_frames, const float *tails, float *tails_out, const void *table,
-                         dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
-                         dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
-                         dmel_stream_t stream) {
+dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
+                       const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
+                       size_t workspace_bytes, dmel_stream_t stream) {
+  return dmel_embed_rows(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, nullptr, 0, out_dtype,
+                         workspace, workspace_bytes, stream);
+}
+
+dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                              int n_clips, int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                              const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, uint8_t *codes_out,
+                              void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
   t_last_launches = 0;
   if (n_clips < 0 || n_frames < 0 || (n_clips == 0 && n_frames > 0)) return DMEL_ERR_INVALID_ARG;
+  if (out_rows && (out_n_rows <= 0 || !aligned(out_rows, 8))) return DMEL_ERR_INVALID_ARG;
   if (!sample_offsets && n_clips > 0) return DMEL_ERR_INVALID_ARG;
   if (!frame_offsets && n_clips > 0) return DMEL_ERR_INVALID_ARG;
   if (n_frames > 0 && !wav) return DMEL_ERR_INVALID_ARG;
@@ -177,9 +189,49 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                                d.sms, s, &launches);
   if (e == cudaSuccess)
     e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype, ws, d.err, d.sms,
-                     s, &launches);
+                     s, &launches, out_rows, out_n_rows);
   t_last_launches = launches;
   return from_cuda(e);
+}
+
+dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                         int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                         dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                         dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
+                         dmel_stream_t stream) {
+  return dmel_forward_rows(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, table, table_dtype,
+                           embed_dim, rms_weight, eps, out, nullptr, 0, out_dtype, codes_out, workspace,
+                           workspace_bytes, stream);
+}
+
+dmel_status dmel_splice_plan(const int64_t *h_sentinel_pos, int n_items, const int64_t *h_frame_offsets,
+                             int64_t seq_len, int64_t *h_token_pos, int64_t *h_frame_rows,
+                             int64_t *h_expanded_len, int64_t *h_audio_tokens) {
+  if (seq_len < 0 || n_items < 0 || !h_frame_offsets || (n_items > 0 && !h_sentinel_pos)) return DMEL_ERR_INVALID_ARG;
+  if (h_frame_offsets[0] != 0) return DMEL_ERR_INVALID_ARG;
+  for (int i = 0; i < n_items; ++i) {
+    if (h_sentinel_pos[i] < 0 || h_sentinel_pos[i] >= seq_len) return DMEL_ERR_INVALID_ARG;
+    if (i > 0 && h_sentinel_pos[i] <= h_sentinel_pos[i - 1]) return DMEL_ERR_INVALID_ARG;
+    if (h_frame_offsets[i + 1] < h_frame_offsets[i]) return DMEL_ERR_INVALID_ARG;
+  }
+  // walk the original positions once; shift = positions gained so far (sum of f_i - 1)
+  int64_t shift = 0;
+  int item = 0;
+  for (int64_t p = 0; p < seq_len; ++p) {
+    if (item < n_items && p == h_sentinel_pos[item]) {
+      const int64_t f0 = h_frame_offsets[item], f = h_frame_offsets[item + 1] - f0;
+      if (h_token_pos) h_token_pos[p] = -1;
+      if (h_frame_rows)
+        for (int64_t j = 0; j < f; ++j) h_frame_rows[f0 + j] = p + shift + j;
+      shift += f - 1;
+      ++item;
+    } else if (h_token_pos) {
+      h_token_pos[p] = p + shift;
+    }
+  }
+  if (h_expanded_len) *h_expanded_len = seq_len + shift;
+  if (h_audio_tokens) *h_audio_tokens = h_frame_offsets[n_items];
+  return DMEL_OK;
 }
 
 dmel_status dmel_embed_noalloc(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,

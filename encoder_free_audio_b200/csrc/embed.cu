@@ -101,6 +101,26 @@ __device__ __forceinline__ void load8_out(const __nv_bfloat16 *p, float (&v)[8])
   }
 }
 
+// ---------------------------------------------------------------- output rows
+
+// Where frame f's vector goes: row f of out, or row rows[f] of an out with n_rows rows (the
+// decoder's input sequence, frames spliced at their sentinels' expanded positions). A row
+// outside [0, n_rows) is not written and is recorded as DMEL_DEVERR_OUT_ROW.
+struct OutMap {
+  const int64_t *rows;
+  int64_t n_rows;
+};
+
+__device__ __forceinline__ int64_t map_row(const OutMap &om, int64_t f, uint32_t *err) {
+  if (!om.rows) return f;
+  const int64_t r = __ldg(om.rows + f);
+  if (r < 0 || r >= om.n_rows) {
+    if (err) record_error(err, DMEL_DEVERR_OUT_ROW);
+    return -1;
+  }
+  return r;
+}
+
 // ---------------------------------------------------------------- CUDA-core path
 
 constexpr int kSimtThreads = 256;
@@ -110,7 +130,7 @@ template <typename TT, typename OT>
 __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t *__restrict__ codes, int64_t F,
                                                                   const TT *__restrict__ table, int D,
                                                                   const TT *__restrict__ g, float eps,
-                                                                  OT *__restrict__ out, uint32_t *err) {
+                                                                  OT *__restrict__ out, OutMap om, uint32_t *err) {
   extern __shared__ __align__(16) float xs[];  // [D] when RMSNorm is on
   __shared__ int rows[kMel];
   __shared__ float red[kSimtThreads / 32];
@@ -124,6 +144,7 @@ __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t 
       }
       rows[threadIdx.x] = kLev * threadIdx.x + c;
     }
+    const int64_t orow = map_row(om, f, threadIdx.x == 0 ? err : nullptr);
     __syncthreads();
     float ss = 0.0f;
     for (int v = threadIdx.x; v < nv; v += kSimtThreads) {
@@ -140,8 +161,8 @@ __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t 
           xs[8 * v + i] = acc[i];
           ss += acc[i] * acc[i];
         }
-      } else {
-        store8(out + f * D + 8 * v, acc);
+      } else if (orow >= 0) {
+        store8(out + orow * D + 8 * v, acc);
       }
     }
     if (g) {
@@ -158,7 +179,7 @@ __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t 
         load8(g + 8 * v, gv);
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = gv[i] * (xs[8 * v + i] * inv);
-        store8(out + f * D + 8 * v, y);
+        if (orow >= 0) store8(out + orow * D + 8 * v, y);
       }
     }
     __syncthreads();
@@ -171,7 +192,7 @@ __global__ void __launch_bounds__(kSimtThreads) embed_simt_kernel(const uint8_t 
 // out_j <- g_j * (out_j / sqrt(ss / D + eps)) in place.
 constexpr int tc_bm = 128;  // frames per tile of the tensor-core kernel (partials layout)
 template <typename OT>
-__global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, int64_t F, int D,
+__global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, OutMap om, int64_t F, int D,
                                                           const __nv_bfloat16 *__restrict__ g,
                                                           const float *__restrict__ partials, int n_ct, float eps) {
   const int lane = threadIdx.x & 31;
@@ -183,7 +204,9 @@ __global__ void __launch_bounds__(256) rms_rescale_kernel(OT *__restrict__ out, 
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.0f / sqrtf(ss / (float)D + eps);
-    OT *row = out + f * D;
+    const int64_t orow = map_row(om, f, nullptr);  // the embedding kernel recorded bad rows
+    if (orow < 0) continue;
+    OT *row = out + orow * D;
     for (int v = lane; v < D / 8; v += 32) {
       float x[8], gv[8], y[8];
       load8_out(row + 8 * v, x);
@@ -268,7 +291,7 @@ __device__ __forceinline__ bool tile_at(int64_t i, int64_t n_m_tiles, int P, int
 template <typename OT, int kMode>
 __global__ void __launch_bounds__(tc::THREADS, 1)
     embed_tc_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
-                    OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                    OT *__restrict__ out, OutMap om, float *__restrict__ partials, int *__restrict__ counters,
                     const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -445,7 +468,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
       tc_fence_after();
       const int64_t f = m * BM + r;
       const bool valid = f < F;
-      OT *orow = out + (valid ? f : 0) * (int64_t)D + nt * BN;
+      const int64_t row = valid ? map_row(om, f, err) : -1;
+      OT *orow = out + (row >= 0 ? row : 0) * (int64_t)D + nt * BN;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
       float scale = 1.0f;
       if (kMode != kPlain) {
@@ -498,7 +522,7 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
         tmem_ld16(tbase + c * 32, v0);
         tmem_ld16(tbase + c * 32 + 16, v1);
         tmem_wait_ld();
-        if (valid) {
+        if (row >= 0) {
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             float x[8];
@@ -576,7 +600,7 @@ __device__ __forceinline__ bool pair_tile_at(int64_t i, int64_t n_pm, int P, int
 template <typename OT, int kMode>
 __global__ void __launch_bounds__(tc2::THREADS, 1)
     embed_tc2_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
-                     OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                     OT *__restrict__ out, OutMap om, float *__restrict__ partials, int *__restrict__ counters,
                      const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -763,7 +787,8 @@ __global__ void __launch_bounds__(tc2::THREADS, 1)
       const int64_t f = m * BM + r;
       const bool valid = f < F;
       const bool live = m < n_m_tiles;  // the pair's second half may hold no frame at all
-      OT *orow = out + (valid ? f : 0) * (int64_t)D + nt * BN;
+      const int64_t row = valid ? map_row(om, f, err) : -1;
+      OT *orow = out + (row >= 0 ? row : 0) * (int64_t)D + nt * BN;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN;
       float scale = 1.0f;
       if (kMode != kPlain && live) {
@@ -814,7 +839,7 @@ __global__ void __launch_bounds__(tc2::THREADS, 1)
           tmem_ld16(tbase + c * 32, v0);
           tmem_ld16(tbase + c * 32 + 16, v1);
           tmem_wait_ld();
-          if (valid) {
+          if (row >= 0) {
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
               float x[8];
@@ -972,7 +997,7 @@ __device__ __forceinline__ uint32_t sp_meta_field(uint32_t c) {
 template <typename OT, int kMode>
 __global__ void __launch_bounds__(sp::THREADS, 1)
     embed_sp_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
-                    OT *__restrict__ out, float *__restrict__ partials, int *__restrict__ counters,
+                    OT *__restrict__ out, OutMap om, float *__restrict__ partials, int *__restrict__ counters,
                     const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace sp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1287,8 +1312,10 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         scale = scl[r];
       }
       if (live) {
-        // rows of this warp: frames m * BM + 32 quad + q, q = 0..31
+        // rows of this warp: frames m * BM + 32 quad + q, q = 0..31; lane q holds row q's
+        // destination (-1: no frame or not written)
         const int64_t f_warp = m * BM + quad * 32;
+        const int64_t my_row = f_warp + lane < F ? map_row(om, f_warp + lane, half == 0 ? err : nullptr) : -1;
 #pragma unroll 1
         for (int c0 = cb; c0 < cb + EPI_COLS && c0 < ncols; c0 += EPI_CHUNK) {
           uint32_t v[2][16];
@@ -1313,8 +1340,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
             const int q = it * (32 / NP) + lane / NP, j = lane % NP;
             const uint4 w = *reinterpret_cast<const uint4 *>(slab + q * RB + (piece(q, j) << 4));
             const int col = c0 + j * (16 / (int)sizeof(OT));
-            if (f_warp + q < F && col < ncols)
-              st_stream16(out + (f_warp + q) * (int64_t)D + n0 + col, w);
+            const int64_t rq = om.rows ? __shfl_sync(0xffffffffu, my_row, q) : (f_warp + q < F ? f_warp + q : -1);
+            if (rq >= 0 && col < ncols) st_stream16(out + rq * (int64_t)D + n0 + col, w);
           }
           __syncwarp();
         }
@@ -1427,7 +1454,7 @@ bool fused_possible(int D, int num_sms, int *grid) {
 bool cooperative_enabled();
 
 template <typename OT, int kMode>
-cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                       const __nv_bfloat16 *g, float eps, uint32_t *err, int grid, cudaStream_t stream) {
   static bool attr[256] = {false};
   cudaError_t e = set_smem_attr_once(embed_tc_kernel<OT, kMode>, tc::SMEM_BYTES, attr);
@@ -1438,44 +1465,44 @@ cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
     const int64_t m_tiles = (F + tc::BM - 1) / tc::BM;
     if ((e = cudaMemsetAsync(sc.counters, 0, (size_t)m_tiles * sizeof(int), stream)) != cudaSuccess) return e;
     if (cooperative_enabled()) {
-      void *args[] = {&tmap, (void *)&codes, (void *)&F, (void *)&D, (void *)&out, (void *)&sc.partials,
+      void *args[] = {&tmap, (void *)&codes, (void *)&F, (void *)&D, (void *)&out, (void *)&om, (void *)&sc.partials,
                       (void *)&sc.counters, (void *)&g, (void *)&eps, (void *)&err};
       return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(embed_tc_kernel<OT, kMode>), dim3(grid),
                                          dim3(tc::THREADS), args, tc::SMEM_BYTES, stream);
     }
   }
-  embed_tc_kernel<OT, kMode><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, sc.partials,
-                                                                             sc.counters, g, eps, err);
+  embed_tc_kernel<OT, kMode><<<grid, tc::THREADS, tc::SMEM_BYTES, stream>>>(tmap, codes, F, D, out, om,
+                                                                             sc.partials, sc.counters, g, eps, err);
   return cudaGetLastError();
 }
 
 template <typename TT, typename OT>
 cudaError_t launch_simt(const uint8_t *codes, int64_t F, const TT *table, int D, const TT *g, float eps, OT *out,
-                        uint32_t *err, int num_sms, cudaStream_t stream) {
+                        OutMap om, uint32_t *err, int num_sms, cudaStream_t stream) {
   const int smem = g ? D * (int)sizeof(float) : 0;
   static bool attr[256] = {false};
   cudaError_t e = set_smem_attr_once(embed_simt_kernel<TT, OT>, kSimtMaxDim * (int)sizeof(float), attr);
   if (e != cudaSuccess) return e;
   const int64_t cap = (int64_t)num_sms * 8;
   const int grid = (int)(F < cap ? F : cap);
-  embed_simt_kernel<TT, OT><<<grid, kSimtThreads, smem, stream>>>(codes, F, table, D, g, eps, out, err);
+  embed_simt_kernel<TT, OT><<<grid, kSimtThreads, smem, stream>>>(codes, F, table, D, g, eps, out, om, err);
   return cudaGetLastError();
 }
 
 template <typename OT>
-cudaError_t launch_rescale(OT *out, int64_t F, int D, const __nv_bfloat16 *g, const float *partials, float eps,
-                           int num_sms, cudaStream_t stream) {
+cudaError_t launch_rescale(OT *out, OutMap om, int64_t F, int D, const __nv_bfloat16 *g, const float *partials,
+                           float eps, int num_sms, cudaStream_t stream) {
   const int64_t blocks_needed = (F + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 8;
   const int grid = (int)(blocks_needed < cap ? blocks_needed : cap);
-  rms_rescale_kernel<OT><<<grid, 256, 0, stream>>>(out, F, D, g, partials, D / tc::BN, eps);
+  rms_rescale_kernel<OT><<<grid, 256, 0, stream>>>(out, om, F, D, g, partials, D / tc::BN, eps);
   return cudaGetLastError();
 }
 
 // CTA-pair launch (clusters of 2); cooperative when the fused schedule needs every group
 // co-resident. Returns cudaErrorNotSupported when the pairs cannot all be resident at once.
 template <typename OT, int kMode>
-cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                        const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
   static bool attr[256] = {false};
   cudaError_t e = set_smem_attr_once(embed_tc2_kernel<OT, kMode>, tc2::SMEM_BYTES, attr);
@@ -1509,14 +1536,14 @@ cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tab
   } else if (resident < 1) {
     return cudaErrorNotSupported;
   }
-  return cudaLaunchKernelEx(&cfg, embed_tc2_kernel<OT, kMode>, tmap, codes, F, D, out, sc.partials, sc.counters, g, eps,
+  return cudaLaunchKernelEx(&cfg, embed_tc2_kernel<OT, kMode>, tmap, codes, F, D, out, om, sc.partials, sc.counters, g, eps,
                             err);
 }
 
 // Sparse CTA-pair launch; same contract as launch_tc2. With RMSNorm every cluster must be
 // resident (tiles of one frame tile wait for each other).
 template <typename OT, int kMode>
-cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, TcScratch sc,
+cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                       const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
   static bool attr[256] = {false};
   cudaError_t e = set_smem_attr_once(embed_sp_kernel<OT, kMode>, sp::SMEM_BYTES, attr);
@@ -1551,7 +1578,7 @@ cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
   } else if (resident < 1) {
     return cudaErrorNotSupported;
   }
-  return cudaLaunchKernelEx(&cfg, embed_sp_kernel<OT, kMode>, tmap, codes, F, D, out, sc.partials, sc.counters, g, eps,
+  return cudaLaunchKernelEx(&cfg, embed_sp_kernel<OT, kMode>, tmap, codes, F, D, out, om, sc.partials, sc.counters, g, eps,
                             err);
 }
 
@@ -1592,7 +1619,7 @@ bool sparse_enabled() {
 // partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel. CTA pairs
 // first; one-CTA tiles when pairs are switched off or cannot launch.
 template <typename OT>
-cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, const __nv_bfloat16 *g,
+cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, OutMap om, const __nv_bfloat16 *g,
                    float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
   const int P = D / tc::BN;
   const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * P;
@@ -1606,8 +1633,8 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
   if (pairs_enabled() && sparse_enabled() && max_clusters >= Psp) {
     const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
     const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
-    e = g ? launch_sp<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, (max_clusters / Psp) * Psp, stream)
-          : launch_sp<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, sp_clusters, stream);
+    e = g ? launch_sp<OT, kFused>(codes, F, T, D, out, om, sc, g, eps, err, (max_clusters / Psp) * Psp, stream)
+          : launch_sp<OT, kPlain>(codes, F, T, D, out, om, sc, nullptr, eps, err, sp_clusters, stream);
     if (e == cudaSuccess) {
       ++*launches;
       return e;
@@ -1616,19 +1643,19 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
   }
   if (!g) {
     if (pairs_enabled()) {
-      e = launch_tc2<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, plain_clusters, stream);
+      e = launch_tc2<OT, kPlain>(codes, F, T, D, out, om, sc, nullptr, eps, err, plain_clusters, stream);
       if (e == cudaSuccess) {
         ++*launches;
         return e;
       }
       (void)cudaGetLastError();  // pairs refused: one-CTA tiles below
     }
-    e = launch_tc<OT, kPlain>(codes, F, T, D, out, sc, nullptr, eps, err, plain_grid, stream);
+    e = launch_tc<OT, kPlain>(codes, F, T, D, out, om, sc, nullptr, eps, err, plain_grid, stream);
     if (e == cudaSuccess) ++*launches;
     return e;
   }
   if (pairs_enabled() && max_clusters / P >= 1) {
-    e = launch_tc2<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, (max_clusters / P) * P, stream);
+    e = launch_tc2<OT, kFused>(codes, F, T, D, out, om, sc, g, eps, err, (max_clusters / P) * P, stream);
     if (e == cudaSuccess) {
       ++*launches;
       return e;
@@ -1637,15 +1664,15 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
   }
   int fgrid = 0;
   if (fused_possible(D, num_sms, &fgrid)) {
-    e = launch_tc<OT, kFused>(codes, F, T, D, out, sc, g, eps, err, fgrid, stream);
+    e = launch_tc<OT, kFused>(codes, F, T, D, out, om, sc, g, eps, err, fgrid, stream);
     if (e == cudaSuccess) ++*launches;
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
     (void)cudaGetLastError();  // clear the refused launch; fall through to the two-kernel form
   }
-  e = launch_tc<OT, kPartials>(codes, F, T, D, out, sc, g, eps, err, plain_grid, stream);
+  e = launch_tc<OT, kPartials>(codes, F, T, D, out, om, sc, g, eps, err, plain_grid, stream);
   if (e == cudaSuccess) ++*launches;
   if (e == cudaSuccess) {
-    e = launch_rescale(out, F, D, g, sc.partials, eps, num_sms, stream);
+    e = launch_rescale(out, om, F, D, g, sc.partials, eps, num_sms, stream);
     if (e == cudaSuccess) ++*launches;
   }
   return e;
@@ -1724,29 +1751,31 @@ size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_d
 
 cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,
                          const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
-                         uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
+                         uint32_t *err, int num_sms, cudaStream_t stream, int *launches, const int64_t *out_rows,
+                         int64_t out_n_rows) {
   if (F <= 0) return cudaSuccess;
+  const OutMap om{out_rows, out_n_rows};
   cudaError_t e;
   if (embed_uses_tensor_cores(table_dtype, D)) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);
     const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
     if (out_dtype == DMEL_BF16)
-      return run_tc(codes, F, T, D, static_cast<__nv_bfloat16 *>(out), g, eps, workspace, err, num_sms, stream,
+      return run_tc(codes, F, T, D, static_cast<__nv_bfloat16 *>(out), om, g, eps, workspace, err, num_sms, stream,
                     launches);
-    return run_tc(codes, F, T, D, static_cast<float *>(out), g, eps, workspace, err, num_sms, stream, launches);
+    return run_tc(codes, F, T, D, static_cast<float *>(out), om, g, eps, workspace, err, num_sms, stream, launches);
   }
   if (table_dtype == DMEL_BF16) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);
     const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
     e = out_dtype == DMEL_BF16
-            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), err, num_sms, stream)
-            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), err, num_sms, stream);
+            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), om, err, num_sms, stream)
+            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), om, err, num_sms, stream);
   } else {
     const auto *T = static_cast<const float *>(table);
     const auto *g = static_cast<const float *>(rms_weight);
     e = out_dtype == DMEL_BF16
-            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), err, num_sms, stream)
-            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), err, num_sms, stream);
+            ? launch_simt(codes, F, T, D, g, eps, static_cast<__nv_bfloat16 *>(out), om, err, num_sms, stream)
+            : launch_simt(codes, F, T, D, g, eps, static_cast<float *>(out), om, err, num_sms, stream);
   }
   if (e == cudaSuccess) ++*launches;
   return e;

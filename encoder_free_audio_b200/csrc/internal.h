@@ -21,9 +21,12 @@ bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim);
 size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm);
 
 // Embedding of n_frames codes; workspace holds embed_workspace_bytes(...) bytes.
+// out_rows: NULL (frame f -> row f of out) or device int64 [n_frames], frame f -> row out_rows[f]
+// of an out with out_n_rows rows.
 cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
                          int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
-                         void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
+                         void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
+                         const int64_t *out_rows = nullptr, int64_t out_n_rows = 0);
 
 // Size of the fixed device scratch used by dmel_embed_noalloc.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;

@@ -25,6 +25,7 @@ DMEL_BF16 = 1
 DMEL_DEVERR_CODE_RANGE = 0x1
 DMEL_DEVERR_WAIT_TIMEOUT = 0x2
 DMEL_DEVERR_OFFSETS = 0x4
+DMEL_DEVERR_OUT_ROW = 0x8
 
 HOP = 800
 WIN = 1600
@@ -63,6 +64,13 @@ def _lib():
         L.dmel_forward.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, vp,
                                    sz, vp]
         L.dmel_forward.restype = i32
+        L.dmel_embed_rows.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, vp, i64, i32, vp, sz, vp]
+        L.dmel_embed_rows.restype = i32
+        L.dmel_forward_rows.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, vp, i64,
+                                        i32, vp, vp, sz, vp]
+        L.dmel_forward_rows.restype = i32
+        L.dmel_splice_plan.argtypes = [vp, i32, vp, i64, vp, vp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+        L.dmel_splice_plan.restype = i32
         L.dmel_embed_noalloc.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp]
         L.dmel_embed_noalloc.restype = i32
         L.dmel_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -173,6 +181,50 @@ def dmel_forward(wav, sample_offsets, frame_offsets, n_frames: int, table, out, 
                              _ptr(rms_weight), float(eps), _ptr(out), _dtype_code(out), _ptr(codes_out),
                              _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dmel_forward")
+
+
+def dmel_embed_rows(codes, table, out, out_rows, rms_weight=None, eps: float = 1e-6, workspace=None, stream=None):
+    """dmel_embed_rows on torch CUDA tensors: as dmel_embed, frame f written to row out_rows[f]
+    (int64 [F] on the device) of out [S, D]."""
+    n = codes.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_embed_rows(_ptr(codes), n, _ptr(table), _dtype_code(table), table.shape[1], _ptr(rms_weight),
+                                float(eps), _ptr(out), _ptr(out_rows), int(out.shape[0]), _dtype_code(out),
+                                _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_embed_rows")
+
+
+def dmel_forward_rows(wav, sample_offsets, frame_offsets, n_frames: int, table, out, out_rows, rms_weight=None,
+                      eps: float = 1e-6, tails=None, tails_out=None, codes_out=None, workspace=None, stream=None):
+    """dmel_forward_rows on torch CUDA tensors: as dmel_forward, frame f written to row
+    out_rows[f] (int64 [n_frames] on the device) of out [S, D]."""
+    n_clips = sample_offsets.shape[0] - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_forward_rows(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames),
+                                  _ptr(tails), _ptr(tails_out), _ptr(table), _dtype_code(table), table.shape[1],
+                                  _ptr(rms_weight), float(eps), _ptr(out), _ptr(out_rows), int(out.shape[0]),
+                                  _dtype_code(out), _ptr(codes_out), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_forward_rows")
+
+
+def dmel_splice_plan(sentinel_pos, frame_offsets, seq_len: int):
+    """Host splice plan: (token_pos [seq_len], frame_rows [F], expanded_len, audio_tokens) for a
+    sequence of seq_len positions with audio sentinels at sentinel_pos (one per clip of
+    frame_offsets)."""
+    sp = np.ascontiguousarray(np.asarray(sentinel_pos, dtype=np.int64))
+    fo = np.ascontiguousarray(np.asarray(frame_offsets, dtype=np.int64))
+    n_items = sp.shape[0]
+    if fo.shape[0] != n_items + 1:
+        raise DmelError(DMEL_ERR_INVALID_ARG, "dmel_splice_plan (frame offsets must have n_items + 1 entries)")
+    token_pos = np.empty(max(int(seq_len), 0), dtype=np.int64)
+    frame_rows = np.empty(int(fo[-1]) if fo.shape[0] else 0, dtype=np.int64)
+    exp_len, audio = ctypes.c_int64(0), ctypes.c_int64(0)
+    rc = _lib().dmel_splice_plan(sp.ctypes.data_as(ctypes.c_void_p), n_items, fo.ctypes.data_as(ctypes.c_void_p),
+                                 int(seq_len), token_pos.ctypes.data_as(ctypes.c_void_p),
+                                 frame_rows.ctypes.data_as(ctypes.c_void_p), ctypes.byref(exp_len),
+                                 ctypes.byref(audio))
+    _check(rc, "dmel_splice_plan")
+    return token_pos, frame_rows, int(exp_len.value), int(audio.value)
 
 
 def dmel_get_device_error(clear: bool = True) -> int:

@@ -67,6 +67,7 @@ typedef enum { DMEL_F32 = 0, DMEL_BF16 = 1 } dmel_dtype;
 #define DMEL_DEVERR_CODE_RANGE 0x1u  /* a code above 15 reached an embedding kernel (used code & 15) */
 #define DMEL_DEVERR_WAIT_TIMEOUT 0x2u /* a pipeline wait inside a kernel gave up (results invalid) */
 #define DMEL_DEVERR_OFFSETS 0x4u     /* device frame offsets disagree with the sample offsets */
+#define DMEL_DEVERR_OUT_ROW 0x8u     /* an output row index outside [0, out_n_rows) (row not written) */
 
 /* Frames of one clip of n_samples samples: floor(n_samples / 800) (20 per second of audio;
  * "Inside Inkling: Audio Design", Part 1 · Modeling). Host only, pure. Returns -1 for
@@ -168,6 +169,45 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                          dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
                          dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
                          dmel_stream_t stream);
+
+/* ---- Sentinel expansion and splice ("Inside Inkling: Audio Design", Part 3 · Inference: at
+ * serve time one audio item is a single sentinel token that expands into f d-mel frame
+ * positions, and the server reports the realised count as audio_tokens).
+ *
+ * dmel_splice_plan (host, pure): a token sequence of seq_len positions holds n_items audio
+ * sentinels at the strictly increasing positions h_sentinel_pos[0 .. n_items); item i is clip i,
+ * whose frames are [h_frame_offsets[i], h_frame_offsets[i + 1]) (from dmel_frame_offsets). Each
+ * sentinel is replaced by its f_i frames in place, so the expanded sequence has
+ * seq_len + sum_i (f_i - 1) positions (a clip with no frame leaves no position). Outputs (each
+ * may be NULL):
+ *   h_token_pos    [seq_len]: the expanded position of each original position, -1 for sentinels
+ *   h_frame_rows   [h_frame_offsets[n_items]]: the expanded position of each frame, in frame order
+ *                  (the out_rows of dmel_embed_rows / dmel_forward_rows)
+ *   h_expanded_len the expanded sequence length
+ *   h_audio_tokens sum_i f_i, the count the server reports
+ * Returns DMEL_ERR_INVALID_ARG (writing nothing) when seq_len < 0, n_items < 0, a sentinel
+ * position is outside [0, seq_len) or not strictly increasing, or the frame offsets do not start
+ * at 0 and increase. */
+dmel_status dmel_splice_plan(const int64_t *h_sentinel_pos, int n_items, const int64_t *h_frame_offsets,
+                             int64_t seq_len, int64_t *h_token_pos, int64_t *h_frame_rows,
+                             int64_t *h_expanded_len, int64_t *h_audio_tokens);
+
+/* dmel_embed and dmel_forward writing frame f's vector to row out_rows[f] of out instead of row f:
+ * out is the decoder's input sequence [out_n_rows x embed_dim] (out_dtype), out_rows a device
+ * int64 [n_frames] array (usually dmel_splice_plan's h_frame_rows, copied to the device). Rows
+ * that no frame maps to are left as they are (the text tokens' embeddings). A row index outside
+ * [0, out_n_rows) is not written and sets DMEL_DEVERR_OUT_ROW; rows mapped twice end up holding
+ * one of the two frames. Every other argument, the workspace included, is as in dmel_embed /
+ * dmel_forward. */
+dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                            int embed_dim, const void *rms_weight, float eps, void *out, const int64_t *out_rows,
+                            int64_t out_n_rows, dmel_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                            dmel_stream_t stream);
+dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                              int n_clips, int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                              const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, uint8_t *codes_out,
+                              void *workspace, size_t workspace_bytes, dmel_stream_t stream);
 
 /* Reads (and, when clear != 0, clears) the device error word of the current device. This call
  * synchronises the device. *h_bits receives DMEL_DEVERR_* bits (0 = no error). */

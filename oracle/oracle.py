@@ -211,3 +211,40 @@ def boundary_distance(lhat: np.ndarray) -> np.ndarray:
     k = np.arange(1, NLEV, dtype=np.float64)
     bnd = LMIN + (LMAX - LMIN) * k / NLEV
     return np.min(np.abs(lhat[..., None] - bnd), axis=-1)
+
+
+def splice(tokens: list, sentinel, frames_per_item: list) -> list:
+    """Sentinel expansion ("Inside Inkling: Audio Design", Part 3 · Inference): at serve time an
+    audio item is one sentinel token that expands into f frame positions. Written out plainly:
+    walk the token list and replace the i-th sentinel by f_i entries ("frame", i, j); every other
+    token is copied as ("token", original position). Returns the expanded list; its length and
+    the positions of its entries are the splice plan. A clip with no frame leaves no entry."""
+    out = []
+    item = 0
+    for pos, tok in enumerate(tokens):
+        if tok == sentinel:
+            for j in range(frames_per_item[item]):
+                out.append(("frame", item, j))
+            item += 1
+        else:
+            out.append(("token", pos))
+    if item != len(frames_per_item):
+        raise ValueError("one sentinel per audio item")
+    return out
+
+
+def splice_plan(seq_len: int, sentinel_pos: list, frames_per_item: list):
+    """The splice plan read off the plain expansion: (token_pos [seq_len] with -1 at sentinels,
+    frame_rows in frame order, expanded_len, audio_tokens)."""
+    sentinel = object()
+    tokens = [sentinel if p in set(sentinel_pos) else p for p in range(seq_len)]
+    expanded = splice(tokens, sentinel, frames_per_item)
+    token_pos = [-1] * seq_len
+    frame_rows = [None] * sum(frames_per_item)
+    starts = np.concatenate([[0], np.cumsum(frames_per_item)]).astype(int)
+    for row, entry in enumerate(expanded):
+        if entry[0] == "token":
+            token_pos[entry[1]] = row
+        else:
+            frame_rows[starts[entry[1]] + entry[2]] = row
+    return token_pos, frame_rows, len(expanded), int(sum(frames_per_item))

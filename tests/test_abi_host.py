@@ -89,6 +89,15 @@ def test_argument_checks_return_invalid_arg_without_gpu(lib):
     assert E(fake, 4, fake, 0, 16392, None, 1e-6, fake, 0, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
     # zero frames is a no-op
     assert E(None, 0, None, 1, 6144, None, 1e-6, None, 1, None, 0, None) == dmel.DMEL_OK
+    # row-mapped output: a row map needs a positive row count and 8-byte alignment
+    R = lib.dmel_embed_rows
+    assert R(fake, 4, fake, 1, 6144, None, 1e-6, fake, fake, 0, 1, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert R(fake, 4, fake, 1, 6144, None, 1e-6, fake, vp((1 << 20) + 4), 10, 1, None, 0,
+             None) == dmel.DMEL_ERR_INVALID_ARG
+    assert R(None, 0, None, 1, 6144, None, 1e-6, None, None, 0, 1, None, 0, None) == dmel.DMEL_OK
+    FR = lib.dmel_forward_rows
+    assert FR(fake, fake, fake, 1, 4, None, None, fake, 1, 6144, None, 1e-6, fake, fake, -3, 1, fake, None, 0,
+              None) == dmel.DMEL_ERR_INVALID_ARG
     Fw = lib.dmel_forward
     assert Fw(fake, fake, fake, 1, 4, None, None, fake, 1, 6144, fake, 1e-6, fake, 1, None, None, 0,
               None) == dmel.DMEL_ERR_INVALID_ARG  # no workspace for codes + partial sums

@@ -335,3 +335,56 @@ def test_rmsnorm_matches_torch(oracle_mod):
 def test_embed_rejects_bad_code(oracle_mod):
     with pytest.raises(ValueError):
         oracle_mod.embed(np.full((1, 80), 16, np.uint8), np.zeros((1280, 8)))
+
+
+# ---------------------------------------------------------------- sentinel expansion (splice)
+
+SPLICE_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "splice_example.json")
+
+
+def test_splice_hand_worked_example(oracle_mod):
+    g = json.load(open(SPLICE_GOLDEN))
+    token_pos, frame_rows, n, audio = oracle_mod.splice_plan(g["seq_len"], g["sentinel_pos"], g["frames_per_item"])
+    assert token_pos == g["token_pos"] and frame_rows == g["frame_rows"]
+    assert n == g["expanded_len"] and audio == g["audio_tokens"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_splice_closed_forms(oracle_mod, seed):
+    r = np.random.default_rng(500 + seed)
+    seq_len = int(r.integers(1, 60))
+    k = int(r.integers(0, seq_len + 1))
+    pos = sorted(r.choice(seq_len, size=k, replace=False).tolist())
+    f = r.integers(0, 9, size=k).tolist()
+    token_pos, frame_rows, n, audio = oracle_mod.splice_plan(seq_len, pos, f)
+    # each sentinel gives way to its f frames: the sequence grows by sum(f - 1)
+    assert n == seq_len + sum(x - 1 for x in f) and audio == sum(f)
+    # every expanded position is used exactly once, by a surviving token or a frame
+    used = [p for p in token_pos if p >= 0] + frame_rows
+    assert sorted(used) == list(range(n))
+    # tokens keep their order, a token before a sentinel keeps its index, and a token moves by
+    # the frames minus sentinels in front of it
+    survivors = [(p, q) for p, q in enumerate(token_pos) if q >= 0]
+    assert all(a[1] < b[1] for a, b in zip(survivors, survivors[1:]))
+    for p, q in survivors:
+        before = [i for i, s in enumerate(pos) if s < p]
+        assert q == p + sum(f[i] - 1 for i in before)
+    # an item's frames are consecutive and start where its sentinel stood (shifted)
+    starts = np.concatenate([[0], np.cumsum(f)]).astype(int)
+    for i, s in enumerate(pos):
+        rows = frame_rows[starts[i]:starts[i + 1]]
+        assert rows == list(range(rows[0], rows[0] + f[i])) if f[i] else rows == []
+        if f[i]:
+            assert rows[0] == s + sum(f[j] - 1 for j in range(i))
+
+
+def test_splice_special_cases(oracle_mod):
+    # no sentinel: the identity
+    tp, fr, n, a = oracle_mod.splice_plan(5, [], [])
+    assert tp == [0, 1, 2, 3, 4] and fr == [] and n == 5 and a == 0
+    # clips with no frame: their sentinels vanish
+    tp, fr, n, a = oracle_mod.splice_plan(4, [0, 2], [0, 0])
+    assert tp == [-1, 0, -1, 1] and fr == [] and n == 2 and a == 0
+    # an audio-only request: one sentinel, 20 frames per second of audio
+    tp, fr, n, a = oracle_mod.splice_plan(1, [0], [40])
+    assert tp == [-1] and fr == list(range(40)) and n == 40 and a == 40

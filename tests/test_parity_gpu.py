@@ -153,6 +153,110 @@ def test_embed_tensor_core_rmsnorm_widths(dim, oracle_mod):
     compare_embed(out.cpu().numpy(), ref, 1e-5)
 
 
+# ------------------------------------------------------------- output rows (sentinel splice)
+
+def _rows_case(F, S, seed):
+    r = np.random.default_rng(seed)
+    return r.choice(S, size=F, replace=False).astype(np.int64)
+
+
+@pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rms", [True, False])
+def test_embed_rows_scatter_into_sequence(out_dt, rms, table_bf16, rmsw_bf16, oracle_mod):
+    """Frames written to arbitrary rows of a longer sequence: the mapped rows hold exactly what
+    dmel_embed gives (same kernels, same arithmetic), within tolerance of the oracle; the other
+    rows keep their contents."""
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    F, S = 700, 1000
+    codes = synth.random_codes(61, F)
+    cd = torch.from_numpy(codes).to(DEV)
+    rows = _rows_case(F, S, 62)
+    ws = torch.empty(max(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, rms, True), 1), dtype=torch.uint8,
+                     device=DEV)
+    seq = torch.full((S, 6144), float("nan"), dtype=out_dt, device=DEV)
+    dmel.dmel_embed_rows(cd, T, seq, torch.from_numpy(rows).to(DEV), rms_weight=g if rms else None, eps=1e-6,
+                         workspace=ws)
+    plain = torch.empty((F, 6144), dtype=out_dt, device=DEV)
+    dmel.dmel_embed(cd, T, plain, rms_weight=g if rms else None, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    got = seq.float().cpu().numpy()
+    np.testing.assert_array_equal(got[rows], plain.float().cpu().numpy())
+    ref = oracle_mod.embed(codes, T64, g64 if rms else None, 1e-6)
+    compare_embed(got[rows], ref, 1e-5 if out_dt == torch.float32 else 1e-2)
+    assert np.isnan(got[np.setdiff1d(np.arange(S), rows)]).all()
+    assert dmel.dmel_get_device_error(clear=True) == 0
+
+
+def test_embed_rows_fp32_table_cuda_cores(oracle_mod):
+    T = synth.table(seed=9, dim=512)
+    gw = synth.rms_weight(seed=10, dim=512)
+    F, S = 77, 200
+    codes = synth.random_codes(63, F)
+    rows = _rows_case(F, S, 64)
+    seq = torch.full((S, 512), float("nan"), dtype=torch.float32, device=DEV)
+    dmel.dmel_embed_rows(torch.from_numpy(codes).to(DEV), torch.from_numpy(T).to(DEV), seq,
+                         torch.from_numpy(rows).to(DEV), rms_weight=torch.from_numpy(gw).to(DEV), eps=1e-6)
+    torch.cuda.synchronize()
+    got = seq.cpu().numpy()
+    compare_embed(got[rows], oracle_mod.embed(codes, T.astype(np.float64), gw.astype(np.float64), 1e-6), 1e-5)
+    assert np.isnan(got[np.setdiff1d(np.arange(S), rows)]).all()
+
+
+def test_embed_rows_out_of_range_rows_are_flagged_not_written(table_bf16, rmsw_bf16):
+    T, _ = table_bf16
+    g, _ = rmsw_bf16
+    F, S = 300, 400
+    rows = _rows_case(F, S, 65)
+    rows[5], rows[200] = S, -1  # one past the end, negative
+    codes = torch.from_numpy(synth.random_codes(66, F)).to(DEV)
+    buf = torch.full((S + 8, 6144), float("nan"), dtype=torch.bfloat16, device=DEV)  # 8 guard rows past S
+    ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True), dtype=torch.uint8, device=DEV)
+    dmel.dmel_get_device_error(clear=True)
+    dmel.dmel_embed_rows(codes, T, buf[:S], torch.from_numpy(rows).to(DEV), rms_weight=g, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    assert dmel.dmel_get_device_error(clear=True) & dmel.DMEL_DEVERR_OUT_ROW
+    got = buf.float().cpu().numpy()
+    assert np.isnan(got[S:]).all()  # nothing past the sequence
+    ok = np.delete(rows, [5, 200])
+    assert np.isfinite(got[ok]).all()
+    assert np.isnan(got[np.setdiff1d(np.arange(S), ok)]).all()
+
+
+def test_forward_rows_splices_clips_at_their_sentinels(table_bf16, rmsw_bf16, oracle_mod):
+    """Waveforms to the decoder's input sequence in one call: the planned rows hold the frames of
+    dmel_forward, text rows keep the text embeddings, and the plan matches the oracle's
+    expansion."""
+    T, _ = table_bf16
+    g, _ = rmsw_bf16
+    wav, off = synth.batch64_10s()
+    n_clips = 6
+    lens = [160000, 32000, 700, 160000, 48000, 16000]  # the third clip is too short for a frame
+    so = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    w = np.concatenate([wav[off[i]:off[i] + lens[i]] for i in range(n_clips)]).astype(np.float32)
+    fo = dmel.dmel_frame_offsets(so)
+    F = int(fo[-1])
+    seq_len = 40
+    sentinels = [2, 9, 10, 21, 30, 39]
+    token_pos, frame_rows, S, audio = dmel.dmel_splice_plan(sentinels, fo, seq_len)
+    otp, ofr, on, oa = oracle_mod.splice_plan(seq_len, sentinels, np.diff(fo).tolist())
+    assert token_pos.tolist() == otp and frame_rows.tolist() == ofr and S == on and audio == oa == F
+    seq = torch.full((S, 6144), 7.0, dtype=torch.bfloat16, device=DEV)  # stands for the text embeddings
+    wd = torch.from_numpy(w).to(DEV)
+    sod, fod = torch.from_numpy(so).to(DEV), torch.from_numpy(fo).to(DEV)
+    ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, False), dtype=torch.uint8, device=DEV)
+    dmel.dmel_forward_rows(wd, sod, fod, F, T, seq, torch.from_numpy(frame_rows).to(DEV), rms_weight=g, eps=1e-6,
+                           workspace=ws)
+    ref = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
+    dmel.dmel_forward(wd, sod, fod, F, T, ref, rms_weight=g, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    got = seq.float().cpu().numpy()
+    np.testing.assert_array_equal(got[frame_rows], ref.float().cpu().numpy())
+    text = token_pos[token_pos >= 0]
+    assert (got[text] == 7.0).all()
+    assert dmel.dmel_get_device_error(clear=True) == 0
+
+
 def test_embed_fp32_table_rmsnorm(oracle_mod):
     T = synth.table(seed=9, dim=512)
     gw = synth.rms_weight(seed=10, dim=512)
