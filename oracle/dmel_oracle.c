@@ -208,6 +208,72 @@ int oracle_codes(const float *wav, const int64_t *soff, int n_clips, const float
   return bad ? -1 : 0;
 }
 
+/* ---- Quantiser variants. The pages leave the level mapping open ("Inside Inkling: Audio
+ * Design", Coda: the quantizer mapping is undocumented, uniform or mu-law or learned, and the
+ * serving default clamps at -1.5 where the released config says -7.0). With the log-mel value
+ * clamped to [lmin, lmax] and u = (L - lmin) / (lmax - lmin):
+ *   mode 0, uniform floor (the default reading): c = min(15, floor((L - lmin) * 16 / (lmax - lmin)))
+ *   mode 1, nearest of the 16 reconstruction points lmin + k (lmax - lmin) / 15, ties upward:
+ *           c = floor((L - lmin) * 15 / (lmax - lmin) + 1/2)
+ *   mode 2, mu-law companding then 16 uniform levels: c = min(15, floor(16 ln(1 + mu u) / ln(1 + mu)))
+ * Codes always end in 0..15. */
+double oracle_log_clamp_q(double M, double lmin, double lmax) {
+  double m = (M > OR_FLOOR) ? M : OR_FLOOR; /* NaN compares false -> floor */
+  double L = log10(m);
+  if (L < lmin) L = lmin;
+  if (L > lmax) L = lmax;
+  return L;
+}
+
+int oracle_quantise_q(double lhat, double lmin, double lmax, int mode, double mu) {
+  double q;
+  if (mode == 1) {
+    q = floor((lhat - lmin) * (double)(OR_NLEV - 1) / (lmax - lmin) + 0.5);
+  } else if (mode == 2) {
+    const double u = (lhat - lmin) / (lmax - lmin);
+    q = floor((double)OR_NLEV * log(1.0 + mu * u) / log(1.0 + mu));
+  } else {
+    q = floor((lhat - lmin) * (double)OR_NLEV / (lmax - lmin));
+  }
+  int c = (int)q;
+  if (c > OR_NLEV - 1) c = OR_NLEV - 1;
+  if (c < 0) c = 0;
+  return c;
+}
+
+/* oracle_codes with a quantiser variant; lhat receives the value clamped to [lmin, lmax]. */
+int oracle_codes_q(const float *wav, const int64_t *soff, int n_clips, const float *tails, const int64_t *frame_ids,
+                   int64_t n_sel, double lmin, double lmax, int mode, double mu, uint8_t *codes, double *lhat) {
+  oracle_init();
+  int64_t *fo = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n_clips + 1));
+  if (!fo) return -1;
+  if (oracle_frame_offsets(soff, n_clips, fo) != 0) { free(fo); return -1; }
+  const int64_t total = fo[n_clips];
+  if (!frame_ids) n_sel = total;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+  for (int64_t i = 0; i < n_sel; ++i) {
+    const int64_t g = frame_ids ? frame_ids[i] : i;
+    if (g < 0 || g >= total) { bad |= 1; continue; }
+    int lo = 0, hi = n_clips - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) / 2;
+      if (fo[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int64_t t = g - fo[lo];
+    double frame[OR_WIN], M[OR_NMEL];
+    for (int n = 0; n < OR_WIN; ++n) frame[n] = frame_sample(wav, soff, tails, lo, OR_HOP * (t - 1) + n);
+    oracle_mel(frame, M);
+    for (int b = 0; b < OR_NMEL; ++b) {
+      const double L = oracle_log_clamp_q(M[b], lmin, lmax);
+      codes[i * OR_NMEL + b] = (uint8_t)oracle_quantise_q(L, lmin, lmax, mode, mu);
+      if (lhat) lhat[i * OR_NMEL + b] = L;
+    }
+  }
+  free(fo);
+  return bad ? -1 : 0;
+}
+
 /* Carried tails out: the 800 samples that end at sample 800 F of each clip (F >= 1), else the
  * tail in (zeros without one). */
 int oracle_tails_out(const float *wav, const int64_t *soff, int n_clips, const float *tails, float *tails_out) {

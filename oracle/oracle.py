@@ -71,6 +71,12 @@ def lib():
         L.oracle_codes.restype = c_int
         L.oracle_tails_out.argtypes = [vp, vp, c_int, vp, vp]
         L.oracle_tails_out.restype = c_int
+        L.oracle_log_clamp_q.argtypes = [c_d, c_d, c_d]
+        L.oracle_log_clamp_q.restype = c_d
+        L.oracle_quantise_q.argtypes = [c_d, c_d, c_d, c_int, c_d]
+        L.oracle_quantise_q.restype = c_int
+        L.oracle_codes_q.argtypes = [vp, vp, c_int, vp, vp, c_i64, c_d, c_d, c_int, c_d, vp, vp]
+        L.oracle_codes_q.restype = c_int
         L.oracle_embed.argtypes = [vp, c_i64, vp, c_int, vp, c_d, vp]
         L.oracle_embed.restype = c_int
         _lib = L
@@ -203,6 +209,60 @@ def embed(codes_: np.ndarray, table: np.ndarray, rms_weight: np.ndarray | None =
     if rc != 0:
         raise ValueError("oracle_embed: code out of range")
     return out
+
+
+# quantiser variants (modes of the C oracle): 0 uniform floor, 1 nearest of 16 reconstruction
+# points, 2 mu-law companding; clamp range [lmin, lmax]
+DEFAULT_QUANT = (LMIN, LMAX, 0, 0.0)
+
+
+def log_clamp_q(M: float, lmin: float, lmax: float) -> float:
+    return float(lib().oracle_log_clamp_q(float(M), float(lmin), float(lmax)))
+
+
+def quantise_q(lhat: float, lmin: float, lmax: float, mode: int, mu: float = 0.0) -> int:
+    return int(lib().oracle_quantise_q(float(lhat), float(lmin), float(lmax), int(mode), float(mu)))
+
+
+def codes_q(wav: np.ndarray, sample_offsets: np.ndarray, quant, tails: np.ndarray | None = None,
+            frame_ids: np.ndarray | None = None):
+    """codes() under a quantiser variant quant = (lmin, lmax, mode, mu); returns (codes, lhat)
+    with lhat clamped to [lmin, lmax]."""
+    lmin, lmax, mode, mu = quant
+    w = np.ascontiguousarray(wav, np.float32)
+    so = np.ascontiguousarray(sample_offsets, np.int64)
+    n_clips = so.shape[0] - 1
+    t = None if tails is None else np.ascontiguousarray(tails, np.float32)
+    if frame_ids is None:
+        n = int(frame_offsets(so)[-1])
+        ids = None
+    else:
+        ids = np.ascontiguousarray(frame_ids, np.int64)
+        n = ids.shape[0]
+    c = np.zeros((n, NMEL), np.uint8)
+    lh = np.zeros((n, NMEL), np.float64)
+    rc = lib().oracle_codes_q(_ptr(w), _ptr(so), n_clips, _ptr(t), _ptr(ids), n, float(lmin), float(lmax),
+                              int(mode), float(mu), _ptr(c), _ptr(lh))
+    if rc != 0:
+        raise ValueError("oracle_codes_q: bad offsets or frame index")
+    return c, lh
+
+
+def level_boundaries_q(lmin: float, lmax: float, mode: int, mu: float = 0.0) -> np.ndarray:
+    """The 15 inner decision boundaries in log-mel units of a quantiser variant (closed forms of
+    the three mappings)."""
+    k = np.arange(1, NLEV, dtype=np.float64)
+    r = lmax - lmin
+    if mode == 1:
+        return lmin + r * (k - 0.5) / (NLEV - 1)
+    if mode == 2:
+        return lmin + r * (np.power(1.0 + mu, k / NLEV) - 1.0) / mu
+    return lmin + r * k / NLEV
+
+
+def boundary_distance_q(lhat: np.ndarray, quant) -> np.ndarray:
+    bnd = level_boundaries_q(*quant)
+    return np.min(np.abs(np.asarray(lhat)[..., None] - bnd), axis=-1)
 
 
 def boundary_distance(lhat: np.ndarray) -> np.ndarray:

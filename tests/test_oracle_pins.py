@@ -388,3 +388,71 @@ def test_splice_special_cases(oracle_mod):
     # an audio-only request: one sentinel, 20 frames per second of audio
     tp, fr, n, a = oracle_mod.splice_plan(1, [0], [40])
     assert tp == [-1] and fr == list(range(40)) and n == 40 and a == 40
+
+
+# ---------------------------------------------------------------- quantiser variants
+
+SERVE_CLAMP = (-1.5, 2.0)  # the serving default's minimum ("Inside Inkling: Audio Design", Coda)
+
+
+def test_quant_default_variant_is_the_default(oracle_mod):
+    wav, off = synth.one_clip_2s()
+    c0, l0 = oracle_mod.codes(wav, off)
+    c1, l1 = oracle_mod.codes_q(wav, off, oracle_mod.DEFAULT_QUANT)
+    assert (c0 == c1).all() and (l0 == l1).all()
+
+
+def test_quant_round_is_nearest_reconstruction_point(oracle_mod):
+    """Mode 1: brute force over the 16 reconstruction points lmin + k (lmax - lmin) / 15."""
+    for lmin, lmax in ((-7.0, 2.0), SERVE_CLAMP):
+        pts = lmin + (lmax - lmin) * np.arange(16) / 15.0
+        for k, p in enumerate(pts):
+            assert oracle_mod.quantise_q(p, lmin, lmax, 1) == k
+        r = np.random.default_rng(11)
+        for L in r.uniform(lmin, lmax, 3000):
+            d = np.abs(L - pts)
+            if np.sort(d)[1] - d.min() < 1e-9:
+                continue  # a tie between two points
+            assert oracle_mod.quantise_q(L, lmin, lmax, 1) == int(np.argmin(d))
+
+
+def test_quant_mulaw_matches_library_companding(oracle_mod):
+    """Mode 2: numpy's log1p companding of u = (L - lmin) / (lmax - lmin), then 16 levels."""
+    mu = 255.0
+    for lmin, lmax in ((-7.0, 2.0), SERVE_CLAMP):
+        r = np.random.default_rng(12)
+        Ls = np.concatenate([r.uniform(lmin, lmax, 3000), [lmin, lmax]])
+        u = (Ls - lmin) / (lmax - lmin)
+        y = 16.0 * np.log1p(mu * u) / np.log1p(mu)
+        ref = np.minimum(15, np.floor(y)).astype(int)
+        near = np.abs(y - np.round(y)) < 1e-9
+        got = np.array([oracle_mod.quantise_q(L, lmin, lmax, 2, mu) for L in Ls])
+        assert (got[~near] == ref[~near]).all()
+        assert got[-2] == 0 and got[-1] == 15
+        # companding spends more levels near the bottom of the range
+        assert (got == 0).mean() < 1.0 / 16 and (got == 15).mean() > 1.0 / 16
+
+
+def test_quant_serving_clamp_special_cases(oracle_mod):
+    q = (SERVE_CLAMP[0], SERVE_CLAMP[1], 0, 0.0)
+    c, lh = oracle_mod.codes_q(np.zeros(16000, np.float32), np.array([0, 16000]), q)
+    assert (c == 0).all() and (lh == -1.5).all()  # silence sits at the new bottom
+    r = np.random.default_rng(5)
+    wav = np.where(r.random(16000 * 4) < 0.5, -1.0, 1.0).astype(np.float32)
+    c, _ = oracle_mod.codes_q(wav, np.array([0, wav.size]), q)
+    assert (c[1:] == 15).mean() >= 0.99
+
+
+def test_quant_serving_clamp_gain_shift_is_one_level(oracle_mod):
+    """With the clamp [-1.5, 2] a level is 3.5 / 16 wide: x -> x * 10^(3.5/32) adds one level."""
+    q = (SERVE_CLAMP[0], SERVE_CLAMP[1], 0, 0.0)
+    w = (SERVE_CLAMP[1] - SERVE_CLAMP[0]) / 16
+    wav, off = synth.one_clip_2s()
+    g = 10.0 ** (w / 2.0)
+    c0, l0 = oracle_mod.codes_q(wav, off, q)
+    c1, l1 = oracle_mod.codes_q((wav.astype(np.float64) * g).astype(np.float32), off, q)
+    inner = (l0 > SERVE_CLAMP[0] + 1e-6) & (l0 < SERVE_CLAMP[1] - w - 1e-6)
+    assert inner.sum() > 300
+    assert np.max(np.abs((l1 - l0)[inner] - w)) < 1e-5
+    safe = inner & (oracle_mod.boundary_distance_q(l0, q) > 1e-4)
+    assert (c1[safe].astype(int) - c0[safe].astype(int) == 1).all()
