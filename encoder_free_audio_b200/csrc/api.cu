@@ -1,4 +1,5 @@
 // C ABI of the dMel front end: argument checks, workspace layout and dispatch to the kernels.
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -80,6 +81,25 @@ dmel_status check_codes_args(const float *wav, const int64_t *sample_offsets, co
 
 dmel_status from_cuda(cudaError_t e) { return e == cudaSuccess ? DMEL_OK : DMEL_ERR_CUDA; }
 
+// dmel_quantizer -> Quant (NULL: the default); false for a quantiser the ABI rejects.
+bool to_quant(const dmel_quantizer *q, Quant *out) {
+  Quant z;
+  if (q) {
+    if (!std::isfinite(q->min_value) || !std::isfinite(q->max_value) || !(q->max_value > q->min_value)) return false;
+    if (q->mode != DMEL_QUANT_FLOOR && q->mode != DMEL_QUANT_ROUND && q->mode != DMEL_QUANT_MULAW) return false;
+    if (q->mode == DMEL_QUANT_MULAW && !(std::isfinite(q->mu) && q->mu > 0.0f)) return false;
+    z.lmin = q->min_value;
+    z.lmax = q->max_value;
+    z.range = q->max_value - q->min_value;
+    z.mode = q->mode;
+    z.mu = q->mode == DMEL_QUANT_MULAW ? q->mu : 0.0f;
+    z.inv_log1p_mu = q->mode == DMEL_QUANT_MULAW ? (float)(1.0 / std::log1p((double)q->mu)) : 0.0f;
+    if (!std::isfinite(z.range)) return false;
+  }
+  *out = z;
+  return true;
+}
+
 }  // namespace
 }  // namespace dmel
 
@@ -112,9 +132,12 @@ size_t dmel_workspace_size(int64_t n_frames, int embed_dim, dmel_dtype table_dty
   return bytes;
 }
 
-dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
-                       int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes, dmel_stream_t stream) {
+dmel_status dmel_codes_q(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                         int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes,
+                         const dmel_quantizer *q, dmel_stream_t stream) {
   t_last_launches = 0;
+  Quant qz;
+  if (!to_quant(q, &qz)) return DMEL_ERR_INVALID_ARG;
   dmel_status st = check_codes_args(wav, sample_offsets, frame_offsets, n_clips, n_frames, codes);
   if (st != DMEL_OK || n_clips == 0) return st;
   DeviceInfo d;
@@ -122,9 +145,14 @@ dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const in
   if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
   int launches = 0;
   cudaError_t e = launch_codes(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, codes, d.err,
-                               d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+                               d.sms, reinterpret_cast<cudaStream_t>(stream), &launches, qz);
   t_last_launches = launches;
   return from_cuda(e);
+}
+
+dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                       int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes, dmel_stream_t stream) {
+  return dmel_codes_q(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, codes, nullptr, stream);
 }
 
 dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
@@ -287,6 +315,14 @@ dmel_status dmel_debug_wait_timeout(uint32_t polls, uint32_t *h_bits) {
   int returned = 0;
   if (run_wait_timeout_selftest(polls, d.err, &returned) != cudaSuccess || returned != 1) return DMEL_ERR_CUDA;
   return dmel_get_device_error(h_bits, 1);
+}
+
+dmel_status dmel_debug_codes_frame_host_q(const float *frame1600, const dmel_quantizer *q, uint8_t *codes80,
+                                          double *lhat80) {
+  Quant qz;
+  if (!frame1600 || !codes80 || !to_quant(q, &qz)) return DMEL_ERR_INVALID_ARG;
+  emulate_codes_frame_host(frame1600, codes80, lhat80, qz);
+  return DMEL_OK;
 }
 
 void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {

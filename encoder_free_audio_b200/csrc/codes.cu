@@ -410,15 +410,31 @@ __host__ __device__ inline void step_e_chunk(int l, const Tables &T, const float
 
 // Step E, second half: channel b = lane, lane + 32, lane + 64 adds its partials, then log10,
 // clamp and quantise.
+// Level of a clamped log-mel value: mode 0 floor((L - lmin) * 16 / range) (for the default
+// [-7, 2] the same fp32 operations as (L + 7) * 16 / 9), mode 1 the nearest of 16 reconstruction
+// points lmin + k range / 15 (ties upward), mode 2 mu-law companding of u = (L - lmin) / range
+// followed by 16 uniform levels.
+__host__ __device__ inline int quant_level(float L, const Quant &q) {
+  float y;
+  if (q.mode == 1) {
+    y = (L - q.lmin) * 15.0f / q.range + 0.5f;
+  } else if (q.mode == 2) {
+    y = 16.0f * (log1pf(q.mu * ((L - q.lmin) / q.range)) * q.inv_log1p_mu);
+  } else {
+    y = (L - q.lmin) * 16.0f / q.range;
+  }
+  const int c = (int)floorf(y);
+  return c > 15 ? 15 : (c < 0 ? 0 : c);
+}
+
 __host__ __device__ inline void step_e_codes(int l, const Tables &T, const float *part, uint8_t *codes_row,
-                                             double *lhat_row) {
+                                             double *lhat_row, const Quant &qz) {
   for (int b = l; b < kMel; b += 32) {
     float m = 0.0f;
     for (int q = T.chanseg[b]; q < T.chanseg[b + 1]; ++q) m += part[q];
     float L = log10f(fmaxf(m, 1e-10f));  // fmaxf drops a NaN energy
-    L = fminf(fmaxf(L, -7.0f), 2.0f);
-    int c = (int)floorf((L + 7.0f) * 16.0f / 9.0f);
-    c = c > 15 ? 15 : (c < 0 ? 0 : c);
+    L = fminf(fmaxf(L, qz.lmin), qz.lmax);
+    const int c = quant_level(L, qz);
     codes_row[b] = (uint8_t)c;
     if (lhat_row) lhat_row[b] = (double)L;
   }
@@ -529,7 +545,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
                                                                              int n_clips, int64_t n_frames,
                                                                              const float *__restrict__ tails,
                                                                              uint8_t *__restrict__ codes,
-                                                                             uint32_t *err) {
+                                                                             Quant qz, uint32_t *err) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -635,7 +651,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     __syncwarp();
     step_e_chunk(lane, T, P, part);
     __syncwarp();
-    step_e_codes(lane, T, part, crow, nullptr);
+    step_e_codes(lane, T, part, crow, nullptr, qz);
     __syncwarp();
   }
 }
@@ -671,7 +687,7 @@ __global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restric
 
 cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *foff, int n_clips, int64_t n_frames,
                          const float *tails, float *tails_out, uint8_t *codes, uint32_t *err, int num_sms,
-                         cudaStream_t stream, int *launches) {
+                         cudaStream_t stream, int *launches, Quant q) {
   cudaError_t e = ensure_device_tables();
   if (e != cudaSuccess) return e;
   static bool attr_set[256] = {false};
@@ -686,7 +702,7 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
     int64_t blocks = (n_frames + kWarpsPerBlock - 1) / kWarpsPerBlock;
     if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM
     codes_kernel_entry<<<(unsigned)blocks, kWarpsPerBlock * 32, kSmemBytes, stream>>>(
-        wav, soff, foff, n_clips, n_frames, tails, codes, err);
+        wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
@@ -704,7 +720,7 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
 // the lanes and units of each step run one after another, and a step's loads all complete
 // before its stores where the kernel separates them with __syncwarp). Diagnostic only: no
 // entry point of the front end calls it.
-void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {
+void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80, Quant q) {
   const HostTables &H = host_tables();
   const Tables T = H.view();
   std::vector<double2> B(800);
@@ -722,7 +738,7 @@ void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *
   for (int l = 0; l < 32; ++l) step_d_load(l, B.data(), R[l]);
   for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<float *>(B.data()));
   for (int l = 0; l < 32; ++l) step_e_chunk(l, T, reinterpret_cast<const float *>(B.data()), part.data());
-  for (int l = 0; l < 32; ++l) step_e_codes(l, T, part.data(), codes80, lhat80);
+  for (int l = 0; l < 32; ++l) step_e_codes(l, T, part.data(), codes80, lhat80, q);
 }
 
 }  // namespace dmel

@@ -8,11 +8,19 @@
 
 namespace dmel {
 
+// The level mapping of the codes (dmel_quantizer, checked): clamp range, mode, mu, and the
+// derived constants the kernel uses. Quant() is the default reading: [-7, 2], uniform floor.
+struct Quant {
+  float lmin = -7.0f, lmax = 2.0f, range = 9.0f;
+  int mode = 0;  // 0 uniform floor, 1 nearest of 16 reconstruction points, 2 mu-law
+  float mu = 0.0f, inv_log1p_mu = 0.0f;
+};
+
 // Codes of n_frames frames (and the carried tails when tails_out != nullptr) on `stream`.
 // Adds the number of kernels launched to *launches.
 cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *foff, int n_clips, int64_t n_frames,
                          const float *tails, float *tails_out, uint8_t *codes, uint32_t *err, int num_sms,
-                         cudaStream_t stream, int *launches);
+                         cudaStream_t stream, int *launches, Quant q = Quant());
 
 // Whether the tensor-core embedding path takes this request.
 bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim);
@@ -37,6 +45,6 @@ cudaError_t noalloc_scratch(void **ptr);
 // Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
 cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);
 
-void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
+void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80, Quant q = Quant());
 
 }  // namespace dmel

@@ -26,6 +26,15 @@ DMEL_DEVERR_CODE_RANGE = 0x1
 DMEL_DEVERR_WAIT_TIMEOUT = 0x2
 DMEL_DEVERR_OFFSETS = 0x4
 DMEL_DEVERR_OUT_ROW = 0x8
+DMEL_QUANT_FLOOR = 0
+DMEL_QUANT_ROUND = 1
+DMEL_QUANT_MULAW = 2
+
+
+class Quantizer(ctypes.Structure):
+    """dmel_quantizer: clamp range [min_value, max_value], mode (DMEL_QUANT_*), mu (mu-law)."""
+    _fields_ = [("min_value", ctypes.c_float), ("max_value", ctypes.c_float), ("mode", ctypes.c_int),
+                ("mu", ctypes.c_float)]
 
 HOP = 800
 WIN = 1600
@@ -83,6 +92,10 @@ def _lib():
         L.dmel_debug_wait_timeout.restype = i32
         L.dmel_debug_codes_frame_host.argtypes = [vp, vp, vp]
         L.dmel_debug_codes_frame_host.restype = None
+        L.dmel_debug_codes_frame_host_q.argtypes = [vp, ctypes.POINTER(Quantizer), vp, vp]
+        L.dmel_debug_codes_frame_host_q.restype = i32
+        L.dmel_codes_q.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, ctypes.POINTER(Quantizer), vp]
+        L.dmel_codes_q.restype = i32
         _L = L
     return _L
 
@@ -150,6 +163,25 @@ def dmel_codes(wav, sample_offsets, frame_offsets, n_frames: int, codes, tails=N
     rc = _lib().dmel_codes(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames), _ptr(tails),
                            _ptr(tails_out), _ptr(codes), _stream(stream))
     _check(rc, "dmel_codes")
+
+
+def _quantizer(q):
+    """None, a Quantizer, or a tuple (min_value, max_value, mode, mu)."""
+    if q is None or isinstance(q, Quantizer):
+        return q
+    lo, hi, mode, mu = q
+    return Quantizer(float(lo), float(hi), int(mode), float(mu))
+
+
+def dmel_codes_q(wav, sample_offsets, frame_offsets, n_frames: int, codes, quantizer=None, tails=None, tails_out=None,
+                 stream=None):
+    """dmel_codes_q on torch CUDA tensors: dmel_codes with the level mapping `quantizer`
+    (None, a Quantizer, or (min_value, max_value, mode, mu))."""
+    n_clips = sample_offsets.shape[0] - 1
+    q = _quantizer(quantizer)
+    rc = _lib().dmel_codes_q(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames), _ptr(tails),
+                             _ptr(tails_out), _ptr(codes), None if q is None else ctypes.byref(q), _stream(stream))
+    _check(rc, "dmel_codes_q")
 
 
 def dmel_embed(codes, table, out, rms_weight=None, eps: float = 1e-6, workspace=None, stream=None):
@@ -250,6 +282,20 @@ def dmel_debug_codes_frame_host(frame1600: np.ndarray):
     lhat = np.zeros(N_MEL, np.float64)
     _lib().dmel_debug_codes_frame_host(fr.ctypes.data_as(ctypes.c_void_p), codes.ctypes.data_as(ctypes.c_void_p),
                                        lhat.ctypes.data_as(ctypes.c_void_p))
+    return codes, lhat
+
+
+def dmel_debug_codes_frame_host_q(frame1600: np.ndarray, quantizer=None):
+    """Host emulation with the level mapping `quantizer` (as dmel_codes_q)."""
+    fr = np.ascontiguousarray(frame1600, np.float32)
+    assert fr.shape == (WIN,)
+    codes = np.zeros(N_MEL, np.uint8)
+    lhat = np.zeros(N_MEL, np.float64)
+    q = _quantizer(quantizer)
+    rc = _lib().dmel_debug_codes_frame_host_q(fr.ctypes.data_as(ctypes.c_void_p), None if q is None else ctypes.byref(q),
+                                              codes.ctypes.data_as(ctypes.c_void_p),
+                                              lhat.ctypes.data_as(ctypes.c_void_p))
+    _check(rc, "dmel_debug_codes_frame_host_q")
     return codes, lhat
 
 

@@ -170,6 +170,32 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                          dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
                          dmel_stream_t stream);
 
+/* ---- Quantiser variants. The pages leave the level mapping open ("Inside Inkling: Audio
+ * Design", Coda: the quantizer mapping is undocumented, uniform or mu-law or learned, and the
+ * serving default clamps the log-mel value at -1.5 where the released config says -7.0). With L
+ * clamped to [min_value, max_value] and u = (L - min_value) / (max_value - min_value):
+ *   DMEL_QUANT_FLOOR  c = min(15, floor(16 u))                      (dmel_codes: [-7, 2])
+ *   DMEL_QUANT_ROUND  c = floor(15 u + 1/2): the nearest of 16 reconstruction points
+ *                     min_value + k (max_value - min_value) / 15, ties upward
+ *   DMEL_QUANT_MULAW  c = min(15, floor(16 ln(1 + mu u) / ln(1 + mu)))
+ * Arithmetic in fp32 like dmel_codes; codes agree with an fp64 evaluation except where the exact
+ * log-mel value lies within 1e-4 of one of the mapping's 15 inner boundaries. */
+typedef enum { DMEL_QUANT_FLOOR = 0, DMEL_QUANT_ROUND = 1, DMEL_QUANT_MULAW = 2 } dmel_quant_mode;
+
+typedef struct {
+  float min_value; /* clamp bottom (the released config: -7.0; the serving default: -1.5) */
+  float max_value; /* clamp top (2.0); finite, > min_value */
+  int mode;        /* dmel_quant_mode */
+  float mu;        /* mu-law parameter (> 0, e.g. 255), ignored by the other modes */
+} dmel_quantizer;
+
+/* dmel_codes with the level mapping q (NULL: the default, exactly dmel_codes). Returns
+ * DMEL_ERR_INVALID_ARG for a non-finite or empty clamp range, an unknown mode or mu <= 0 in
+ * mu-law mode. Codes from here feed dmel_embed / dmel_embed_rows unchanged. */
+dmel_status dmel_codes_q(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets, int n_clips,
+                         int64_t n_frames, const float *tails, float *tails_out, uint8_t *codes,
+                         const dmel_quantizer *q, dmel_stream_t stream);
+
 /* ---- Sentinel expansion and splice ("Inside Inkling: Audio Design", Part 3 · Inference: at
  * serve time one audio item is a single sentinel token that expands into f d-mel frame
  * positions, and the server reports the realised count as audio_tokens).

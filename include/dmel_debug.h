@@ -20,6 +20,11 @@ extern "C" {
  * clamped log10 mel energies. Lets the kernel's arithmetic be checked without a GPU. */
 void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80);
 
+/* The same with the level mapping q of dmel_codes_q (NULL: the default). Returns
+ * DMEL_ERR_INVALID_ARG for a quantiser dmel_codes_q would reject. */
+dmel_status dmel_debug_codes_frame_host_q(const float *frame1600, const dmel_quantizer *q, uint8_t *codes80,
+                                          double *lhat80);
+
 /* Failure-detection self test: launches one thread that waits, with a limit of `polls`
  * mbarrier polls, on a barrier phase that can never complete (two arrivals expected, one
  * made). The wait must give up and the kernel return; the call synchronises, then reads and

@@ -4,12 +4,17 @@ max(|o_j|, rms of the oracle row))."""
 import numpy as np
 
 
-def compare_codes(gpu_codes: np.ndarray, ora_codes: np.ndarray, ora_lhat: np.ndarray, band: float = 1e-4):
+def compare_codes(gpu_codes: np.ndarray, ora_codes: np.ndarray, ora_lhat: np.ndarray, band: float = 1e-4,
+                  boundaries: np.ndarray | None = None):
     """Returns (number of flipped cells, boolean mask of frames with a flip). Fails on any
-    mismatch whose oracle value lies farther than `band` from every inner level boundary."""
+    mismatch whose oracle value lies farther than `band` from every inner level boundary
+    (the default mapping's, -7 + 9k/16, unless `boundaries` gives a variant's)."""
     assert gpu_codes.shape == ora_codes.shape, (gpu_codes.shape, ora_codes.shape)
-    k = np.arange(1, 16, dtype=np.float64)
-    bnd = -7.0 + 9.0 * k / 16.0
+    if boundaries is None:
+        k = np.arange(1, 16, dtype=np.float64)
+        bnd = -7.0 + 9.0 * k / 16.0
+    else:
+        bnd = np.asarray(boundaries, np.float64)
     mism = gpu_codes != ora_codes
     if not mism.any():
         return 0, np.zeros(gpu_codes.shape[0], bool)

@@ -157,3 +157,48 @@ def test_kernel_arithmetic_on_host_tones_and_noise(lib, oracle_mod):
         gc, gl = dmel.dmel_debug_codes_frame_host(fr)
         oc, ol = oracle_mod.codes(fr, np.array([0, 1600]), tails=None, frame_ids=np.array([1]))
         _compare_codes(gc, gl, oc[0], ol[0], oracle_mod)
+
+
+# ---------------------------------------------------------------- quantiser variants on the host
+
+QUANTS = [(-7.0, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0), (-1.5, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0),
+          (-7.0, 2.0, dmel.DMEL_QUANT_ROUND, 0.0), (-1.5, 2.0, dmel.DMEL_QUANT_ROUND, 0.0),
+          (-7.0, 2.0, dmel.DMEL_QUANT_MULAW, 255.0), (-1.5, 2.0, dmel.DMEL_QUANT_MULAW, 255.0)]
+
+
+@pytest.mark.parametrize("q", QUANTS)
+def test_kernel_quantiser_variants_on_host_match_oracle(lib, oracle_mod, q):
+    wav, off = synth.one_clip_2s()
+    frames = _frames(wav, off, np.arange(40), oracle_mod)
+    oc, ol = oracle_mod.codes_q(wav, off, q)
+    for i in range(40):
+        gc, gl = dmel.dmel_debug_codes_frame_host_q(frames[i], q)
+        dist = oracle_mod.boundary_distance_q(ol[i], q)
+        assert not ((gc != oc[i]) & (dist > 1e-4)).any(), "code mismatch away from a level boundary"
+        inner = (ol[i] > q[0]) & (ol[i] < q[1])
+        np.testing.assert_allclose(gl[inner], ol[i][inner], rtol=0, atol=2e-6)
+
+
+def test_default_quantiser_is_bit_identical_on_host(lib):
+    wav, off = synth.one_clip_2s()
+    r = np.random.default_rng(3)
+    for t in range(1, 40, 7):
+        fr = wav[800 * (t - 1):800 * (t + 1)].astype(np.float32)
+        c0, l0 = dmel.dmel_debug_codes_frame_host(fr)
+        c1, l1 = dmel.dmel_debug_codes_frame_host_q(fr, None)
+        c2, l2 = dmel.dmel_debug_codes_frame_host_q(fr, (-7.0, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0))
+        assert (c0 == c1).all() and (c0 == c2).all() and (l0 == l1).all() and (l0 == l2).all()
+
+
+@pytest.mark.parametrize("q", [(2.0, 2.0, 0, 0.0), (3.0, -7.0, 0, 0.0), (float("nan"), 2.0, 0, 0.0),
+                               (-7.0, float("inf"), 0, 0.0), (-7.0, 2.0, 3, 0.0), (-7.0, 2.0, 2, 0.0),
+                               (-7.0, 2.0, 2, -1.0)])
+def test_bad_quantisers_are_rejected_without_gpu(lib, q):
+    fr = np.zeros(1600, np.float32)
+    with pytest.raises(dmel.DmelError):
+        dmel.dmel_debug_codes_frame_host_q(fr, q)
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)
+    qq = dmel.Quantizer(*q)
+    assert lib.dmel_codes_q(fake, fake, fake, 1, 4, None, None, fake, ctypes.byref(qq),
+                            None) == dmel.DMEL_ERR_INVALID_ARG

@@ -98,6 +98,42 @@ def test_codes_no_frames_is_noop():
     assert g.shape == (0, 80)
 
 
+# ---------------------------------------------------------------- codes: quantiser variants
+
+QUANTS = [(-1.5, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0), (-7.0, 2.0, dmel.DMEL_QUANT_ROUND, 0.0),
+          (-1.5, 2.0, dmel.DMEL_QUANT_ROUND, 0.0), (-7.0, 2.0, dmel.DMEL_QUANT_MULAW, 255.0),
+          (-1.5, 2.0, dmel.DMEL_QUANT_MULAW, 255.0)]
+
+
+def _codes_q_gpu(wav, off, q):
+    fo = dmel.dmel_frame_offsets(off)
+    F = int(fo[-1])
+    codes = torch.empty((F, 80), dtype=torch.uint8, device=DEV)
+    dmel.dmel_codes_q(torch.from_numpy(wav).to(DEV), torch.from_numpy(off).to(DEV), torch.from_numpy(fo).to(DEV), F,
+                      codes, quantizer=q)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy()
+
+
+def test_codes_q_default_is_dmel_codes():
+    wav, off = synth.batch64_10s(n_clips=16)
+    base, _ = _codes_gpu(wav, off)
+    assert (_codes_q_gpu(wav, off, None) == base).all()
+    assert (_codes_q_gpu(wav, off, (-7.0, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0)) == base).all()
+
+
+@pytest.mark.parametrize("q", QUANTS)
+def test_codes_q_variants_match_oracle(q, oracle_mod):
+    """The level mappings the pages leave open, on 16 clips of the batch workload (3,200 frames:
+    silence, clipped full scale, pink noise and chirps): equal to the oracle's codes except where
+    the oracle's log-mel value lies within 1e-4 of one of the variant's own boundaries."""
+    wav, off = synth.batch64_10s(n_clips=16)
+    got = _codes_q_gpu(wav, off, q)
+    oc, ol = oracle_mod.codes_q(wav, off, q)
+    flips, _ = compare_codes(got, oc, ol, boundaries=oracle_mod.level_boundaries_q(*q))
+    print(f"quantiser {q}: {flips} boundary flips of {oc.size} cells")
+
+
 # ------------------------------------------------------------------------- embedding
 
 @pytest.mark.parametrize("dim", [8, 24, 1000, 256, 512])
