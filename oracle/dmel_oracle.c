@@ -311,3 +311,41 @@ int oracle_embed(const uint8_t *codes, int64_t n_frames, const double *table, in
   }
   return bad ? -1 : 0;
 }
+
+/* ---- ShortConv ("Inside Inkling: Audio Design", Part 3 · Inference): per-channel causal
+ * convolution of width W = 4 with the input added back,
+ *     y[t, c] = x[t, c] + sum_{d=0}^{3} w[c, d] * x[t - d, c],
+ * over each sequence s of tokens [off[s], off[s+1]). Inputs before a sequence's first token
+ * come from its carried state (state[s][3 + j] = x[j] for j = -3, -2, -1; all zero without a
+ * state). state_out[s] receives the last three inputs the sequence ends with (taking them from
+ * the state in when the sequence is shorter than three). Everything in fp64. */
+int oracle_shortconv(const double *x, const int64_t *off, int n_seq, int C, const double *w, const double *state,
+                     double *y, double *state_out) {
+  for (int s = 0; s < n_seq; ++s) {
+    const int64_t t0 = off[s], T = off[s + 1] - off[s];
+    if (T < 0) return -1;
+    for (int64_t t = 0; t < T; ++t)
+      for (int c = 0; c < C; ++c) {
+        double acc = x[(t0 + t) * C + c];
+        for (int d = 0; d < 4; ++d) {
+          const int64_t j = t - d;
+          double xv;
+          if (j >= 0) xv = x[(t0 + j) * C + c];
+          else xv = state ? state[((int64_t)s * 3 + 3 + j) * C + c] : 0.0;
+          acc += w[c * 4 + d] * xv;
+        }
+        y[(t0 + t) * C + c] = acc;
+      }
+    if (state_out)
+      for (int i = 0; i < 3; ++i) {
+        const int64_t j = T - 3 + i; /* position of state row i relative to the sequence start */
+        for (int c = 0; c < C; ++c) {
+          double v;
+          if (j >= 0) v = x[(t0 + j) * C + c];
+          else v = state ? state[((int64_t)s * 3 + 3 + j) * C + c] : 0.0;
+          state_out[((int64_t)s * 3 + i) * C + c] = v;
+        }
+      }
+  }
+  return 0;
+}

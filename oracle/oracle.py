@@ -77,6 +77,8 @@ def lib():
         L.oracle_quantise_q.restype = c_int
         L.oracle_codes_q.argtypes = [vp, vp, c_int, vp, vp, c_i64, c_d, c_d, c_int, c_d, vp, vp]
         L.oracle_codes_q.restype = c_int
+        L.oracle_shortconv.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, vp]
+        L.oracle_shortconv.restype = c_int
         L.oracle_embed.argtypes = [vp, c_i64, vp, c_int, vp, c_d, vp]
         L.oracle_embed.restype = c_int
         _lib = L
@@ -308,3 +310,22 @@ def splice_plan(seq_len: int, sentinel_pos: list, frames_per_item: list):
         else:
             frame_rows[starts[entry[1]] + entry[2]] = row
     return token_pos, frame_rows, len(expanded), int(sum(frames_per_item))
+
+
+def shortconv(x: np.ndarray, seq_offsets, w: np.ndarray, state: np.ndarray | None = None):
+    """ShortConv of tokens x [T, C] split into sequences by seq_offsets [n + 1], weights
+    w [C, 4], carried states [n, 3, C] or None (zeros). Returns (y [T, C], state_out [n, 3, C]),
+    all fp64 ("Inside Inkling: Audio Design", Part 3 · Inference: y = x + sum_d w_d x_{t-d})."""
+    xx = np.ascontiguousarray(x, np.float64)
+    off = np.ascontiguousarray(seq_offsets, np.int64)
+    n = off.shape[0] - 1
+    C = xx.shape[1]
+    ww = np.ascontiguousarray(w, np.float64)
+    assert ww.shape == (C, 4)
+    st = None if state is None else np.ascontiguousarray(state, np.float64)
+    y = np.zeros_like(xx)
+    so = np.zeros((n, 3, C), np.float64)
+    rc = lib().oracle_shortconv(_ptr(xx), _ptr(off), n, C, _ptr(ww), _ptr(st), _ptr(y), _ptr(so))
+    if rc != 0:
+        raise ValueError("oracle_shortconv: bad offsets")
+    return y, so

@@ -456,3 +456,66 @@ def test_quant_serving_clamp_gain_shift_is_one_level(oracle_mod):
     assert np.max(np.abs((l1 - l0)[inner] - w)) < 1e-5
     safe = inner & (oracle_mod.boundary_distance_q(l0, q) > 1e-4)
     assert (c1[safe].astype(int) - c0[safe].astype(int) == 1).all()
+
+
+# ---------------------------------------------------------------- ShortConv (Part 3 · Inference)
+
+def _conv_numpy(x, w, hist):
+    """Per channel: numpy's full convolution of [history, x] with (1 + w0, w1, w2, w3), cut to
+    the positions of x (a library routine for the same causal filter)."""
+    T, C = x.shape
+    out = np.zeros((T, C))
+    for c in range(C):
+        h = np.array([1.0 + w[c, 0], w[c, 1], w[c, 2], w[c, 3]])
+        full = np.convolve(np.concatenate([hist[:, c], x[:, c]]), h)
+        out[:, c] = full[3:3 + T]
+    return out
+
+
+def test_shortconv_matches_numpy_convolution(oracle_mod):
+    r = np.random.default_rng(21)
+    C = 24
+    lens = [0, 1, 2, 3, 17, 5]
+    off = np.concatenate([[0], np.cumsum(lens)])
+    x = r.standard_normal((off[-1], C))
+    w = r.standard_normal((C, 4))
+    st = r.standard_normal((len(lens), 3, C))
+    y, so = oracle_mod.shortconv(x, off, w, st)
+    for s, T in enumerate(lens):
+        seg = x[off[s]:off[s + 1]]
+        np.testing.assert_allclose(y[off[s]:off[s + 1]], _conv_numpy(seg, w, st[s]), rtol=1e-12, atol=1e-12)
+        full = np.concatenate([st[s], seg])
+        np.testing.assert_array_equal(so[s], full[-3:])
+
+
+def test_shortconv_impulse_response_and_identity(oracle_mod):
+    C = 8
+    w = np.arange(C * 4, dtype=np.float64).reshape(C, 4) / 10.0
+    x = np.zeros((10, C))
+    x[4] = 1.0
+    y, _ = oracle_mod.shortconv(x, [0, 10], w)
+    # the impulse reappears with gain 1 + w0 at its own step and w_d d steps later
+    expect = np.zeros((10, C))
+    expect[4] = 1.0 + w[:, 0]
+    for d in (1, 2, 3):
+        expect[4 + d] = w[:, d]
+    np.testing.assert_array_equal(y, expect)
+    y0, _ = oracle_mod.shortconv(np.random.default_rng(2).standard_normal((7, C)), [0, 7], np.zeros((C, 4)))
+    x0 = np.random.default_rng(2).standard_normal((7, C))
+    np.testing.assert_array_equal(y0, x0)  # zero weights: the identity
+
+
+def test_shortconv_streaming_equals_offline(oracle_mod):
+    """Decoding token by token (or in chunks) with the carried state gives the offline result."""
+    r = np.random.default_rng(23)
+    C, T = 16, 29
+    x = r.standard_normal((T, C))
+    w = r.standard_normal((C, 4))
+    y_all, s_all = oracle_mod.shortconv(x, [0, T], w)
+    st = np.zeros((1, 3, C))
+    ys = []
+    for a, b in ((0, 1), (1, 2), (2, 9), (9, 9), (9, 10), (10, 29)):
+        yc, st = oracle_mod.shortconv(x[a:b], [0, b - a], w, st)
+        ys.append(yc)
+    np.testing.assert_allclose(np.concatenate(ys), y_all, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(st, s_all)
