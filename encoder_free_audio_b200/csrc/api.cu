@@ -232,6 +232,38 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                            workspace_bytes, stream);
 }
 
+dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq, int64_t n_tokens, int channels,
+                           const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
+                           dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (n_seq < 0 || n_tokens < 0 || channels <= 0 || channels % 8 != 0 || !dtype_ok(dtype)) return DMEL_ERR_INVALID_ARG;
+  if (n_seq == 0 && n_tokens > 0) return DMEL_ERR_INVALID_ARG;
+  if (n_seq == 0) return DMEL_OK;
+  if (!seq_offsets || !weights || !aligned(weights, 16)) return DMEL_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return DMEL_ERR_INVALID_ARG;
+  if ((state && !aligned(state, 16)) || (state_out && !aligned(state_out, 16))) return DMEL_ERR_INVALID_ARG;
+  const size_t es = dtype == DMEL_BF16 ? 2 : 4;
+  const size_t tok_bytes = (size_t)n_tokens * (size_t)channels * es;
+  const size_t st_bytes = (size_t)n_seq * 3 * (size_t)channels * es;
+  auto overlap = [](const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return a && b && na && nb && pa < pb + nb && pb < pa + na;
+  };
+  if (overlap(y, tok_bytes, x, tok_bytes) || overlap(y, tok_bytes, state, st_bytes) ||
+      overlap(y, tok_bytes, state_out, st_bytes) || overlap(state_out, st_bytes, x, tok_bytes))
+    return DMEL_ERR_INVALID_ARG;
+  if (state_out && state && state_out != state && overlap(state_out, st_bytes, state, st_bytes))
+    return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  cudaError_t e = launch_shortconv(x, seq_offsets, n_seq, n_tokens, channels, weights, state, state_out, y, dtype,
+                                   d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
 dmel_status dmel_splice_plan(const int64_t *h_sentinel_pos, int n_items, const int64_t *h_frame_offsets,
                              int64_t seq_len, int64_t *h_token_pos, int64_t *h_frame_rows,
                              int64_t *h_expanded_len, int64_t *h_audio_tokens) {

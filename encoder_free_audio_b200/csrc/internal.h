@@ -42,6 +42,13 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 // Device address of that scratch on the current device (looked up once per device).
 cudaError_t noalloc_scratch(void **ptr);
 
+// ShortConv of n_tokens tokens (sequences by device seq_offsets [n_seq + 1]) on `stream`: y, and
+// the carried state out when state_out != nullptr (may be the state in). Adds the kernels
+// launched to *launches.
+cudaError_t launch_shortconv(const void *x, const int64_t *seq_offsets, int n_seq, int64_t n_tokens, int channels,
+                             const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
+                             uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
+
 // Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
 cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);
 

@@ -80,6 +80,8 @@ def _lib():
         L.dmel_forward_rows.restype = i32
         L.dmel_splice_plan.argtypes = [vp, i32, vp, i64, vp, vp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
         L.dmel_splice_plan.restype = i32
+        L.dmel_shortconv.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp, vp, i32, vp]
+        L.dmel_shortconv.restype = i32
         L.dmel_embed_noalloc.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp]
         L.dmel_embed_noalloc.restype = i32
         L.dmel_get_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
@@ -237,6 +239,15 @@ def dmel_forward_rows(wav, sample_offsets, frame_offsets, n_frames: int, table, 
                                   _ptr(rms_weight), float(eps), _ptr(out), _ptr(out_rows), int(out.shape[0]),
                                   _dtype_code(out), _ptr(codes_out), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dmel_forward_rows")
+
+
+def dmel_shortconv(x, seq_offsets, weights, y, state=None, state_out=None, stream=None):
+    """dmel_shortconv on torch CUDA tensors: x and y [T, C] (fp32 or bf16), seq_offsets int64
+    [n + 1], weights fp32 [C, 4], state / state_out [n, 3, C] in x's dtype or None."""
+    n_seq = seq_offsets.shape[0] - 1
+    rc = _lib().dmel_shortconv(_ptr(x), _ptr(seq_offsets), n_seq, int(x.shape[0]), int(x.shape[1]), _ptr(weights),
+                               _ptr(state), _ptr(state_out), _ptr(y), _dtype_code(x), _stream(stream))
+    _check(rc, "dmel_shortconv")
 
 
 def dmel_splice_plan(sentinel_pos, frame_offsets, seq_len: int):

@@ -235,6 +235,26 @@ dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, c
                               const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, uint8_t *codes_out,
                               void *workspace, size_t workspace_bytes, dmel_stream_t stream);
 
+/* ---- ShortConv ("Inside Inkling: Audio Design", Part 3 · Inference: the decoder's per-channel
+ * causal convolutions of width W = 4, applied after the key/value projections and on the
+ * residual-branch outputs, with a small per-request convolution state):
+ *     y[t, c] = x[t, c] + sum_{d=0}^{3} weights[c * 4 + d] * x[t - d, c]
+ * within each sequence s of tokens [seq_offsets[s], seq_offsets[s + 1]).
+ * x            [n_tokens x channels] in dtype (fp32 or bf16), device, 16-byte aligned
+ * seq_offsets  device int64 [n_seq + 1], 0 = seq_offsets[0] <= ... <= seq_offsets[n_seq] = n_tokens
+ * channels     a positive multiple of 8
+ * weights      device fp32 [channels x 4], 16-byte aligned
+ * state        NULL (new requests: zeros before each sequence) or device [n_seq x 3 x channels] in
+ *              dtype: row 3 + j holds x[j] for j = -3, -2, -1 of sequence s
+ * state_out    NULL or [n_seq x 3 x channels]: the last three inputs each sequence ends with
+ *              (taken from the state where a sequence is shorter than three); may be state
+ * y            [n_tokens x channels] in dtype; must not overlap x or state
+ * Sums in fp32, y rounded to dtype (bf16: nearest even). Offsets that do not describe the token
+ * range read as zero inputs and set DMEL_DEVERR_OFFSETS. Asynchronous on stream. */
+dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq, int64_t n_tokens, int channels,
+                           const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
+                           dmel_stream_t stream);
+
 /* Reads (and, when clear != 0, clears) the device error word of the current device. This call
  * synchronises the device. *h_bits receives DMEL_DEVERR_* bits (0 = no error). */
 dmel_status dmel_get_device_error(uint32_t *h_bits, int clear);

@@ -202,3 +202,20 @@ def test_bad_quantisers_are_rejected_without_gpu(lib, q):
     qq = dmel.Quantizer(*q)
     assert lib.dmel_codes_q(fake, fake, fake, 1, 4, None, None, fake, ctypes.byref(qq),
                             None) == dmel.DMEL_ERR_INVALID_ARG
+
+
+def test_shortconv_argument_checks_without_gpu(lib):
+    vp = ctypes.c_void_p
+    a, b, c = vp(1 << 20), vp(1 << 24), vp(1 << 28)
+    S = lib.dmel_shortconv
+    # channels not a multiple of 8, negative sizes, tokens without sequences
+    assert S(a, a, 1, 10, 12, b, None, None, c, 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert S(a, a, -1, 10, 16, b, None, None, c, 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert S(a, a, 0, 10, 16, b, None, None, c, 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    # misaligned weights, missing output
+    assert S(a, a, 1, 10, 16, vp((1 << 24) + 4), None, None, c, 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert S(a, a, 1, 10, 16, b, None, None, None, 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    # y overlapping x (in place is not allowed)
+    assert S(a, a, 1, 10, 16, b, None, None, vp((1 << 20) + 64), 1, None) == dmel.DMEL_ERR_INVALID_ARG
+    # no sequences: a no-op
+    assert S(None, None, 0, 0, 16, None, None, None, None, 1, None) == dmel.DMEL_OK
