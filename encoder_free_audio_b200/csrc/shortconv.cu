@@ -100,7 +100,7 @@ __device__ __forceinline__ void sc_fetch(const T *x, const T *state, const int64
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kScThreads) shortconv_kernel(const T *__restrict__ x, const int64_t *__restrict__ off,
+__global__ void __launch_bounds__(kScThreads, 3) shortconv_kernel(const T *__restrict__ x, const int64_t *__restrict__ off,
                                                                int n_seq, int64_t n_tok, int C,
                                                                const float *__restrict__ w, const T *state,
                                                                T *__restrict__ y, uint32_t *err) {
