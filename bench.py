@@ -166,7 +166,7 @@ def streaming_latency(torch, dev, T, G, FrontEnd, dmel, warmup: int, calls: int 
             "tokens_per_s": S.n * calls / (sum(ms) / 1e3), "launches_per_call": dmel.dmel_last_launch_count()}
 
 
-def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20) -> dict:
+def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20, with_oracle: bool = False) -> dict:
     """ShortConv (the decoder's width-4 per-channel causal conv) over the batch's 12,800 frame
     vectors as 64 sequences of 200 tokens, bf16, with carried state in and out: HBM-bound, so
     reported against the measured copy bandwidth. Inputs larger than L2 are rotated between calls."""
@@ -190,10 +190,22 @@ def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20) 
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in evs) / steps
     algo = 2 * T * C * 2 + C * 16 + 2 * n_seq * 3 * C * 2  # x in, y out, weights, state in + out
-    return {"workload": "12,800 tokens x 6144 channels bf16, 64 sequences, state in/out", "us_per_call": ms * 1e3,
+    line = {"workload": "12,800 tokens x 6144 channels bf16, 64 sequences, state in/out", "us_per_call": ms * 1e3,
             "achieved_gbs": algo / (ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
             "frac": algo / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "bytes_per_call": algo,
             "launches_per_call": dmel.dmel_last_launch_count()}
+    if with_oracle:
+        # the oracle beside it: 8 of the 64 sequences on the host (fp64, one thread), as tokens/s
+        from oracle import oracle
+        xh = xs[0][: 8 * (T // n_seq)].float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.shortconv(xh, np.arange(0, xh.shape[0] + 1, T // n_seq), w.cpu().numpy(),
+                         st[:8].float().cpu().numpy())
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": xh.shape[0] / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"8 of 64 sequences ({xh.shape[0]} tokens x {C} channels)"}
+        line["tokens_per_s"] = T / (ms / 1e3)
+    return line
 
 
 def load_workload():
@@ -337,7 +349,8 @@ def run_ours(args):
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
     # ---------------------------------------------------------- streaming shape (context line)
     stream_line = streaming_latency(torch, dev, T, G, FrontEnd, dmel, args.warmup)
-    shortconv_line = shortconv_context(torch, dev, dmel, peaks(), args.warmup)
+    shortconv_line = shortconv_context(torch, dev, dmel, peaks(), args.warmup,
+                                       with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
     err_bits = dmel.dmel_get_device_error(clear=True)
 
     if rank != 0:

@@ -329,3 +329,68 @@ def shortconv(x: np.ndarray, seq_offsets, w: np.ndarray, state: np.ndarray | Non
     if rc != 0:
         raise ValueError("oracle_shortconv: bad offsets")
     return y, so
+
+
+# ---------------------------------------------------------------- hMLP patchifier (vision)
+
+HMLP_PATCH = 40
+HMLP_LN_EPS = 1e-6
+
+
+def _bf16(a: np.ndarray) -> np.ndarray:
+    """Round to bfloat16 (nearest even) and back to float64: the activations' storage type."""
+    a32 = np.ascontiguousarray(a, np.float32)
+    u = a32.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def _gelu(x: np.ndarray) -> np.ndarray:
+    from math import erf, sqrt
+    v = np.vectorize(lambda t: 0.5 * t * (1.0 + erf(t / sqrt(2.0))))
+    return v(x) if x.size else x
+
+
+def _layernorm(x: np.ndarray, g: np.ndarray, b: np.ndarray) -> np.ndarray:
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + HMLP_LN_EPS) * g + b
+
+
+def hmlp(images: np.ndarray, params: dict) -> np.ndarray:
+    """The hierarchical MLP patchifier ("Inside Inkling: Audio Design", Part 1 · Modeling: a
+    4-layer hMLP over 40x40 patches; "Why Thinking Machines Built Inkling Without a Vision
+    Encoder": linear layers progressively merge pixels into one embedding per patch), in fp64:
+      stage 1: every 5x5 pixel block, its 75 values in (row, column, channel) order, times W1 + b1
+      stages 2-4: every 2x2 group of the previous stage's grid, the four vectors concatenated in
+               (top-left, top-right, bottom-left, bottom-right) order, times Ws + bs
+    LayerNorm (eps 1e-6, gamma, beta) and the exact GELU follow stages 1-3; every stage's output
+    is stored in bf16 (the input to the next stage and the final embedding). images: [n, H, W, 3]
+    with H, W multiples of 40; returns [n * (H / 40) * (W / 40), D] with patches in raster order."""
+    n, H, W, ch = images.shape
+    assert ch == 3 and H % HMLP_PATCH == 0 and W % HMLP_PATCH == 0
+    out = []
+    for i in range(n):
+        for pr in range(H // HMLP_PATCH):
+            for pc in range(W // HMLP_PATCH):
+                patch = np.asarray(images[i, 40 * pr:40 * pr + 40, 40 * pc:40 * pc + 40, :], np.float64)
+                # stage 1: 8 x 8 grid of 5 x 5 blocks
+                grid = np.zeros((8, 8, params["W1"].shape[1]))
+                for br in range(8):
+                    for bc in range(8):
+                        v = patch[5 * br:5 * br + 5, 5 * bc:5 * bc + 5, :].reshape(-1)
+                        grid[br, bc] = v @ params["W1"] + params["b1"]
+                grid = _bf16(_gelu(_layernorm(grid, params["g1"], params["be1"])))
+                for s in (2, 3, 4):
+                    m = grid.shape[0] // 2
+                    nxt = np.zeros((m, m, params[f"W{s}"].shape[1]))
+                    for r in range(m):
+                        for c in range(m):
+                            v = np.concatenate([grid[2 * r, 2 * c], grid[2 * r, 2 * c + 1],
+                                                grid[2 * r + 1, 2 * c], grid[2 * r + 1, 2 * c + 1]])
+                            nxt[r, c] = v @ params[f"W{s}"] + params[f"b{s}"]
+                    if s < 4:
+                        nxt = _gelu(_layernorm(nxt, params[f"g{s}"], params[f"be{s}"]))
+                    grid = _bf16(nxt)
+                out.append(grid[0, 0])
+    return np.stack(out) if out else np.zeros((0, params["W4"].shape[1]))

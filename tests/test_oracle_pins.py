@@ -519,3 +519,63 @@ def test_shortconv_streaming_equals_offline(oracle_mod):
         ys.append(yc)
     np.testing.assert_allclose(np.concatenate(ys), y_all, rtol=0, atol=1e-12)
     np.testing.assert_array_equal(st, s_all)
+
+
+# ---------------------------------------------------------------- hMLP patchifier
+
+def _hmlp_params(r, d1, d2, d3, D):
+    p = {"W1": r.standard_normal((75, d1)) / np.sqrt(75), "b1": 0.1 * r.standard_normal(d1),
+         "g1": 1 + 0.1 * r.standard_normal(d1), "be1": 0.1 * r.standard_normal(d1),
+         "W2": r.standard_normal((4 * d1, d2)) / np.sqrt(4 * d1), "b2": 0.1 * r.standard_normal(d2),
+         "g2": 1 + 0.1 * r.standard_normal(d2), "be2": 0.1 * r.standard_normal(d2),
+         "W3": r.standard_normal((4 * d2, d3)) / np.sqrt(4 * d2), "b3": 0.1 * r.standard_normal(d3),
+         "g3": 1 + 0.1 * r.standard_normal(d3), "be3": 0.1 * r.standard_normal(d3),
+         "W4": r.standard_normal((4 * d3, D)) / np.sqrt(4 * d3), "b4": 0.1 * r.standard_normal(D)}
+    return p
+
+
+def test_hmlp_matches_strided_convolutions(oracle_mod):
+    """The hMLP as torch's conv2d with kernel = stride (5, 2, 2, 2), layer norm over channels and
+    the exact GELU, bf16 storage between stages: an independent formulation on the image grid."""
+    import torch
+    import torch.nn.functional as Fn
+    r = np.random.default_rng(31)
+    d1, d2, d3, D = 8, 12, 16, 24
+    p = _hmlp_params(r, d1, d2, d3, D)
+    img = oracle_mod._bf16(r.uniform(-1, 1, (2, 80, 120, 3)))
+    got = oracle_mod.hmlp(img, p)
+    x = torch.from_numpy(img).permute(0, 3, 1, 2)  # NCHW, float64
+    # stage 1 weight: row (5 kr + kc) * 3 + ch of W1 -> conv weight [out, ch, kr, kc]
+    w1 = torch.from_numpy(p["W1"].reshape(5, 5, 3, d1)).permute(3, 2, 0, 1)
+    def bf(t):
+        return torch.from_numpy(oracle_mod._bf16(t.numpy()))
+    def ln_gelu(t, g, b):
+        t = t.permute(0, 2, 3, 1)
+        t = Fn.layer_norm(t, (t.shape[-1],), torch.from_numpy(g), torch.from_numpy(b), eps=1e-6)
+        return Fn.gelu(t).permute(0, 3, 1, 2)
+    h = bf(ln_gelu(Fn.conv2d(x, w1, torch.from_numpy(p["b1"]), stride=5), p["g1"], p["be1"]))
+    for s, d_in in ((2, d1), (3, d2), (4, d3)):
+        d_out = p[f"W{s}"].shape[1]
+        # rows of Ws: child k = 2 kr + kc (tl, tr, bl, br), then its d_in channels
+        ws = torch.from_numpy(p[f"W{s}"].reshape(2, 2, d_in, d_out)).permute(3, 2, 0, 1)
+        h = Fn.conv2d(h, ws, torch.from_numpy(p[f"b{s}"]), stride=2)
+        h = bf(ln_gelu(h, p[f"g{s}"], p[f"be{s}"]) if s < 4 else h)
+    ref = h.permute(0, 2, 3, 1).reshape(-1, D).numpy()  # patches in raster order
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-2 * np.abs(ref).max())
+    # away from bf16 rounding ties the two agree to the last bit of the storage type
+    assert (np.abs(got - ref) <= 2 ** -7 * np.maximum(np.abs(ref), 1e-3)).mean() > 0.99
+
+
+def test_hmlp_closed_forms(oracle_mod):
+    r = np.random.default_rng(32)
+    d1, d2, d3, D = 4, 4, 4, 6
+    p = _hmlp_params(r, d1, d2, d3, D)
+    p["W4"][:] = 0.0  # the last stage ignores its input: every patch is b4 (rounded to bf16)
+    img = r.uniform(-1, 1, (1, 40, 80, 3))
+    out = oracle_mod.hmlp(img, p)
+    np.testing.assert_array_equal(out, np.tile(oracle_mod._bf16(p["b4"]), (2, 1)))
+    # patches are independent: swapping the two 40 x 40 halves swaps the outputs
+    p2 = _hmlp_params(r, d1, d2, d3, D)
+    a = oracle_mod.hmlp(img, p2)
+    b = oracle_mod.hmlp(np.concatenate([img[:, :, 40:], img[:, :, :40]], axis=2), p2)
+    np.testing.assert_array_equal(a, b[::-1])
