@@ -208,6 +208,55 @@ def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20, 
     return line
 
 
+def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_oracle: bool = False) -> dict:
+    """The hMLP patchifier of the vision path on 4 images of 800 x 800 (1,600 patches of 40 x 40),
+    widths 1536 / 1536 / 1536 / 6144, bf16, synthetic weights: dense GEMMs, so reported against the
+    sustained bf16 tensor peak."""
+    n, H, W = 4, 800, 800
+    d1 = d2 = d3 = DIM // 4
+    g = torch.Generator(device=dev).manual_seed(11)
+    def rn(*shape, scale=1.0):
+        return (scale * torch.randn(shape, device=dev, generator=g)).contiguous()
+    params = {"W1": rn(75, d1, scale=75 ** -0.5).to(torch.bfloat16), "W2": rn(4 * d1, d2, scale=(4 * d1) ** -0.5).to(
+        torch.bfloat16), "W3": rn(4 * d2, d3, scale=(4 * d2) ** -0.5).to(torch.bfloat16),
+        "W4": rn(4 * d3, DIM, scale=(4 * d3) ** -0.5).to(torch.bfloat16)}
+    for k, d in (("b1", d1), ("b2", d2), ("b3", d3), ("b4", DIM)):
+        params[k] = rn(d, scale=0.1)
+    for s_, d in ((1, d1), (2, d2), (3, d3)):
+        params[f"g{s_}"] = (1 + rn(d, scale=0.1)).contiguous()
+        params[f"be{s_}"] = rn(d, scale=0.1)
+    img = rn(n, H, W, 3).clamp(-1, 1).to(torch.bfloat16).contiguous()
+    P = n * (H // 40) * (W // 40)
+    out = torch.empty((P, DIM), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(dmel.dmel_hmlp_workspace_size(P, params), dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        dmel.dmel_hmlp(img, params, out, ws)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    s = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    for k in range(steps):
+        evs[k][0].record(s)
+        dmel.dmel_hmlp(img, params, out, ws)
+        evs[k][1].record(s)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / steps
+    flop = 2 * P * (64 * 75 * d1 + 16 * 4 * d1 * d2 + 4 * 4 * d2 * d3 + 4 * d3 * DIM)
+    line = {"workload": "4 images 800x800 bf16 = 1,600 patches, widths 1536/1536/1536/6144", "us_per_call": ms * 1e3,
+            "patches_per_s": P / (ms / 1e3), "achieved_tflops": flop / (ms / 1e3) / 1e12,
+            "peak_tflops": pk["bf16_tflops_sustained"],
+            "frac": flop / (ms / 1e3) / 1e12 / pk["bf16_tflops_sustained"], "flop_per_call": flop,
+            "launches_per_call": dmel.dmel_last_launch_count(), "gemms": "4 cuBLASLt calls per invocation"}
+    if with_oracle:
+        from oracle import oracle
+        host = {k: v.double().cpu().numpy() for k, v in params.items()}
+        t0 = time.perf_counter()
+        oracle.hmlp(img[:1, :40, :40].double().cpu().numpy(), host)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": 1.0 / dt, "unit": "patches/s", "cores": 1, "kind": "oracle",
+                                "sample": "1 patch of 40 x 40"}
+    return line
+
+
 def load_workload():
     from encoder_free_audio_b200 import synth
     wav, off = synth.batch64_10s()
@@ -351,6 +400,8 @@ def run_ours(args):
     stream_line = streaming_latency(torch, dev, T, G, FrontEnd, dmel, args.warmup)
     shortconv_line = shortconv_context(torch, dev, dmel, peaks(), args.warmup,
                                        with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    hmlp_line = hmlp_context(torch, dev, dmel, peaks(), args.warmup,
+                             with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
     err_bits = dmel.dmel_get_device_error(clear=True)
 
     if rank != 0:
@@ -397,6 +448,7 @@ def run_ours(args):
         "stages_ms": {"codes": statistics.mean(codes_ms), "embed": statistics.mean(embed_ms)},
         "streaming": stream_line,
         "shortconv": shortconv_line,
+        "hmlp": hmlp_line,
         "device_error_bits": err_bits,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -264,6 +264,45 @@ dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq,
   return from_cuda(e);
 }
 
+namespace {
+bool hmlp_weights_ok(const dmel_hmlp_weights *w) {
+  if (!w) return false;
+  const int dims[4] = {w->d1, w->d2, w->d3, w->dim};
+  for (int d : dims)
+    if (d <= 0 || d % 8 != 0) return false;
+  const void *ptrs[14] = {w->w1, w->w2, w->w3, w->w4, w->b1, w->b2, w->b3, w->b4,
+                          w->g1, w->g2, w->g3, w->be1, w->be2, w->be3};
+  for (const void *p : ptrs)
+    if (!p || !aligned(p, 16)) return false;
+  return true;
+}
+}  // namespace
+
+size_t dmel_hmlp_workspace_size(int64_t n_patches, const dmel_hmlp_weights *w) {
+  if (n_patches <= 0 || !hmlp_weights_ok(w)) return 0;
+  return hmlp_workspace_bytes(n_patches, *w);
+}
+
+dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, const dmel_hmlp_weights *w, void *out,
+                      void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (n_images < 0 || height < 0 || width < 0 || height % 40 != 0 || width % 40 != 0) return DMEL_ERR_INVALID_ARG;
+  if (!hmlp_weights_ok(w)) return DMEL_ERR_INVALID_ARG;
+  const int64_t P = (int64_t)n_images * (height / 40) * (width / 40);
+  if (P == 0) return DMEL_OK;
+  if (!images || !out || !aligned(images, 16) || !aligned(out, 16)) return DMEL_ERR_INVALID_ARG;
+  const size_t need = hmlp_workspace_bytes(P, *w);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  cudaError_t e = launch_hmlp(images, n_images, height, width, *w, out, workspace, d.sms,
+                              reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
 dmel_status dmel_splice_plan(const int64_t *h_sentinel_pos, int n_items, const int64_t *h_frame_offsets,
                              int64_t seq_len, int64_t *h_token_pos, int64_t *h_frame_rows,
                              int64_t *h_expanded_len, int64_t *h_audio_tokens) {

@@ -49,6 +49,12 @@ cudaError_t launch_shortconv(const void *x, const int64_t *seq_offsets, int n_se
                              const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
                              uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
 
+// hMLP patchifier: workspace bytes for n_patches, and the launch (gather, four cuBLASLt GEMMs,
+// four row kernels) on `stream`.
+size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w);
+cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp_weights &w, void *out,
+                        void *workspace, int num_sms, cudaStream_t stream, int *launches);
+
 // Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
 cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);
 

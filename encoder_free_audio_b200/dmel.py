@@ -80,6 +80,10 @@ def _lib():
         L.dmel_forward_rows.restype = i32
         L.dmel_splice_plan.argtypes = [vp, i32, vp, i64, vp, vp, ctypes.POINTER(i64), ctypes.POINTER(i64)]
         L.dmel_splice_plan.restype = i32
+        L.dmel_hmlp_workspace_size.argtypes = [i64, ctypes.POINTER(HmlpWeights)]
+        L.dmel_hmlp_workspace_size.restype = sz
+        L.dmel_hmlp.argtypes = [vp, i32, i32, i32, ctypes.POINTER(HmlpWeights), vp, vp, sz, vp]
+        L.dmel_hmlp.restype = i32
         L.dmel_shortconv.argtypes = [vp, vp, i32, i64, i32, vp, vp, vp, vp, i32, vp]
         L.dmel_shortconv.restype = i32
         L.dmel_embed_noalloc.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp]
@@ -165,6 +169,34 @@ def dmel_codes(wav, sample_offsets, frame_offsets, n_frames: int, codes, tails=N
     rc = _lib().dmel_codes(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames), _ptr(tails),
                            _ptr(tails_out), _ptr(codes), _stream(stream))
     _check(rc, "dmel_codes")
+
+
+class HmlpWeights(ctypes.Structure):
+    """dmel_hmlp_weights: widths and device pointers of the hMLP patchifier's parameters."""
+    _fields_ = [("d1", ctypes.c_int), ("d2", ctypes.c_int), ("d3", ctypes.c_int), ("dim", ctypes.c_int)] + \
+               [(k, ctypes.c_void_p) for k in ("w1", "w2", "w3", "w4", "b1", "b2", "b3", "b4", "g1", "g2", "g3",
+                                              "be1", "be2", "be3")]
+
+
+def hmlp_weights(params: dict) -> HmlpWeights:
+    """HmlpWeights of torch CUDA tensors: W1..W4 bf16 [75 x d1], [4 d1 x d2], [4 d2 x d3],
+    [4 d3 x dim]; b1..b4, g1..g3, be1..be3 fp32."""
+    d = [int(params[f"W{s}"].shape[1]) for s in (1, 2, 3, 4)]
+    return HmlpWeights(*d, *[_ptr(params[k]) for k in ("W1", "W2", "W3", "W4", "b1", "b2", "b3", "b4", "g1", "g2",
+                                                          "g3", "be1", "be2", "be3")])
+
+
+def dmel_hmlp_workspace_size(n_patches: int, params: dict) -> int:
+    return int(_lib().dmel_hmlp_workspace_size(int(n_patches), ctypes.byref(hmlp_weights(params))))
+
+
+def dmel_hmlp(images, params: dict, out, workspace, stream=None):
+    """dmel_hmlp on torch CUDA tensors: images bf16 [n, H, W, 3], out bf16 [patches, dim]."""
+    n, H, W, _ = images.shape
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_hmlp(_ptr(images), int(n), int(H), int(W), ctypes.byref(hmlp_weights(params)), _ptr(out),
+                          _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_hmlp")
 
 
 def _quantizer(q):

@@ -255,6 +255,33 @@ dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq,
                            const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
                            dmel_stream_t stream);
 
+/* ---- hMLP patchifier (vision; "Inside Inkling: Audio Design", Part 1 · Modeling: a 4-layer
+ * hMLP over 40x40 patches; "Why Thinking Machines Built Inkling Without a Vision Encoder":
+ * linear layers progressively merge pixels into one embedding per patch). The pages give no
+ * widths: the caller chooses them. Stage 1 maps every 5x5 pixel block of a patch (75 values in
+ * row, column, channel order) to d1 features; stages 2, 3, 4 map every 2x2 group of the previous
+ * stage's grid (the four vectors concatenated top-left, top-right, bottom-left, bottom-right) to
+ * d2, d3 and dim features. Bias, LayerNorm (eps 1e-6, gain, shift) and the exact GELU follow
+ * stages 1-3, bias alone stage 4; every stage's output is stored in bf16, products sum in fp32. */
+typedef struct {
+  int d1, d2, d3, dim;            /* stage widths, each a positive multiple of 8 */
+  const void *w1, *w2, *w3, *w4;  /* bf16 row-major [75 x d1], [4 d1 x d2], [4 d2 x d3], [4 d3 x dim] */
+  const float *b1, *b2, *b3, *b4; /* fp32 biases [d1], [d2], [d3], [dim] */
+  const float *g1, *g2, *g3;      /* fp32 LayerNorm gains [d1], [d2], [d3] */
+  const float *be1, *be2, *be3;   /* fp32 LayerNorm shifts */
+} dmel_hmlp_weights;              /* all device pointers, 16-byte aligned */
+
+/* Bytes of device workspace dmel_hmlp needs for n_patches patches (0 when none). */
+size_t dmel_hmlp_workspace_size(int64_t n_patches, const dmel_hmlp_weights *w);
+
+/* images   bf16 [n_images x height x width x 3] (channel last), device, 16-byte aligned;
+ *          height and width multiples of 40
+ * out      bf16 [n_images * (height / 40) * (width / 40) x dim], patches in raster order
+ * The four products run as dense bf16 GEMMs (cuBLASLt); gathering the pixel blocks and the bias,
+ * LayerNorm and GELU between them run in the library's kernels. Asynchronous on stream. */
+dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, const dmel_hmlp_weights *w, void *out,
+                      void *workspace, size_t workspace_bytes, dmel_stream_t stream);
+
 /* Reads (and, when clear != 0, clears) the device error word of the current device. This call
  * synchronises the device. *h_bits receives DMEL_DEVERR_* bits (0 = no error). */
 dmel_status dmel_get_device_error(uint32_t *h_bits, int clear);

@@ -219,3 +219,28 @@ def test_shortconv_argument_checks_without_gpu(lib):
     assert S(a, a, 1, 10, 16, b, None, None, vp((1 << 20) + 64), 1, None) == dmel.DMEL_ERR_INVALID_ARG
     # no sequences: a no-op
     assert S(None, None, 0, 0, 16, None, None, None, None, 1, None) == dmel.DMEL_OK
+
+
+def test_hmlp_argument_checks_without_gpu(lib):
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)
+    w = dmel.HmlpWeights(16, 16, 16, 32, *([a] * 14))
+    H = lib.dmel_hmlp
+    # height / width not multiples of 40
+    assert H(a, 1, 40, 50, ctypes.byref(w), a, a, 1 << 30, None) == dmel.DMEL_ERR_INVALID_ARG
+    # a width that is not a multiple of 8, a missing or misaligned parameter
+    bad = dmel.HmlpWeights(16, 12, 16, 32, *([a] * 14))
+    assert H(a, 1, 40, 40, ctypes.byref(bad), a, a, 1 << 30, None) == dmel.DMEL_ERR_INVALID_ARG
+    miss = dmel.HmlpWeights(16, 16, 16, 32, *([a] * 13 + [None]))
+    assert H(a, 1, 40, 40, ctypes.byref(miss), a, a, 1 << 30, None) == dmel.DMEL_ERR_INVALID_ARG
+    odd = dmel.HmlpWeights(16, 16, 16, 32, *([vp((1 << 20) + 4)] + [a] * 13))
+    assert H(a, 1, 40, 40, ctypes.byref(odd), a, a, 1 << 30, None) == dmel.DMEL_ERR_INVALID_ARG
+    # no workspace for a real request
+    assert H(a, 1, 40, 40, ctypes.byref(w), a, None, 0, None) == dmel.DMEL_ERR_INVALID_ARG
+    # the workspace grows with the patch count and covers the fp32 stage outputs
+    n1 = lib.dmel_hmlp_workspace_size(1, ctypes.byref(w))
+    n10 = lib.dmel_hmlp_workspace_size(10, ctypes.byref(w))
+    assert 0 < n1 < n10 and n10 >= 10 * 64 * 16 * 4
+    assert lib.dmel_hmlp_workspace_size(0, ctypes.byref(w)) == 0
+    # no image: a no-op
+    assert H(None, 0, 40, 40, ctypes.byref(w), None, None, 0, None) == dmel.DMEL_OK
