@@ -245,7 +245,8 @@ def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_
             "patches_per_s": P / (ms / 1e3), "achieved_tflops": flop / (ms / 1e3) / 1e12,
             "peak_tflops": pk["bf16_tflops_sustained"],
             "frac": flop / (ms / 1e3) / 1e12 / pk["bf16_tflops_sustained"], "flop_per_call": flop,
-            "launches_per_call": dmel.dmel_last_launch_count(), "gemms": "4 cuBLASLt calls per invocation"}
+            "launches_per_call": dmel.dmel_last_launch_count(),
+            "gemms": "stage 1 in one tcgen05 kernel; stages 2-4 as 3 cuBLASLt calls per invocation"}
     if with_oracle:
         from oracle import oracle
         host = {k: v.double().cpu().numpy() for k, v in params.items()}
@@ -397,11 +398,20 @@ def run_ours(args):
     barrier()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
     # ---------------------------------------------------------- streaming shape (context line)
+    # each context line runs inside an NVTX range of its name, so a profiler can list its launches
+    # alone (ncu --nvtx --nvtx-include "hmlp/")
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push("streaming")
     stream_line = streaming_latency(torch, dev, T, G, FrontEnd, dmel, args.warmup)
+    nvtx.range_pop()
+    nvtx.range_push("shortconv")
     shortconv_line = shortconv_context(torch, dev, dmel, peaks(), args.warmup,
                                        with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    nvtx.range_pop()
+    nvtx.range_push("hmlp")
     hmlp_line = hmlp_context(torch, dev, dmel, peaks(), args.warmup,
                              with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    nvtx.range_pop()
     err_bits = dmel.dmel_get_device_error(clear=True)
 
     if rank != 0:

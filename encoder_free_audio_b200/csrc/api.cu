@@ -297,7 +297,7 @@ dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, c
   if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
   if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
   int launches = 0;
-  cudaError_t e = launch_hmlp(images, n_images, height, width, *w, out, workspace, d.sms,
+  cudaError_t e = launch_hmlp(images, n_images, height, width, *w, out, workspace, d.err, d.sms,
                               reinterpret_cast<cudaStream_t>(stream), &launches);
   t_last_launches = launches;
   return from_cuda(e);
@@ -394,6 +394,18 @@ dmel_status dmel_debug_codes_frame_host_q(const float *frame1600, const dmel_qua
   if (!frame1600 || !codes80 || !to_quant(q, &qz)) return DMEL_ERR_INVALID_ARG;
   emulate_codes_frame_host(frame1600, codes80, lhat80, qz);
   return DMEL_OK;
+}
+
+dmel_status dmel_debug_gelu(const float *x, float *y, int64_t n, dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (n < 0) return DMEL_ERR_INVALID_ARG;
+  if (n == 0) return DMEL_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  t_last_launches = 1;
+  return from_cuda(launch_gelu_debug(x, y, n, d.sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 void dmel_debug_codes_frame_host(const float *frame1600, uint8_t *codes80, double *lhat80) {

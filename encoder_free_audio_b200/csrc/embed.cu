@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(tc::THREADS, 1)
                     const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace tc;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, as an offset from the shared array (keeps the shared address space)
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   const uint32_t bar0 = smem_addr(bars);
@@ -604,7 +605,8 @@ __global__ void __launch_bounds__(tc2::THREADS, 1)
                      const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace tc2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, as an offset from the shared array (keeps the shared address space)
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -1001,7 +1003,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
                     const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
   using namespace sp;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, as an offset from the shared array (keeps the shared address space)
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -1362,9 +1365,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
 EncodeTiledFn encode_tiled_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -1378,6 +1379,8 @@ EncodeTiledFn encode_tiled_fn() {
   });
   return fn;
 }
+
+namespace {
 
 template <typename K>
 cudaError_t set_smem_attr_once(K kernel, int bytes, bool *flags) {

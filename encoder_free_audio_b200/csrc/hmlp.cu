@@ -4,14 +4,15 @@
 // Stage 1 maps every 5x5 pixel block (75 values, row / column / channel order) to d1 features;
 // stages 2-4 map every 2x2 group of the previous stage's grid (four vectors concatenated in
 // top-left, top-right, bottom-left, bottom-right order) to d2, d3 and finally dim features.
-// Bias, LayerNorm (eps 1e-6) and the exact GELU follow stages 1-3, bias alone stage 4; every
-// stage's output is stored in bf16.
+// Bias, LayerNorm (eps 1e-6) and GELU follow stages 1-3, bias alone stage 4; every stage's
+// output is stored in bf16.
 //
 // Within a patch the blocks are kept in Morton (quad-tree) order, so the four children of a
 // 2x2 group are four consecutive rows and every merge is the previous stage's output read as
-// [rows / 4 x 4 d]: no data moves between stages. The four products are plain dense GEMMs
-// (cuBLASLt, bf16 x bf16 -> fp32); the pixel gather and the fused bias / LayerNorm / GELU /
-// rounding run in this file's kernels.
+// [rows / 4 x 4 d]: no data moves between stages. Stage 1 runs as one tcgen05 kernel (pixel
+// gather, K = 80 product, LayerNorm and GELU in its epilogue) when d1 is a multiple of 256 up to
+// 1536, else as a gather, a cuBLASLt GEMM and a row kernel; stages 2-4 are cuBLASLt GEMMs
+// (bf16 x bf16 -> fp32) followed by this file's bias / LayerNorm / GELU / rounding row kernel.
 #include <cublasLt.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -55,8 +56,36 @@ __global__ void __launch_bounds__(256) hmlp_gather_kernel(const __nv_bfloat16 *_
   }
 }
 
+// GELU(u) = u * Phi(u), Phi the standard normal distribution function, with
+// Phi(u) = 1 - erfc(u / sqrt 2) / 2 for u >= 0 and erfc(|u| / sqrt 2) / 2 for u < 0, and erfc(z)
+// for z >= 0 from Abramowitz & Stegun, Handbook of Mathematical Functions, formula 7.1.26
+// (Hastings): erfc(z) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2), t = 1 / (1 + p z),
+// absolute error at most 1.5e-7. One reciprocal and one exp2 on the special-function unit.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// With h = erfc(|u| / sqrt 2) / 2, GELU(u) = max(u, 0) - |u| h for either sign of u; the 1/2
+// is folded into the coefficients and 1/sqrt 2 into p.
+__device__ __forceinline__ float gelu_erf(float u) {
+  constexpr float kPr = 0.3275911f * 0.70710678118654752f;  // p / sqrt 2: t = 1 / (1 + p |u| / sqrt 2)
+  constexpr float kH1 = 0.5f * 0.254829592f, kH2 = 0.5f * -0.284496736f, kH3 = 0.5f * 1.421413741f,
+                  kH4 = 0.5f * -1.453152027f, kH5 = 0.5f * 1.061405429f;
+  constexpr float kNegHalfLog2e = -0.72134752044448170f;  // exp(-u^2 / 2) = 2^(u^2 * this)
+  const float t = rcp_approx(fmaf(kPr, fabsf(u), 1.0f));
+  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, kH5, kH4), kH3), kH2), kH1);
+  const float h = poly * ex2_approx(u * (u * kNegHalfLog2e));
+  return fmaf(-fabsf(u), h, fmaxf(u, 0.0f));
+}
+
 // One warp per row of d fp32 sums: + bias, then (kNorm) LayerNorm with gain / shift and the
-// exact GELU, rounded to bf16. Mean first, then the mean squared deviation (two passes).
+// GELU, rounded to bf16. Mean first, then the mean squared deviation (two passes).
 template <bool kNorm>
 __global__ void __launch_bounds__(256) hmlp_row_kernel(const float *__restrict__ in, int64_t rows, int d,
                                                        const float *__restrict__ bias, const float *__restrict__ g,
@@ -93,10 +122,7 @@ __global__ void __launch_bounds__(256) hmlp_row_kernel(const float *__restrict__
         const float4 gg = *reinterpret_cast<const float4 *>(g + j), bb = *reinterpret_cast<const float4 *>(be + j);
         const float gv[4] = {gg.x, gg.y, gg.z, gg.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float u = (t[k] - mean) * rstd * gv[k] + bv[k];
-          t[k] = 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
-        }
+        for (int k = 0; k < 4; ++k) t[k] = gelu_erf((t[k] - mean) * rstd * gv[k] + bv[k]);
       }
       __nv_bfloat162 lo = __floats2bfloat162_rn(t[0], t[1]), hi = __floats2bfloat162_rn(t[2], t[3]);
       uint2 pk;
@@ -104,6 +130,436 @@ __global__ void __launch_bounds__(256) hmlp_row_kernel(const float *__restrict__
       pk.y = *reinterpret_cast<uint32_t *>(&hi);
       *reinterpret_cast<uint2 *>(y + j) = pk;
     }
+  }
+}
+
+// Debug: y = GELU(x) with the kernels' formula, one thread per value.
+__global__ void hmlp_gelu_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = gelu_erf(x[i]);
+}
+
+// ---------------------------------------------------------------- stage 1, fused (tcgen05)
+//
+// One tile is two patches = 128 pixel blocks (TMEM lanes). Four gather warps copy the tile's
+// pixels (two patches of 40 rows x 240 bytes) into shared memory and build the 128 x 80 bf16
+// operand A there (K-major, 128-byte swizzle; values 64..79 in a second K block). A TMA warp
+// streams W1 (padded to 80 rows) in chunks of 256 columns; one thread issues the
+// 128 x 256 x 80 products into a double-buffered TMEM accumulator. The LayerNorm needs the
+// whole row of d1 sums, which does not fit in TMEM, so each tile runs its d1 / 256 chunks
+// twice: the first pass gives the row statistics (mean and sum of squared deviations per
+// 32 values, merged pairwise), the second recomputes the same sums and writes
+// bf16(GELU(LayerNorm(x + b1))). The product is tiny (K = 80), so the second pass costs far
+// less than storing and re-reading the fp32 sums.
+namespace s1 {
+constexpr int BM = 128;                 // pixel blocks per tile (two patches)
+constexpr int BN = 256;                 // columns per accumulator job
+constexpr int KP = 80;                  // K: 75 values + 5 zeros
+constexpr int A_KB = BM * 128;          // one 64-wide K block of A: 128 rows x 128 B
+constexpr int A_STAGE = 2 * A_KB;       // K blocks 0 (values 0..63) and 1 (values 64..79)
+constexpr int A_SLOTS = 2;
+constexpr int B_BOX = KP * 128;         // 80 K-rows x 64 columns
+constexpr int B_STAGE = (BN / 64) * B_BOX;
+constexpr int B_STAGES = 2;
+constexpr int STG_ROW = 240;            // bytes of one patch row (40 pixels x 3 x bf16)
+constexpr int STG = 2 * kPatch * STG_ROW;
+#ifndef HMLP_S1_EPI_WARPS
+#define HMLP_S1_EPI_WARPS 8
+#endif
+#ifndef HMLP_S1_BATCH
+#define HMLP_S1_BATCH 32
+#endif
+constexpr int EPI_WARPS = HMLP_S1_EPI_WARPS;  // EPI_WARPS / 4 per TMEM lane quadrant
+constexpr int BATCH = HMLP_S1_BATCH;          // columns per TMEM load in the epilogue
+constexpr int EPI_PARTS = EPI_WARPS / 4;
+constexpr int EPI_COLS = BN / EPI_PARTS;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr int THREADS = 32 * (6 + EPI_WARPS);
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + A_SLOTS * A_STAGE;
+constexpr int OFF_OUT = OFF_B + B_STAGES * B_STAGE;
+// output staging: per epilogue warp two buffers of 32 rows x BATCH bf16 (64-byte swizzle),
+// written to global memory by TMA bulk stores
+constexpr int OUT_BUF = 32 * BATCH * 2;
+constexpr int OFF_STG = OFF_OUT + EPI_WARPS * 2 * OUT_BUF;
+constexpr int OFF_STAT = OFF_STG + STG;  // [parts][128 rows] (mean, M2)
+constexpr int OFF_BAR = OFF_STAT + EPI_PARTS * BM * 8;
+constexpr int N_BARS = 2 * B_STAGES + 2 * A_SLOTS + 4 + 1;
+constexpr int MAX_D1 = 1536;            // b1, g1, be1 of up to this many columns staged in shared memory
+constexpr int OFF_PAR = OFF_BAR + 256;
+constexpr int SMEM_USED = OFF_PAR + 3 * MAX_D1 * 4;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(N_BARS * 8 + 4 <= 256, "barrier area");
+static_assert((EPI_PARTS == 2 || EPI_PARTS == 4) && BATCH == 32 && EPI_COLS % BATCH == 0, "epilogue split");
+static_assert(OFF_OUT % 1024 == 0 && OUT_BUF % 512 == 0, "64-byte swizzle atoms of the output staging");
+static_assert(B_STAGE % 1024 == 0 && A_KB % 1024 == 0 && OFF_B % 1024 == 0, "swizzle atoms stay 1024-B aligned");
+}  // namespace s1
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(s1::EPI_THREADS) : "memory"); }
+
+// Barrier of a named group that also ANDs a flag across it, so the whole group takes the same
+// branch after a bounded wait.
+template <int kId, int kCount>
+__device__ __forceinline__ bool group_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"((uint32_t)v), "n"(kId), "n"(kCount)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ void gather_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// TMA bulk tensor store of a 2D box from shared memory (no multicast), and its bulk-group
+// bookkeeping: commit, wait until the source may be overwritten (.read) or until done.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int32_t x, int32_t y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// BATCH consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld_batch(uint32_t taddr, float (&x)[s1::BATCH]) {
+  uint32_t a[16];
+  tmem_ld16(taddr, a);
+  if constexpr (s1::BATCH == 32) {
+    uint32_t b[16];
+    tmem_ld16(taddr + 16, b);
+    tmem_wait_ld();
+#pragma unroll
+    for (int k = 0; k < 16; ++k) x[16 + k] = __uint_as_float(b[k]);
+  } else {
+    tmem_wait_ld();
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) x[k] = __uint_as_float(a[k]);
+}
+
+__global__ void __launch_bounds__(s1::THREADS, 1)
+    hmlp_stage1_kernel(const __grid_constant__ CUtensorMap w1map, const __grid_constant__ CUtensorMap omap,
+                       const __nv_bfloat16 *__restrict__ img, int H, int W, int64_t P, int d1,
+                       const float *__restrict__ b1, const float *__restrict__ g1, const float *__restrict__ be1,
+                       uint32_t *err) {
+  using namespace s1;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base, as an offset from the shared array (keeps the shared address space)
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bar0 = smem_addr(smem + OFF_BAR);
+  auto full_b = [&](int s) { return bar0 + 8u * s; };
+  auto empty_b = [&](int s) { return bar0 + 8u * (B_STAGES + s); };
+  auto full_a = [&](int s) { return bar0 + 8u * (2 * B_STAGES + s); };
+  auto empty_a = [&](int s) { return bar0 + 8u * (2 * B_STAGES + A_SLOTS + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * B_STAGES + 2 * A_SLOTS + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * B_STAGES + 2 * A_SLOTS + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (N_BARS - 1);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+
+  const int NC = d1 / BN;                      // column chunks per row
+  float *par = reinterpret_cast<float *>(smem + OFF_PAR);  // b1 | g1 | be1
+  for (int i = threadIdx.x; i < d1; i += blockDim.x) {
+    par[i] = b1[i];
+    par[d1 + i] = g1[i];
+    par[2 * d1 + i] = be1[i];
+  }
+  const int64_t n_tiles = (P + 1) / 2;
+  const int64_t rows1 = P * kBlocks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < B_STAGES; ++s) {
+      mbar_init(full_b(s), 1);
+      mbar_init(empty_b(s), 1);
+    }
+    for (int s = 0; s < A_SLOTS; ++s) {
+      mbar_init(full_a(s), 128);
+      mbar_init(empty_a(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), EPI_THREADS);
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&w1map);
+    tma_prefetch_desc(&omap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA: W1 chunks, 2 NC per tile
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, pending = 0, pending_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < n_tiles; t += gridDim.x) {
+        for (int j = 0; j < 2 * NC; ++j) {
+          if (!mbar_wait(empty_b(stage), phase ^ 1u, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_b(stage), B_STAGE);
+          const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
+          const int c0 = (j % NC) * BN;
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q) tma_load_2d(dst + q * B_BOX, &w1map, c0 + 64 * q, 0, full_b(stage), pol);
+          pending |= 1u << stage;
+          pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == B_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int s = 0; s < B_STAGES; ++s)
+        if (pending & (1u << s)) mbar_wait(full_b(s), (pending_phase >> s) & 1u, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 1);
+      int stage = 0;
+      uint32_t phase = 0, g = 0;
+      bool ok = true;
+      uint32_t it = 0;
+      for (int64_t t = blockIdx.x; ok && t < n_tiles; t += gridDim.x, ++it) {
+        const uint32_t slot = it & 1u;
+        if (!mbar_wait(full_a(slot), (it >> 1) & 1u, err)) break;
+        const uint32_t a0 = smem_addr(smem + OFF_A + slot * A_STAGE);
+        for (int j = 0; j < 2 * NC; ++j, ++g) {
+          const uint32_t acc = g & 1u;
+          if (!mbar_wait(tempty(acc), ((g >> 1) & 1u) ^ 1u, err) || !mbar_wait(full_b(stage), phase, err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b0 = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < KP / 16; ++k) {
+            // A: K-major, 128-byte swizzle, 8-row groups 1024 B apart; K steps of 32 B within a
+            // 64-wide block, the fifth step at the start of the second block.
+            const uint64_t adesc = smem_desc(k < 4 ? a0 + 32u * k : a0 + A_KB, 16u, 1024u, kSwizzle128B);
+            // B: MN-major, 128-byte swizzle; 64-column boxes B_BOX apart, 8 K-rows 1024 B apart,
+            // 16 K-rows (2 KB) per step.
+            const uint64_t bdesc = smem_desc(b0 + 2048u * k, (uint32_t)B_BOX, 1024u, kSwizzle128B);
+            tc_mma_f16(tmem_base + acc * BN, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+          }
+          tc_commit(empty_b(stage));
+          tc_commit(tfull(acc));
+          if (++stage == B_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(empty_a(slot));
+      }
+      tc_commit(done_bar);
+      mbar_wait(done_bar, 0, err);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------ pixel gather: row t of A per thread
+    const int t = threadIdx.x - 64;
+    const int pw = W / kPatch, ph = H / kPatch;
+    uint4 *stg = reinterpret_cast<uint4 *>(smem + OFF_STG);
+    const __nv_bfloat16 *stg_h = reinterpret_cast<const __nv_bfloat16 *>(smem + OFF_STG);
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const uint32_t slot = it & 1u;
+      if (!group_and<2, 128>(mbar_wait(empty_a(slot), ((it >> 1) & 1u) ^ 1u, err))) break;
+      // two patches x 40 rows x 15 16-byte pieces, coalesced
+      for (int idx = t; idx < 2 * kPatch * 15; idx += 128) {
+        const int pp = idx / (kPatch * 15), rem = idx % (kPatch * 15);
+        const int row = rem / 15, q = rem % 15;
+        const int64_t p = 2 * tile + pp;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (p < P) {
+          const int64_t im = p / ((int64_t)ph * pw);
+          const int pr = (int)((p / pw) % ph), pc = (int)(p % pw);
+          const __nv_bfloat16 *src = img + ((im * H + kPatch * pr + row) * (int64_t)W + kPatch * pc) * 3;
+          v = __ldg(reinterpret_cast<const uint4 *>(src) + q);
+        }
+        stg[(pp * kPatch + row) * 15 + q] = v;
+      }
+      gather_bar();
+      {
+        const int pp = t >> 6, m = t & 63;
+        const __nv_bfloat16 *base = stg_h + (pp * kPatch + 5 * demorton_r(m)) * (STG_ROW / 2) + 15 * demorton_c(m);
+        uint8_t *arow = smem + OFF_A + slot * A_STAGE + (t >> 3) * 1024 + (t & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < KP / 8; ++c) {
+          // values 8c .. 8c + 7 of the row (75 and on are zero) as one 16-byte chunk
+          uint32_t wv[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const int e = 8 * c + 2 * h;
+            const float lo = e < 75 ? __bfloat162float(base[(e / 15) * (STG_ROW / 2) + e % 15]) : 0.0f;
+            const float hi =
+                e + 1 < 75 ? __bfloat162float(base[((e + 1) / 15) * (STG_ROW / 2) + (e + 1) % 15]) : 0.0f;
+            wv[h] = pack_bf16(lo, hi);
+          }
+          const int kb = c >> 3, cc = c & 7;
+          *reinterpret_cast<uint4 *>(arow + kb * A_KB + ((cc ^ (t & 7)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(full_a(slot));
+      gather_bar();  // the staging buffer is free for the next tile
+    }
+  } else {
+    // ------------------------------------------------ epilogue: row r, EPI_COLS columns per job
+    // Each warp waits for the accumulator itself; a warp whose wait gave up skips the work but
+    // keeps arriving and joining the statistics barrier, so no thread is left at a barrier.
+    const int ew = warp - 6;
+    const int quad = warp & 3, part = ew >> 2;
+    const int r = quad * 32 + lane;
+    float2 *stat = reinterpret_cast<float2 *>(smem + OFF_STAT);
+    const uint32_t obuf = smem_addr(smem + OFF_OUT + ew * 2 * OUT_BUF);
+    const uint32_t par_b = smem_addr(par), par_g = par_b + 4u * d1, par_e = par_b + 8u * d1;
+    uint32_t g = 0, n_stored = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+      float n_run = 0.0f, mean_run = 0.0f, m2_run = 0.0f, mean = 0.0f, rstd = 1.0f;
+      for (int j = 0; j < 2 * NC; ++j, ++g) {
+        const uint32_t acc = g & 1u;
+        ok = __all_sync(0xffffffffu, ok && mbar_wait(tfull(acc), (g >> 1) & 1u, err));
+        tc_fence_after();
+        const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * BN + EPI_COLS * part;
+        const int col0 = (j % NC) * BN + EPI_COLS * part;
+        // the 32 rows of this warp exist (a ragged last tile has one patch: rows 64..127 do not)
+        const int64_t row0 = tile * BM + quad * 32;
+        if (ok && j < NC) {
+          // pass 1: per BATCH values the mean and sum of squared deviations, merged into the run
+#pragma unroll 1
+          for (int c = 0; c < EPI_COLS / BATCH; ++c) {
+            float x[BATCH];
+            tmem_ld_batch(tb + BATCH * c, x);
+            float s = 0.0f;
+#pragma unroll
+            for (int k = 0; k < BATCH; k += 4) {
+              const float4 b = lds4(par_b + 4u * (col0 + BATCH * c + k));
+              x[k] += b.x; x[k + 1] += b.y; x[k + 2] += b.z; x[k + 3] += b.w;
+              s += (x[k] + x[k + 1]) + (x[k + 2] + x[k + 3]);
+            }
+            const float mb = s * (1.0f / BATCH);
+            float q = 0.0f;
+#pragma unroll
+            for (int k = 0; k < BATCH; ++k) {
+              const float dv = x[k] - mb;
+              q = fmaf(dv, dv, q);
+            }
+            const float n_new = n_run + (float)BATCH, delta = mb - mean_run;
+            mean_run += delta * ((float)BATCH / n_new);
+            m2_run += q + delta * delta * (n_run * (float)BATCH / n_new);
+            n_run = n_new;
+          }
+        } else if (ok && row0 < rows1) {
+          // pass 2: the same sums again, normalised, GELU, bf16
+#pragma unroll 1
+          for (int c = 0; c < EPI_COLS / BATCH; ++c) {
+            float x[BATCH];
+            tmem_ld_batch(tb + BATCH * c, x);
+            uint32_t pk[BATCH / 2];
+#pragma unroll
+            for (int k = 0; k < BATCH; k += 4) {
+              const int col = col0 + BATCH * c + k;
+              const float4 b = lds4(par_b + 4u * col), gg = lds4(par_g + 4u * col), bb = lds4(par_e + 4u * col);
+              const float bv[4] = {b.x, b.y, b.z, b.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w},
+                          ev[4] = {bb.x, bb.y, bb.z, bb.w};
+              float y[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) y[e] = gelu_erf(fmaf((x[k + e] + bv[e] - mean) * rstd, gv[e], ev[e]));
+              pk[k / 2] = pack_bf16(y[0], y[1]);
+              pk[k / 2 + 1] = pack_bf16(y[2], y[3]);
+            }
+            // row r of the warp's 32 x 32 box, 16-byte chunk v at v ^ ((r >> 1) & 3) (64-byte swizzle);
+            // the buffer written two batches ago must have been read by its store first
+            const uint32_t buf = obuf + (n_stored & 1u) * OUT_BUF;
+            if (lane == 0 && n_stored >= 2) bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint32_t a = buf + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * v]), "r"(pk[4 * v + 1]),
+                           "r"(pk[4 * v + 2]), "r"(pk[4 * v + 3])
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&omap, col0 + BATCH * c, (int32_t)row0, buf);
+              bulk_commit();
+            }
+            ++n_stored;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty(acc));
+        if (j == NC - 1) {
+          // the row's parts (n_run values each), merged pairwise in a fixed order
+          stat[part * BM + r] = make_float2(mean_run, m2_run);
+          epi_bar();
+          float m[EPI_PARTS], q[EPI_PARTS];
+#pragma unroll
+          for (int a = 0; a < EPI_PARTS; ++a) {
+            const float2 v = stat[a * BM + r];
+            m[a] = v.x;
+            q[a] = v.y;
+          }
+          float cnt = n_run;
+#pragma unroll
+          for (int w = 1; w < EPI_PARTS; w *= 2) {
+#pragma unroll
+            for (int a = 0; a < EPI_PARTS; a += 2 * w) {
+              const float d = m[a + w] - m[a];
+              m[a] += 0.5f * d;
+              q[a] += q[a + w] + d * d * (0.5f * cnt);
+            }
+            cnt *= 2.0f;
+          }
+          mean = m[0];
+          rstd = 1.0f / sqrtf(q[0] / (float)d1 + 1e-6f);
+          epi_bar();  // every thread has read the statistics before the next tile writes them
+        }
+      }
+    }
+    if (lane == 0) bulk_wait<0>();  // stores done before the block's shared memory goes away
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -162,24 +618,41 @@ cudaError_t lt_gemm(cublasLtHandle_t h, const __nv_bfloat16 *A, int64_t M, int K
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct HmlpLayout {
-  size_t a1, h13, h2, f32, lt, total;
+  size_t a1, h13, h2, f32, lt, w1p, total;
 };
+
+// Stage 1 runs fused (hmlp_stage1_kernel) when d1 is a whole number of 256-column chunks, at
+// most 1536;
+// otherwise as gather + cuBLASLt GEMM + row kernel.
+bool stage1_fused(const dmel_hmlp_weights &w) { return w.d1 % s1::BN == 0 && w.d1 <= s1::MAX_D1; }
 
 HmlpLayout hmlp_layout(int64_t P, const dmel_hmlp_weights &w) {
   const size_t rows1 = (size_t)P * kBlocks, rows2 = (size_t)P * 16, rows3 = (size_t)P * 4;
+  const bool fused = stage1_fused(w);
   HmlpLayout L;
-  L.a1 = r256(rows1 * kK1Pad * 2);
+  L.a1 = fused ? 0 : r256(rows1 * kK1Pad * 2);
   const size_t h1 = rows1 * (size_t)w.d1, h3 = rows3 * (size_t)w.d3;
   L.h13 = r256((h1 > h3 ? h1 : h3) * 2);
   L.h2 = r256(rows2 * (size_t)w.d2 * 2);
-  size_t f = rows1 * (size_t)w.d1;
+  size_t f = fused ? 0 : rows1 * (size_t)w.d1;
   if (rows2 * (size_t)w.d2 > f) f = rows2 * (size_t)w.d2;
   if (rows3 * (size_t)w.d3 > f) f = rows3 * (size_t)w.d3;
   if ((size_t)P * (size_t)w.dim > f) f = (size_t)P * (size_t)w.dim;
   L.f32 = r256(f * 4);
   L.lt = kLtWorkspace;
-  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.lt;
+  L.w1p = r256((size_t)kK1Pad * (size_t)w.d1 * 2);
+  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.lt + L.w1p;
   return L;
+}
+
+cudaError_t stage1_smem_attr() {
+  static bool done[256] = {false};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || done[dev & 255]) return e;
+  e = cudaFuncSetAttribute(hmlp_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1::SMEM_BYTES);
+  if (e == cudaSuccess) done[dev & 255] = true;
+  return e;
 }
 
 template <bool kNorm>
@@ -187,18 +660,25 @@ cudaError_t launch_rows(const float *in, int64_t rows, int d, const float *b, co
                         __nv_bfloat16 *out, int num_sms, cudaStream_t stream) {
   const int64_t blocks = (rows + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 16;
-  hmlp_row_kernel<kNorm><<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(in, rows, d, b, g, be, out);
+  const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
+  hmlp_row_kernel<kNorm><<<grid, 256, 0, stream>>>(in, rows, d, b, g, be, out);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_gelu_debug(const float *x, float *y, int64_t n, int num_sms, cudaStream_t stream) {
+  const int64_t blocks = (n + 255) / 256, cap = (int64_t)num_sms * 8;
+  hmlp_gelu_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w) {
   return n_patches > 0 ? hmlp_layout(n_patches, w).total : 0;
 }
 
 cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp_weights &w, void *out,
-                        void *workspace, int num_sms, cudaStream_t stream, int *launches) {
+                        void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
   const int64_t P = (int64_t)n * (H / kPatch) * (W / kPatch);
   if (P <= 0) return cudaSuccess;
   cublasLtHandle_t h;
@@ -211,22 +691,54 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
   auto *H2 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13);
   auto *F = reinterpret_cast<float *>(base + L.a1 + L.h13 + L.h2);
   void *lt_ws = base + L.a1 + L.h13 + L.h2 + L.f32;
-  const auto *W1 = static_cast<const __nv_bfloat16 *>(w.w1);
+  // W1 padded to 80 rows (5 zero rows) so the stage-1 product has a 16-byte aligned K
+  auto *W1 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13 + L.h2 + L.f32 + L.lt);
+  if ((e = cudaMemcpyAsync(W1, w.w1, (size_t)kK1 * w.d1 * 2, cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
+    return e;
+  if ((e = cudaMemsetAsync(W1 + (size_t)kK1 * w.d1, 0, (size_t)(kK1Pad - kK1) * w.d1 * 2, stream)) != cudaSuccess)
+    return e;
   const auto *W2 = static_cast<const __nv_bfloat16 *>(w.w2);
   const auto *W3 = static_cast<const __nv_bfloat16 *>(w.w3);
   const auto *W4 = static_cast<const __nv_bfloat16 *>(w.w4);
-  {
+  const int64_t rows1 = P * kBlocks, rows2 = P * 16, rows3 = P * 4;
+  if (stage1_fused(w)) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)w.d1, (cuuint64_t)kK1Pad};
+    const cuuint64_t strides[1] = {(cuuint64_t)w.d1 * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kK1Pad};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W1, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    // the stage-1 output [rows1 x d1] bf16, stored in boxes of 32 rows x 32 columns
+    CUtensorMap omap;
+    const cuuint64_t odims[2] = {(cuuint64_t)w.d1, (cuuint64_t)rows1};
+    const cuuint32_t obox[2] = {(cuuint32_t)s1::BATCH, 32};
+    if (enc(&omap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H13, odims, strides, obox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    if ((e = stage1_smem_attr()) != cudaSuccess) return e;
+    const int64_t tiles = (P + 1) / 2;
+    const unsigned grid = (unsigned)(tiles < num_sms ? tiles : num_sms);
+    hmlp_stage1_kernel<<<grid, s1::THREADS, s1::SMEM_BYTES, stream>>>(
+        map, omap, static_cast<const __nv_bfloat16 *>(images), H, W, P, w.d1, w.b1, w.g1, w.be1, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+  } else {
     const int64_t items = P * kBlocks;
     const int64_t cap = (int64_t)num_sms * 16;
     const int64_t blocks = (items + 255) / 256;
     hmlp_gather_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(images), n, H, W, A1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ++*launches;
+    if ((e = lt_gemm(h, A1, rows1, kK1Pad, kK1Pad, W1, w.d1, F, lt_ws, stream)) != cudaSuccess) return e;
+    if ((e = launch_rows<true>(F, rows1, w.d1, w.b1, w.g1, w.be1, H13, num_sms, stream)) != cudaSuccess) return e;
+    *launches += 2;
   }
-  const int64_t rows1 = P * kBlocks, rows2 = P * 16, rows3 = P * 4;
-  if ((e = lt_gemm(h, A1, rows1, kK1, kK1Pad, W1, w.d1, F, lt_ws, stream)) != cudaSuccess) return e;
-  if ((e = launch_rows<true>(F, rows1, w.d1, w.b1, w.g1, w.be1, H13, num_sms, stream)) != cudaSuccess) return e;
   if ((e = lt_gemm(h, H13, rows2, 4 * w.d1, 4 * w.d1, W2, w.d2, F, lt_ws, stream)) != cudaSuccess) return e;
   if ((e = launch_rows<true>(F, rows2, w.d2, w.b2, w.g2, w.be2, H2, num_sms, stream)) != cudaSuccess) return e;
   if ((e = lt_gemm(h, H2, rows3, 4 * w.d2, 4 * w.d2, W3, w.d3, F, lt_ws, stream)) != cudaSuccess) return e;
@@ -235,7 +747,7 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
   if ((e = launch_rows<false>(F, P, w.dim, w.b4, nullptr, nullptr, static_cast<__nv_bfloat16 *>(out), num_sms,
                               stream)) != cudaSuccess)
     return e;
-  *launches += 4;  // the four row kernels (the four GEMMs are cuBLASLt's)
+  *launches += 3;  // the row kernels of stages 2-4 (their GEMMs are cuBLASLt's)
   return cudaSuccess;
 }
 

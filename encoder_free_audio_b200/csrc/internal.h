@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "dmel.h"
@@ -49,11 +50,21 @@ cudaError_t launch_shortconv(const void *x, const int64_t *seq_offsets, int n_se
                              const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
                              uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
 
-// hMLP patchifier: workspace bytes for n_patches, and the launch (gather, four cuBLASLt GEMMs,
-// four row kernels) on `stream`.
+// hMLP patchifier: workspace bytes for n_patches, and the launch on `stream` (stage 1 fused in
+// one tcgen05 kernel when d1 is a multiple of 256, else gather + GEMM + row kernel; stages 2-4
+// as cuBLASLt GEMMs + row kernels).
 size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w);
 cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp_weights &w, void *out,
-                        void *workspace, int num_sms, cudaStream_t stream, int *launches);
+                        void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
+
+// cuTensorMapEncodeTiled, looked up once from the driver (nullptr when unavailable).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// GELU of n values with the hMLP kernels' formula (diagnostic).
+cudaError_t launch_gelu_debug(const float *x, float *y, int64_t n, int num_sms, cudaStream_t stream);
 
 // Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
 cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);

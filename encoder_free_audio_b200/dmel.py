@@ -96,6 +96,8 @@ def _lib():
         L.dmel_last_launch_count.restype = i32
         L.dmel_debug_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.POINTER(ctypes.c_uint32)]
         L.dmel_debug_wait_timeout.restype = i32
+        L.dmel_debug_gelu.argtypes = [vp, vp, ctypes.c_int64, vp]
+        L.dmel_debug_gelu.restype = i32
         L.dmel_debug_codes_frame_host.argtypes = [vp, vp, vp]
         L.dmel_debug_codes_frame_host.restype = None
         L.dmel_debug_codes_frame_host_q.argtypes = [vp, ctypes.POINTER(Quantizer), vp, vp]
@@ -340,6 +342,17 @@ def dmel_debug_codes_frame_host_q(frame1600: np.ndarray, quantizer=None):
                                               lhat.ctypes.data_as(ctypes.c_void_p))
     _check(rc, "dmel_debug_codes_frame_host_q")
     return codes, lhat
+
+
+def dmel_debug_gelu(x, y=None):
+    """GELU of a contiguous fp32 device tensor with the hMLP kernels' formula (diagnostic, see
+    dmel_debug.h); returns y."""
+    import torch
+    if y is None:
+        y = torch.empty_like(x)
+    rc = _lib().dmel_debug_gelu(_ptr(x), _ptr(y), x.numel(), _stream(None))
+    _check(rc, "dmel_debug_gelu")
+    return y
 
 
 def dmel_debug_wait_timeout(polls: int = 1 << 16) -> int:

@@ -261,8 +261,9 @@ dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq,
  * widths: the caller chooses them. Stage 1 maps every 5x5 pixel block of a patch (75 values in
  * row, column, channel order) to d1 features; stages 2, 3, 4 map every 2x2 group of the previous
  * stage's grid (the four vectors concatenated top-left, top-right, bottom-left, bottom-right) to
- * d2, d3 and dim features. Bias, LayerNorm (eps 1e-6, gain, shift) and the exact GELU follow
- * stages 1-3, bias alone stage 4; every stage's output is stored in bf16, products sum in fp32. */
+ * d2, d3 and dim features. Bias, LayerNorm (eps 1e-6, gain, shift) and GELU (u Phi(u), with
+ * erfc from Abramowitz & Stegun 7.1.26: absolute error at most 1.5e-7) follow stages 1-3, bias
+ * alone stage 4; every stage's output is stored in bf16, products sum in fp32. */
 typedef struct {
   int d1, d2, d3, dim;            /* stage widths, each a positive multiple of 8 */
   const void *w1, *w2, *w3, *w4;  /* bf16 row-major [75 x d1], [4 d1 x d2], [4 d2 x d3], [4 d3 x dim] */
@@ -277,8 +278,9 @@ size_t dmel_hmlp_workspace_size(int64_t n_patches, const dmel_hmlp_weights *w);
 /* images   bf16 [n_images x height x width x 3] (channel last), device, 16-byte aligned;
  *          height and width multiples of 40
  * out      bf16 [n_images * (height / 40) * (width / 40) x dim], patches in raster order
- * The four products run as dense bf16 GEMMs (cuBLASLt); gathering the pixel blocks and the bias,
- * LayerNorm and GELU between them run in the library's kernels. Asynchronous on stream. */
+ * Stage 1 (d1 a multiple of 256, at most 1536) runs in one tensor-core kernel of the library;
+ * otherwise, and for stages 2-4, the products run as dense bf16 GEMMs (cuBLASLt) with the bias,
+ * LayerNorm and GELU in the library's kernels. Asynchronous on stream. */
 dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, const dmel_hmlp_weights *w, void *out,
                       void *workspace, size_t workspace_bytes, dmel_stream_t stream);
 

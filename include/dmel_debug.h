@@ -32,6 +32,11 @@ dmel_status dmel_debug_codes_frame_host_q(const float *frame1600, const dmel_qua
  * faults or hangs: the context stays usable. */
 dmel_status dmel_debug_wait_timeout(uint32_t polls, uint32_t *h_bits);
 
+/* y[i] = GELU(x[i]) for i < n with the formula the hMLP kernels use (u Phi(u), erfc from
+ * Abramowitz & Stegun 7.1.26, absolute error at most 1.5e-7 in erfc), so it can be checked
+ * against the exact function. x, y: device fp32 [n], 16-byte aligned. Asynchronous on stream. */
+dmel_status dmel_debug_gelu(const float *x, float *y, int64_t n, dmel_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
