@@ -49,6 +49,17 @@ int oracle_threads(void) {
 #endif
 }
 
+/* Sets the number of threads the frame loops use (n >= 1); returns the number now in effect. */
+int oracle_set_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+  return omp_get_max_threads();
+#else
+  (void)n;
+  return 1;
+#endif
+}
+
 /* Frames of one clip: floor(N / hop); negative lengths are an error (-1). */
 int64_t oracle_frames_for_length(int64_t n_samples) {
   if (n_samples < 0) return -1;

@@ -51,6 +51,8 @@ def lib():
         c_d, c_i64, c_int = ctypes.c_double, ctypes.c_int64, ctypes.c_int
         vp = ctypes.c_void_p
         L.oracle_threads.restype = c_int
+        L.oracle_set_threads.argtypes = [c_int]
+        L.oracle_set_threads.restype = c_int
         L.oracle_frames_for_length.argtypes = [c_i64]
         L.oracle_frames_for_length.restype = c_i64
         L.oracle_window.argtypes = [vp]
@@ -92,6 +94,11 @@ def _ptr(a):
 def threads() -> int:
     """OpenMP threads the oracle's frame loops use."""
     return int(lib().oracle_threads())
+
+
+def set_threads(n: int) -> int:
+    """Sets the OpenMP threads of the frame loops (n >= 1); returns the count now in effect."""
+    return int(lib().oracle_set_threads(int(n)))
 
 
 def frames_for_length(n: int) -> int:

@@ -262,6 +262,25 @@ def test_frame_subset_equals_full_run(oracle_mod):
         oracle_mod.codes(wav, off, frame_ids=np.array([40]))
 
 
+def test_thread_count_changes_nothing(oracle_mod):
+    """The oracle's threads split frames only: one thread and all threads give bit-identical
+    codes, log-mel values and embeddings (the host baseline times both)."""
+    wav, off = synth.one_clip_2s()
+    table = np.random.default_rng(9).standard_normal((1280, 16))
+    n_all = oracle_mod.threads()
+    c_all, l_all = oracle_mod.codes(wav, off)
+    e_all = oracle_mod.embed(c_all, table, np.ones(16))
+    try:
+        assert oracle_mod.set_threads(1) == 1
+        c_one, l_one = oracle_mod.codes(wav, off)
+        e_one = oracle_mod.embed(c_one, table, np.ones(16))
+    finally:
+        assert oracle_mod.set_threads(n_all) == n_all
+    np.testing.assert_array_equal(c_one, c_all)
+    np.testing.assert_array_equal(l_one, l_all)
+    np.testing.assert_array_equal(e_one, e_all)
+
+
 def test_frame_alignment_closed_form(oracle_mod):
     """Frame t of a clip sees samples [800 (t - 1), 800 (t + 1)): a clip that is silent except
     for a bin-centred tone in [800 t0, 800 t0 + 800) lights frames t0 and t0 + 1 only."""
