@@ -44,8 +44,10 @@ EMBED_BYTES_PER_FRAME = 80 + DIM * 2
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
 SPARSE_PEAK_RATIO = 2.0
 # DRAM bytes (read + write) of one launch of the dominant kernel on this workload, from the ncu
-# capture summarised in profiles/ (None when the kernel changed since the capture)
-EMBED_TRAFFIC_PER_LAUNCH = 18_343_168 + 104_999_168  # embed_sp_kernel fused, 12,800 frames
+# capture summarised in profiles/ (None when the kernel changed since the capture). The capture
+# (18,343,168 + 104,999,168 B) predates the kernel's shared-space base pointer, so it is None
+# until the kernel is captured again.
+EMBED_TRAFFIC_PER_LAUNCH = None
 
 
 def peaks():
