@@ -615,13 +615,15 @@ struct HmlpLayout {
 };
 
 // Stage 1 runs fused (hmlp_stage1_kernel) when d1 is a whole number of 256-column chunks, at
-// most 1536;
-// otherwise as gather + cuBLASLt GEMM + row kernel.
-bool stage1_fused(const dmel_hmlp_weights &w) { return w.d1 % s1::BN == 0 && w.d1 <= s1::MAX_D1; }
+// most 1536, and the block rows fit the TMA store's 32-bit row coordinate; otherwise as
+// gather + cuBLASLt GEMM + row kernel.
+bool stage1_fused(int64_t P, const dmel_hmlp_weights &w) {
+  return w.d1 % s1::BN == 0 && w.d1 <= s1::MAX_D1 && P * kBlocks <= (int64_t)INT32_MAX;
+}
 
 HmlpLayout hmlp_layout(int64_t P, const dmel_hmlp_weights &w) {
   const size_t rows1 = (size_t)P * kBlocks, rows2 = (size_t)P * 16, rows3 = (size_t)P * 4;
-  const bool fused = stage1_fused(w);
+  const bool fused = stage1_fused(P, w);
   HmlpLayout L;
   L.a1 = fused ? 0 : r256(rows1 * kK1Pad * 2);
   const size_t h1 = rows1 * (size_t)w.d1, h3 = rows3 * (size_t)w.d3;
@@ -694,7 +696,7 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
   const auto *W3 = static_cast<const __nv_bfloat16 *>(w.w3);
   const auto *W4 = static_cast<const __nv_bfloat16 *>(w.w4);
   const int64_t rows1 = P * kBlocks, rows2 = P * 16, rows3 = P * 4;
-  if (stage1_fused(w)) {
+  if (stage1_fused(P, w)) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap map;
