@@ -278,7 +278,8 @@ size_t dmel_hmlp_workspace_size(int64_t n_patches, const dmel_hmlp_weights *w);
 /* images   bf16 [n_images x height x width x 3] (channel last), device, 16-byte aligned;
  *          height and width multiples of 40
  * out      bf16 [n_images * (height / 40) * (width / 40) x dim], patches in raster order
- * Stage 1 (d1 a multiple of 256, at most 1536) runs in one tensor-core kernel of the library;
+ * Stage 1 (d1 a multiple of 256, at most 1536; fewer than 2^31 pixel blocks) runs in one
+ * tensor-core kernel of the library;
  * otherwise, and for stages 2-4, the products run as dense bf16 GEMMs (cuBLASLt) with the bias,
  * LayerNorm and GELU in the library's kernels. Asynchronous on stream. */
 dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, const dmel_hmlp_weights *w, void *out,
