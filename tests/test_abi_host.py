@@ -242,5 +242,16 @@ def test_hmlp_argument_checks_without_gpu(lib):
     n10 = lib.dmel_hmlp_workspace_size(10, ctypes.byref(w))
     assert 0 < n1 < n10 and n10 >= 10 * 64 * 16 * 4
     assert lib.dmel_hmlp_workspace_size(0, ctypes.byref(w)) == 0
+    # d1 a multiple of 256 (at most 1536): stage 1 runs fused and needs neither the gathered
+    # blocks nor the fp32 stage-1 sums; a d1 just off that grid takes the general path
+    P = 10
+    fused = dmel.HmlpWeights(256, 64, 64, 64, *([a] * 14))
+    general = dmel.HmlpWeights(264, 64, 64, 64, *([a] * 14))
+    too_wide = dmel.HmlpWeights(1792, 64, 64, 64, *([a] * 14))
+    nf = lib.dmel_hmlp_workspace_size(P, ctypes.byref(fused))
+    ng = lib.dmel_hmlp_workspace_size(P, ctypes.byref(general))
+    nw = lib.dmel_hmlp_workspace_size(P, ctypes.byref(too_wide))
+    assert ng - nf >= P * 64 * 256 * 2  # more than half the fp32 stage-1 sums the general path keeps
+    assert nw >= nf + P * 64 * 1792 * 4  # past 1536 columns the fp32 sums are back
     # no image: a no-op
     assert H(None, 0, 40, 40, ctypes.byref(w), None, None, 0, None) == dmel.DMEL_OK
