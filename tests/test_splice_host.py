@@ -56,3 +56,20 @@ def test_frame_counts_from_clip_lengths():
 def test_rejects_bad_plans(pos, fo, seq_len):
     with pytest.raises(dmel.DmelError):
         dmel.dmel_splice_plan(pos, fo, seq_len)
+
+
+@pytest.mark.parametrize("seq_len,pos,f", [
+    (0, [], []),                        # empty sequence, no audio
+    (4, [], []),                        # text only: identity
+    (3, [0, 1, 2], [2, 0, 3]),          # every position a sentinel, one clip without frames
+    (5, [0, 4], [1, 1]),                # one-frame clips at both ends: the length is unchanged
+    (6, [5], [0]),                      # a frameless clip at the end drops the last position
+    (2, [0], [100000]),                 # one long clip
+])
+def test_edge_cases_match_oracle(oracle_mod, seq_len, pos, f):
+    tp, fr, n, a = dmel.dmel_splice_plan(pos, _fo(f), seq_len)
+    otp, ofr, on, oa = oracle_mod.splice_plan(seq_len, pos, f)
+    assert tp.tolist() == otp and fr.tolist() == ofr and n == on and a == oa
+    # every expanded position is filled exactly once, by a text token or by a frame
+    filled = sorted([p for p in tp.tolist() if p >= 0] + fr.tolist())
+    assert filled == list(range(n))
