@@ -159,6 +159,26 @@ def test_kernel_arithmetic_on_host_tones_and_noise(lib, oracle_mod):
         _compare_codes(gc, gl, oc[0], ol[0], oracle_mod)
 
 
+def test_kernel_arithmetic_on_host_extremes(lib, oracle_mod):
+    """Frames at the ends of the range: a NaN sample (every energy NaN: read as the floor, so
+    code 0 everywhere), a constant 1e30 frame (the fp32 mel sums overflow, L clamps at the top),
+    and a 1e-30 frame (the energies underflow, L clamps at the bottom): the same codes as the
+    oracle, all in 0..15."""
+    r = np.random.default_rng(12)
+    nan_frame = r.uniform(-0.5, 0.5, 1600).astype(np.float32)
+    nan_frame[777] = np.nan
+    cases = [nan_frame, np.full(1600, 1e30, np.float32),
+             (1e-30 * r.standard_normal(1600)).astype(np.float32)]
+    for fr in cases:
+        gc, _ = dmel.dmel_debug_codes_frame_host(fr)
+        oc, _ = oracle_mod.codes(fr, np.array([0, 1600]), tails=None, frame_ids=np.array([1]))
+        np.testing.assert_array_equal(gc, oc[0])
+        assert gc.max() <= 15
+    assert (dmel.dmel_debug_codes_frame_host(cases[0])[0] == 0).all()
+    assert (dmel.dmel_debug_codes_frame_host(cases[1])[0] == 15).all()
+    assert (dmel.dmel_debug_codes_frame_host(cases[2])[0] == 0).all()
+
+
 # ---------------------------------------------------------------- quantiser variants on the host
 
 QUANTS = [(-7.0, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0), (-1.5, 2.0, dmel.DMEL_QUANT_FLOOR, 0.0),
