@@ -149,7 +149,8 @@ __global__ void hmlp_gelu_kernel(const float *__restrict__ x, float *__restrict_
 // whole row of d1 sums, which does not fit in TMEM, so each tile runs its d1 / 256 chunks
 // twice: the first pass gives the row statistics (mean and sum of squared deviations per
 // 32 values, merged pairwise), the second recomputes the same sums and writes
-// bf16(GELU(LayerNorm(x + b1))). The product is tiny (K = 80), so the second pass costs far
+// bf16(GELU(LayerNorm(x + b1))), each warp's 32 x 32 box staged in shared memory and stored
+// with a TMA bulk-tensor store. The product is tiny (K = 80), so the second pass costs far
 // less than storing and re-reading the fp32 sums.
 namespace s1 {
 constexpr int BM = 128;                 // pixel blocks per tile (two patches)
