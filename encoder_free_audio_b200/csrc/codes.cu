@@ -690,14 +690,8 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
                          cudaStream_t stream, int *launches, Quant q) {
   cudaError_t e = ensure_device_tables();
   if (e != cudaSuccess) return e;
-  static bool attr_set[256] = {false};
-  int dev = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if (!attr_set[dev & 255]) {
-    e = cudaFuncSetAttribute(codes_kernel_entry, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set[dev & 255] = true;
-  }
+  static std::atomic<bool> attr_set[256];
+  if ((e = set_smem_attr_once(codes_kernel_entry, kSmemBytes, attr_set)) != cudaSuccess) return e;
   if (n_frames > 0) {
     int64_t blocks = (n_frames + kWarpsPerBlock - 1) / kWarpsPerBlock;
     if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM

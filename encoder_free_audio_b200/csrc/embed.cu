@@ -1382,17 +1382,6 @@ EncodeTiledFn encode_tiled_fn() {
 
 namespace {
 
-template <typename K>
-cudaError_t set_smem_attr_once(K kernel, int bytes, bool *flags) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (flags[dev & 255]) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) flags[dev & 255] = true;
-  return e;
-}
-
 // Tensor map of the bf16 table [1280 x D]: boxes of box_cols columns x box_rows rows, with the
 // swizzle whose span is one box row (64 columns: 128 bytes; 32 columns: 64 bytes).
 bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D, int box_rows = tc::BK, int box_cols = 64) {
@@ -1441,17 +1430,19 @@ TcScratch tc_scratch(void *ws, int64_t F, int D) {
 // Whether the fused RMSNorm schedule can run: every block of a group of D/256 blocks must be
 // resident at once (cooperative launch, one block per SM).
 bool fused_possible(int D, int num_sms, int *grid) {
-  static int coop[256] = {0};  // 0 unknown, 1 yes, 2 no
+  static std::atomic<int> coop[256];  // 0 unknown, 1 yes, 2 no
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (coop[dev & 255] == 0) {
+  int c = coop[dev & 255].load(std::memory_order_relaxed);
+  if (c == 0) {
     int v = 0;
-    coop[dev & 255] = (cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && v) ? 1 : 2;
+    c = (cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && v) ? 1 : 2;
+    coop[dev & 255].store(c, std::memory_order_relaxed);
   }
   const int P = D / tc::BN;
   const int G = num_sms / P;
   *grid = G * P;
-  return coop[dev & 255] == 1 && G >= 1;
+  return c == 1 && G >= 1;
 }
 
 bool cooperative_enabled();
@@ -1459,7 +1450,7 @@ bool cooperative_enabled();
 template <typename OT, int kMode>
 cudaError_t launch_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                       const __nv_bfloat16 *g, float eps, uint32_t *err, int grid, cudaStream_t stream) {
-  static bool attr[256] = {false};
+  static std::atomic<bool> attr[256];
   cudaError_t e = set_smem_attr_once(embed_tc_kernel<OT, kMode>, tc::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
   CUtensorMap tmap;
@@ -1483,7 +1474,7 @@ template <typename TT, typename OT>
 cudaError_t launch_simt(const uint8_t *codes, int64_t F, const TT *table, int D, const TT *g, float eps, OT *out,
                         OutMap om, uint32_t *err, int num_sms, cudaStream_t stream) {
   const int smem = g ? D * (int)sizeof(float) : 0;
-  static bool attr[256] = {false};
+  static std::atomic<bool> attr[256];
   cudaError_t e = set_smem_attr_once(embed_simt_kernel<TT, OT>, kSimtMaxDim * (int)sizeof(float), attr);
   if (e != cudaSuccess) return e;
   const int64_t cap = (int64_t)num_sms * 8;
@@ -1507,7 +1498,7 @@ cudaError_t launch_rescale(OT *out, OutMap om, int64_t F, int D, const __nv_bflo
 template <typename OT, int kMode>
 cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                        const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
-  static bool attr[256] = {false};
+  static std::atomic<bool> attr[256];
   cudaError_t e = set_smem_attr_once(embed_tc2_kernel<OT, kMode>, tc2::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
   CUtensorMap tmap;
@@ -1548,7 +1539,7 @@ cudaError_t launch_tc2(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tab
 template <typename OT, int kMode>
 cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om, TcScratch sc,
                       const __nv_bfloat16 *g, float eps, uint32_t *err, int clusters, cudaStream_t stream) {
-  static bool attr[256] = {false};
+  static std::atomic<bool> attr[256];
   cudaError_t e = set_smem_attr_once(embed_sp_kernel<OT, kMode>, sp::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
   CUtensorMap tmap;

@@ -642,13 +642,8 @@ HmlpLayout hmlp_layout(int64_t P, const dmel_hmlp_weights &w) {
 }
 
 cudaError_t stage1_smem_attr() {
-  static bool done[256] = {false};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || done[dev & 255]) return e;
-  e = cudaFuncSetAttribute(hmlp_stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, s1::SMEM_BYTES);
-  if (e == cudaSuccess) done[dev & 255] = true;
-  return e;
+  static std::atomic<bool> done[256];
+  return set_smem_attr_once(hmlp_stage1_kernel, s1::SMEM_BYTES, done);
 }
 
 template <bool kNorm>

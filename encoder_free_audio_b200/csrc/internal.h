@@ -1,6 +1,7 @@
 // Host-side interface between the library's translation units (not part of the C ABI).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -56,6 +57,20 @@ cudaError_t launch_shortconv(const void *x, const int64_t *seq_offsets, int n_se
 size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w);
 cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp_weights &w, void *out,
                         void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches);
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device. `done` is that
+// kernel's own flag array [256] (by device ordinal); concurrent first calls from several host
+// threads may both set the attribute, which is harmless.
+template <typename K>
+cudaError_t set_smem_attr_once(K kernel, int bytes, std::atomic<bool> *done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (done[dev & 255].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev & 255].store(true, std::memory_order_release);
+  return e;
+}
 
 // cuTensorMapEncodeTiled, looked up once from the driver (nullptr when unavailable).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,

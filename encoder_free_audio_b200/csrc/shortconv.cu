@@ -221,15 +221,9 @@ cudaError_t launch_sc(const T *x, const int64_t *off, int n_seq, int64_t n_tok, 
     const int64_t cap = (int64_t)num_sms * 8;
     const int64_t blocks = (items + kScThreads - 1) / kScThreads;
     const int smem = kScDepth * kScThreads * 16 * ((int)sizeof(T) / 2);
-    static bool attr[256] = {false};
-    int dev = 0;
-    cudaError_t e0 = cudaGetDevice(&dev);
+    static std::atomic<bool> attr[256];
+    const cudaError_t e0 = set_smem_attr_once(shortconv_kernel<T>, smem, attr);
     if (e0 != cudaSuccess) return e0;
-    if (!attr[dev & 255]) {
-      e0 = cudaFuncSetAttribute(shortconv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e0 != cudaSuccess) return e0;
-      attr[dev & 255] = true;
-    }
     shortconv_kernel<T><<<(unsigned)(blocks < cap ? blocks : cap), kScThreads, smem, stream>>>(x, off, n_seq, n_tok, C,
                                                                                              w, state, y, err);
     cudaError_t e = cudaGetLastError();

@@ -25,6 +25,9 @@
  *   - n_clips == 0 or n_frames == 0 is a valid call that does nothing.
  *   - No entry point allocates device memory. Scratch space comes from the caller's workspace;
  *     dmel_workspace_size() says how much.
+ *   - Calls may come from several host threads at once (each with its own buffers): the
+ *     per-device one-time setup (constant tables, kernel attributes, the cuBLASLt handle of
+ *     dmel_hmlp) is guarded, and dmel_last_launch_count() reports the calling thread's last call.
  *   - Environment (read once per process): DMEL_EMBED_MMA=dense runs the tensor-core embedding
  *     as a dense one-hot product instead of the 2:4-sparse one; DMEL_EMBED_TILE=single runs it
  *     dense on one-CTA tiles instead of CTA pairs; DMEL_COOPERATIVE=0 launches the fused
