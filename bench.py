@@ -2,10 +2,18 @@
 """Benchmark of the dMel front end on B200: dMel tokens/s (waveform to 6144-d bf16 vector) and
 the fraction of the HBM roofline.
 
-Workload: 64 clips x 10 s of 16 kHz fp32 audio (pink noise + chirps, 10% silent clips, 5%
-clipped), 12,800 frames, bf16 table 1280 x 6144 ~ N(0, 0.02), RMSNorm on (eps 1e-6), bf16 out.
-A step is one dmel_forward over the whole batch with inputs resident in HBM; L2 is flushed
-(256 MB write) between timed steps and each step is timed with its own CUDA events.
+Headline workload: ragged1024, 1024 clips of 1-30 s of 16 kHz fp32 audio (pink noise, harmonic
+tones, both, silence), concatenated with an offsets array and no padding: 318,044 frames, bf16
+table 1280 x 6144 ~ N(0, 0.02), RMSNorm on (eps 1e-6), bf16 out. A step is one dmel_forward over
+the whole batch with inputs resident in HBM (1.0 GB in, 3.9 GB out: larger than L2), each step
+timed with its own CUDA events on the launching stream. `e2e` is the same batch through
+dmel_forward_host: page-locked host waveforms in, the 6144-d vectors back in page-locked host
+memory, every copy inside the timed region.
+
+Context lines (each with its own roofline fractions and CPU baseline): one_clip_2s (latency of a
+40-frame call, fp32 table and output, no RMSNorm), batch64_10s (12,800 frames), long_20min
+(24,000 frames), streams4096 (1000 successive calls of 4096 streams x 800 new samples plus the
+carried tail), and the ShortConv and hMLP kernels.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -30,24 +38,39 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "dMel tokens/sec (waveform to 6144-d bf16 embed); % of HBM roofline"
-WORKLOAD = ("batch64_10s: 64 clips x 10 s of 16 kHz mono fp32 (pink noise + linear chirp, 10% silent, "
-            "5% clipped), 12,800 frames, bf16 table 1280x6144 N(0,0.02), RMSNorm on (eps 1e-6, w~N(1,0.1)), "
-            "bf16 out")
 DIM = 6144
-# algorithmic HBM bytes per frame of the whole path (bf16 out): 800 new fp32 samples in,
-# 6144 bf16 out
-PATH_BYTES_PER_FRAME = 800 * 4 + DIM * 2
-# embedding stage (the dominant kernels): codes in (80 B), bf16 vector out
-EMBED_BYTES_PER_FRAME = 80 + DIM * 2
+DESCR = {
+    "one_clip_2s": "one_clip_2s: 1 clip, 2.0 s of 16 kHz mono fp32 (3 sines + N(0, 0.01^2) noise), 40 frames, "
+                   "fp32 table 1280x6144 N(0,0.02), no RMSNorm, fp32 out",
+    "batch64_10s": "batch64_10s: 64 clips x 10 s of 16 kHz mono fp32 (pink noise + linear chirp, 10% silent, "
+                   "5% clipped), 12,800 frames, bf16 table 1280x6144 N(0,0.02), RMSNorm on (eps 1e-6, "
+                   "w~N(1,0.1)), bf16 out",
+    "long_20min": "long_20min: 1 clip of 20 min of 16 kHz mono fp32 (AR(12) noise bursts of 50-400 ms, 20% "
+                  "silence), 24,000 frames, bf16 table, RMSNorm on, bf16 out",
+    "ragged1024": "ragged1024: 1024 clips of 1-30 s of 16 kHz mono fp32 (pink noise, harmonic tones, both, "
+                  "silence), concatenated with offsets and no padding, 318,044 frames, bf16 table 1280x6144 "
+                  "N(0,0.02), RMSNorm on (eps 1e-6, w~N(1,0.1)), bf16 out",
+    "streams4096": "streams4096: 4096 streams x (800 new + 800 carried samples) per call, 1000 successive calls, "
+                   "white noise + tone, bf16 table, RMSNorm on, bf16 out",
+}
+HEADLINE = "ragged1024"
+# algorithmic HBM bytes per frame: the path (800 new fp32 samples in, the vector out), and each
+# stage: codes (samples in, 80 code bytes out), embedding (codes in, vector out)
+IN_BYTES = 800 * 4
+CODES_BYTES = 80
+
+
+def out_bytes(out_es: int) -> int:
+    return DIM * out_es
+
+
+# DRAM bytes (read + write) per frame of each dominant kernel, from the ncu captures summarised
+# in profiles/ (batch64_10s; per launch = per frame x frames). None when the kernel changed since.
+TRAFFIC_PER_FRAME = {"embed": None, "codes": None}
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144 logical flops, run as a
 # 2:4-sparse product whose peak is twice the dense bf16 peak (nominal 4.5 vs 2.25 PFLOP/s)
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
 SPARSE_PEAK_RATIO = 2.0
-# DRAM bytes (read + write) of one launch of the dominant kernel on this workload, from the ncu
-# capture summarised in profiles/ (None when the kernel changed since the capture). The capture
-# (18,343,168 + 104,999,168 B) predates the kernel's shared-space base pointer, so it is None
-# until the kernel is captured again.
-EMBED_TRAFFIC_PER_LAUNCH = None
 
 
 def peaks():
@@ -118,70 +141,233 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def cpu_baseline(wav, off, table64, g64, budget_s: float = 12.0) -> dict:
-    """The oracle as it stands (codes + embedding + RMSNorm, fp64) on a bounded random sample of
-    the workload's frames, on this host's cores."""
+# ------------------------------------------------------------------------------------ workloads
+
+def load_workload(name: str) -> dict:
+    """Host inputs of a workload: waveforms, sample offsets, table (fp32), RMSNorm weight or None,
+    output element size."""
+    from encoder_free_audio_b200 import synth
+    if name == "one_clip_2s":
+        wav, off = synth.one_clip_2s()
+        return {"wav": wav, "off": off, "table": synth.table(), "g": None, "bf16": False}
+    fn = {"batch64_10s": synth.batch64_10s, "long_20min": synth.long_20min, "ragged1024": synth.ragged1024}[name]
+    wav, off = fn()
+    return {"wav": wav, "off": off, "table": synth.table(), "g": synth.rms_weight(), "bf16": True}
+
+
+def oracle_sample(wav, off, table64, g64, budget_s: float, seed: int, tails=None) -> dict:
+    """The oracle as it stands (codes + embedding [+ RMSNorm], fp64) on a bounded random sample of
+    the workload's frames, on this host's cores; tokens/s."""
     from oracle import oracle
     oracle.build()
     fo = oracle.frame_offsets(off)
     F = int(fo[-1])
-    rng = np.random.default_rng(77)
+    rng = np.random.default_rng(seed)
 
     def run(n):
         ids = np.sort(rng.choice(F, n, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        c = oracle.codes(wav, off, frame_ids=ids, want_lhat=False)
+        c = oracle.codes(wav, off, tails=tails, frame_ids=ids, want_lhat=False)
         oracle.embed(c, table64, g64, 1e-6)
         return time.perf_counter() - t0
 
-    n0 = 64
+    n0 = min(F, 32)
     t0 = run(n0)
     n = int(min(F, max(n0, n0 * budget_s / max(t0, 1e-6))))
     t = run(n)
-    cores = oracle.threads()
-    line = {"value": n / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} random frames of the {F}-frame workload (codes + embedding + RMSNorm, fp64)"}
-    # the same oracle on one core, on a smaller sample (about a quarter of the budget)
-    oracle.set_threads(1)
-    try:
-        n1 = int(min(F, max(16, n * (budget_s / 4) / max(t * cores, 1e-6))))
-        t1 = run(n1)
-    finally:
-        oracle.set_threads(cores)
-    line["one_core"] = {"value": n1 / t1, "unit": "tokens/s", "cores": 1, "sample": f"{n1} random frames"}
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} random frames of the {F}-frame workload (codes + embedding"
+                      f"{' + RMSNorm' if g64 is not None else ''}, fp64)"}
+
+
+def host_tables(torch, wl):
+    """The table and RMSNorm weight as the oracle sees them: the bf16 values (exactly) in fp64."""
+    dt = torch.bfloat16 if wl["bf16"] else torch.float32
+    tb = torch.from_numpy(wl["table"]).to(dt).double().numpy()
+    gb = None if wl["g"] is None else torch.from_numpy(wl["g"]).to(dt).double().numpy()
+    return tb, gb
+
+
+class Timer:
+    """CUDA-event timing of calls on one stream (after warm-up; optional L2 flush before each)."""
+
+    def __init__(self, torch, stream, flush=None):
+        self.torch, self.stream, self.flush = torch, stream, flush
+
+    def run(self, fn, steps: int, warmup: int, launches: list | None = None):
+        torch = self.torch
+        for _ in range(warmup):
+            if self.flush is not None:
+                self.flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            if self.flush is not None:
+                self.flush.zero_()
+            evs[i][0].record(self.stream)
+            fn()
+            evs[i][1].record(self.stream)
+            if launches is not None:
+                from encoder_free_audio_b200 import dmel
+                launches.append(dmel.dmel_last_launch_count())
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in evs]
+
+
+def stage_lines(F, codes_ms, embed_ms, out_es, pk) -> dict:
+    """Roofline of each stage (algorithmic bytes of one launch / its mean event-timed duration)."""
+    def line(name, ms, bytes_per_frame, kernel):
+        s = statistics.mean(ms) / 1e3
+        achieved = bytes_per_frame * F / s / 1e9
+        tr = TRAFFIC_PER_FRAME.get(name)
+        return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None if tr is None else tr * F,
+                "ms": statistics.mean(ms), "kernel": kernel, "peak_source": pk["source"]}
+    return {"codes": line("codes", codes_ms, IN_BYTES + CODES_BYTES, "codes_kernel_entry (fp64 DFT, fp32 mel/log/levels)"),
+            "embed": line("embed", embed_ms, CODES_BYTES + out_bytes(out_es), "dmel_embed call (tensor-core one-hot "
+                          "product with fused RMSNorm)")}
+
+
+def run_batch(torch, dev, dmel, FrontEnd, name, wl, steps, warmup, pk, flush, with_cpu, cpu_budget,
+              with_e2e=True, e2e_steps=None):
+    """One batch workload: device-resident steps, the two stages alone, e2e from host memory."""
+    stream = torch.cuda.current_stream()
+    dt = torch.bfloat16 if wl["bf16"] else torch.float32
+    T = torch.from_numpy(wl["table"]).to(dt).to(dev)
+    G = None if wl["g"] is None else torch.from_numpy(wl["g"]).to(dt).to(dev)
+    fe = FrontEnd(T, G, 1e-6, dt)
+    plan = fe.plan(wl["off"])
+    F = plan.n_frames
+    out_es = 2 if wl["bf16"] else 4
+    wav_d = torch.from_numpy(wl["wav"]).to(dev)
+    timer = Timer(torch, stream, flush)
+    launches: list = []
+    step_ms = timer.run(lambda: fe.forward(wav_d, plan), steps, warmup, launches)
+    # the two stages alone (same kernels), each bracketed by events on the launching stream
+    codes_ms = timer.run(lambda: dmel.dmel_codes(wav_d, plan.sample_offsets, plan.frame_offsets, F, plan.codes),
+                         steps, warmup)
+    embed_ms = timer.run(lambda: dmel.dmel_embed(plan.codes, T, plan.out, rms_weight=G, eps=1e-6,
+                                                 workspace=plan.workspace), steps, warmup)
+    res = {"frames": F, "step_ms": step_ms, "launches": launches, "stages": stage_lines(F, codes_ms, embed_ms, out_es, pk),
+           "path_bytes_per_frame": IN_BYTES + out_bytes(out_es)}
+    del wav_d
+    if with_e2e:
+        # end to end: page-locked host waveforms in, vectors back in page-locked host memory
+        wav_h = torch.from_numpy(wl["wav"]).pin_memory()
+        out_h = torch.empty((F, DIM), dtype=dt, pin_memory=True)
+        ws = torch.empty(max(1, dmel.dmel_forward_host_workspace_size(wl["off"], DIM, dmel._dtype_code(T),
+                                                                       dmel._dtype_code(out_h), G is not None)),
+                         dtype=torch.uint8, device=dev)
+        fwd = lambda: dmel.dmel_forward_host(wav_h, wl["off"], T, out_h, rms_weight=G, eps=1e-6, workspace=ws)
+        e2e_ms = Timer(torch, stream, None).run(fwd, e2e_steps or steps, min(warmup, 3))
+        res["e2e"] = {"ms": e2e_ms, "h2d_bytes_per_step": int(wl["wav"].nbytes),
+                      "d2h_bytes_per_step": int(F * DIM * out_es)}
+        del wav_h, out_h, ws
+    if with_cpu:
+        tb, gb = host_tables(torch, wl)
+        res["cpu_baseline"] = oracle_sample(wl["wav"], wl["off"], tb, gb, cpu_budget, 77)
+    del plan, fe
+    torch.cuda.empty_cache()
+    return res
+
+
+def context_line(name, r, pk, world) -> dict:
+    F = r["frames"]
+    ms = statistics.mean(r["step_ms"])
+    st = r["stages"]
+    dom = max(st, key=lambda k: st[k]["ms"])
+    line = {"workload": DESCR[name], "frames": F, "tokens_per_s": F / (ms / 1e3), "ms_per_call": ms,
+            "hbm_roofline_frac": r["path_bytes_per_frame"] * F / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+            "roofline": st[dom], "stages": {k: {"ms": v["ms"], "frac": v["frac"]} for k, v in st.items()},
+            "launches_per_call": r["launches"][-1] if r["launches"] else None}
+    if "e2e" in r:
+        e = r["e2e"]
+        line["e2e"] = {"value": F / (statistics.mean(e["ms"]) / 1e3), "unit": "tokens/s",
+                       "ms_per_call": statistics.mean(e["ms"]), "h2d_bytes_per_step": e["h2d_bytes_per_step"],
+                       "d2h_bytes_per_step": e["d2h_bytes_per_step"]}
+    if "cpu_baseline" in r:
+        line["cpu_baseline"] = r["cpu_baseline"]
     return line
 
 
-def streaming_latency(torch, dev, T, G, FrontEnd, dmel, warmup: int, calls: int = 200) -> dict:
-    """Streaming shape: 4096 streams, each call brings 800 new samples per stream plus the
-    carried 800-sample tail (one frame per stream). Per-call device time with CUDA events."""
+def latency_line(torch, dev, dmel, FrontEnd, pk, calls: int, with_cpu: bool) -> dict:
+    """one_clip_2s: a single 40-frame call (fp32 table and output, no RMSNorm): p50 / p99 device
+    latency per call, and the same from host memory (dmel_forward_host)."""
+    wl = load_workload("one_clip_2s")
+    stream = torch.cuda.current_stream()
+    T = torch.from_numpy(wl["table"]).to(dev)
+    fe = FrontEnd(T, None, 1e-6, torch.float32)
+    plan = fe.plan(wl["off"])
+    F = plan.n_frames
+    wav_d = torch.from_numpy(wl["wav"]).to(dev)
+    timer = Timer(torch, stream, None)
+    ms = sorted(timer.run(lambda: fe.forward(wav_d, plan), calls, 10))
+    wav_h = torch.from_numpy(wl["wav"]).pin_memory()
+    out_h = torch.empty((F, DIM), dtype=torch.float32, pin_memory=True)
+    ws = torch.empty(max(1, dmel.dmel_forward_host_workspace_size(wl["off"], DIM, dmel.DMEL_F32, dmel.DMEL_F32, False)),
+                     dtype=torch.uint8, device=dev)
+    e2e = sorted(timer.run(lambda: dmel.dmel_forward_host(wav_h, wl["off"], T, out_h, workspace=ws), calls, 10))
+    p50, p99 = ms[len(ms) // 2], ms[min(len(ms) - 1, int(0.99 * len(ms)))]
+    path = (IN_BYTES + out_bytes(4)) * F
+    line = {"workload": DESCR["one_clip_2s"], "frames": F, "calls": calls, "p50_us": 1e3 * p50, "p99_us": 1e3 * p99,
+            "tokens_per_s": F / (statistics.mean(ms) / 1e3),
+            "hbm_roofline_frac": path / (p50 / 1e3) / 1e9 / pk["hbm_gbs"],
+            "e2e": {"p50_us": 1e3 * e2e[len(e2e) // 2], "value": F / (statistics.mean(e2e) / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(wl["wav"].nbytes), "d2h_bytes_per_step": int(F * DIM * 4)},
+            "note": "latency-bound: one 40-frame call; the HBM fraction is the call's bytes over its p50 latency"}
+    if with_cpu:
+        tb, _ = host_tables(torch, wl)
+        line["cpu_baseline"] = oracle_sample(wl["wav"], wl["off"], tb, None, 2.0, 71)
+    return line
+
+
+def streaming_line(torch, dev, dmel, FrontEnd, pk, calls: int, warmup: int, with_cpu: bool) -> dict:
+    """streams4096: 4096 streams, each call brings 800 new samples per stream plus the carried
+    800-sample tail (one frame per stream); `calls` successive calls, per-call device time with
+    CUDA events. The calls' inputs are generated up front and kept on the device."""
     from encoder_free_audio_b200 import synth
     S = synth.Streams4096()
+    wl = {"table": synth.table(), "g": synth.rms_weight(), "bf16": True}
+    T = torch.from_numpy(wl["table"]).to(torch.bfloat16).to(dev)
+    G = torch.from_numpy(wl["g"]).to(torch.bfloat16).to(dev)
     fe = FrontEnd(T, G, 1e-6, torch.bfloat16)
     plan = fe.plan(synth.offsets_from_lengths([800] * S.n))
-    xs = [torch.from_numpy(S.call(k)).to(dev).reshape(-1) for k in range(8)]
+    n_in = min(calls, 64)  # distinct inputs, cycled (13 MB each)
+    xs = [torch.from_numpy(S.call(k)).to(dev).reshape(-1) for k in range(n_in)]
     tails = torch.zeros((S.n, 800), device=dev)
+    stream = torch.cuda.current_stream()
     for k in range(warmup):
-        fe.forward(xs[k % 8], plan, tails=tails, tails_out=tails)
+        fe.forward(xs[k % n_in], plan, tails=tails, tails_out=tails)
+    tails.zero_()
+    torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
-    st = torch.cuda.current_stream()
-    torch.cuda.synchronize()
     for k in range(calls):
-        evs[k][0].record(st)
-        fe.forward(xs[k % 8], plan, tails=tails, tails_out=tails)
-        evs[k][1].record(st)
+        evs[k][0].record(stream)
+        fe.forward(xs[k % n_in], plan, tails=tails, tails_out=tails)
+        evs[k][1].record(stream)
     torch.cuda.synchronize()
-    ms = sorted(a.elapsed_time(b) for a, b in evs)
-    return {"workload": "streams4096: 4096 streams x (800 new + 800 carried samples) per call, bf16, RMSNorm",
-            "frames_per_call": S.n, "calls": calls, "p50_us": 1e3 * ms[len(ms) // 2],
-            "p99_us": 1e3 * ms[min(len(ms) - 1, int(0.99 * len(ms)))],
-            "tokens_per_s": S.n * calls / (sum(ms) / 1e3), "launches_per_call": dmel.dmel_last_launch_count()}
+    ms = [a.elapsed_time(b) for a, b in evs]
+    srt = sorted(ms)
+    per_frame = IN_BYTES + 2 * 800 * 4 + out_bytes(2)  # new samples, tail in and out, vector out
+    line = {"workload": DESCR["streams4096"], "frames_per_call": S.n, "calls": calls,
+            "p50_us": 1e3 * srt[len(srt) // 2], "p99_us": 1e3 * srt[min(len(srt) - 1, int(0.99 * len(srt)))],
+            "tokens_per_s": S.n * calls / (sum(ms) / 1e3),
+            "hbm_roofline_frac": per_frame * S.n * calls / (sum(ms) / 1e3) / 1e9 / pk["hbm_gbs"],
+            "launches_per_call": dmel.dmel_last_launch_count()}
+    if with_cpu:
+        tb, gb = host_tables(torch, wl)
+        wav = S.call(0).reshape(-1)
+        line["cpu_baseline"] = oracle_sample(wav, synth.offsets_from_lengths([800] * S.n), tb, gb, 2.0, 72,
+                                             tails=np.zeros((S.n, 800), np.float32))
+        line["cpu_baseline"]["sample"] += " (call 0, zero tails)"
+    return line
 
 
 def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20, with_oracle: bool = False) -> dict:
-    """ShortConv (the decoder's width-4 per-channel causal conv) over the batch's 12,800 frame
-    vectors as 64 sequences of 200 tokens, bf16, with carried state in and out: HBM-bound, so
-    reported against the measured copy bandwidth. Inputs larger than L2 are rotated between calls."""
+    """ShortConv (the decoder's width-4 per-channel causal conv) over 12,800 frame vectors as 64
+    sequences of 200 tokens, bf16, with carried state in and out: HBM-bound, so reported against
+    the measured copy bandwidth. Inputs larger than L2 are rotated between calls."""
     T, C, n_seq = 12800, DIM, 64
     g = torch.Generator(device=dev).manual_seed(9)
     xs = [torch.randn((T, C), device=dev, generator=g).to(torch.bfloat16) for _ in range(2)]
@@ -205,7 +391,7 @@ def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20, 
     line = {"workload": "12,800 tokens x 6144 channels bf16, 64 sequences, state in/out", "us_per_call": ms * 1e3,
             "achieved_gbs": algo / (ms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
             "frac": algo / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "bytes_per_call": algo,
-            "launches_per_call": dmel.dmel_last_launch_count()}
+            "tokens_per_s": T / (ms / 1e3), "launches_per_call": dmel.dmel_last_launch_count()}
     if with_oracle:
         # the oracle beside it: 8 of the 64 sequences on the host (fp64, one thread), as tokens/s
         from oracle import oracle
@@ -216,7 +402,6 @@ def shortconv_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 20, 
         dt = time.perf_counter() - t0
         line["cpu_baseline"] = {"value": xh.shape[0] / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": f"8 of 64 sequences ({xh.shape[0]} tokens x {C} channels)"}
-        line["tokens_per_s"] = T / (ms / 1e3)
     return line
 
 
@@ -227,6 +412,7 @@ def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_
     n, H, W = 4, 800, 800
     d1 = d2 = d3 = DIM // 4
     g = torch.Generator(device=dev).manual_seed(11)
+
     def rn(*shape, scale=1.0):
         return (scale * torch.randn(shape, device=dev, generator=g)).contiguous()
     params = {"W1": rn(75, d1, scale=75 ** -0.5).to(torch.bfloat16), "W2": rn(4 * d1, d2, scale=(4 * d1) ** -0.5).to(
@@ -270,32 +456,27 @@ def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_
     return line
 
 
-def load_workload():
-    from encoder_free_audio_b200 import synth
-    wav, off = synth.batch64_10s()
-    table = synth.table()
-    g = synth.rms_weight()
-    return wav, off, table, g
-
+# ------------------------------------------------------------------------------------ arms
 
 def run_reference(args):
+    """The oracle on the host cores, on the headline workload: each step a bounded random sample
+    of its frames (codes + embedding + RMSNorm, fp64)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from oracle import oracle
     import torch
-    wav, off, table, g = load_workload()
-    tb = torch.from_numpy(table).to(torch.bfloat16).float().numpy().astype(np.float64)
-    gb = torch.from_numpy(g).to(torch.bfloat16).float().numpy().astype(np.float64)
+    wl = load_workload(HEADLINE)
+    tb, gb = host_tables(torch, wl)
     oracle.build()
-    F = int(oracle.frame_offsets(off)[-1])
+    F = int(oracle.frame_offsets(wl["off"])[-1])
     rng = np.random.default_rng(78)
-    per_step = 128
+    per_step = 96
     times = []
     for i in range(args.warmup + args.steps):
         ids = np.sort(rng.choice(F, per_step, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        c = oracle.codes(wav, off, frame_ids=ids, want_lhat=False)
+        c = oracle.codes(wl["wav"], wl["off"], frame_ids=ids, want_lhat=False)
         oracle.embed(c, tb, gb, 1e-6)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
@@ -306,7 +487,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "step": f"{per_step} random frames of the workload per step"},
+        "config": {"workload": DESCR[HEADLINE], "step": f"{per_step} random frames of the workload per step"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
                          "sample": f"{per_step} random frames per step, {args.steps} timed steps"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -326,21 +507,14 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     from encoder_free_audio_b200 import build, dmel, replicas
     from encoder_free_audio_b200.frontend import FrontEnd
     build.build()
-
-    wav, off, table, g = load_workload()
-    T = torch.from_numpy(table).to(torch.bfloat16).to(dev)
-    G = torch.from_numpy(g).to(torch.bfloat16).to(dev)
-    fe = FrontEnd(T, G, 1e-6, torch.bfloat16)
-    plan = fe.plan(off)
-    F = plan.n_frames
-    wav_d = torch.from_numpy(wav).to(dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    pk = peaks()
+    solo = rank == 0 and world == 1
+    with_cpu = solo and not args.no_cpu_baseline
 
     def barrier():
         torch.cuda.synchronize()
@@ -348,13 +522,8 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        return replicas.max_over_ranks(x, world, dev)
-
-    # ---------------------------------------------------------- device-resident timed region
-    for _ in range(args.warmup):
-        flush.zero_()
-        fe.forward(wav_d, plan)
+    # ---------------------------------------------------------- headline: ragged1024
+    wl = load_workload(HEADLINE)
     barrier()
     uuid = None
     try:
@@ -363,66 +532,36 @@ def run_ours(args):
         uuid = None
     sampler = ClockSampler(uuid)
     sampler.start()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    launches = 0
-    barrier()
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        fe.forward(wav_d, plan)
-        evs[i][1].record(stream)
-        launches += dmel.dmel_last_launch_count()
-    barrier()
-    step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(sum(step_ms))
-
-    # ---------------------------------------------------------- stage breakdown (same kernels)
-    # dmel_codes and dmel_embed called separately, each bracketed by events on the stream the
-    # kernels run on: the embedding stage is the dominant one.
-    ws = plan.workspace
-    codes_ms, embed_ms = [], []
-    for i in range(args.warmup + args.steps):
-        flush.zero_()
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        e0.record(stream)
-        dmel.dmel_codes(wav_d, plan.sample_offsets, plan.frame_offsets, F, plan.codes)
-        e1.record(stream)
-        dmel.dmel_embed(plan.codes, T, plan.out, rms_weight=G, eps=1e-6, workspace=ws)
-        e2.record(stream)
-        e2.synchronize()
-        if i >= args.warmup:
-            codes_ms.append(e0.elapsed_time(e1))
-            embed_ms.append(e1.elapsed_time(e2))
+    head = run_batch(torch, dev, dmel, FrontEnd, HEADLINE, wl, args.steps, args.warmup, pk, None, False, 0.0,
+                     with_e2e=True, e2e_steps=max(3, args.steps // 2))
     clocks = sampler.stop()
+    barrier()
+    F = head["frames"]
+    total_ms = replicas.max_over_ranks(sum(head["step_ms"]), world, dev)
+    e2e_ms = replicas.max_over_ranks(sum(head["e2e"]["ms"]), world, dev)
+    e2e_steps = len(head["e2e"]["ms"])
 
-    # ---------------------------------------------------------- end to end from host memory
-    wav_h = torch.from_numpy(wav).pin_memory()
-    codes_h = torch.empty((F, 80), dtype=torch.uint8).pin_memory()
-    for _ in range(args.warmup):
-        fe.forward_host(wav_h, plan, codes_h)
-    barrier()
-    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_evs[i][0].record(stream)
-        fe.forward_host(wav_h, plan, codes_h)
-        e2e_evs[i][1].record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
-    # ---------------------------------------------------------- streaming shape (context line)
-    # each context line runs inside an NVTX range of its name, so a profiler can list its launches
-    # alone (ncu --nvtx --nvtx-include "hmlp/")
+    # ---------------------------------------------------------- context lines
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     nvtx = torch.cuda.nvtx
+    ctx = {}
+    for name in ("batch64_10s", "long_20min"):
+        nvtx.range_push(name)
+        r = run_batch(torch, dev, dmel, FrontEnd, name, load_workload(name), args.steps, args.warmup, pk, flush,
+                      with_cpu, 3.0)
+        ctx[name] = context_line(name, r, pk, world)
+        nvtx.range_pop()
+    nvtx.range_push("one_clip_2s")
+    ctx["one_clip_2s"] = latency_line(torch, dev, dmel, FrontEnd, pk, max(100, 10 * args.steps), with_cpu)
+    nvtx.range_pop()
     nvtx.range_push("streaming")
-    stream_line = streaming_latency(torch, dev, T, G, FrontEnd, dmel, args.warmup)
+    ctx["streams4096"] = streaming_line(torch, dev, dmel, FrontEnd, pk, args.stream_calls, args.warmup, with_cpu)
     nvtx.range_pop()
     nvtx.range_push("shortconv")
-    shortconv_line = shortconv_context(torch, dev, dmel, peaks(), args.warmup,
-                                       with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    ctx["shortconv"] = shortconv_context(torch, dev, dmel, pk, args.warmup, with_oracle=with_cpu)
     nvtx.range_pop()
     nvtx.range_push("hmlp")
-    hmlp_line = hmlp_context(torch, dev, dmel, peaks(), args.warmup,
-                             with_oracle=rank == 0 and world == 1 and not args.no_cpu_baseline)
+    ctx["hmlp"] = hmlp_context(torch, dev, dmel, pk, args.warmup, with_oracle=with_cpu)
     nvtx.range_pop()
     err_bits = dmel.dmel_get_device_error(clear=True)
 
@@ -432,10 +571,10 @@ def run_ours(args):
             dist.destroy_process_group()
         return 0
 
-    pk = peaks()
     value = replicas.job_throughput([F * args.steps] * world, total_ms / 1e3)
-    emb_avg_s = statistics.mean(embed_ms) / 1e3
-    emb_achieved = EMBED_BYTES_PER_FRAME * F / emb_avg_s / 1e9
+    st = head["stages"]
+    dom = max(st, key=lambda k: st[k]["ms"])
+    emb_s = st["embed"]["ms"] / 1e3
     line = {
         "metric": METRIC,
         "value": value,
@@ -449,34 +588,30 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "frames_per_gpu": F, "parallelism": f"replicas x{world}",
-                   "l2": "flushed between timed steps (256 MB write)",
+        "config": {"workload": DESCR[HEADLINE], "frames_per_gpu": F, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (1.02 GB of samples in, 3.9 GB of vectors out per step)",
                    "compute": "fp64 transform, 2:4-sparse bf16 x bf16 -> fp32 tensor-core sum, bf16 out"},
-        "hbm_roofline_frac": PATH_BYTES_PER_FRAME * value / world / (pk["hbm_gbs"] * 1e9),
+        "hbm_roofline_frac": head["path_bytes_per_frame"] * value / world / (pk["hbm_gbs"] * 1e9),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
-        "e2e": {"value": world * F * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(wav.nbytes), "d2h_bytes_per_step": int(F * 80)},
-        "gpu_launches": launches,
-        "roofline": {"bound": "hbm", "achieved": emb_achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": emb_achieved / pk["hbm_gbs"], "traffic": EMBED_TRAFFIC_PER_LAUNCH,
-                     "kernel": "embed_sp_kernel (2:4-sparse tcgen05, fused RMSNorm, CTA pairs), timed as the dmel_embed call",
-                     "peak_source": pk["source"]},
-        "roofline_tensor": {"achieved": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12,
+        "e2e": {"value": world * F * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": head["e2e"]["h2d_bytes_per_step"],
+                "d2h_bytes_per_step": head["e2e"]["d2h_bytes_per_step"],
+                "api": "dmel_forward_host (page-locked host samples in, page-locked host vectors out)"},
+        "gpu_launches": int(sum(head["launches"])),
+        "roofline": {k: v for k, v in st[dom].items() if k != "ms"},
+        "roofline_stages": st,
+        "roofline_tensor": {"achieved": ONEHOT_FLOP_PER_FRAME * F / emb_s / 1e12,
                             "peak": SPARSE_PEAK_RATIO * pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                            "frac": ONEHOT_FLOP_PER_FRAME * F / emb_avg_s / 1e12
+                            "frac": ONEHOT_FLOP_PER_FRAME * F / emb_s / 1e12
                             / (SPARSE_PEAK_RATIO * pk["bf16_tflops_sustained"]),
-                            "note": "one-hot product, 2*1280*6144 logical flops per frame, against the 2:4-sparse "
-                                    "bf16 peak = measured sustained dense bf16 x 2 (nominal ratio)"},
-        "stages_ms": {"codes": statistics.mean(codes_ms), "embed": statistics.mean(embed_ms)},
-        "streaming": stream_line,
-        "shortconv": shortconv_line,
-        "hmlp": hmlp_line,
+                            "note": "embedding's one-hot product, 2*1280*6144 logical flops per frame, against the "
+                                    "2:4-sparse bf16 peak = measured sustained dense bf16 x 2 (nominal ratio)"},
+        "context": ctx,
         "device_error_bits": err_bits,
     }
-    if not args.no_cpu_baseline and world == 1:
-        tb = T.float().cpu().numpy().astype(np.float64)
-        gb = G.float().cpu().numpy().astype(np.float64)
-        line["cpu_baseline"] = cpu_baseline(wav, off, tb, gb)
+    if with_cpu:
+        tb, gb = host_tables(torch, wl)
+        line["cpu_baseline"] = oracle_sample(wl["wav"], wl["off"], tb, gb, 12.0, 77)
     print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -490,6 +625,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--stream-calls", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps

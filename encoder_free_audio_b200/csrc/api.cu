@@ -232,6 +232,54 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                            workspace_bytes, stream);
 }
 
+namespace {
+// Host sample offsets of dmel_forward_host: start 0, non-decreasing.
+bool host_offsets_ok(const int64_t *so, int n_clips) {
+  if (!so || n_clips < 0 || so[0] != 0) return false;
+  for (int c = 0; c < n_clips; ++c)
+    if (so[c + 1] < so[c]) return false;
+  return true;
+}
+constexpr int64_t kDefaultChunkFrames = 8192;
+}  // namespace
+
+size_t dmel_forward_host_workspace_size(const int64_t *h_sample_offsets, int n_clips, int embed_dim,
+                                        dmel_dtype table_dtype, dmel_dtype out_dtype, int with_rmsnorm,
+                                        int64_t chunk_frames) {
+  if (!host_offsets_ok(h_sample_offsets, n_clips) || embed_dim <= 0 || chunk_frames < 0) return 0;
+  if (!dtype_ok(table_dtype) || !dtype_ok(out_dtype)) return 0;
+  return forward_host_workspace_bytes(h_sample_offsets, n_clips, embed_dim, table_dtype, out_dtype, with_rmsnorm,
+                                      chunk_frames ? chunk_frames : kDefaultChunkFrames);
+}
+
+dmel_status dmel_forward_host(const float *h_wav, const int64_t *h_sample_offsets, int n_clips, const void *table,
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *h_out,
+                              dmel_dtype out_dtype, uint8_t *h_codes, int64_t chunk_frames, void *workspace,
+                              size_t workspace_bytes, dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (!host_offsets_ok(h_sample_offsets, n_clips) || chunk_frames < 0) return DMEL_ERR_INVALID_ARG;
+  int64_t F = 0;
+  for (int c = 0; c < n_clips; ++c) F += dmel_frames_for_length(h_sample_offsets[c + 1] - h_sample_offsets[c]);
+  if (F > 0 && (!h_wav || !h_out)) return DMEL_ERR_INVALID_ARG;
+  // the embedding arguments (the codes live in the workspace)
+  dmel_status st = check_embed_args(nullptr, false, F, table, table_dtype, embed_dim, rms_weight, eps, h_out,
+                                    out_dtype);
+  if (st != DMEL_OK || F == 0) return st;
+  if (workspace && !aligned(workspace, 256)) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  bool too_small = false;
+  cudaError_t e = run_forward_host(h_wav, h_sample_offsets, n_clips, table, table_dtype, embed_dim, rms_weight, eps,
+                                   h_out, out_dtype, h_codes, chunk_frames ? chunk_frames : kDefaultChunkFrames,
+                                   workspace, workspace_bytes, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream),
+                                   &launches, &too_small);
+  if (too_small) return DMEL_ERR_INVALID_ARG;
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
 dmel_status dmel_shortconv(const void *x, const int64_t *seq_offsets, int n_seq, int64_t n_tokens, int channels,
                            const float *weights, const void *state, void *state_out, void *y, dmel_dtype dtype,
                            dmel_stream_t stream) {
@@ -393,6 +441,14 @@ dmel_status dmel_debug_codes_frame_host_q(const float *frame1600, const dmel_qua
   Quant qz;
   if (!frame1600 || !codes80 || !to_quant(q, &qz)) return DMEL_ERR_INVALID_ARG;
   emulate_codes_frame_host(frame1600, codes80, lhat80, qz);
+  return DMEL_OK;
+}
+
+dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_clips, int64_t chunk_frames,
+                                         int64_t *h_plan, int64_t cap, int64_t *h_len) {
+  if (!host_offsets_ok(h_sample_offsets, n_clips) || chunk_frames <= 0 || !h_len || cap < 0 || (cap > 0 && !h_plan))
+    return DMEL_ERR_INVALID_ARG;
+  *h_len = debug_forward_host_plan(h_sample_offsets, n_clips, chunk_frames, h_plan, cap);
   return DMEL_OK;
 }
 

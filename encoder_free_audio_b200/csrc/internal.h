@@ -38,6 +38,21 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *tab
                          void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
                          const int64_t *out_rows = nullptr, int64_t out_n_rows = 0);
 
+// dmel_forward_host: workspace bytes for this batch (0 when it has no frame) and the pipelined
+// run (host samples in, host vectors and codes out; streams and events of the library's own).
+// *too_small is set (and nothing queued) when the workspace is smaller than the first reports.
+size_t forward_host_workspace_bytes(const int64_t *h_sample_offsets, int n_clips, int embed_dim,
+                                    dmel_dtype table_dtype, dmel_dtype out_dtype, int with_rmsnorm,
+                                    int64_t chunk_frames);
+cudaError_t run_forward_host(const float *h_wav, const int64_t *h_sample_offsets, int n_clips, const void *table,
+                             dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *h_out,
+                             dmel_dtype out_dtype, uint8_t *h_codes, int64_t chunk_frames, void *workspace,
+                             size_t workspace_bytes, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
+                             bool *too_small);
+// The plan of run_forward_host flattened for dmel_debug_forward_host_plan; returns its length.
+int64_t debug_forward_host_plan(const int64_t *h_sample_offsets, int n_clips, int64_t chunk_frames, int64_t *h_plan,
+                                int64_t cap);
+
 // Size of the fixed device scratch used by dmel_embed_noalloc.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 

@@ -104,6 +104,12 @@ def _lib():
         L.dmel_debug_codes_frame_host_q.restype = i32
         L.dmel_codes_q.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, ctypes.POINTER(Quantizer), vp]
         L.dmel_codes_q.restype = i32
+        L.dmel_forward_host_workspace_size.argtypes = [vp, i32, i32, i32, i32, i32, i64]
+        L.dmel_forward_host_workspace_size.restype = sz
+        L.dmel_forward_host.argtypes = [vp, vp, i32, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, i64, vp, sz, vp]
+        L.dmel_forward_host.restype = i32
+        L.dmel_debug_forward_host_plan.argtypes = [vp, i32, i64, vp, i64, ctypes.POINTER(i64)]
+        L.dmel_debug_forward_host_plan.restype = i32
         _L = L
     return _L
 
@@ -171,6 +177,30 @@ def dmel_codes(wav, sample_offsets, frame_offsets, n_frames: int, codes, tails=N
     rc = _lib().dmel_codes(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames), _ptr(tails),
                            _ptr(tails_out), _ptr(codes), _stream(stream))
     _check(rc, "dmel_codes")
+
+
+def dmel_forward_host_workspace_size(sample_offsets, embed_dim: int, table_dtype: int, out_dtype: int,
+                                     with_rmsnorm: bool, chunk_frames: int = 0) -> int:
+    """Device workspace bytes of dmel_forward_host for these host sample offsets."""
+    so = np.ascontiguousarray(np.asarray(sample_offsets, dtype=np.int64))
+    return int(_lib().dmel_forward_host_workspace_size(so.ctypes.data_as(ctypes.c_void_p), so.shape[0] - 1,
+                                                       int(embed_dim), int(table_dtype), int(out_dtype),
+                                                       int(bool(with_rmsnorm)), int(chunk_frames)))
+
+
+def dmel_forward_host(wav_host, sample_offsets, table, out_host, rms_weight=None, eps: float = 1e-6, codes_host=None,
+                      chunk_frames: int = 0, workspace=None, stream=None):
+    """dmel_forward_host: wav_host a host (pinned) fp32 torch tensor, sample_offsets host int64
+    (numpy or list), table / rms_weight / workspace torch CUDA tensors, out_host a host tensor
+    [F, D] (bf16 or fp32), codes_host None or host uint8 [F, 80]. Asynchronous on the stream."""
+    so = np.ascontiguousarray(np.asarray(sample_offsets, dtype=np.int64))
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_forward_host(ctypes.c_void_p(wav_host.data_ptr()), so.ctypes.data_as(ctypes.c_void_p),
+                                  so.shape[0] - 1, _ptr(table), _dtype_code(table), int(table.shape[1]),
+                                  _ptr(rms_weight), ctypes.c_float(eps), ctypes.c_void_p(out_host.data_ptr()),
+                                  _dtype_code(out_host), _ptr(codes_host), int(chunk_frames), _ptr(workspace),
+                                  ws_bytes, _stream(stream))
+    _check(rc, "dmel_forward_host")
 
 
 class HmlpWeights(ctypes.Structure):
@@ -361,3 +391,25 @@ def dmel_debug_wait_timeout(polls: int = 1 << 16) -> int:
     rc = _lib().dmel_debug_wait_timeout(int(polls), ctypes.byref(bits))
     _check(rc, "dmel_debug_wait_timeout")
     return int(bits.value)
+
+
+def dmel_debug_forward_host_plan(sample_offsets, chunk_frames: int) -> list:
+    """dmel_forward_host's chunk plan (diagnostic, see dmel_debug.h) as a list of dicts with keys
+    f0, f1, s_lo, s_hi, tail, so, fo."""
+    so = np.ascontiguousarray(np.asarray(sample_offsets, dtype=np.int64))
+    n = ctypes.c_int64(0)
+    _check(_lib().dmel_debug_forward_host_plan(so.ctypes.data_as(ctypes.c_void_p), so.shape[0] - 1,
+                                               int(chunk_frames), None, 0, ctypes.byref(n)),
+           "dmel_debug_forward_host_plan")
+    buf = np.zeros(max(1, n.value), np.int64)
+    _check(_lib().dmel_debug_forward_host_plan(so.ctypes.data_as(ctypes.c_void_p), so.shape[0] - 1,
+                                               int(chunk_frames), buf.ctypes.data_as(ctypes.c_void_p), n.value,
+                                               ctypes.byref(n)), "dmel_debug_forward_host_plan")
+    out, i = [], 0
+    while i < n.value:
+        f0, f1, s_lo, s_hi, tail, k = (int(v) for v in buf[i:i + 6])
+        i += 6
+        out.append({"f0": f0, "f1": f1, "s_lo": s_lo, "s_hi": s_hi, "tail": bool(tail),
+                    "so": buf[i:i + k + 1].copy(), "fo": buf[i + k + 1:i + 2 * k + 2].copy()})
+        i += 2 * k + 2
+    return out

@@ -173,6 +173,43 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                          dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
                          dmel_stream_t stream);
 
+/* ---- End to end from host memory: dmel_forward for a batch held in host memory, returning the
+ * frame vectors (and optionally the codes) to host memory, with the copies overlapped with the
+ * kernels ("Inside Inkling: Audio Design", Part 1 · Modeling for what is computed; Part 3 ·
+ * Inference describes featurisation as work done on the host at render time, which is where
+ * such batches come from).
+ *
+ * h_wav             host fp32 samples of all clips, concatenated with no padding
+ * h_sample_offsets  host int64 [n_clips + 1] (start 0, non-decreasing)
+ * table, table_dtype, embed_dim, rms_weight, eps, out_dtype: as in dmel_embed (device memory)
+ * h_out             host [F x embed_dim] in out_dtype, F = the frame count dmel_frame_offsets gives;
+ *                   16-byte aligned
+ * h_codes           NULL, or host uint8 [F x 80] to receive the codes
+ * chunk_frames      frames per pipeline chunk (0: 8192); a chunk may start or end inside a clip
+ *                   (its first frame then takes the 800 samples before it from the clip), and the
+ *                   results do not depend on it
+ * workspace         device scratch of dmel_forward_host_workspace_size(...) bytes with the same
+ *                   offsets, widths, types, RMSNorm flag and chunk_frames, 256-byte aligned
+ *
+ * The frames are cut into chunks; per chunk the samples go to the device on a copy stream of the
+ * library's own, the codes and embedding kernels run on `stream`, and the vectors come back on a
+ * second copy stream; two device buffer sets alternate, so chunk i + 1 is copied in and chunk
+ * i - 1 copied out while chunk i computes. Host buffers should be page-locked (cudaHostAlloc or
+ * cudaHostRegister) for the copies to overlap; pageable memory gives the same results, copied
+ * synchronously. Asynchronous like every call: the results are in host memory once `stream`
+ * reaches the point of the call (cudaStreamSynchronize(stream) waits for them). The host arrays
+ * must stay valid and unchanged until then. The first call on a device creates the two copy
+ * streams. Errors: DMEL_ERR_INVALID_ARG for bad offsets, a NULL h_wav / h_out with frames to
+ * compute, the embedding's argument errors, a negative chunk_frames or a workspace smaller than
+ * reported. */
+size_t dmel_forward_host_workspace_size(const int64_t *h_sample_offsets, int n_clips, int embed_dim,
+                                        dmel_dtype table_dtype, dmel_dtype out_dtype, int with_rmsnorm,
+                                        int64_t chunk_frames);
+dmel_status dmel_forward_host(const float *h_wav, const int64_t *h_sample_offsets, int n_clips, const void *table,
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *h_out,
+                              dmel_dtype out_dtype, uint8_t *h_codes, int64_t chunk_frames, void *workspace,
+                              size_t workspace_bytes, dmel_stream_t stream);
+
 /* ---- Quantiser variants. The pages leave the level mapping open ("Inside Inkling: Audio
  * Design", Coda: the quantizer mapping is undocumented, uniform or mu-law or learned, and the
  * serving default clamps the log-mel value at -1.5 where the released config says -7.0). With L

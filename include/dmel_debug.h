@@ -37,6 +37,20 @@ dmel_status dmel_debug_wait_timeout(uint32_t polls, uint32_t *h_bits);
  * against the exact function. x, y: device fp32 [n], 16-byte aligned. Asynchronous on stream. */
 dmel_status dmel_debug_gelu(const float *x, float *y, int64_t n, dmel_stream_t stream);
 
+/* The chunk plan dmel_forward_host follows for these host sample offsets (host only, pure).
+ * Writes, chunk after chunk, into h_plan (at most cap int64 values):
+ *   f0, f1          the chunk's frames [f0, f1) of the batch
+ *   s_lo, s_hi      the host samples [s_lo, s_hi) it copies to the device
+ *   tail            1 when its first piece starts inside its clip (the first 800 copied samples
+ *                   are then that piece's tail, the rest its samples), else 0
+ *   n               its number of pieces (one per clip with frames in the chunk)
+ *   so[n + 1]       the pieces' sample offsets within the copied samples (after the tail)
+ *   fo[n + 1]       the pieces' frame offsets within the chunk
+ * *h_len receives the number of int64 values the whole plan needs (so a call with cap 0 sizes
+ * it). Returns DMEL_ERR_INVALID_ARG for bad offsets or chunk_frames <= 0. */
+dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_clips, int64_t chunk_frames,
+                                         int64_t *h_plan, int64_t cap, int64_t *h_len);
+
 #ifdef __cplusplus
 }
 #endif

@@ -365,21 +365,22 @@ def test_forward_batch64_10s(table_bf16, rmsw_bf16, oracle_mod):
 
 
 def test_forward_host_pipelined_equals_single_call(table_bf16, rmsw_bf16):
-    """The host path (copies of run i + 1 overlapping the kernels of run i) gives the same
-    vectors and codes, bit for bit, as one device-side call on the whole batch."""
+    """The host path (copies of chunk i + 1 and i - 1 overlapping the kernels of chunk i) gives
+    the same vectors and codes, bit for bit, as one device-side call on the whole batch."""
     T, _ = table_bf16
     g, _ = rmsw_bf16
     wav, off = synth.ragged1024(n_clips=40)
     fe = FrontEnd(T, g, 1e-6, torch.bfloat16)
     one = fe.plan(off)
     fe.forward(torch.from_numpy(wav).to(DEV), one)
-    for chunks in (1, 3, 7):
-        p = fe.plan(off, chunks=chunks)
+    for chunk in (97, 1000, 0):
+        p = fe.plan(off, chunk_frames=chunk, host_path=True)
+        out_h = torch.empty((p.n_frames, T.shape[1]), dtype=torch.bfloat16).pin_memory()
         codes_h = torch.empty((p.n_frames, 80), dtype=torch.uint8).pin_memory()
-        fe.forward_host(torch.from_numpy(wav).pin_memory(), p, codes_h)
+        fe.forward_host(torch.from_numpy(wav).pin_memory(), p, out_h, codes_h)
         torch.cuda.synchronize()
-        assert torch.equal(p.out, one.out), chunks
-        assert torch.equal(codes_h, one.codes.cpu()), chunks
+        assert torch.equal(out_h, one.out.cpu()), chunk
+        assert torch.equal(codes_h, one.codes.cpu()), chunk
 
 
 def test_forward_long_20min(table_bf16, rmsw_bf16, oracle_mod):
