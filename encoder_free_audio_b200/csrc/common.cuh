@@ -313,6 +313,7 @@ __host__ __device__ constexpr uint64_t smem_desc(uint32_t addr, uint32_t lbo_byt
 }
 constexpr uint32_t kSwizzle128B = 2;
 constexpr uint32_t kSwizzle64B = 4;
+constexpr uint32_t kSwizzle32B = 6;
 
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, A K-major,
 // B K-major (b_mn_major = 0) or MN-major (1), shape M x N.

@@ -879,10 +879,10 @@ __global__ void __launch_bounds__(tc2::THREADS, 1)
 // (0, 1) with zeros), so the 16 logical columns become 8 stored bf16 (16 bytes) with the 1 at
 // position 2 (c >> 2) + (c & 1), and 16 bits of metadata (a nibble of two 2-bit row positions
 // per group). The metadata lives in TMEM, one 32-bit column per MMA (logical K = 32, two bins).
-// Tiles are 256 frames x 176 columns: two fp32 accumulators at TMEM columns 0 and 256 leave
-// columns 496..511 for a four-stage metadata ring. With RMSNorm, groups of ceil(D / 176)
-// clusters (35 at D = 6144, two groups on 148 SMs) own fixed column slices and walk the same
-// frame tiles together; each row's sum of squares
+// Tiles are 256 frames x 192 columns: two fp32 accumulators at TMEM columns 0 and 256, three
+// 32-column A slots at 192, 224 and 448 and a three-stage metadata ring at 480..491. With
+// RMSNorm, groups of ceil(D / 192) clusters (32 at D = 6144, two groups, 64 clusters, on 148
+// SMs) own fixed column slices and walk the same frame tiles together; each row's sum of squares
 // over a slice is published into a buffer pre-filled with a sentinel and the other slices'
 // sums are read as they appear (all clusters are co-resident under the cooperative launch).
 // An mbarrier wait in the thread that issues tcgen05.mma stalls that thread behind its queued
@@ -1363,6 +1363,426 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- column-stationary sparse product
+//
+// The same 2:4-sparse one-hot product as embed_sp_kernel, with the table read from memory once
+// per launch instead of once per frame tile. Cluster c (a CTA pair) owns the column slice
+// [n0_c, n0_c + N_c) of the output: the D / 32 units of 32 columns are spread over the clusters,
+// so N_c is 64 or 96 at D = 6144 on 74 clusters. Each CTA keeps its N_c / 2 columns of all 1280
+// table rows resident in shared memory (MN-major, 32-byte swizzle atoms of 16 columns, 120 KB at
+// most), and every cluster walks every 256-frame pair tile. Per tile the 8 producer warps write
+// the compressed one-hot A and its metadata into TMEM (even and odd stages by two warps of each
+// lane quarter), the MMA warp issues M = 256, N = N_c, logical K = 32 sparse MMAs from a waiter
+// warp's handoffs, and three TMEM accumulators let the MMAs run two tiles ahead of the epilogue.
+//
+// RMSNorm, without a buffer that grows with the batch: each cluster publishes its rows' sums of
+// squares over its slice as 64-bit words (value bits | (pair tile + 1) << 32) in a ring of four
+// pair tiles; cluster c reduces rows R = c, c + ncl, ... of each pair tile (one warp per row
+// sums the ncl partials in a fixed order) and publishes the total the same way; each CTA then
+// reads the totals of its 128 rows. A ring slot is rewritten for tile t + 4 only after every
+// cluster has read tile t: a cluster publishes tile t + 4 only after it finished tile t + 3,
+// whose totals need every cluster's partial of tile t + 3, which a cluster writes only after it
+// finished tile t + 2. The ring is zeroed before each launch, so no tag from an earlier launch
+// can match.
+namespace cs {
+constexpr int BM = 128;                      // frames per CTA (TMEM lanes)
+constexpr int MAX_N = 96;                    // columns per cluster, at most
+constexpr int UNIT = 32;                     // slice widths are multiples of 32 columns
+constexpr int ATOM = 16;                     // 32-byte swizzle atom: 16 columns x 8 rows
+constexpr int B_ATOM_BYTES = kRows * 32;     // one resident atom column: 1280 rows x 32 bytes
+constexpr int MAX_ATOMS = MAX_N / 2 / ATOM;  // 3 per CTA
+constexpr int BKL = 128;                     // logical K per stage: 8 bins
+constexpr int KSTAGES = kRows / BKL;         // 10
+constexpr int B_BOX = BKL * 32;              // TMA box: 16 columns x 128 rows = 4 KB
+constexpr int STAGES_A = 4;                  // A + metadata slots in TMEM
+constexpr int N_ACC = 3;
+constexpr uint32_t ACC_STRIDE = 128;         // accumulators at TMEM columns 0, 128, 256 (N <= 96 used)
+constexpr uint32_t META_COL = 96;            // metadata slots at 96, 100, 104, 108 (after accumulator 0)
+constexpr uint32_t A_COL0 = 384;             // A slots at 384, 416, 448, 480 (32 columns each)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int PROD_WARPS = 8;                // warps 0..7: lane quarter w & 3, stage parity w >> 2
+constexpr int W_EPI0 = 8;                    // warps 8..15: lane quarter w & 3, column half
+constexpr int EPI_WARPS = 8;
+constexpr int W_TMA = 16, W_MMA = 17, W_WAIT = 18;
+constexpr int THREADS = 32 * 19;
+constexpr int RING = 4;                      // pair tiles in the RMSNorm exchange ring
+constexpr int MAX_CLUSTERS = 128;            // ring sized for up to 256 SMs
+constexpr int OFF_B = 0;
+constexpr int OFF_BAR = OFF_B + MAX_ATOMS * B_ATOM_BYTES;
+constexpr int N_BARS = 2 * STAGES_A + KSTAGES + 2 * N_ACC + 1;
+constexpr int OFF_G = OFF_BAR + 256;         // RMSNorm weights of the slice (fp32)
+constexpr int OFF_EPI = OFF_G + MAX_N * 4;   // row sums of the two column halves [2][128], scales [128]
+constexpr int STG_ROW_MAX = MAX_N / 2 * 4 + 16;  // staging row: up to 48 fp32 + 16 bytes of pad
+constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;
+constexpr int SMEM_USED = OFF_STG + EPI_WARPS * 32 * STG_ROW_MAX;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;
+static_assert(KSTAGES * BKL == kRows && KSTAGES % 2 == 0, "stages cover the table; parity splits them");
+static_assert(MAX_N <= (int)META_COL && META_COL + 4 * STAGES_A <= ACC_STRIDE && N_ACC * ACC_STRIDE <= A_COL0 &&
+                  A_COL0 + 32 * STAGES_A <= TMEM_COLS, "TMEM map");
+static_assert(N_BARS * 8 + 16 <= 256, "barrier area");
+static_assert(OFF_STG % 16 == 0 && SMEM_BYTES <= 227 * 1024, "shared memory budget");
+}  // namespace cs
+
+// Ring bytes of the column-stationary kernel's RMSNorm exchange (partials, then totals).
+__host__ __device__ constexpr size_t cs_ring_words(int ncl) {
+  return (size_t)cs::RING * 2 * cs::BM * (size_t)ncl + (size_t)cs::RING * 2 * cs::BM;
+}
+
+// Named barriers 2..5 ("stage slot j is ready", waiter arrives, MMA warp syncs) and 6..9
+// ("stage slot j was issued", MMA warp arrives, waiter syncs), j = stage mod 4.
+__device__ __forceinline__ void cs_ready_arrive(int j) { asm volatile("bar.arrive %0, 64;" ::"r"(2 + j) : "memory"); }
+__device__ __forceinline__ void cs_ready_sync(int j) { asm volatile("bar.sync %0, 64;" ::"r"(2 + j) : "memory"); }
+__device__ __forceinline__ void cs_issued_arrive(int j) { asm volatile("bar.arrive %0, 64;" ::"r"(6 + j) : "memory"); }
+__device__ __forceinline__ void cs_issued_sync(int j) { asm volatile("bar.sync %0, 64;" ::"r"(6 + j) : "memory"); }
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// The 16 metadata bits of one bin at level c (see sp_meta_field), computed without a branch.
+__device__ __forceinline__ uint32_t cs_meta16(uint32_t c) {
+  return 0x4444u | (((c & 2u) * 5u) << ((c >> 2) << 2));
+}
+
+template <typename OT, bool kRms>
+__global__ void __launch_bounds__(cs::THREADS, 1)
+    embed_cs_kernel(const __grid_constant__ CUtensorMap tmap, const uint8_t *__restrict__ codes, int64_t F, int D,
+                    OT *__restrict__ out, OutMap om, unsigned long long *__restrict__ ring,
+                    const __nv_bfloat16 *__restrict__ gw, float eps, uint32_t *err) {
+  using namespace cs;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+  // this cluster's column slice
+  const int U = D / UNIT, uq = U / ncl, ur = U % ncl;
+  const int N = UNIT * (uq + (cid < ur ? 1 : 0));
+  const int n0 = UNIT * (cid * uq + (cid < ur ? cid : ur));
+  const int NH = N / 2;  // columns each CTA holds, and each epilogue warp of a lane quarter stores
+  const int64_t n_pm = (F + 2 * BM - 1) / (2 * BM);
+  const int64_t n_m_tiles = (F + BM - 1) / BM;
+
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  const uint32_t bar0 = smem_addr(bars);
+  auto full_a = [&](int s) { return bar0 + 8u * s; };
+  auto empty_a = [&](int s) { return bar0 + 8u * (STAGES_A + s); };
+  auto bfull = [&](int k) { return bar0 + 8u * (2 * STAGES_A + k); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * STAGES_A + KSTAGES + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * STAGES_A + KSTAGES + N_ACC + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES_A + KSTAGES + 2 * N_ACC);
+  auto in_leader = [&](uint32_t local_bar) { return mapa_shared(local_bar, 0); };
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+  float *gsm = reinterpret_cast<float *>(smem + OFF_G);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES_A; ++s) {
+      mbar_init(full_a(s), 8);  // the 4 producer warps of a stage parity in each CTA
+      mbar_init(empty_a(s), 1);
+    }
+    for (int k = 0; k < KSTAGES; ++k) mbar_init(bfull(k), 1);  // the leader's expect-tx for both halves
+    for (int a = 0; a < N_ACC; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 2 * EPI_WARPS);  // epilogue warps of both CTAs
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (kRms && threadIdx.x < N) gsm[threadIdx.x] = __bfloat162float(gw[n0 + threadIdx.x]);
+  if (warp == W_MMA) {
+    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == W_TMA && lane == 0) tma_prefetch_desc(&tmap);
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const uint32_t b_base = smem_addr(smem + OFF_B);
+
+  if (warp == W_TMA) {
+    // ------------------------------------------------ this CTA's columns of the whole table, once
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      const int atoms = NH / ATOM;
+      const int c0 = n0 + (int)rank * NH;
+      for (int k = 0; k < KSTAGES; ++k) {
+        if (leader) mbar_arrive_expect_tx(bfull(k), 2u * atoms * B_BOX);
+        for (int a = 0; a < atoms; ++a)
+          tma_load_2d_pair(b_base + a * B_ATOM_BYTES + k * B_BOX, &tmap, c0 + ATOM * a, k * BKL, in_leader(bfull(k)),
+                           pol);
+      }
+    }
+  } else if (warp == W_MMA) {
+    // ------------------------------------------------ MMA issue (even CTA): stages come from the waiter
+    if (leader) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BM, (uint32_t)N, 1) | kIdescSparse;
+      int sa = 0;
+      for (int64_t i = 0; i < n_pm; ++i) {
+        const uint32_t acc = (uint32_t)(i % N_ACC);
+        const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
+        for (int s = 0; s < KSTAGES; ++s) {
+          cs_ready_sync(sa);
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t a0 = tmem_base + A_COL0 + 32u * sa;
+#pragma unroll
+            for (int k = 0; k < BKL / 32; ++k) {
+              // 32 table rows per MMA (32 x 32 bytes in each atom column); atom columns B_ATOM_BYTES apart
+              const uint64_t bdesc =
+                  smem_desc(b_base + (uint32_t)(s * BKL + 32 * k) * 32u, (uint32_t)B_ATOM_BYTES, 256u, kSwizzle32B);
+              const uint32_t mcol = META_COL + 4u * sa + k;
+              tc_mma_sp_pair_ts(d_tmem, a0 + 8u * k, bdesc, idesc | (mcol & 1u), tmem_base + (mcol & ~1u),
+                                (s | k) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair_both(empty_a(sa), 3);
+            if (s == KSTAGES - 1) tc_commit_pair_both(tfull(acc), 3);
+          }
+          __syncwarp();
+          cs_issued_arrive(sa);
+          sa = (sa + 1) & (STAGES_A - 1);
+        }
+      }
+      if (lane == 0) {
+        tc_commit_pair(done_bar);
+        mbar_wait(done_bar, 0, err);
+      }
+    }
+  } else if (warp == W_WAIT) {
+    // ------------------------------------------------ waits on behalf of the MMA warp (even CTA)
+    if (leader) {
+      bool ok = true;  // after a timed-out wait: no more waiting, stages still handed over
+      uint32_t pmask = 0;
+      int64_t n = 0;
+      for (int64_t i = 0; i < n_pm; ++i) {
+        const uint32_t acc = (uint32_t)(i % N_ACC), acc_phase = (uint32_t)((i / N_ACC) & 1);
+        for (int s = 0; s < KSTAGES; ++s, ++n) {
+          const int sa = (int)(n & (STAGES_A - 1));
+          if (n >= STAGES_A) cs_issued_sync(sa);  // stage n - 4 (same slot) was issued
+          if (lane == 0 && ok) {
+            if (s == 0) ok = mbar_wait(tempty(acc), acc_phase ^ 1u, err);
+            ok = ok && mbar_wait(full_a(sa), (pmask >> sa) & 1u, err);
+            if (i == 0) ok = ok && mbar_wait(bfull(s), 0, err);
+          }
+          pmask ^= 1u << sa;
+          __syncwarp();
+          cs_ready_arrive(sa);
+        }
+      }
+      for (int64_t q = n > STAGES_A ? n - STAGES_A : 0; q < n; ++q) cs_issued_sync((int)(q & (STAGES_A - 1)));
+    }
+  } else if (warp < PROD_WARPS) {
+    // ------------------------------------------------ compressed one-hot A + metadata into TMEM
+    const int quad = warp & 3, par = warp >> 2;  // stages with s % 2 == par
+    const int r = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(quad * 32) << 16);
+    // metadata lane order: lane t takes rows (t & 7) + 16 (t >> 4) and + 8 for bin (t >> 3) & 1
+    // of the MMA's two: one exchange with lane t ^ 8, then a byte permute
+    const uint32_t msel = (lane & 8) ? 0x3276u : 0x5410u;
+    uint32_t pmask = 0;
+    bool ok = true;
+    // codes of this row for this warp's stages s = par + 2 j: bytes 8 s .. 8 s + 7
+    auto load_codes = [&](int64_t i_, uint2 (&u)[5]) {
+      const int64_t f_ = (2 * i_ + rank) * BM + r;
+      if (i_ < n_pm && f_ < F) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(codes + f_ * kMel) + par;
+#pragma unroll
+        for (int j = 0; j < 5; ++j) u[j] = __ldg(src + 2 * j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 5; ++j) u[j] = make_uint2(0u, 0u);
+      }
+    };
+    uint2 next[5];
+    load_codes(0, next);
+    for (int64_t i = 0; ok && i < n_pm; ++i) {
+      const bool valid = (2 * i + rank) * BM + r < F;
+      uint2 cw[5];
+#pragma unroll
+      for (int j = 0; j < 5; ++j) cw[j] = next[j];
+      load_codes(i + 1, next);
+      if (valid) {
+        uint32_t bad = 0;
+#pragma unroll
+        for (int j = 0; j < 5; ++j) bad |= (cw[j].x | cw[j].y) & 0xF0F0F0F0u;
+        if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
+      }
+      const uint32_t one_mask = valid ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        const int s = par + 2 * j;
+        const int sa = (int)((i * KSTAGES + s) & (STAGES_A - 1));
+        if (!__all_sync(0xffffffffu, mbar_wait(empty_a(sa), ((pmask >> sa) & 1u) ^ 1u, err))) { ok = false; break; }
+        pmask ^= 1u << sa;
+        // bin b of the stage at level c: stored bf16 8b .. 8b + 7 (columns 4b .. 4b + 3), the 1
+        // in column 4b + (c >> 2), low half when c is even
+        uint32_t av[32], cc[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          const uint32_t c = ((b < 4 ? cw[j].x : cw[j].y) >> (8 * (b & 3))) & 15u;
+          cc[b] = c;
+          const uint32_t one = (0x3F80u << ((c & 1u) << 4)) & one_mask;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) av[4 * b + g] = (c >> 2) == (uint32_t)g ? one : 0u;
+        }
+        tmem_st32(lane_base + A_COL0 + 32u * sa, av);
+        uint32_t m[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t pk = cs_meta16(cc[2 * k]) | (cs_meta16(cc[2 * k + 1]) << 16);
+          const uint32_t p = __shfl_xor_sync(0xffffffffu, pk, 8);
+          m[k] = __byte_perm(pk, p, msel);
+        }
+        tmem_st4(lane_base + META_COL + 4u * sa, m[0], m[1], m[2], m[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(in_leader(full_a(sa)));
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue: 32 rows x NH columns per warp
+    const int ew = warp - W_EPI0;
+    const int quad = warp & 3, half = ew >> 2;
+    const int r = quad * 32 + lane;
+    float *ssp = reinterpret_cast<float *>(smem + OFF_EPI);  // [2][128]
+    float *scl = ssp + 2 * BM;                               // [128]
+    constexpr int OB = (int)sizeof(OT);
+    const int row_bytes = NH * OB, stride = row_bytes + 16, pieces = row_bytes / 16;
+    uint8_t *stg = smem + OFF_STG + ew * 32 * STG_ROW_MAX;
+    unsigned long long *part = ring;                                   // [RING][256][ncl]
+    unsigned long long *tot = ring + (size_t)RING * 2 * BM * ncl;      // [RING][256]
+    bool ok = true;
+    bool gave_up = false;  // a row-sum wait of this thread timed out: results are invalid, stop waiting
+    for (int64_t i = 0; ok && i < n_pm; ++i) {
+      const uint32_t acc = (uint32_t)(i % N_ACC), acc_phase = (uint32_t)((i / N_ACC) & 1);
+      if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
+      tc_fence_after();
+      const int64_t m = 2 * i + rank;
+      const bool live = m < n_m_tiles;  // uniform over the CTA
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + half * NH;
+      float scale = 1.0f;
+      if (kRms) {
+        const unsigned long long tag = (unsigned long long)(i + 1) << 32;
+        const int slot = (int)(i % RING);
+        if (live) {
+          float ss = 0.0f;
+          for (int c = 0; c < NH; c += 16) {
+            uint32_t v[16];
+            tmem_ld16(tbase + c, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 16; ++q) ss = fmaf(__uint_as_float(v[q]), __uint_as_float(v[q]), ss);
+          }
+          ssp[half * BM + r] = ss;
+        }
+        sp_epi_barrier();
+        const int R = (int)rank * BM + r;  // row of the pair tile
+        const bool row_ok = live && i * 2 * BM + R < F;
+        if (half == 0 && row_ok)
+          st_relaxed_u64(part + ((size_t)slot * 2 * BM + R) * ncl + cid,
+                         tag | __float_as_uint(ssp[r] + ssp[BM + r]));
+        // this cluster's rows of the reduction in this CTA's half: R = cid + ncl k, one per warp
+        for (int k = ew; ; k += EPI_WARPS) {
+          const int Rr = cid + ncl * k;
+          if (Rr >= 2 * BM) break;
+          if (Rr / BM != (int)rank) continue;
+          if (i * 2 * BM + Rr >= F) break;
+          const unsigned long long *src = part + ((size_t)slot * 2 * BM + Rr) * ncl;
+          float sum = 0.0f;
+          for (int c0 = 0; c0 < ncl; c0 += 32) {
+            const int c = c0 + lane;
+            unsigned long long v = 0;
+            if (c < ncl) {
+              uint32_t polls = 0;
+              for (;;) {
+                v = ld_relaxed_u64(src + c);
+                if ((v & 0xFFFFFFFF00000000ull) == tag) break;
+                if (gave_up || ++polls > kMaxPolls) {  // after one timeout this thread stops waiting
+                  if (!gave_up) record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+                  gave_up = true;
+                  v = 0;
+                  break;
+                }
+                __nanosleep(64);
+              }
+            }
+            sum += __uint_as_float((uint32_t)v);
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          if (lane == 0) st_relaxed_u64(tot + (size_t)slot * 2 * BM + Rr, tag | __float_as_uint(sum));
+        }
+        if (half == 0 && row_ok) {
+          uint32_t polls = 0;
+          unsigned long long v;
+          for (;;) {
+            v = ld_relaxed_u64(tot + (size_t)slot * 2 * BM + R);
+            if ((v & 0xFFFFFFFF00000000ull) == tag) break;
+            if (gave_up || ++polls > kMaxPolls) {
+              if (!gave_up) record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+              gave_up = true;
+              break;
+            }
+            __nanosleep(64);
+          }
+          scl[r] = 1.0f / sqrtf(__uint_as_float((uint32_t)v) / (float)D + eps);
+        }
+        sp_epi_barrier();
+        scale = scl[r];
+      }
+      if (live) {
+        const int64_t f_warp = m * BM + quad * 32;
+        const int64_t my_row = f_warp + lane < F ? map_row(om, f_warp + lane, half == 0 ? err : nullptr) : -1;
+        const int cb = half * NH;  // column of the slice where this warp's columns start
+        for (int c = 0; c < NH; c += 16) {
+          uint32_t v[16];
+          tmem_ld16(tbase + c, v);
+          tmem_wait_ld();
+          float x[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            x[e] = __uint_as_float(v[e]);
+            if (kRms) x[e] = gsm[cb + c + e] * (x[e] * scale);
+          }
+          uint8_t *dst = stg + lane * stride + c * OB;
+#pragma unroll
+          for (int h = 0; h < 16 * OB / 16; ++h) {
+            float x8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x8[e] = x[(h * (16 / OB) + e) & 15];
+            *reinterpret_cast<uint4 *>(dst + 16 * h) = pack16<OT>(x8);
+          }
+        }
+        __syncwarp();
+        for (int p = lane; p < 32 * pieces; p += 32) {
+          const int q = p / pieces, j = p - q * pieces;
+          const uint4 w = *reinterpret_cast<const uint4 *>(stg + q * stride + 16 * j);
+          const int64_t rq = om.rows ? __shfl_sync(0xffffffffu, my_row, q) : (f_warp + q < F ? f_warp + q : -1);
+          if (rq >= 0) st_stream16(out + rq * (int64_t)D + n0 + cb + j * (16 / OB), w);
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(in_leader(tempty(acc)));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 }  // namespace
@@ -1383,7 +1803,8 @@ EncodeTiledFn encode_tiled_fn() {
 namespace {
 
 // Tensor map of the bf16 table [1280 x D]: boxes of box_cols columns x box_rows rows, with the
-// swizzle whose span is one box row (64 columns: 128 bytes; 32 columns: 64 bytes).
+// swizzle whose span is one box row (64 columns: 128 bytes; 32 columns: 64 bytes; 16 columns:
+// 32 bytes).
 bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D, int box_rows = tc::BK, int box_cols = 64) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
@@ -1391,7 +1812,9 @@ bool make_table_map(CUtensorMap *tmap, const __nv_bfloat16 *table, int D, int bo
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUtensorMapSwizzle sw = box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapSwizzle sw = box_cols == 16   ? CU_TENSOR_MAP_SWIZZLE_32B
+                               : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(table), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1407,8 +1830,9 @@ struct TcScratch {
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Partial sums are laid out [frame tile][column tile][128]; the sparse kernel's 240-column tiles
-// are the most numerous, so the region is sized for them and the 256-column kernels use a prefix.
+// Partial sums are laid out [frame tile][column tile][128]; the streamed sparse kernel's
+// 192-column tiles are the most numerous, so the region is sized for them and the 256-column
+// kernels use a prefix.
 size_t tc_partials_bytes(int64_t F, int D) {
   const size_t m_tiles = (size_t)((F + tc::BM - 1) / tc::BM);
   return round256(m_tiles * (size_t)sp_col_tiles(D) * tc::BM * sizeof(float));
@@ -1576,6 +2000,60 @@ cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
                             err);
 }
 
+// Clusters the column-stationary kernel runs on: every resident pair, at most one per 32 columns;
+// 0 when a slice would be wider than cs::MAX_N (the resident table would not fit).
+int cs_clusters(int D, int resident) {
+  const int U = D / cs::UNIT;
+  int ncl = resident < U ? resident : U;
+  if (ncl > cs::MAX_CLUSTERS) ncl = cs::MAX_CLUSTERS;
+  if (ncl < 1) return 0;
+  const int widest = cs::UNIT * (U / ncl + (U % ncl ? 1 : 0));
+  return widest <= cs::MAX_N ? ncl : 0;
+}
+
+// Column-stationary launch: one cluster per resident CTA pair (cooperative with RMSNorm, whose
+// exchange needs every cluster resident). cudaErrorNotSupported when it cannot take the request.
+template <typename OT, bool kRms>
+cudaError_t launch_cs(const uint8_t *codes, int64_t F, const __nv_bfloat16 *table, int D, OT *out, OutMap om,
+                      unsigned long long *ring, const __nv_bfloat16 *g, float eps, uint32_t *err, int num_sms,
+                      cudaStream_t stream) {
+  if (D % cs::UNIT != 0) return cudaErrorNotSupported;
+  static std::atomic<bool> attr[256];
+  cudaError_t e = set_smem_attr_once(embed_cs_kernel<OT, kRms>, cs::SMEM_BYTES, attr);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(cs::THREADS);
+  cfg.dynamicSmemBytes = cs::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeCooperative;
+  at[1].val.cooperative = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(2 * (num_sms / 2));
+  int resident = 0;
+  if (cudaOccupancyMaxActiveClusters(&resident, embed_cs_kernel<OT, kRms>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
+  }
+  if (resident > num_sms / 2) resident = num_sms / 2;
+  const int ncl = cs_clusters(D, resident);
+  if (ncl == 0) return cudaErrorNotSupported;
+  cfg.gridDim = dim3(2 * ncl);
+  CUtensorMap tmap;
+  if (!make_table_map(&tmap, table, D, cs::BKL, cs::ATOM)) return cudaErrorInvalidValue;
+  if (kRms) {
+    cfg.numAttrs = cooperative_enabled() ? 2 : 1;
+    if ((e = cudaMemsetAsync(ring, 0, cs_ring_words(ncl) * sizeof(unsigned long long), stream)) != cudaSuccess)
+      return e;
+  }
+  return cudaLaunchKernelEx(&cfg, embed_cs_kernel<OT, kRms>, tmap, codes, F, D, out, om, ring, g, eps, err);
+}
+
 // Fused kernels are launched cooperatively, which guarantees that every block of a group is
 // resident while the group exchanges row sums. DMEL_COOPERATIVE=0 (read once per process)
 // launches the same kernel and grid without that attribute, which profilers that cannot replay
@@ -1609,6 +2087,16 @@ bool sparse_enabled() {
   return on;
 }
 
+// The column-stationary kernel unless the environment sets DMEL_EMBED_TABLE=streamed (read once
+// per process; for comparisons and tests).
+bool stationary_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("DMEL_EMBED_TABLE");
+    return !(v && strcmp(v, "streamed") == 0);
+  }();
+  return on;
+}
+
 // Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
 // partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel. CTA pairs
 // first; one-CTA tiles when pairs are switched off or cannot launch.
@@ -1623,6 +2111,16 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
   const int plain_clusters = (int)(pair_tiles < max_clusters ? pair_tiles : max_clusters);
   const TcScratch sc = g ? tc_scratch(workspace, F, D) : TcScratch{nullptr, nullptr};
   cudaError_t e;
+  if (pairs_enabled() && sparse_enabled() && stationary_enabled()) {
+    e = g ? launch_cs<OT, true>(codes, F, T, D, out, om, reinterpret_cast<unsigned long long *>(workspace), g, eps,
+                                err, num_sms, stream)
+          : launch_cs<OT, false>(codes, F, T, D, out, om, nullptr, nullptr, eps, err, num_sms, stream);
+    if (e == cudaSuccess) {
+      ++*launches;
+      return e;
+    }
+    (void)cudaGetLastError();  // refused: the streamed-table kernels below
+  }
   const int Psp = sp_col_tiles(D);
   if (pairs_enabled() && sparse_enabled() && max_clusters >= Psp) {
     const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
@@ -1740,7 +2238,10 @@ bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
 
 size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
   if (!with_rmsnorm || !embed_uses_tensor_cores(table_dtype, embed_dim) || n_frames <= 0) return 0;
-  return tc_scratch_bytes(n_frames, embed_dim);
+  // the column-stationary kernel's exchange ring, or the streamed-table kernels' partial sums
+  const size_t ring = cs_ring_words(cs::MAX_CLUSTERS) * sizeof(unsigned long long);
+  const size_t parts = tc_scratch_bytes(n_frames, embed_dim);
+  return ring > parts ? ring : parts;
 }
 
 cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,

@@ -24,7 +24,9 @@
  *     dmel_get_device_error() reads, and carry on with a clamped value.
  *   - n_clips == 0 or n_frames == 0 is a valid call that does nothing.
  *   - No entry point allocates device memory. Scratch space comes from the caller's workspace;
- *     dmel_workspace_size() says how much.
+ *     dmel_workspace_size() says how much. The one exception is dmel_embed_noalloc, whose
+ *     scratch is a fixed array inside the library (see there); dmel_forward_host also creates
+ *     two copy streams per device on its first call.
  *   - Calls may come from several host threads at once (each with its own buffers): the
  *     per-device one-time setup (constant tables, kernel attributes, the cuBLASLt handle of
  *     dmel_hmlp) is guarded, and dmel_last_launch_count() reports the calling thread's last call.

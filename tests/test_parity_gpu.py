@@ -172,11 +172,13 @@ def test_embed_tensor_core_model_dim(out_dt, rms, table_bf16, rmsw_bf16, oracle_
     print(f"tensor-core embed out={out_dt} rms={rms}: worst {worst:.2e}")
 
 
-@pytest.mark.parametrize("dim", [256, 768, 2048])
+@pytest.mark.parametrize("dim", [256, 768, 2048, 4096, 7168])
 def test_embed_tensor_core_rmsnorm_widths(dim, oracle_mod):
-    """Fused RMSNorm where a frame tile's row sums come from several column tiles (sparse
-    kernel: 192-column tiles, so 256 = 192 + 64, 768 = 4 x 192, 2048 = 10 x 192 + 128, partial
-    last tiles included; dense kernels: 1, 3 and 8 tiles of 256) and a ragged last frame tile."""
+    """Fused RMSNorm where a frame tile's row sums come from several column slices, and a ragged
+    last frame tile. Resident-table kernel: slices of 32 columns on 8, 24 and 64 clusters (256,
+    768, 2048), 64 and 32 (4096), and 7168, whose slices would be wider than the table space
+    allows, falls back to the streamed kernel; streamed sparse kernel: 192-column tiles, partial
+    last tiles included; dense kernels: 1, 3, 8, 16 and 28 tiles of 256."""
     T, T64 = bf16_table(synth.table(seed=12, dim=dim))
     gw = torch.from_numpy(synth.rms_weight(seed=13, dim=dim)).to(torch.bfloat16)
     F = 700

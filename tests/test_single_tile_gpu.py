@@ -1,7 +1,9 @@
 """The other tensor-core kernels against the oracle: the embedding parity tests run again in a
-fresh process with the 2:4-sparse product switched off (DMEL_EMBED_MMA=dense: dense CTA-pair
-tiles) and with CTA pairs switched off (DMEL_EMBED_TILE=single: dense one-CTA tiles), so every
-tile shape of the tcgen05 path stays covered."""
+fresh process with the resident-table kernel switched off (DMEL_EMBED_TABLE=streamed: the
+2:4-sparse kernel that streams table blocks per frame tile), with the 2:4-sparse product switched
+off (DMEL_EMBED_MMA=dense: dense CTA-pair tiles) and with CTA pairs switched off
+(DMEL_EMBED_TILE=single: dense one-CTA tiles), so every tile shape of the tcgen05 path stays
+covered."""
 import os
 import subprocess
 import sys
@@ -19,6 +21,10 @@ def _run_embed_parity(**env_overrides):
                         os.path.join(ROOT, "tests", "test_parity_gpu.py"), "-k", "embed or batch64"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+def test_embedding_parity_with_streamed_table_tiles():
+    _run_embed_parity(DMEL_EMBED_TABLE="streamed")
 
 
 def test_embedding_parity_with_dense_pair_tiles():
