@@ -19,15 +19,19 @@
 //       k2b + 4 k2a;
 //   D   X_k = (Z_k + conj Z_{800-k}) / 2 + W_1600^k (Z_k - conj Z_{800-k}) / (2 i),
 //       P_k = |X_k|^2; lane l of round r reads Z at row r, column l and its partner
-//       Z_{800-k} at row 25 - r, column 31 - l (both bank-conflict free);
-//   E   the 1571 non-zero mel weights, as one list sorted by channel, are cut into 32 equal
-//       chunks; lane l sums its chunk into per-channel partials, then 80 channel sums, log10,
-//       clamp, quantise (fp32).
+//       Z_{800-k} at row 25 - r, column 31 - l (both bank-conflict free), so each lane owns
+//       two runs of 13 adjacent bins (k = 25 k2 + r ascending and 800 - k descending);
+//   E   every bin lies between two adjacent mel points, so it feeds at most two adjacent
+//       channels (the falling edge of one triangle, the rising edge of the next); each lane
+//       folds its two runs into fp32 channel partials as it computes P_k (no P array), writing a
+//       partial when its run crosses into a new channel, then 80 channel sums, log10, clamp,
+//       quantise (fp32).
 // Each frame's 1600 samples are first copied into the warp's buffer with coalesced loads.
 // Every root of unity comes from one fp64 table of W_1600^k, k = 0..800 (W_800 = W_1600^2,
 // W_32 = W_1600^50, W_25 = W_1600^64, W^{1600 - k} = conj W^k). The buffer is swizzled so the
 // column accesses of A, C1 and C2 are free of shared-memory bank conflicts.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -38,52 +42,48 @@
 namespace dmel {
 namespace {
 
-#ifndef DMEL_CODES_WARPS
-#define DMEL_CODES_WARPS 12
-#endif
-constexpr int kWarpsPerBlock = DMEL_CODES_WARPS;
-constexpr int kMelNnzMax = 1600;
-constexpr int kMaxSegs = 128;      // channel segments of the 32 mel chunks (<= 80 + 31)
+// Warps (frames in flight) per block, one block per SM: 12 (168 registers per thread) or 14
+// (the shared-memory limit; the register file then allows 146 per thread and some spill).
+constexpr int kWarpsDefault = 12;
+constexpr int kWarpsMore = 14;
+constexpr int kRunLen = 13;        // bins per lane run (rounds r = 0..12 of step D)
+constexpr int kMaxFlush = 16;      // channel partials one lane writes per run, at most
+constexpr int kMaxSegs = 256;      // channel partials per frame (+ one slot for edge flushes)
 
 // Shared memory of one block: the constant tables once, then one 800-element complex buffer
 // per warp (Y, then Z in place, then P in place; the mel partials follow P).
 constexpr int kSmW = 0;                                    // double2 [801]: W_1600^k
 constexpr int kSmHann = kSmW + 801 * 16;                   // double2 [800]: (w[2m], w[2m+1])
 constexpr int kSmTwA = kSmHann + 800 * 16;                 // double2 [25 * 32]: W_800^{l k1}
-constexpr int kSmMelW = kSmTwA + 800 * 16;                 // float [kMelNnzMax]: weights
-constexpr int kSmMelK = kSmMelW + kMelNnzMax * 4;          // short [kMelNnzMax]: bin of each weight
-constexpr int kSmMelB = kSmMelK + kMelNnzMax * 2;          // uchar [kMelNnzMax]: channel of each weight
-constexpr int kSmChunk = kSmMelB + kMelNnzMax;             // int [33]: chunk bounds per lane
-constexpr int kSmSegFirst = kSmChunk + 36 * 4;             // int [33]: first segment of each lane
-constexpr int kSmChanSeg = kSmSegFirst + 36 * 4;           // int [81]: segment range per channel
+constexpr int kSmMelW2 = kSmTwA + 800 * 16;                // float2 [2][13][32]: bin weights per lane run
+constexpr int kSmSlot = kSmMelW2 + 2 * kRunLen * 32 * 8;   // ushort [32][2][kMaxFlush]: partial slots
+constexpr int kSmFlush = kSmSlot + 32 * 2 * kMaxFlush * 2; // uint [2][32]: run positions of new channels
+constexpr int kSmChanSeg = kSmFlush + 64 * 4;              // int [81]: slot range per channel
 constexpr int kSmTables = (kSmChanSeg + 84 * 4 + 127) / 128 * 128;
 constexpr int kWarpBufBytes = 800 * 16;
-constexpr int kPartOffset = 3216;                          // mel partials (floats) after P[801]
-constexpr int kSmemBytes = kSmTables + kWarpsPerBlock * kWarpBufBytes;
-static_assert(kPartOffset + kMaxSegs * 4 <= kWarpBufBytes, "mel partials fit behind P");
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+__host__ __device__ constexpr int smem_bytes(int warps) { return kSmTables + warps * kWarpBufBytes; }
+static_assert(kMaxSegs * 4 <= 2 * 32 * 16, "mel partials fit in rows 0 and 1 of the warp's buffer");
+static_assert(smem_bytes(kWarpsMore) <= 227 * 1024, "shared memory budget");
 
 // Constant tables, filled once per device from host-computed fp64 values.
 __device__ double2 d_w1600[kBins];
 __device__ double2 d_hann2[800];
 __device__ double2 d_twa[800];
-__device__ float d_melw[kMelNnzMax];
-__device__ short d_melk[kMelNnzMax];
-__device__ unsigned char d_melb[kMelNnzMax];
-__device__ int d_chunk[33];
-__device__ int d_segfirst[33];
+__device__ float2 d_melw2[2 * kRunLen * 32];
+__device__ unsigned short d_slot[32 * 2 * kMaxFlush];
+__device__ unsigned int d_flush[64];
 __device__ int d_chanseg[81];
 
 struct Tables {
   const double2 *w;      // W_1600^k = exp(-2 pi i k / 1600), k = 0..800
   const double2 *hann2;  // periodic Hann pairs (w[2m], w[2m+1]), m = 0..799
   const double2 *twa;    // W_800^{l k1} at [k1 * 32 + l]
-  const float *melw;     // non-zero mel weights (fp32), sorted by channel then bin
-  const short *melk;     // their bins
-  const unsigned char *melb;  // their channels
-  const int *chunk;      // lane l sums entries [chunk[l], chunk[l + 1])
-  const int *segfirst;   // lane l owns the partial-sum slots [segfirst[l], segfirst[l + 1])
-  const int *chanseg;    // channel b adds the partials [chanseg[b], chanseg[b + 1])
+  // mel weights of the bins of lane l's runs, run q (0: ascending, 1: descending) round r, at
+  // [(q * 13 + r) * 32 + l]: (weight to the lower channel, weight to the channel above it)
+  const float2 *melw2;
+  const unsigned short *slot;  // partial slots of lane l's run q, in order, at [(l * 2 + q) * kMaxFlush]
+  const unsigned int *flush;   // bit r of [q * 32 + l]: the run enters a new channel at round r
+  const int *chanseg;          // channel b adds the partials [chanseg[b], chanseg[b + 1])
 };
 
 // W_1600^idx for idx in [0, 1600).
@@ -337,27 +337,28 @@ __host__ __device__ inline void step_c2_lane(int l, double2 *B) {
   }
 }
 
-// Step D, first half for lane l: pairs (k, 800 - k). Round r = 1..12 takes Z at row r, column
-// l (k = r + 25 k2 with k2 = (l >> 2) + 8 (l & 3)) and its partner Z_{800-k} at row 25 - r,
+// Step D for lane l: pairs (k, 800 - k). Round r = 1..12 takes Z at row r, column l
+// (k = r + 25 k2 with k2 = (l >> 2) + 8 (l & 3)) and its partner Z_{800-k} at row 25 - r,
 // column 31 - l; round 0 takes row 0 (k = 25 k2, k2 <= 16; the partner is Z_{800-k} in row 0).
-struct PairRegs {
-  double2 a[13], b[13];
+// Rounds 0 and 1 are loaded first by every lane (rows 0, 1 and 24), so after a __syncwarp rows 0
+// and 1 can hold the channel partials while rounds 2..12 are read one at a time.
+struct Pair01 {
+  double2 a0, b0, a1, b1;
 };
 
 __host__ __device__ inline int dk2(int l) { return (l >> 2) + 8 * (l & 3); }
 
-__host__ __device__ inline void step_d_load(int l, const double2 *B, PairRegs &R) {
+__host__ __device__ inline void step_d_load01(int l, const double2 *B, Pair01 &R) {
   const int k2 = dk2(l);
   if (k2 <= 16) {
-    R.a[0] = B[slot(0, l)];
-    R.b[0] = B[zslot((800 - 25 * k2) % 800)];
+    R.a0 = B[slot(0, l)];
+    R.b0 = B[zslot((800 - 25 * k2) % 800)];
   }
-#pragma unroll
-  for (int r = 1; r <= 12; ++r) {
-    R.a[r] = B[slot(r, l)];
-    R.b[r] = B[slot(25 - r, 31 - l)];
-  }
+  R.a1 = B[slot(1, l)];
+  R.b1 = B[slot(24, 31 - l)];
 }
+
+constexpr int kPartRows = 2;  // rows 0 and 1 of the buffer: 64 x 16 bytes for the channel partials
 
 // |X_k|^2 of the real 1600-point DFT from a = Z_k and b = Z_{800-k}.
 __host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, double2 b) {
@@ -370,42 +371,56 @@ __host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, d
   return xr * xr + xi * xi;
 }
 
-// Step D, second half: P_k and P_{800 - k} (fp32) in natural order over the buffer.
-__host__ __device__ inline void step_d_store(int l, const Tables &T, const PairRegs &R, float *P) {
+// Bin of lane l's run q at round r (-1 when the round has none): run 0 ascends from 25 k2, run 1
+// descends from 800 - 25 k2; round 0 exists for k2 <= 16 (run 0) and k2 <= 15 (run 1: for
+// k2 = 16 both would be bin 400).
+__host__ __device__ inline int run_bin(int l, int q, int r) {
   const int k2 = dk2(l);
-  if (k2 <= 16) {
-    const int k = 25 * k2;
-    P[k] = (float)power_bin(T, k, R.a[0], R.b[0]);
-    if (k != 400) P[800 - k] = (float)power_bin(T, 800 - k, R.b[0], R.a[0]);
-  }
-#pragma unroll
-  for (int r = 1; r <= 12; ++r) {
-    const int k = r + 25 * k2;
-    P[k] = (float)power_bin(T, k, R.a[r], R.b[r]);
-    P[800 - k] = (float)power_bin(T, 800 - k, R.b[r], R.a[r]);
-  }
+  if (r == 0 && (q == 0 ? k2 > 16 : k2 > 15)) return -1;
+  return q == 0 ? 25 * k2 + r : 800 - 25 * k2 - r;
 }
 
-// Step E, first half for lane l: the entries [chunk[l], chunk[l + 1]) of the weight list,
-// summed per channel into the partial-sum slots segfirst[l], segfirst[l] + 1, ... Every lane
-// walks the same number of entries (within one), so the loop does not diverge.
-__host__ __device__ inline void step_e_chunk(int l, const Tables &T, const float *P, float *part) {
-  const int e0 = T.chunk[l], e1 = T.chunk[l + 1];
-  int seg = T.segfirst[l];
-  int cur = T.melb[e0];
-  float acc = 0.0f;
-#pragma unroll 4
-  for (int e = e0; e < e1; ++e) {
-    const float v = T.melw[e] * P[T.melk[e]];
-    const int b = T.melb[e];
-    if (b != cur) {
-      part[seg++] = acc;
-      acc = 0.0f;
-      cur = b;
+// Steps D and E for lane l: P of the lane's 26 bins (fp64 -> fp32) folded into channel partials.
+// Each run carries two accumulators, for its current lower channel and the channel above; where
+// the run enters a new channel (flush bit r) the finished one is written to its slot (ascending
+// run: the lower; descending run: the upper); at the end of the run both are written.
+__host__ __device__ inline void step_de_lane(int l, const Tables &T, const Pair01 &R, const double2 *B,
+                                             float *part) {
+  const int k2 = dk2(l);
+  float lo[2] = {0.0f, 0.0f}, hi[2] = {0.0f, 0.0f};
+  int nf[2] = {0, 0};
+  const unsigned int fl[2] = {T.flush[l], T.flush[32 + l]};
+  const unsigned short *sl[2] = {T.slot + (l * 2) * kMaxFlush, T.slot + (l * 2 + 1) * kMaxFlush};
+#pragma unroll
+  for (int r = 0; r < kRunLen; ++r) {
+    const int k = 25 * k2 + r;
+    const double2 a = r == 0 ? R.a0 : r == 1 ? R.a1 : B[slot(r, l)];
+    const double2 b = r == 0 ? R.b0 : r == 1 ? R.b1 : B[slot(25 - r, 31 - l)];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (r == 0 && (q == 0 ? k2 > 16 : k2 > 15)) continue;
+      const float p = q == 0 ? (float)power_bin(T, k, a, b) : (float)power_bin(T, 800 - k, b, a);
+      if ((fl[q] >> r) & 1u) {
+        if (q == 0) {
+          part[sl[0][nf[0]++]] = lo[0];
+          lo[0] = hi[0];
+          hi[0] = 0.0f;
+        } else {
+          part[sl[1][nf[1]++]] = hi[1];
+          hi[1] = lo[1];
+          lo[1] = 0.0f;
+        }
+      }
+      const float2 w = T.melw2[(q * kRunLen + r) * 32 + l];
+      lo[q] = fmaf(w.x, p, lo[q]);
+      hi[q] = fmaf(w.y, p, hi[q]);
     }
-    acc += v;
   }
-  part[seg] = acc;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    part[sl[q][nf[q]++]] = lo[q];
+    part[sl[q][nf[q]]] = hi[q];
+  }
 }
 
 // Step E, second half: channel b = lane, lane + 32, lane + 64 adds its partials, then log10,
@@ -444,13 +459,12 @@ __host__ __device__ inline void step_e_codes(int l, const Tables &T, const float
 
 struct HostTables {
   std::vector<double2> w, hann2, twa;
-  std::vector<float> melw;
-  std::vector<short> melk;
-  std::vector<unsigned char> melb;
-  int chunk[33], segfirst[33], chanseg[81];
-  Tables view() const {
-    return Tables{w.data(), hann2.data(), twa.data(), melw.data(), melk.data(), melb.data(), chunk, segfirst, chanseg};
-  }
+  std::vector<float2> melw2;
+  std::vector<unsigned short> slot;
+  std::vector<unsigned int> flush;
+  int chanseg[81];
+  bool ok = true;  // every check of the mel layout held
+  Tables view() const { return Tables{w.data(), hann2.data(), twa.data(), melw2.data(), slot.data(), flush.data(), chanseg}; }
 };
 
 void build_host_tables(HostTables &H) {
@@ -466,41 +480,70 @@ void build_host_tables(HostTables &H) {
       const int j = (l * k1) % 800;
       H.twa[k1 * 32 + l] = make_double2(std::cos(two_pi * j / 800), -std::sin(two_pi * j / 800));
     }
-  // HTK mel points: 82 points equally spaced in mel on [0, 8000] Hz; non-zero triangle weights
-  // listed channel by channel, bins ascending
+  // HTK mel points: 82 points equally spaced in mel on [0, 8000] Hz; triangle b rises from point
+  // b to its peak (1) at point b + 1 and falls to point b + 2, evaluated at f_k = 10 k Hz
   const double mel_top = 2595.0 * std::log10(1.0 + 8000.0 / 700.0);
   double fp[kMel + 2];
   for (int i = 0; i < kMel + 2; ++i) fp[i] = 700.0 * (std::pow(10.0, (mel_top * i / (kMel + 1)) / 2595.0) - 1.0);
-  H.melw.clear();
-  H.melk.clear();
-  H.melb.clear();
-  for (int b = 0; b < kMel; ++b)
-    for (int k = 0; k < kBins; ++k) {
-      const double f = 10.0 * k;
-      const double up = (f - fp[b]) / (fp[b + 1] - fp[b]);
-      const double down = (fp[b + 2] - f) / (fp[b + 2] - fp[b + 1]);
-      const double h = up < down ? up : down;
-      if (h > 0.0) {
-        H.melw.push_back((float)h);
-        H.melk.push_back((short)k);
-        H.melb.push_back((unsigned char)b);
-      }
-    }
-  const int nnz = (int)H.melw.size();
-  for (int l = 0; l <= 32; ++l) H.chunk[l] = (int)((int64_t)l * nnz / 32);
-  // partial-sum slots: one per maximal run of one channel inside a chunk, numbered lane by lane
-  int seg = 0;
-  for (int b = 0; b <= kMel; ++b) H.chanseg[b] = -1;
-  for (int l = 0; l < 32; ++l) {
-    H.segfirst[l] = seg;
-    for (int e = H.chunk[l]; e < H.chunk[l + 1]; ++e) {
-      if (e > H.chunk[l] && H.melb[e] != H.melb[e - 1]) ++seg;
-      if (H.chanseg[H.melb[e]] < 0) H.chanseg[H.melb[e]] = seg;
-    }
-    ++seg;
+  auto tri = [&](int b, int k) {  // weight of bin k in channel b (0 outside the triangle)
+    if (b < 0 || b >= kMel) return 0.0;
+    const double f = 10.0 * k;
+    const double up = (f - fp[b]) / (fp[b + 1] - fp[b]);
+    const double down = (fp[b + 2] - f) / (fp[b + 2] - fp[b + 1]);
+    const double h = up < down ? up : down;
+    return h > 0.0 ? h : 0.0;
+  };
+  // every bin k lies in one gap (fp[g], fp[g + 1]] (g = -1 for bin 0): it can feed channel g - 1
+  // (falling edge) and channel g (rising edge) only; lower channel of bin k: g - 1
+  std::vector<int> chl(kBins);
+  for (int k = 0; k < kBins; ++k) {
+    int g = -1;
+    while (g + 1 < kMel + 1 && fp[g + 1] < 10.0 * k) ++g;
+    chl[k] = g - 1;
+    for (int b = 0; b < kMel; ++b)  // no weight outside the two channels of the gap
+      if (b != g - 1 && b != g && tri(b, k) != 0.0) H.ok = false;
   }
-  H.segfirst[32] = seg;
-  H.chanseg[kMel] = seg;
+  // per lane and run: weights, the rounds where the run enters a new channel, the channel of each
+  // partial it writes (-1 / 80: outside 0..79, sent to a trash slot)
+  H.melw2.assign(2 * kRunLen * 32, make_float2(0.0f, 0.0f));
+  H.flush.assign(64, 0u);
+  std::vector<int> fch[32][2];
+  for (int l = 0; l < 32; ++l)
+    for (int q = 0; q < 2; ++q) {
+      int prev = -100, c = 0;
+      for (int r = 0; r < kRunLen; ++r) {
+        const int k = run_bin(l, q, r);
+        if (k < 0) continue;
+        c = chl[k];
+        H.melw2[(q * kRunLen + r) * 32 + l] = make_float2((float)tri(c, k), (float)tri(c + 1, k));
+        if (prev != -100 && c != prev) {
+          if (c != prev + (q == 0 ? 1 : -1)) H.ok = false;  // one channel per step
+          H.flush[q * 32 + l] |= 1u << r;
+          fch[l][q].push_back(q == 0 ? prev : prev + 1);  // the channel that is finished
+        }
+        prev = c;
+      }
+      fch[l][q].push_back(c);
+      fch[l][q].push_back(c + 1);
+      if ((int)fch[l][q].size() > kMaxFlush) H.ok = false;
+    }
+  // slots numbered channel by channel (lane, run and order within the run ascending), so that
+  // channel b adds the contiguous slots [chanseg[b], chanseg[b + 1]); then one trash slot
+  H.slot.assign(32 * 2 * kMaxFlush, 0);
+  int nslot = 0;
+  for (int b = 0; b < kMel; ++b) {
+    H.chanseg[b] = nslot;
+    for (int l = 0; l < 32; ++l)
+      for (int q = 0; q < 2; ++q)
+        for (size_t i = 0; i < fch[l][q].size(); ++i)
+          if (fch[l][q][i] == b) H.slot[(l * 2 + q) * kMaxFlush + i] = (unsigned short)nslot++;
+  }
+  H.chanseg[kMel] = nslot;
+  for (int l = 0; l < 32; ++l)
+    for (int q = 0; q < 2; ++q)
+      for (size_t i = 0; i < fch[l][q].size(); ++i)
+        if (fch[l][q][i] < 0 || fch[l][q][i] >= kMel) H.slot[(l * 2 + q) * kMaxFlush + i] = (unsigned short)nslot;
+  if (nslot + 1 > kMaxSegs) H.ok = false;
 }
 
 const HostTables &host_tables() {
@@ -521,15 +564,13 @@ cudaError_t ensure_device_tables() {
   std::lock_guard<std::mutex> lock(g_upload_mu);
   if (g_uploaded[dev]) return cudaSuccess;
   const HostTables &H = host_tables();
-  if (H.melw.size() > (size_t)kMelNnzMax || H.chanseg[kMel] > kMaxSegs) return cudaErrorInvalidValue;
+  if (!H.ok) return cudaErrorInvalidValue;
   if ((e = cudaMemcpyToSymbol(d_w1600, H.w.data(), sizeof(double2) * kBins)) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_hann2, H.hann2.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_twa, H.twa.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_melw, H.melw.data(), sizeof(float) * H.melw.size())) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_melk, H.melk.data(), sizeof(short) * H.melk.size())) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_melb, H.melb.data(), H.melb.size())) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_chunk, H.chunk, sizeof(H.chunk))) != cudaSuccess) return e;
-  if ((e = cudaMemcpyToSymbol(d_segfirst, H.segfirst, sizeof(H.segfirst))) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_melw2, H.melw2.data(), sizeof(float2) * H.melw2.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_slot, H.slot.data(), sizeof(unsigned short) * H.slot.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_flush, H.flush.data(), sizeof(unsigned int) * H.flush.size())) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_chanseg, H.chanseg, sizeof(H.chanseg))) != cudaSuccess) return e;
   g_uploaded[dev] = true;
   return cudaSuccess;
@@ -539,6 +580,7 @@ cudaError_t ensure_device_tables() {
 
 // ---------------------------------------------------------------- kernels
 
+template <int kWarpsPerBlock>
 __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(const float *__restrict__ wav,
                                                                              const int64_t *__restrict__ soff,
                                                                              const int64_t *__restrict__ foff,
@@ -554,36 +596,28 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     double2 *w = reinterpret_cast<double2 *>(smem + kSmW);
     double2 *h2 = reinterpret_cast<double2 *>(smem + kSmHann);
     double2 *ta = reinterpret_cast<double2 *>(smem + kSmTwA);
-    float *mw = reinterpret_cast<float *>(smem + kSmMelW);
-    short *mk = reinterpret_cast<short *>(smem + kSmMelK);
-    unsigned char *mb = reinterpret_cast<unsigned char *>(smem + kSmMelB);
-    int *ch = reinterpret_cast<int *>(smem + kSmChunk);
-    int *sf = reinterpret_cast<int *>(smem + kSmSegFirst);
+    float2 *mw = reinterpret_cast<float2 *>(smem + kSmMelW2);
+    unsigned short *sl = reinterpret_cast<unsigned short *>(smem + kSmSlot);
+    unsigned int *fl = reinterpret_cast<unsigned int *>(smem + kSmFlush);
     int *cs = reinterpret_cast<int *>(smem + kSmChanSeg);
     for (int i = threadIdx.x; i < kBins; i += blockDim.x) w[i] = d_w1600[i];
     for (int i = threadIdx.x; i < 800; i += blockDim.x) {
       h2[i] = d_hann2[i];
       ta[i] = d_twa[i];
     }
-    for (int i = threadIdx.x; i < kMelNnzMax; i += blockDim.x) {
-      mw[i] = d_melw[i];
-      mk[i] = d_melk[i];
-      mb[i] = d_melb[i];
-    }
-    for (int i = threadIdx.x; i < 33; i += blockDim.x) ch[i] = d_chunk[i];
-    for (int i = threadIdx.x; i < 33; i += blockDim.x) sf[i] = d_segfirst[i];
+    for (int i = threadIdx.x; i < 2 * kRunLen * 32; i += blockDim.x) mw[i] = d_melw2[i];
+    for (int i = threadIdx.x; i < 32 * 2 * kMaxFlush; i += blockDim.x) sl[i] = d_slot[i];
+    for (int i = threadIdx.x; i < 64; i += blockDim.x) fl[i] = d_flush[i];
     for (int i = threadIdx.x; i < 81; i += blockDim.x) cs[i] = d_chanseg[i];
   }
   __syncthreads();
   const Tables T{reinterpret_cast<const double2 *>(smem + kSmW), reinterpret_cast<const double2 *>(smem + kSmHann),
-                 reinterpret_cast<const double2 *>(smem + kSmTwA), reinterpret_cast<const float *>(smem + kSmMelW),
-                 reinterpret_cast<const short *>(smem + kSmMelK),
-                 reinterpret_cast<const unsigned char *>(smem + kSmMelB), reinterpret_cast<const int *>(smem + kSmChunk),
-                 reinterpret_cast<const int *>(smem + kSmSegFirst), reinterpret_cast<const int *>(smem + kSmChanSeg)};
+                 reinterpret_cast<const double2 *>(smem + kSmTwA), reinterpret_cast<const float2 *>(smem + kSmMelW2),
+                 reinterpret_cast<const unsigned short *>(smem + kSmSlot),
+                 reinterpret_cast<const unsigned int *>(smem + kSmFlush), reinterpret_cast<const int *>(smem + kSmChanSeg)};
   double2 *B = reinterpret_cast<double2 *>(smem + kSmTables + warp * kWarpBufBytes);
-  float *P = reinterpret_cast<float *>(B);  // P (fp32) over the buffer after step D
-  float *S = reinterpret_cast<float *>(B);  // the frame's raw samples before step A
-  float *part = reinterpret_cast<float *>(smem + kSmTables + warp * kWarpBufBytes + kPartOffset);
+  float *S = reinterpret_cast<float *>(B);     // the frame's raw samples before step A
+  float *part = reinterpret_cast<float *>(B);  // channel partials: rows 0 and 1, once rounds 0 and 1 are read
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int64_t gw = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
@@ -643,13 +677,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     step_c2_lane(lane, B);
     __syncwarp();
     {
-      PairRegs R;
-      step_d_load(lane, B, R);
-      __syncwarp();  // every Z value is in registers before P overwrites the buffer
-      step_d_store(lane, T, R, P);
+      Pair01 R;
+      step_d_load01(lane, B, R);
+      __syncwarp();  // rows 0, 1 and 24 are read before the partials overwrite rows 0 and 1
+      step_de_lane(lane, T, R, B, part);
     }
-    __syncwarp();
-    step_e_chunk(lane, T, P, part);
     __syncwarp();
     step_e_codes(lane, T, part, crow, nullptr, qz);
     __syncwarp();
@@ -685,18 +717,37 @@ __global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restric
 
 // ---------------------------------------------------------------- host entry points
 
+// Warps per block of the codes kernel: kWarpsDefault unless the environment sets
+// DMEL_CODES_WARPS=14 (read once per process; for measurement).
+int codes_warps() {
+  static const int w = [] {
+    const char *v = getenv("DMEL_CODES_WARPS");
+    return (v && atoi(v) == kWarpsMore) ? kWarpsMore : kWarpsDefault;
+  }();
+  return w;
+}
+
 cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *foff, int n_clips, int64_t n_frames,
                          const float *tails, float *tails_out, uint8_t *codes, uint32_t *err, int num_sms,
                          cudaStream_t stream, int *launches, Quant q) {
   cudaError_t e = ensure_device_tables();
   if (e != cudaSuccess) return e;
-  static std::atomic<bool> attr_set[256];
-  if ((e = set_smem_attr_once(codes_kernel_entry, kSmemBytes, attr_set)) != cudaSuccess) return e;
+  static std::atomic<bool> attr12[256], attr14[256];
+  const bool more = codes_warps() == kWarpsMore;
+  if ((e = more ? set_smem_attr_once(codes_kernel_entry<kWarpsMore>, smem_bytes(kWarpsMore), attr14)
+                : set_smem_attr_once(codes_kernel_entry<kWarpsDefault>, smem_bytes(kWarpsDefault), attr12)) !=
+      cudaSuccess)
+    return e;
   if (n_frames > 0) {
-    int64_t blocks = (n_frames + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    const int W = more ? kWarpsMore : kWarpsDefault;
+    int64_t blocks = (n_frames + W - 1) / W;
     if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM
-    codes_kernel_entry<<<(unsigned)blocks, kWarpsPerBlock * 32, kSmemBytes, stream>>>(
-        wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
+    if (more)
+      codes_kernel_entry<kWarpsMore><<<(unsigned)blocks, kWarpsMore * 32, smem_bytes(kWarpsMore), stream>>>(
+          wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
+    else
+      codes_kernel_entry<kWarpsDefault><<<(unsigned)blocks, kWarpsDefault * 32, smem_bytes(kWarpsDefault), stream>>>(
+          wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
@@ -718,8 +769,8 @@ void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *
   const HostTables &H = host_tables();
   const Tables T = H.view();
   std::vector<double2> B(800);
-  std::vector<PairRegs> R(32);
-  std::vector<float> part(kMaxSegs);
+  std::vector<Pair01> R(32);
+  std::vector<float> part(kMaxSegs, 0.0f);
   std::vector<double> arb(32 * 25), aib(32 * 25);
   for (int l = 0; l < 32; ++l)
     step_a_load(l, frame1600, T, *reinterpret_cast<double(*)[25]>(&arb[25 * l]),
@@ -729,9 +780,9 @@ void emulate_codes_frame_host(const float *frame1600, uint8_t *codes80, double *
                B.data());
   for (int l = 0; l < 32; ++l) step_c1_lane(l, T, B.data());
   for (int l = 0; l < 32; ++l) step_c2_lane(l, B.data());
-  for (int l = 0; l < 32; ++l) step_d_load(l, B.data(), R[l]);
-  for (int l = 0; l < 32; ++l) step_d_store(l, T, R[l], reinterpret_cast<float *>(B.data()));
-  for (int l = 0; l < 32; ++l) step_e_chunk(l, T, reinterpret_cast<const float *>(B.data()), part.data());
+  for (int l = 0; l < 32; ++l) step_d_load01(l, B.data(), R[l]);
+  for (int l = 0; l < 32; ++l) step_de_lane(l, T, R[l], B.data(), reinterpret_cast<float *>(B.data()));
+  for (int i = 0; i < kMaxSegs; ++i) part[i] = reinterpret_cast<const float *>(B.data())[i];
   for (int l = 0; l < 32; ++l) step_e_codes(l, T, part.data(), codes80, lhat80, q);
 }
 
