@@ -26,7 +26,8 @@
 //       folds its two runs into fp32 channel partials as it computes P_k (no P array), writing a
 //       partial when its run crosses into a new channel, then 80 channel sums, log10, clamp,
 //       quantise (fp32).
-// Each frame's 1600 samples are first copied into the warp's buffer with coalesced loads.
+// Each lane reads its 50 samples of a frame straight from global memory (for each j the warp
+// reads 64 consecutive samples; half of them were read by the previous frame and sit in L1).
 // Every root of unity comes from one fp64 table of W_1600^k, k = 0..800 (W_800 = W_1600^2,
 // W_32 = W_1600^50, W_25 = W_1600^64, W^{1600 - k} = conj W^k). The buffer is swizzled so the
 // column accesses of A, C1 and C2 are free of shared-memory bank conflicts.
@@ -197,20 +198,30 @@ __host__ __device__ inline void dft8(double (&r)[8], double (&i)[8]) {
   }
 }
 
-// Copies the 1600 raw samples of frame t of a clip, x[800 (t - 1) + n], into S[n] with
-// coalesced loads (lane l takes n = l + 32 i). Samples before the clip come from the carried
-// tail (tail points one past its last sample) or are zero.
-__device__ inline void stage_frame(int l, const float *base, const float *tail, int64_t start, float *S) {
-  if (start >= 0) {
-    const float *src = base + start;
-#pragma unroll 10
-    for (int n = l; n < 1600; n += 32) S[n] = __ldg(src + n);
-  } else {
-    // first frame of a clip (start = -800): the carried tail (or zeros), then the new samples
-#pragma unroll 5
-    for (int n = l; n < 800; n += 32) S[n] = tail ? __ldg(tail + (n - 800)) : 0.0f;
-#pragma unroll 5
-    for (int n = 800 + l; n < 1600; n += 32) S[n] = __ldg(base + (n - 800));
+// Step A, first half, straight from global memory: lane l reads the samples
+// x[800 (t - 1) + 64 j + 2 l] and the next one of frame t (start = 800 (t - 1)), j = 0..24 (the
+// warp reads 64 consecutive samples per j; the previous frame of the warp usually left them in
+// L1). Samples before the clip come from the carried tail (tail points one past its last sample)
+// or are zero. Windowed as in step_a_load.
+__device__ inline void step_a_load_global(int l, const float *base, const float *tail, int64_t start,
+                                          const Tables &T, double (&ar)[25], double (&ai)[25]) {
+#pragma unroll
+  for (int j = 0; j < 25; ++j) {
+    const int n = 64 * j + 2 * l;  // even: n and n + 1 fall on the same side of sample 800
+    float x0, x1;
+    if (start >= 0) {
+      x0 = __ldg(base + start + n);
+      x1 = __ldg(base + start + n + 1);
+    } else if (n >= 800) {  // first frame of a clip (start = -800): the new samples
+      x0 = __ldg(base + (n - 800));
+      x1 = __ldg(base + (n - 799));
+    } else {  // ... after the carried tail or zeros
+      x0 = tail ? __ldg(tail + (n - 800)) : 0.0f;
+      x1 = tail ? __ldg(tail + (n - 799)) : 0.0f;
+    }
+    const double2 w = T.hann2[32 * j + l];  // periodic Hann at n and n + 1
+    ar[j] = w.x * (double)x0;
+    ai[j] = w.y * (double)x1;
   }
 }
 
@@ -616,7 +627,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
                  reinterpret_cast<const unsigned short *>(smem + kSmSlot),
                  reinterpret_cast<const unsigned int *>(smem + kSmFlush), reinterpret_cast<const int *>(smem + kSmChanSeg)};
   double2 *B = reinterpret_cast<double2 *>(smem + kSmTables + warp * kWarpBufBytes);
-  float *S = reinterpret_cast<float *>(B);     // the frame's raw samples before step A
   float *part = reinterpret_cast<float *>(B);  // channel partials: rows 0 and 1, once rounds 0 and 1 are read
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
@@ -662,13 +672,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     // the next frame of this clip needs samples [800 (t + 1), 800 (t + 2)): start them into L1
     if (g + 1 < g1 && (int64_t)kHop * (t + 2) <= len && lane < 25)
       asm volatile("prefetch.global.L1 [%0];" ::"l"(wav + soff[clip] + (int64_t)kHop * (t + 1) + 32 * lane));
-    stage_frame(lane, wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr, (int64_t)kHop * (t - 1),
-                S);
-    __syncwarp();
+    __syncwarp();  // the previous frame's partials are read before this frame's DFT outputs land
     {
       double ar[25], ai[25];
-      step_a_load(lane, S, T, ar, ai);
-      __syncwarp();  // every lane has its samples before the DFT outputs overwrite them
+      step_a_load_global(lane, wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr,
+                         (int64_t)kHop * (t - 1), T, ar, ai);
       step_a_dft(lane, T, ar, ai, B);
     }
     __syncwarp();

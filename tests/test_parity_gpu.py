@@ -342,8 +342,11 @@ def _check_forward(wav, off, plan, T64, g64, rtol, oracle_mod, frame_ids=None, e
     ids = np.arange(gsel.shape[0]) if embed_ids is None else embed_ids
     ids = ids[~flipped[ids]]
     rows = ids if frame_ids is None else frame_ids[ids]
-    ref = oracle_mod.embed(oc[ids], T64, g64, 1e-6)
-    worst = compare_embed(plan.out[torch.from_numpy(rows).to(DEV)].float().cpu().numpy(), ref, rtol)
+    worst = 0.0
+    for c0 in range(0, len(ids), 2048):  # the fp64 oracle vectors, 2048 frames at a time
+        ref = oracle_mod.embed(oc[ids[c0:c0 + 2048]], T64, g64, 1e-6)
+        got = plan.out[torch.from_numpy(rows[c0:c0 + 2048]).to(DEV)].float().cpu().numpy()
+        worst = max(worst, compare_embed(got, ref, rtol))
     print(f"{label}: frames {plan.n_frames}, code cells checked {gsel.size}, flips {flips}, "
           f"embeddings checked {len(ids)}, worst {worst:.2e}")
 
@@ -356,14 +359,14 @@ def test_forward_one_clip_2s_fp32(oracle_mod):
 
 
 def test_forward_batch64_10s(table_bf16, rmsw_bf16, oracle_mod):
+    """Every frame: codes against the oracle, and every frame's vector (bar the few with a code
+    flip at a level boundary) against the oracle's vector of the oracle's codes."""
     T, T64 = table_bf16
     g, g64 = rmsw_bf16
     wav, off = synth.batch64_10s()
     plan = _forward(wav, off, T, g, torch.bfloat16)
     assert plan.n_frames == 12800
-    r = np.random.default_rng(51)
-    emb = np.sort(r.choice(12800, 1536, replace=False))
-    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, embed_ids=emb, label="batch64_10s")
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, label="batch64_10s")
 
 
 def test_forward_host_pipelined_equals_single_call(table_bf16, rmsw_bf16):
@@ -386,14 +389,13 @@ def test_forward_host_pipelined_equals_single_call(table_bf16, rmsw_bf16):
 
 
 def test_forward_long_20min(table_bf16, rmsw_bf16, oracle_mod):
+    """Every one of the 24,000 frames, codes and vectors, against the oracle."""
     T, T64 = table_bf16
     g, g64 = rmsw_bf16
     wav, off = synth.long_20min()
     plan = _forward(wav, off, T, g, torch.bfloat16)
     assert plan.n_frames == 24000
-    r = np.random.default_rng(52)
-    emb = np.sort(r.choice(24000, 1024, replace=False))
-    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, embed_ids=emb, label="long_20min")
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, label="long_20min")
 
 
 def test_forward_ragged1024(table_bf16, rmsw_bf16, oracle_mod):
