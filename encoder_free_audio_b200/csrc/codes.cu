@@ -369,7 +369,6 @@ __host__ __device__ inline void step_d_load01(int l, const double2 *B, Pair01 &R
   R.b1 = B[slot(24, 31 - l)];
 }
 
-constexpr int kPartRows = 2;  // rows 0 and 1 of the buffer: 64 x 16 bytes for the channel partials
 
 // |X_k|^2 of the real 1600-point DFT from a = Z_k and b = Z_{800-k}.
 __host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, double2 b) {
