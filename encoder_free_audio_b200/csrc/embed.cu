@@ -2087,12 +2087,15 @@ bool sparse_enabled() {
   return on;
 }
 
-// The column-stationary kernel unless the environment sets DMEL_EMBED_TABLE=streamed (read once
-// per process; for comparisons and tests).
+// The column-stationary kernel only when the environment sets DMEL_EMBED_TABLE=resident (read
+// once per process). Measured on B200 it is slower than the streamed-table kernel: a 2:4-sparse
+// pair MMA (M = 256, logical K = 32) takes about 97 cycles whatever N is up to 128 (116 at
+// N = 192, 148 at N = 256), so the 64- and 96-column slices the resident table allows leave the
+// tensor pipe half idle.
 bool stationary_enabled() {
   static const bool on = [] {
     const char *v = getenv("DMEL_EMBED_TABLE");
-    return !(v && strcmp(v, "streamed") == 0);
+    return v && strcmp(v, "resident") == 0;
   }();
   return on;
 }

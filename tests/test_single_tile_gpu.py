@@ -1,6 +1,6 @@
 """The other tensor-core kernels against the oracle: the embedding parity tests run again in a
-fresh process with the resident-table kernel switched off (DMEL_EMBED_TABLE=streamed: the
-2:4-sparse kernel that streams table blocks per frame tile), with the 2:4-sparse product switched
+fresh process with the resident-table kernel switched on (DMEL_EMBED_TABLE=resident: each CTA
+pair keeps its column slice of the table in shared memory), with the 2:4-sparse product switched
 off (DMEL_EMBED_MMA=dense: dense CTA-pair tiles) and with CTA pairs switched off
 (DMEL_EMBED_TILE=single: dense one-CTA tiles), so every tile shape of the tcgen05 path stays
 covered."""
@@ -23,8 +23,8 @@ def _run_embed_parity(**env_overrides):
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
-def test_embedding_parity_with_streamed_table_tiles():
-    _run_embed_parity(DMEL_EMBED_TABLE="streamed")
+def test_embedding_parity_with_resident_table_slices():
+    _run_embed_parity(DMEL_EMBED_TABLE="resident")
 
 
 def test_embedding_parity_with_dense_pair_tiles():
