@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(PKG, "_build")
 LIB = os.path.join(OUT_DIR, "libdmel.so")
-SOURCES = ["api.cu", "codes.cu", "embed.cu", "pipeline.cu", "shortconv.cu", "hmlp.cu"]
+SOURCES = ["api.cu", "codes.cu", "embed.cu", "norm.cu", "pipeline.cu", "shortconv.cu", "hmlp.cu"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-O2", f"-I{INCLUDE}", f"-I{CSRC}"]
 

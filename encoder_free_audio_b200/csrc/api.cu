@@ -388,7 +388,7 @@ dmel_status dmel_embed_noalloc(const uint8_t *codes, int64_t n_frames, const voi
   dmel_status st =
       check_embed_args(codes, true, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype);
   if (st != DMEL_OK || n_frames == 0) return st;
-  const size_t need = embed_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
+  const size_t need = embed_exchange_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
   if (need > kNoAllocScratchBytes) return DMEL_ERR_TOO_LARGE;
   DeviceInfo d;
   if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
@@ -397,7 +397,8 @@ dmel_status dmel_embed_noalloc(const uint8_t *codes, int64_t n_frames, const voi
   if (need > 0 && noalloc_scratch(&scratch) != cudaSuccess) return DMEL_ERR_CUDA;
   int launches = 0;
   cudaError_t e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype,
-                               scratch, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches);
+                               scratch, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches, nullptr, 0,
+                               false);
   t_last_launches = launches;
   return from_cuda(e);
 }
@@ -449,6 +450,27 @@ dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_
   if (!host_offsets_ok(h_sample_offsets, n_clips) || chunk_frames <= 0 || !h_len || cap < 0 || (cap > 0 && !h_plan))
     return DMEL_ERR_INVALID_ARG;
   *h_len = debug_forward_host_plan(h_sample_offsets, n_clips, chunk_frames, h_plan, cap);
+  return DMEL_OK;
+}
+
+dmel_status dmel_debug_gram(const void *table, int embed_dim, float *gram, dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (!table || !gram || embed_dim <= 0 || embed_dim % 64 != 0 || !aligned(table, 16) || !aligned(gram, 16))
+    return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  cudaError_t e = launch_gram(table, embed_dim, gram, d.err, reinterpret_cast<cudaStream_t>(stream), &launches);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+
+dmel_status dmel_debug_norm_sumsq_host(const uint8_t *codes80, const float *h_gram, double *h_sumsq) {
+  if (!codes80 || !h_gram || !h_sumsq) return DMEL_ERR_INVALID_ARG;
+  for (int b = 0; b < kMel; ++b)
+    if (codes80[b] > 15) return DMEL_ERR_INVALID_ARG;
+  *h_sumsq = norm_sumsq_host(codes80, h_gram);
   return DMEL_OK;
 }
 

@@ -245,7 +245,8 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 enum TcMode : int {
   kPlain = 0,     // no RMSNorm: store x
   kPartials = 1,  // store x and each row's sum of squares over the tile (rms_rescale_kernel follows)
-  kFused = 2      // groups of D/256 blocks exchange the row sums and store the normalised rows
+  kFused = 2,     // groups of D/256 blocks exchange the row sums and store the normalised rows
+  kScaled = 3     // every row's RMSNorm scale is given (computed from the codes beforehand)
 };
 
 __device__ __forceinline__ void epi_barrier() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -1264,6 +1265,14 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       const int ncols = D - n0 < BN ? D - n0 : BN;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + cb;
       float scale = 1.0f;
+      if (kMode == kScaled) {
+        // the column tile changes from tile to tile: its RMSNorm weights, and this row's scale
+        const int t = (warp - 6) * 32 + lane;
+        if (t < BN_EPI) gsm[t] = t < ncols ? __bfloat162float(gw[n0 + t]) : 0.0f;
+        const int64_t f = (2 * mp + rank) * BM + r;
+        scale = live && f < F ? __ldg(partials + f) : 0.0f;
+        sp_epi_barrier();
+      }
       if (kMode == kFused && live) {
         float ss = 0.0f;
 #pragma unroll
@@ -1333,7 +1342,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
             for (int e = 0; e < E; ++e) {
               const int cc = h * E + e;
               x[e] = __uint_as_float(v[cc >> 4][cc & 15]);
-              if (kMode == kFused) x[e] = gsm[c0 + cc] * (x[e] * scale);
+              if (kMode == kFused || kMode == kScaled) x[e] = gsm[c0 + cc] * (x[e] * scale);
             }
             *reinterpret_cast<uint4 *>(slab + lane * RB + (piece(lane, h) << 4)) = pack16<OT>(x);
           }
@@ -2100,12 +2109,24 @@ bool stationary_enabled() {
   return on;
 }
 
+// RMSNorm scales from G = T T^T unless the environment sets DMEL_EMBED_NORM=exchange (read once
+// per process; for comparisons and tests): then the CTAs that own a row's column tiles exchange
+// their partial sums of squares inside the embedding kernel.
+bool gram_enabled() {
+  static const bool on = [] {
+    const char *v = getenv("DMEL_EMBED_NORM");
+    return !(v && strcmp(v, "exchange") == 0);
+  }();
+  return on;
+}
+
 // Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
 // partial-sum kernel followed by rms_rescale_kernel; no RMSNorm: the plain kernel. CTA pairs
 // first; one-CTA tiles when pairs are switched off or cannot launch.
 template <typename OT>
 cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, OutMap om, const __nv_bfloat16 *g,
-                   float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
+                   float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
+                   bool allow_gram) {
   const int P = D / tc::BN;
   const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * P;
   const int plain_grid = (int)(tiles < num_sms ? tiles : num_sms);
@@ -2125,6 +2146,28 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
     (void)cudaGetLastError();  // refused: the streamed-table kernels below
   }
   const int Psp = sp_col_tiles(D);
+  if (g && allow_gram && gram_enabled() && pairs_enabled() && sparse_enabled() && max_clusters >= 1) {
+    // RMSNorm scales from the codes and G = T T^T first, then the product on every cluster with
+    // no exchange of row sums
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *G = reinterpret_cast<float *>(ws);
+    void *parts = ws + gram_bytes();
+    float *scale = reinterpret_cast<float *>(ws + gram_bytes() + norm_scale_bytes(F) - round256((size_t)F * 4));
+    int l = 0;
+    e = launch_gram(T, D, G, err, stream, &l);
+    if (e == cudaSuccess) e = launch_norm_scale(codes, F, D, G, eps, parts, scale, stream, &l);
+    if (e == cudaSuccess) {
+      const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
+      const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
+      e = launch_sp<OT, kScaled>(codes, F, T, D, out, om, TcScratch{scale, nullptr}, g, eps, err, sp_clusters, stream);
+      if (e == cudaSuccess) {
+        *launches += l + 1;
+        return e;
+      }
+    }
+    if (e != cudaErrorNotSupported) return e;
+    (void)cudaGetLastError();  // sparse pairs refused: the exchange kernels below
+  }
   if (pairs_enabled() && sparse_enabled() && max_clusters >= Psp) {
     const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
     const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
@@ -2239,7 +2282,7 @@ bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim) {
   return table_dtype == DMEL_BF16 && embed_dim > 0 && embed_dim % tc::BN == 0;
 }
 
-size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
+size_t embed_exchange_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
   if (!with_rmsnorm || !embed_uses_tensor_cores(table_dtype, embed_dim) || n_frames <= 0) return 0;
   // the column-stationary kernel's exchange ring, or the streamed-table kernels' partial sums
   const size_t ring = cs_ring_words(cs::MAX_CLUSTERS) * sizeof(unsigned long long);
@@ -2247,10 +2290,18 @@ size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_d
   return ring > parts ? ring : parts;
 }
 
+size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
+  const size_t ex = embed_exchange_workspace_bytes(n_frames, embed_dim, table_dtype, with_rmsnorm);
+  if (ex == 0) return 0;
+  // or G, the per-frame partial sums of squares and the scales of the G path
+  const size_t gp = gram_bytes() + norm_scale_bytes(n_frames);
+  return ex > gp ? ex : gp;
+}
+
 cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,
                          const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
                          uint32_t *err, int num_sms, cudaStream_t stream, int *launches, const int64_t *out_rows,
-                         int64_t out_n_rows) {
+                         int64_t out_n_rows, bool allow_gram) {
   if (F <= 0) return cudaSuccess;
   const OutMap om{out_rows, out_n_rows};
   cudaError_t e;
@@ -2259,8 +2310,9 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dme
     const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
     if (out_dtype == DMEL_BF16)
       return run_tc(codes, F, T, D, static_cast<__nv_bfloat16 *>(out), om, g, eps, workspace, err, num_sms, stream,
-                    launches);
-    return run_tc(codes, F, T, D, static_cast<float *>(out), om, g, eps, workspace, err, num_sms, stream, launches);
+                    launches, allow_gram);
+    return run_tc(codes, F, T, D, static_cast<float *>(out), om, g, eps, workspace, err, num_sms, stream, launches,
+                  allow_gram);
   }
   if (table_dtype == DMEL_BF16) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);

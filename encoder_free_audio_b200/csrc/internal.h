@@ -30,13 +30,29 @@ bool embed_uses_tensor_cores(dmel_dtype table_dtype, int embed_dim);
 // Scratch bytes the embedding needs (RMSNorm partial sums of the tensor-core path).
 size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm);
 
-// Embedding of n_frames codes; workspace holds embed_workspace_bytes(...) bytes.
+// Scratch the embedding needs when its RMSNorm scales come from an exchange of row sums between
+// the CTAs of a row (no G): what dmel_embed_noalloc's fixed scratch must hold.
+size_t embed_exchange_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm);
+
+// Embedding of n_frames codes; workspace holds embed_workspace_bytes(...) bytes (with allow_gram
+// false, embed_exchange_workspace_bytes(...)).
 // out_rows: NULL (frame f -> row f of out) or device int64 [n_frames], frame f -> row out_rows[f]
 // of an out with out_n_rows rows.
 cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
                          int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
                          void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
-                         const int64_t *out_rows = nullptr, int64_t out_n_rows = 0);
+                         const int64_t *out_rows = nullptr, int64_t out_n_rows = 0, bool allow_gram = true);
+
+// G = T T^T (fp32 [1280 x 1280], the 55 blocks of 128 x 128 rows with row block <= column block
+// written) of a bf16 table T [1280 x D], D a multiple of 64; and the RMSNorm scale of each frame,
+// 1 / sqrt(sum_b sum_b' G[r_b, r_b'] / D + eps), from its codes (scratch: norm_scale_bytes(F)
+// minus the F scales at its end).
+size_t gram_bytes();
+size_t norm_scale_bytes(int64_t n_frames);
+cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaStream_t stream, int *launches);
+cudaError_t launch_norm_scale(const uint8_t *codes, int64_t n_frames, int D, const float *G, float eps, void *scratch,
+                              float *scale, cudaStream_t stream, int *launches);
+double norm_sumsq_host(const uint8_t *codes80, const float *G);
 
 // dmel_forward_host: workspace bytes for this batch (0 when it has no frame) and the pipelined
 // run (host samples in, host vectors and codes out; streams and events of the library's own).

@@ -110,6 +110,10 @@ def _lib():
         L.dmel_forward_host.restype = i32
         L.dmel_debug_forward_host_plan.argtypes = [vp, i32, i64, vp, i64, ctypes.POINTER(i64)]
         L.dmel_debug_forward_host_plan.restype = i32
+        L.dmel_debug_gram.argtypes = [vp, i32, vp, vp]
+        L.dmel_debug_gram.restype = i32
+        L.dmel_debug_norm_sumsq_host.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_double)]
+        L.dmel_debug_norm_sumsq_host.restype = i32
         _L = L
     return _L
 
@@ -413,3 +417,19 @@ def dmel_debug_forward_host_plan(sample_offsets, chunk_frames: int) -> list:
                     "so": buf[i:i + k + 1].copy(), "fo": buf[i + k + 1:i + 2 * k + 2].copy()})
         i += 2 * k + 2
     return out
+
+
+def dmel_debug_gram(table, gram, stream=None):
+    """G = T T^T of a bf16 CUDA table [1280, D] into the CUDA fp32 tensor gram [1280, 1280] (the
+    upper blocks; diagnostic, see dmel_debug.h)."""
+    _check(_lib().dmel_debug_gram(_ptr(table), int(table.shape[1]), _ptr(gram), _stream(stream)), "dmel_debug_gram")
+
+
+def dmel_debug_norm_sumsq_host(codes80: np.ndarray, gram: np.ndarray) -> float:
+    """The device's per-frame sum of squares from G, evaluated on the host (diagnostic)."""
+    c = np.ascontiguousarray(codes80, np.uint8)
+    g = np.ascontiguousarray(gram, np.float32)
+    out = ctypes.c_double(0.0)
+    _check(_lib().dmel_debug_norm_sumsq_host(c.ctypes.data_as(ctypes.c_void_p), g.ctypes.data_as(ctypes.c_void_p),
+                                             ctypes.byref(out)), "dmel_debug_norm_sumsq_host")
+    return out.value

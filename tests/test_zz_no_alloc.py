@@ -61,20 +61,16 @@ def test_noalloc_matches_workspace_entry_point_twice(lib, oracle_mod):
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch(lib):
+    """The fixed scratch holds the row sums of squares the CTAs of a row exchange: 128-frame tiles
+    x ceil(6144 / 192) = 32 column tiles x 128 floats, plus one counter per tile, which is 4 MiB
+    or less up to 32,640 frames at width 6144 and more from 32,641 frames on."""
     T = torch.zeros((1280, 6144), dtype=torch.bfloat16, device=DEV)
     g = torch.ones(6144, dtype=torch.bfloat16, device=DEV)
-    # the smallest frame count whose scratch (what dmel_workspace_size reports) exceeds 4 MiB
-    F = 1
-    while dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True) <= (4 << 20):
-        F *= 2
-    lo, hi = F // 2, F
-    while hi - lo > 1:
-        mid = (lo + hi) // 2
-        lo, hi = (mid, hi) if dmel.dmel_workspace_size(mid, 6144, dmel.DMEL_BF16, True, True) <= (4 << 20) else (lo, mid)
-    F = hi
+    F = 32641
     codes = torch.zeros((F, 80), dtype=torch.uint8, device=DEV)
     out = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
     assert _call_noalloc(lib, codes, T, out, g) == dmel.DMEL_ERR_TOO_LARGE
+    assert _call_noalloc(lib, codes[:32640], T, out[:32640], g) == dmel.DMEL_OK
     # without RMSNorm the request needs no scratch and runs
     assert _call_noalloc(lib, codes[:300], T, out[:300], None) == dmel.DMEL_OK
     torch.cuda.synchronize()
