@@ -455,7 +455,7 @@ dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_
 
 dmel_status dmel_debug_gram(const void *table, int embed_dim, float *gram, dmel_stream_t stream) {
   t_last_launches = 0;
-  if (!table || !gram || embed_dim <= 0 || embed_dim % 64 != 0 || !aligned(table, 16) || !aligned(gram, 16))
+  if (!table || !gram || embed_dim <= 0 || embed_dim % 128 != 0 || !aligned(table, 16) || !aligned(gram, 256))
     return DMEL_ERR_INVALID_ARG;
   DeviceInfo d;
   if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;

@@ -2109,15 +2109,20 @@ bool stationary_enabled() {
   return on;
 }
 
-// RMSNorm scales from G = T T^T unless the environment sets DMEL_EMBED_NORM=exchange (read once
-// per process; for comparisons and tests): then the CTAs that own a row's column tiles exchange
-// their partial sums of squares inside the embedding kernel.
+// RMSNorm scales from G = T T^T for calls of at least kGramMinFrames frames (below that, the
+// fixed cost of G, ~30 us, outweighs what the exchange of row sums costs the embedding kernel),
+// unless the environment sets DMEL_EMBED_NORM=exchange; DMEL_EMBED_NORM=gram takes the G path at
+// every size (read once per process; for comparisons and tests).
+int64_t kGramMinFrames = 16384;
 bool gram_enabled() {
-  static const bool on = [] {
+  static const int mode = [] {
     const char *v = getenv("DMEL_EMBED_NORM");
-    return !(v && strcmp(v, "exchange") == 0);
+    if (v && strcmp(v, "exchange") == 0) return 0;
+    if (v && strcmp(v, "gram") == 0) return 2;
+    return 1;
   }();
-  return on;
+  if (mode == 2) kGramMinFrames = 1;
+  return mode != 0;
 }
 
 // Tensor-core embedding of F frames: fused RMSNorm when the group schedule fits, else the
@@ -2146,7 +2151,8 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
     (void)cudaGetLastError();  // refused: the streamed-table kernels below
   }
   const int Psp = sp_col_tiles(D);
-  if (g && allow_gram && gram_enabled() && pairs_enabled() && sparse_enabled() && max_clusters >= 1) {
+  if (g && allow_gram && gram_enabled() && F >= kGramMinFrames && pairs_enabled() && sparse_enabled() &&
+      max_clusters >= 1) {
     // RMSNorm scales from the codes and G = T T^T first, then the product on every cluster with
     // no exchange of row sums
     uint8_t *ws = static_cast<uint8_t *>(workspace);

@@ -44,7 +44,8 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *tab
                          const int64_t *out_rows = nullptr, int64_t out_n_rows = 0, bool allow_gram = true);
 
 // G = T T^T (fp32 [1280 x 1280], the 55 blocks of 128 x 128 rows with row block <= column block
-// written) of a bf16 table T [1280 x D], D a multiple of 64; and the RMSNorm scale of each frame,
+// written; gram_bytes() holds it and a second partial product after it) of a bf16 table
+// T [1280 x D], D a multiple of 128; and the RMSNorm scale of each frame,
 // 1 / sqrt(sum_b sum_b' G[r_b, r_b'] / D + eps), from its codes (scratch: norm_scale_bytes(F)
 // minus the F scales at its end).
 size_t gram_bytes();

@@ -10,13 +10,20 @@
 // CTAs that own different columns of a row.
 //
 //   gram_kernel     G = T T^T in fp32 on the tensor cores (bf16 x bf16, fp32 accumulate in TMEM),
-//                   one CTA per 128 x 128 block of the upper block triangle (55 blocks): the
-//                   block of bin groups (g, g'), g <= g', 8 bins x 16 levels each way.
+//                   one CTA per 128 x 128 block of the upper block triangle (55 blocks: the block
+//                   of bin groups (g, g'), g <= g', 8 bins x 16 levels each way) and half of the
+//                   D columns (two partial products, 110 CTAs);
+//   gram_combine    the two halves added; the 1,280 diagonal entries G[r, r] = sum_j T[r, j]^2
+//                   replaced by fp64 sums of the same products: the tensor cores' fp32 accumulation
+//                   over thousands of products drifts by ~1e-5 relative, and the diagonal carries
+//                   almost all of a frame's sum of squares (80 terms of ~D * var(T) each, against
+//                   off-diagonal terms of either sign ~sqrt(D) times smaller).
 //   norm_partials   per 512-frame chunk and group of 5 blocks: each block staged in shared
 //                   memory, each frame's 64 (or, on the diagonal, 36) terms looked up and added
 //                   in a fixed order; one partial sum per frame and group.
 //   norm_finalize   scale_f = 1 / sqrt((sum of the 11 partials, in group order) / D + eps).
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -29,7 +36,7 @@ namespace {
 namespace gm {
 constexpr int BT = 128;                 // block: 128 table rows x 128 table rows
 constexpr int BK = 64;                  // K per stage: 64 bf16 = one 128-byte swizzle row
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int OP_STAGE = BT * BK * 2;   // 16 KB per operand and stage
 constexpr int OFF_A = 0;
 constexpr int OFF_B = STAGES * OP_STAGE;
@@ -55,7 +62,8 @@ __host__ __device__ inline void gram_block(int q, int &g, int &h) {
 }
 
 __global__ void __launch_bounds__(gm::THREADS, 1)
-    gram_kernel(const __grid_constant__ CUtensorMap tmap, int D, float *__restrict__ G, uint32_t *err) {
+    gram_kernel(const __grid_constant__ CUtensorMap tmap, int D, float *__restrict__ G0, float *__restrict__ G1,
+                uint32_t *err) {
   using namespace gm;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -67,8 +75,10 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
   const uint32_t tfull = bar0 + 8u * (2 * STAGES);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
   int g, h;
-  gram_block(blockIdx.x, g, h);
-  const int kblocks = D / BK;
+  gram_block(blockIdx.x >> 1, g, h);
+  const int half = blockIdx.x & 1;  // which half of the D columns (K) this CTA sums
+  const int kblocks = D / BK / 2, kb0 = half * kblocks;
+  float *__restrict__ G = half ? G1 : G0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -98,8 +108,8 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
       for (int kb = 0; kb < kblocks; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1u, err)) break;
         mbar_arrive_expect_tx(full(stage), 2 * OP_STAGE);
-        tma_load_2d(smem_addr(smem + OFF_A + stage * OP_STAGE), &tmap, kb * BK, g * BT, full(stage), pol);
-        tma_load_2d(smem_addr(smem + OFF_B + stage * OP_STAGE), &tmap, kb * BK, h * BT, full(stage), pol);
+        tma_load_2d(smem_addr(smem + OFF_A + stage * OP_STAGE), &tmap, (kb0 + kb) * BK, g * BT, full(stage), pol);
+        tma_load_2d(smem_addr(smem + OFF_B + stage * OP_STAGE), &tmap, (kb0 + kb) * BK, h * BT, full(stage), pol);
         pending |= 1u << stage;
         pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -157,6 +167,43 @@ __global__ void __launch_bounds__(gm::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+}
+
+// G0 <- G0 + G1 on the 55 upper blocks (one thread per 4 entries).
+__global__ void __launch_bounds__(256) gram_combine_kernel(float *__restrict__ G0, const float *__restrict__ G1) {
+  const int per_block = gm::BT * gm::BT / 4;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < gm::BLOCKS * per_block; i += gridDim.x * blockDim.x) {
+    int g, h;
+    gram_block(i / per_block, g, h);
+    const int e = i % per_block, r = e / (gm::BT / 4), c4 = e % (gm::BT / 4);
+    const size_t at = (size_t)(g * gm::BT + r) * kRows + h * gm::BT + 4 * c4;
+    float4 a = *reinterpret_cast<const float4 *>(G0 + at);
+    const float4 b = *reinterpret_cast<const float4 *>(G1 + at);
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    *reinterpret_cast<float4 *>(G0 + at) = a;
+  }
+}
+
+// G[r, r] = sum_j T[r, j]^2 in fp64 (each bf16 square is exact; the sum is rounded once): one
+// warp per row, each lane a strided share of the D columns, then a fixed reduction tree.
+__global__ void __launch_bounds__(256) gram_diag_kernel(const __nv_bfloat16 *__restrict__ T, int D,
+                                                         float *__restrict__ G) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= kRows) return;
+  const __nv_bfloat16 *row = T + (size_t)r * D;
+  double s = 0.0;
+  for (int j = 2 * lane; j < D; j += 64) {
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(row + j);
+    const double a = (double)__bfloat162float(v.x), b = (double)__bfloat162float(v.y);
+    s += a * a + b * b;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) G[(size_t)r * kRows + r] = (float)s;
 }
 
 // ---------------------------------------------------------------- per-frame sums of squares
@@ -283,14 +330,14 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 }  // namespace
 
-size_t gram_bytes() { return round256((size_t)kRows * kRows * sizeof(float)); }
+size_t gram_bytes() { return 2 * round256((size_t)kRows * kRows * sizeof(float)); }
 
 size_t norm_scale_bytes(int64_t F) {
   return round256((size_t)nm::NGROUPS * (size_t)F * sizeof(float)) + round256((size_t)F * sizeof(float));
 }
 
 cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaStream_t stream, int *launches) {
-  if (D % gm::BK != 0) return cudaErrorInvalidValue;
+  if (D % (2 * gm::BK) != 0) return cudaErrorInvalidValue;
   static std::atomic<bool> attr[256];
   cudaError_t e = set_smem_attr_once(gram_kernel, gm::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
@@ -306,9 +353,14 @@ cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaS
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  gram_kernel<<<gm::BLOCKS, gm::THREADS, gm::SMEM_BYTES, stream>>>(tmap, D, G, err);
+  float *G1 = G + round256((size_t)kRows * kRows * sizeof(float)) / sizeof(float);
+  gram_kernel<<<2 * gm::BLOCKS, gm::THREADS, gm::SMEM_BYTES, stream>>>(tmap, D, G, G1, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ++*launches;
+  gram_combine_kernel<<<148 * 2, 256, 0, stream>>>(G, G1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  gram_diag_kernel<<<kRows / 8, 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(table), D, G);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  *launches += 3;
   return cudaSuccess;
 }
 

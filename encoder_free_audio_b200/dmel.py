@@ -420,8 +420,9 @@ def dmel_debug_forward_host_plan(sample_offsets, chunk_frames: int) -> list:
 
 
 def dmel_debug_gram(table, gram, stream=None):
-    """G = T T^T of a bf16 CUDA table [1280, D] into the CUDA fp32 tensor gram [1280, 1280] (the
-    upper blocks; diagnostic, see dmel_debug.h)."""
+    """G = T T^T of a bf16 CUDA table [1280, D] into gram[0] of the CUDA fp32 tensor gram
+    [2, 1280, 1280] (the upper blocks; gram[1] is scratch; diagnostic, see dmel_debug.h)."""
+    assert gram.shape == (2, 1280, 1280)
     _check(_lib().dmel_debug_gram(_ptr(table), int(table.shape[1]), _ptr(gram), _stream(stream)), "dmel_debug_gram")
 
 

@@ -54,10 +54,10 @@ dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_
 /* RMSNorm from the Gram matrix: the embedding's RMSNorm scales come from G = T T^T (the table's
  * 1280 x 1280 Gram matrix, fp32), because a frame's sum of squares is
  * sum_j x_j^2 = sum_b sum_b' G[16 b + c_b, 16 b' + c_b'].
- * dmel_debug_gram writes G for a bf16 table [1280 x embed_dim] (embed_dim a multiple of 64) into the
- * device array gram [1280 x 1280] (row-major; the 55 blocks of 128 x 128 entries whose row block
- * is at most their column block are written, the others left as they are), asynchronously on
- * stream. dmel_debug_norm_sumsq_host evaluates, on the host, the sum of squares of one frame
+ * dmel_debug_gram writes G for a bf16 table [1280 x embed_dim] (embed_dim a multiple of 128) into
+ * the first half of the device array gram [2 x 1280 x 1280] (row-major; the 55 blocks of 128 x 128
+ * entries whose row block is at most their column block are written, the others left as they
+ * are; the second half is scratch), asynchronously on stream. dmel_debug_norm_sumsq_host evaluates, on the host, the sum of squares of one frame
  * with codes codes80 from a host copy of such a G, in the order the device sums it (blocks of
  * 8 x 8 bins, diagonal terms once, other pairs twice), into *h_sumsq. */
 dmel_status dmel_debug_gram(const void *table, int embed_dim, float *gram, dmel_stream_t stream);

@@ -1,6 +1,7 @@
 """The other tensor-core kernels against the oracle: the embedding parity tests run again in a
-fresh process with the RMSNorm scales taken from an exchange of row sums between the CTAs of a
-row instead of from G (DMEL_EMBED_NORM=exchange), with the resident-table kernel switched on (DMEL_EMBED_TABLE=resident: each CTA
+fresh process with the RMSNorm scales taken from the table's Gram matrix at every call size
+(DMEL_EMBED_NORM=gram; by default only calls of 16,384 frames or more do), with the resident-table
+kernel switched on (DMEL_EMBED_TABLE=resident: each CTA
 pair keeps its column slice of the table in shared memory), with the 2:4-sparse product switched
 off (DMEL_EMBED_MMA=dense: dense CTA-pair tiles) and with CTA pairs switched off
 (DMEL_EMBED_TILE=single: dense one-CTA tiles), so every tile shape of the tcgen05 path stays
@@ -24,8 +25,8 @@ def _run_embed_parity(**env_overrides):
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
-def test_embedding_parity_with_row_sum_exchange():
-    _run_embed_parity(DMEL_EMBED_NORM="exchange")
+def test_embedding_parity_with_gram_norm_at_every_size():
+    _run_embed_parity(DMEL_EMBED_NORM="gram")
 
 
 def test_embedding_parity_with_resident_table_slices():
