@@ -18,12 +18,14 @@
 //                   over thousands of products drifts by ~1e-5 relative, and the diagonal carries
 //                   almost all of a frame's sum of squares (80 terms of ~D * var(T) each, against
 //                   off-diagonal terms of either sign ~sqrt(D) times smaller).
-//   norm_partials   per 512-frame chunk and group of 5 blocks: each block staged in shared
-//                   memory, each frame's 64 (or, on the diagonal, 36) terms looked up and added
-//                   in a fixed order; one partial sum per frame and group.
-//   norm_finalize   scale_f = 1 / sqrt((sum of the 11 partials, in group order) / D + eps).
+//   norm_partials   per G block and chunk of 4096 frames: the block staged in shared memory once,
+//                   each frame's 64 (on the diagonal 36) terms looked up with eight independent
+//                   accumulators; one partial sum per frame and block.
+//   norm_finalize   scale_f = 1 / sqrt((sum of the 55 partials, in block order) / D + eps).
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -209,119 +211,88 @@ __global__ void __launch_bounds__(256) gram_diag_kernel(const __nv_bfloat16 *__r
 // ---------------------------------------------------------------- per-frame sums of squares
 
 namespace nm {
-constexpr int FRAMES = 512;             // frames per CTA
-constexpr int THREADS = 256;            // two frames per thread
-constexpr int PER_GROUP = 5;            // G blocks per CTA
-constexpr int NGROUPS = (gm::BLOCKS + PER_GROUP - 1) / PER_GROUP;  // 11
+constexpr int FRAMES = 4096;            // frames per CTA
+constexpr int THREADS = 256;            // 16 frames per thread
 constexpr int LD = gm::BT + 4;          // staged row stride (floats): 528 bytes, spreads the banks
 constexpr int BLK_FLOATS = gm::BT * LD;
-constexpr int OFF_CODES = 0;            // uint8 [80][FRAMES], transposed
-constexpr int OFF_G = kMel * FRAMES;    // float [2][BT][LD]
-constexpr int SMEM_BYTES = OFF_G + 2 * BLK_FLOATS * 4;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(OFF_G % 16 == 0, "16-byte aligned staging");
+constexpr int SMEM_BYTES = BLK_FLOATS * 4;  // one G block: 67.6 KB, three CTAs per SM
+static_assert(SMEM_BYTES * 3 <= 227 * 1024, "three CTAs per SM");
 }  // namespace nm
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem_dst)), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all_but_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// G block (g, h) -> shared memory [128][LD], 16-byte copies spread over the CTA.
-__device__ __forceinline__ void stage_block(float *dst, const float *__restrict__ G, int q) {
-  int g, h;
-  gram_block(q, g, h);
-  const float *src = G + (size_t)(g * gm::BT) * kRows + h * gm::BT;
-  for (int i = threadIdx.x; i < gm::BT * (gm::BT / 4); i += nm::THREADS) {
-    const int r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
-    cp_async16(dst + r * nm::LD + 4 * c4, src + (size_t)r * kRows + 4 * c4);
+// Sum of one frame's terms in G block (g, h) (bin groups g <= h, 8 bins each): ci / cj are the
+// row / column offsets 16 i + c and 16 j + c' of the frame's levels in the staged block [128][LD].
+// Off the diagonal: all 64 pairs, doubled; on it: the 8 diagonal terms once and the 28 pairs
+// i < j twice. Eight accumulators (one per j) keep the additions independent; they are combined
+// in a fixed tree.
+__host__ __device__ inline float block_terms(const float *blk, const int (&ri)[8], const int (&cj)[8], bool diag) {
+  float a[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) a[j] = 0.0f;
+  if (!diag) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] += blk[ri[i] + cj[j]];
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = i + 1; j < 8; ++j) a[j] += blk[ri[i] + cj[j]];
   }
+  float s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+  s *= 2.0f;
+  if (diag) {
+    float d[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i & 1] += blk[ri[i] + cj[i]];
+    s += d[0] + d[1];
+  }
+  return s;
 }
 
-__global__ void __launch_bounds__(nm::THREADS, 1)
+// One CTA per (G block q, chunk of 4096 frames): the block is staged once, then each thread
+// takes 16 frames, reads the 16 codes of the block's two bin groups straight from the codes
+// rows (two 8-byte loads) and writes the frame's partial sum for this block.
+__global__ void __launch_bounds__(nm::THREADS, 3)
     norm_partials_kernel(const uint8_t *__restrict__ codes, int64_t F, const float *__restrict__ G,
                          float *__restrict__ partials) {
   using namespace nm;
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t *csm = smem + OFF_CODES;
-  float *gbuf = reinterpret_cast<float *>(smem + OFF_G);
+  extern __shared__ __align__(16) float blk[];
+  const int q = blockIdx.y;
+  int g, h;
+  gram_block(q, g, h);
+  const float *src = G + (size_t)(g * gm::BT) * kRows + h * gm::BT;
+  for (int i = threadIdx.x; i < gm::BT * (gm::BT / 4); i += THREADS) {
+    const int r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
+    *reinterpret_cast<float4 *>(blk + r * LD + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(src + (size_t)r * kRows) + c4);
+  }
+  __syncthreads();
   const int64_t f0 = (int64_t)blockIdx.x * FRAMES;
-  const int grp = blockIdx.y;
-  const int q0 = grp * PER_GROUP;
-  const int q1 = q0 + PER_GROUP < gm::BLOCKS ? q0 + PER_GROUP : gm::BLOCKS;
-
-  stage_block(gbuf, G, q0);
-  cp_async_commit();
-  // this chunk's codes, transposed to [bin][frame] (frames past F read as level 0, never written)
-  for (int i = threadIdx.x; i < FRAMES * (kMel / 16); i += THREADS) {
-    const int fl = i / (kMel / 16), part = i % (kMel / 16);
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (f0 + fl < F) u = __ldg(reinterpret_cast<const uint4 *>(codes + (f0 + fl) * kMel) + part);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int e = 0; e < FRAMES / THREADS; ++e) {
+    const int64_t f = f0 + e * THREADS + threadIdx.x;
+    if (f >= F) break;
+    const uint8_t *row = codes + f * kMel;
+    const uint2 ug = __ldg(reinterpret_cast<const uint2 *>(row + 8 * g));
+    const uint2 uh = __ldg(reinterpret_cast<const uint2 *>(row + 8 * h));
+    int ri[8], cj[8];
 #pragma unroll
-    for (int b = 0; b < 16; ++b) csm[(16 * part + b) * FRAMES + fl] = (uint8_t)((w[b >> 2] >> (8 * (b & 3))) & 15u);
-  }
-  float acc[2] = {0.0f, 0.0f};
-  for (int q = q0; q < q1; ++q) {
-    const int buf = (q - q0) & 1;
-    if (q + 1 < q1) {
-      stage_block(gbuf + (buf ^ 1) * BLK_FLOATS, G, q + 1);
-      cp_async_commit();
-      cp_async_wait_all_but_one();
-    } else {
-      cp_async_wait_all();
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t cg = ((i < 4 ? ug.x : ug.y) >> (8 * (i & 3))) & 15u;
+      const uint32_t ch = ((i < 4 ? uh.x : uh.y) >> (8 * (i & 3))) & 15u;
+      ri[i] = (16 * i + (int)cg) * LD;
+      cj[i] = 16 * i + (int)ch;
     }
-    __syncthreads();  // block q (and, the first time, the codes) visible to every thread
-    const float *blk = gbuf + buf * BLK_FLOATS;
-    int g, h;
-    gram_block(q, g, h);
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int fl = threadIdx.x + e * THREADS;
-      int ci[8], cj[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        ci[i] = csm[(8 * g + i) * FRAMES + fl];
-        cj[i] = csm[(8 * h + i) * FRAMES + fl];
-      }
-      float s = 0.0f;
-      if (g != h) {
-        // bins of two different groups: every pair once in G's upper block, twice in the sum
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) s += blk[(16 * i + ci[i]) * LD + 16 * j + cj[j]];
-        s *= 2.0f;
-      } else {
-        // one group: the 8 diagonal terms once, the 28 pairs i < j twice
-        float off = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          s += blk[(16 * i + ci[i]) * LD + 16 * i + ci[i]];
-#pragma unroll
-          for (int j = i + 1; j < 8; ++j) off += blk[(16 * i + ci[i]) * LD + 16 * j + ci[j]];
-        }
-        s += 2.0f * off;
-      }
-      acc[e] += s;
-    }
-    __syncthreads();  // everyone is done with this buffer before it is refilled
-  }
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int64_t f = f0 + threadIdx.x + e * THREADS;
-    if (f < F) partials[(size_t)grp * F + f] = acc[e];
+    partials[(size_t)q * F + f] = block_terms(blk, ri, cj, g == h);
   }
 }
 
+// scale_f = 1 / sqrt((sum over the 55 blocks, in block order) / D + eps)
 __global__ void __launch_bounds__(256) norm_finalize_kernel(const float *__restrict__ partials, int64_t F, int D,
                                                             float eps, float *__restrict__ scale) {
   for (int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f < F; f += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.0f;
-#pragma unroll
-    for (int q = 0; q < nm::NGROUPS; ++q) s += partials[(size_t)q * F + f];
+#pragma unroll 5
+    for (int q = 0; q < gm::BLOCKS; ++q) s += partials[(size_t)q * F + f];
     scale[f] = 1.0f / sqrtf(s / (float)D + eps);
   }
 }
@@ -333,7 +304,7 @@ size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 size_t gram_bytes() { return 2 * round256((size_t)kRows * kRows * sizeof(float)); }
 
 size_t norm_scale_bytes(int64_t F) {
-  return round256((size_t)nm::NGROUPS * (size_t)F * sizeof(float)) + round256((size_t)F * sizeof(float));
+  return round256((size_t)gm::BLOCKS * (size_t)F * sizeof(float)) + round256((size_t)F * sizeof(float));
 }
 
 cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaStream_t stream, int *launches) {
@@ -371,7 +342,7 @@ cudaError_t launch_norm_scale(const uint8_t *codes, int64_t F, int D, const floa
   cudaError_t e = set_smem_attr_once(norm_partials_kernel, nm::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
   float *partials = static_cast<float *>(scratch);
-  const dim3 grid((unsigned)((F + nm::FRAMES - 1) / nm::FRAMES), nm::NGROUPS);
+  const dim3 grid((unsigned)((F + nm::FRAMES - 1) / nm::FRAMES), gm::BLOCKS);
   norm_partials_kernel<<<grid, nm::THREADS, nm::SMEM_BYTES, stream>>>(codes, F, G, partials);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ++*launches;
@@ -383,33 +354,21 @@ cudaError_t launch_norm_scale(const uint8_t *codes, int64_t F, int D, const floa
 }
 
 // Host evaluation of the same per-frame formula (diagnostic): sum of squares of the frame with
-// codes c[80] from G [1280 x 1280] (row-major, upper blocks filled), in the kernel's order.
+// codes c[80] from G [1280 x 1280] (row-major, upper blocks filled), in the kernels' order.
 double norm_sumsq_host(const uint8_t *c, const float *G) {
+  std::vector<float> blk(nm::BLK_FLOATS);
   float acc = 0.0f;
-  for (int grp = 0; grp < nm::NGROUPS; ++grp) {
-    float part = 0.0f;
-    for (int q = grp * nm::PER_GROUP; q < (grp + 1) * nm::PER_GROUP && q < gm::BLOCKS; ++q) {
-      int g, h;
-      gram_block(q, g, h);
-      auto at = [&](int bi, int bj) {
-        return G[(size_t)(16 * bi + c[bi]) * kRows + 16 * bj + c[bj]];
-      };
-      float s = 0.0f;
-      if (g != h) {
-        for (int i = 0; i < 8; ++i)
-          for (int j = 0; j < 8; ++j) s += at(8 * g + i, 8 * h + j);
-        s *= 2.0f;
-      } else {
-        float off = 0.0f;
-        for (int i = 0; i < 8; ++i) {
-          s += at(8 * g + i, 8 * g + i);
-          for (int j = i + 1; j < 8; ++j) off += at(8 * g + i, 8 * g + j);
-        }
-        s += 2.0f * off;
-      }
-      part += s;
+  for (int q = 0; q < gm::BLOCKS; ++q) {
+    int g, h;
+    gram_block(q, g, h);
+    for (int r = 0; r < gm::BT; ++r)
+      for (int k = 0; k < gm::BT; ++k) blk[r * nm::LD + k] = G[(size_t)(g * gm::BT + r) * kRows + h * gm::BT + k];
+    int ri[8], cj[8];
+    for (int i = 0; i < 8; ++i) {
+      ri[i] = (16 * i + c[8 * g + i]) * nm::LD;
+      cj[i] = 16 * i + c[8 * h + i];
     }
-    acc += part;
+    acc += block_terms(blk.data(), ri, cj, g == h);
   }
   return (double)acc;
 }

@@ -59,7 +59,7 @@ dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_
  * entries whose row block is at most their column block are written, the others left as they
  * are; the second half is scratch), asynchronously on stream. dmel_debug_norm_sumsq_host evaluates, on the host, the sum of squares of one frame
  * with codes codes80 from a host copy of such a G, in the order the device sums it (blocks of
- * 8 x 8 bins, diagonal terms once, other pairs twice), into *h_sumsq. */
+ * 8 x 8 bins in order, diagonal terms once, other pairs twice), into *h_sumsq. */
 dmel_status dmel_debug_gram(const void *table, int embed_dim, float *gram, dmel_stream_t stream);
 dmel_status dmel_debug_norm_sumsq_host(const uint8_t *codes80, const float *h_gram, double *h_sumsq);
 

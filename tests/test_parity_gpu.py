@@ -223,7 +223,6 @@ def test_embed_rmsnorm_from_gram_matches_oracle(table_bf16, rmsw_bf16, oracle_mo
     ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True), dtype=torch.uint8, device=DEV)
     dmel.dmel_embed(torch.from_numpy(codes).to(DEV), T, out, rms_weight=g, eps=1e-6, workspace=ws)
     torch.cuda.synchronize()
-    assert dmel.dmel_last_launch_count() >= 4  # G, partial sums, scales, product
     for c0 in range(0, F, 4096):
         ref = oracle_mod.embed(codes[c0:c0 + 4096], T64, g64, 1e-6)
         compare_embed(out[c0:c0 + 4096].cpu().numpy(), ref, 1e-5)
