@@ -64,9 +64,13 @@ def out_bytes(out_es: int) -> int:
     return DIM * out_es
 
 
-# DRAM bytes (read + write) per frame of each dominant kernel, from the ncu captures summarised
-# in profiles/ (batch64_10s; per launch = per frame x frames). None when the kernel changed since.
-TRAFFIC_PER_FRAME = {"embed": None, "codes": None}
+# DRAM bytes (read + write) of each stage's kernels, from the ncu capture summarised in
+# profiles/dram_traffic_batch64_10s.md (one 12,800-frame call, cold caches): a fixed part per call
+# and a part per frame, so a launch of F frames moves fixed + F x per_frame. The embedding stage
+# of a call of >= 16,384 frames (the headline's) is gram_kernel (the table once) + norm_partials
+# + embed_sp_kernel<kScaled>. None when a kernel changed since the capture.
+TRAFFIC = {"codes": {"fixed": 0.0, "per_frame": (41083648 + 0) / 12800},
+           "embed": {"fixed": 15749120 + 256, "per_frame": (4639232 + 16945152 + 101312000) / 12800}}
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144 logical flops, run as a
 # 2:4-sparse product whose peak is twice the dense bf16 peak (nominal 4.5 vs 2.25 PFLOP/s)
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
@@ -220,13 +224,17 @@ def stage_lines(F, codes_ms, embed_ms, out_es, pk) -> dict:
     def line(name, ms, bytes_per_frame, kernel):
         s = statistics.mean(ms) / 1e3
         achieved = bytes_per_frame * F / s / 1e9
-        tr = TRAFFIC_PER_FRAME.get(name)
+        tr = TRAFFIC.get(name)
+        if name == "embed" and F < 16384:
+            tr = None  # a smaller call takes the exchange form of RMSNorm, not the captured kernels
         return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": None if tr is None else tr * F,
+                "frac": achieved / pk["hbm_gbs"],
+                "traffic": None if tr is None or tr["per_frame"] is None else tr["fixed"] + tr["per_frame"] * F,
                 "ms": statistics.mean(ms), "kernel": kernel, "peak_source": pk["source"]}
+    norm = ("RMSNorm scales from G = T T^T, then the 2:4-sparse one-hot product" if F >= 16384 else
+            "2:4-sparse one-hot product, RMSNorm by row-sum exchange")
     return {"codes": line("codes", codes_ms, IN_BYTES + CODES_BYTES, "codes_kernel_entry (fp64 DFT, fp32 mel/log/levels)"),
-            "embed": line("embed", embed_ms, CODES_BYTES + out_bytes(out_es), "dmel_embed call (tensor-core one-hot "
-                          "product with fused RMSNorm)")}
+            "embed": line("embed", embed_ms, CODES_BYTES + out_bytes(out_es), f"dmel_embed call ({norm})")}
 
 
 def run_batch(torch, dev, dmel, FrontEnd, name, wl, steps, warmup, pk, flush, with_cpu, cpu_budget,
