@@ -466,6 +466,37 @@ def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_
 
 # ------------------------------------------------------------------------------------ arms
 
+def run_profile(args):
+    """Profiling mode (no timing, no JSON line): dmel_codes and dmel_embed (RMSNorm, bf16 out) on
+    one workload, args.steps times, so a profiler can capture the path's kernels on a call of that
+    size. The form of RMSNorm follows the library's rule for the call size (DMEL_EMBED_NORM
+    overrides it)."""
+    import torch
+    from encoder_free_audio_b200 import build, dmel
+    build.build()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    wl = load_workload(args.profile)
+    fo = dmel.dmel_frame_offsets(wl["off"])
+    F = int(fo[-1])
+    dt = torch.bfloat16 if wl["bf16"] else torch.float32
+    T = torch.from_numpy(wl["table"]).to(dt).to(dev)
+    G = None if wl["g"] is None else torch.from_numpy(wl["g"]).to(dt).to(dev)
+    w = torch.from_numpy(wl["wav"]).to(dev)
+    so, fod = torch.from_numpy(wl["off"]).to(dev), torch.from_numpy(fo).to(dev)
+    codes = torch.empty((F, 80), dtype=torch.uint8, device=dev)
+    out = torch.empty((F, DIM), dtype=dt, device=dev)
+    n = dmel.dmel_workspace_size(F, DIM, dmel._dtype_code(T), G is not None, True)
+    ws = torch.empty(max(1, n), dtype=torch.uint8, device=dev)
+    for _ in range(args.steps):
+        dmel.dmel_codes(w, so, fod, F, codes)
+        dmel.dmel_embed(codes, T, out, rms_weight=G, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    print(f"profile {args.profile}: {F} frames x {args.steps} calls, device error bits "
+          f"{dmel.dmel_get_device_error(clear=True)}", flush=True)
+    return 0
+
+
 def run_reference(args):
     """The oracle on the host cores, on the headline workload: each step a bounded random sample
     of its frames (codes + embedding + RMSNorm, fp64)."""
@@ -635,8 +666,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--stream-calls", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["batch64_10s", "long_20min", "one_clip_2s", "ragged1024"], default=None,
+                    help="run the path's kernels on one workload --steps times, untimed (for profilers)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
