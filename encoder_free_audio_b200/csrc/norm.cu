@@ -266,14 +266,22 @@ __global__ void __launch_bounds__(nm::THREADS, 3)
     const int r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
     *reinterpret_cast<float4 *>(blk + r * LD + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(src + (size_t)r * kRows) + c4);
   }
+  const int64_t f0 = (int64_t)blockIdx.x * FRAMES + threadIdx.x;
+  // the codes of this thread's next frame are loaded while the current frame's terms are summed
+  auto load = [&](int e, uint2 &ug, uint2 &uh) {
+    const int64_t f = f0 + (int64_t)e * THREADS;
+    if (e < FRAMES / THREADS && f < F) {
+      const uint8_t *row = codes + f * kMel;
+      ug = __ldg(reinterpret_cast<const uint2 *>(row + 8 * g));
+      uh = __ldg(reinterpret_cast<const uint2 *>(row + 8 * h));
+    }
+  };
+  uint2 ug = make_uint2(0u, 0u), uh = make_uint2(0u, 0u);
+  load(0, ug, uh);
   __syncthreads();
-  const int64_t f0 = (int64_t)blockIdx.x * FRAMES;
   for (int e = 0; e < FRAMES / THREADS; ++e) {
-    const int64_t f = f0 + e * THREADS + threadIdx.x;
+    const int64_t f = f0 + (int64_t)e * THREADS;
     if (f >= F) break;
-    const uint8_t *row = codes + f * kMel;
-    const uint2 ug = __ldg(reinterpret_cast<const uint2 *>(row + 8 * g));
-    const uint2 uh = __ldg(reinterpret_cast<const uint2 *>(row + 8 * h));
     int ri[8], cj[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -282,6 +290,7 @@ __global__ void __launch_bounds__(nm::THREADS, 3)
       ri[i] = (16 * i + (int)cg) * LD;
       cj[i] = 16 * i + (int)ch;
     }
+    load(e + 1, ug, uh);
     partials[(size_t)q * F + f] = block_terms(blk, ri, cj, g == h);
   }
 }
