@@ -59,6 +59,21 @@ def test_shortconv_ragged_matches_oracle(dt, with_state, oracle_mod):
 
 
 @pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_shortconv_channel_slices_and_long_runs(dt, oracle_mod):
+    """2056 channels (a full 2048-channel slice and one of 8), sequences long enough that each
+    block's run of tokens starts inside a sequence and crosses into the next one."""
+    lens = [0, 2, 900, 1, 1500, 3, 0, 777]
+    C = 2056
+    off, x, w, st = _case(84, lens, C, dt)
+    for with_state in (True, False):
+        y, so = _run(off, x, w, st, dt, with_state=with_state)
+        ry, rso = oracle_mod.shortconv(x, off, w, st if with_state else None)
+        compare_embed(y, ry, 1e-5 if dt == torch.float32 else 1e-2)
+        np.testing.assert_array_equal(so, rso.astype(np.float32))
+    assert dmel.dmel_get_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
 def test_shortconv_decode_token_by_token_equals_offline(dt):
     """Serving: one call per decode step with the state updated in place gives, bit for bit,
     what one call over the whole sequences gives."""
