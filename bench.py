@@ -468,7 +468,7 @@ def hmlp_context(torch, dev, dmel, pk: dict, warmup: int, steps: int = 10, with_
             "peak_tflops": pk["bf16_tflops_sustained"],
             "frac": flop / (ms / 1e3) / 1e12 / pk["bf16_tflops_sustained"], "flop_per_call": flop,
             "launches_per_call": dmel.dmel_last_launch_count(),
-            "gemms": "stage 1 in one tcgen05 kernel; stages 2-4 as 3 cuBLASLt calls per invocation"}
+            "gemms": "stage 1 in one tcgen05 kernel; stages 2-4 on the tcgen05 CTA-pair GEMM, each followed by its row kernel"}
     if with_oracle:
         from oracle import oracle
         host = {k: v.double().cpu().numpy() for k, v in params.items()}

@@ -474,6 +474,21 @@ dmel_status dmel_debug_norm_sumsq_host(const uint8_t *codes80, const float *h_gr
   return DMEL_OK;
 }
 
+dmel_status dmel_debug_gemm(const void *a, int64_t m, int k, int lda, const void *b, int n, float *c,
+                            dmel_stream_t stream) {
+  t_last_launches = 0;
+  if (m < 0 || m > (int64_t)INT32_MAX || k <= 0 || n <= 0 || lda < k || k % 8 || n % 8 || lda % 8)
+    return DMEL_ERR_INVALID_ARG;
+  if (m == 0) return DMEL_OK;
+  if (!a || !b || !c || !aligned(a, 16) || !aligned(b, 16) || !aligned(c, 16)) return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  const cudaError_t e = launch_gemm_debug(a, m, k, lda, b, n, c, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) t_last_launches = 1;
+  return from_cuda(e);
+}
+
 dmel_status dmel_debug_gelu(const float *x, float *y, int64_t n, dmel_stream_t stream) {
   t_last_launches = 0;
   if (n < 0) return DMEL_ERR_INVALID_ARG;

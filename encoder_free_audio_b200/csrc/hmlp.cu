@@ -11,14 +11,12 @@
 // 2x2 group are four consecutive rows and every merge is the previous stage's output read as
 // [rows / 4 x 4 d]: no data moves between stages. Stage 1 runs as one tcgen05 kernel (pixel
 // gather, K = 80 product, LayerNorm and GELU in its epilogue) when d1 is a multiple of 256 up to
-// 1536, else as a gather, a cuBLASLt GEMM and a row kernel; stages 2-4 are cuBLASLt GEMMs
-// (bf16 x bf16 -> fp32) followed by this file's bias / LayerNorm / GELU / rounding row kernel.
-#include <cublasLt.h>
+// 1536, else as a gather, this file's GEMM and a row kernel; stages 2-4 run this file's tcgen05
+// GEMM (bf16 x bf16 -> fp32, CTA pairs) followed by its bias / LayerNorm / GELU / rounding row
+// kernel.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -30,7 +28,6 @@ constexpr int kPatch = 40;
 constexpr int kBlocks = 64;   // 5x5 blocks per patch (8 x 8)
 constexpr int kK1 = 75;       // values per block
 constexpr int kK1Pad = 80;    // row stride of the gathered blocks (16-byte rows)
-constexpr size_t kLtWorkspace = size_t(32) << 20;
 
 __host__ __device__ inline int demorton_r(int m) { return ((m >> 1) & 1) | ((m >> 2) & 2) | ((m >> 3) & 4); }
 __host__ __device__ inline int demorton_c(int m) { return (m & 1) | ((m >> 1) & 2) | ((m >> 2) & 4); }
@@ -557,67 +554,323 @@ __global__ void __launch_bounds__(s1::THREADS, 1)
   }
 }
 
-// cuBLASLt handle per device (created on first use, kept for the process).
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt[256] = {nullptr};
+// ---------------------------------------------------------------- stage GEMMs (tcgen05, CTA pairs)
+//
+// C [M x N] fp32 = A [M x K] bf16 (row-major, K contiguous) * B [K x N] bf16 (row-major, N
+// contiguous), for the merges of stages 2-4 (and stage 1 when it does not run fused). A pair of
+// CTAs computes a 256 x 192 tile: each CTA loads its 128 rows of A (K-major, 128-byte swizzle)
+// and its 96-column half of B (N-major, 64-byte swizzle) per 64-wide K block by TMA; the even
+// CTA's thread issues M = 256, N = 192, K = 16 MMAs into a double-buffered TMEM accumulator of
+// both CTAs. Four epilogue warps per CTA move their 32 rows x 192 columns out of TMEM in 32 x 32
+// fp32 boxes through shared memory and TMA bulk-tensor stores. Rows past M and columns past N
+// (and K past the end) are zero-filled by the loads and clipped by the stores, so any M, N and
+// K that are multiples of 8 work.
+// Tile configuration for pair tiles of 256 x kBN (kBN = 192 or 256): as many K stages as fit
+// beside the output staging (one 4 KB box buffer per epilogue warp, two when that costs no stage).
+template <int kBN>
+struct G2 {
+  static constexpr int BM = 128;                      // rows per CTA (256 per pair)
+  static constexpr int BN = kBN;                      // columns per pair tile
+  static constexpr int BNH = BN / 2;                  // columns of B each CTA loads
+  static constexpr int BK = 64;                       // K per stage: one 128-byte row of A
+  static constexpr int A_STAGE = BM * BK * 2;         // 16 KB
+  static constexpr int B_BOX_COLS = 32;               // 64-byte rows
+  static constexpr int B_BOX = B_BOX_COLS * BK * 2;   // 32 columns x 64 K rows = 4 KB
+  static constexpr int B_BOXES = BNH / B_BOX_COLS;
+  static constexpr int B_STAGE = B_BOXES * B_BOX;
+  static constexpr int STAGE = A_STAGE + B_STAGE;
+  static constexpr int EPI_WARPS = 4;                 // one per TMEM lane quadrant
+  static constexpr int OUT_COLS = 32;                 // fp32 output box: 32 rows x 32 columns (128-byte rows)
+  static constexpr int OUT_BUF = 32 * OUT_COLS * 4;   // 4 KB
+  static constexpr int BUDGET = 227 * 1024 - 1024 - 256;
+  static constexpr int OUT_BUFS =
+      (BUDGET - EPI_WARPS * 2 * OUT_BUF) / STAGE == (BUDGET - EPI_WARPS * OUT_BUF) / STAGE ? 2 : 1;
+  static constexpr int STAGES = (BUDGET - EPI_WARPS * OUT_BUFS * OUT_BUF) / STAGE;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+  static constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
+  static constexpr int OFF_BAR = OFF_OUT + EPI_WARPS * OUT_BUFS * OUT_BUF;
+  static constexpr int N_BARS = 2 * STAGES + 4 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS);  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+  static constexpr uint32_t ACC_STRIDE = 256;           // accumulators at TMEM columns 0 and 256
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(N_BARS * 8 + 8 <= 256, "barrier area");
+  static_assert(A_STAGE % 1024 == 0 && B_STAGE % 1024 == 0 && OFF_OUT % 1024 == 0 && OUT_BUF % 1024 == 0,
+                "swizzle atoms stay aligned");
+  static_assert(B_BOXES * B_BOX_COLS == BNH && BN <= (int)ACC_STRIDE && STAGES >= 4, "tile split");
+};
 
-cudaError_t lt_handle(cublasLtHandle_t *h) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(g_lt_mu);
-  if (!g_lt[dev & 255] && cublasLtCreate(&g_lt[dev & 255]) != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
-  *h = g_lt[dev & 255];
+__device__ __forceinline__ bool g2_tile_at(int64_t i, int64_t n_tiles, int n_tn, int64_t &mp, int &nt) {
+  const int64_t t = (int64_t)(blockIdx.x >> 1) + i * (int64_t)(gridDim.x >> 1);
+  mp = t / n_tn;  // consecutive clusters share a row block of A (read once into L2)
+  nt = (int)(t % n_tn);
+  return t < n_tiles;
+}
+
+template <int kBN>
+__global__ void __launch_bounds__(G2<kBN>::THREADS, 1)
+    hmlp_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                     const __grid_constant__ CUtensorMap cmap, int64_t M, int N, int K, uint32_t *err) {
+  using G = G2<kBN>;
+  constexpr int BM = G::BM, BN = G::BN, BNH = G::BNH, BK = G::BK, STAGES = G::STAGES;
+  constexpr int A_STAGE = G::A_STAGE, B_STAGE = G::B_STAGE, B_BOX = G::B_BOX, B_BOX_COLS = G::B_BOX_COLS;
+  constexpr int B_BOXES = G::B_BOXES, EPI_WARPS = G::EPI_WARPS, OUT_COLS = G::OUT_COLS, OUT_BUF = G::OUT_BUF;
+  constexpr int OUT_BUFS = G::OUT_BUFS, OFF_A = G::OFF_A, OFF_B = G::OFF_B, OFF_OUT = G::OFF_OUT;
+  constexpr int OFF_BAR = G::OFF_BAR, N_BARS = G::N_BARS;
+  constexpr uint32_t ACC_STRIDE = G::ACC_STRIDE, TMEM_COLS = G::TMEM_COLS;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t bar0 = smem_addr(smem + OFF_BAR);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_BAR + N_BARS * 8);
+  const int n_tn = (N + BN - 1) / BN;
+  const int64_t n_tiles = ((M + 2 * BM - 1) / (2 * BM)) * n_tn;
+  const int KB = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full(s), 1);   // the even CTA's expect-tx for both CTAs' loads
+      mbar_init(empty(s), 1);  // the even CTA's commit, multicast to both
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull(a), 1);
+      mbar_init(tempty(a), 2 * EPI_WARPS);  // the epilogue warps of both CTAs (even CTA's barrier)
+    }
+    mbar_init(done_bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_addr(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+    tma_prefetch_desc(&cmap);
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA: this CTA's A rows and B half
+    if (lane == 0) {
+      const uint64_t keep = policy_evict_last();  // B is re-read by every row block
+      int stage = 0;
+      uint32_t phase = 0, pending = 0, pending_phase = 0;
+      bool ok = true;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; ok && g2_tile_at(i, n_tiles, n_tn, mp, nt); ++i) {
+        const int32_t row = (int32_t)((2 * mp + rank) * BM);
+        const int32_t col = nt * BN + (int32_t)rank * BNH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1u, err)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(full(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full(stage), 2 * (A_STAGE + B_STAGE));
+          const uint32_t a_dst = smem_addr(smem + OFF_A + stage * A_STAGE);
+          const uint32_t b_dst = smem_addr(smem + OFF_B + stage * B_STAGE);
+          tma_load_2d_pair(a_dst, &amap, kb * BK, row, fb, keep);
+#pragma unroll
+          for (int q = 0; q < B_BOXES; ++q)
+            tma_load_2d_pair(b_dst + q * B_BOX, &bmap, col + B_BOX_COLS * q, kb * BK, fb, keep);
+          pending |= 1u << stage;
+          pending_phase = (pending_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // the even CTA's barriers count every load; it waits for the last ones before leaving
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (pending & (1u << s)) mbar_wait(full(s), (pending_phase >> s) & 1u, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * BM, BN, 1);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int64_t mp;
+      int nt;
+      for (int64_t i = 0; ok && g2_tile_at(i, n_tiles, n_tn, mp, nt); ++i) {
+        const uint32_t acc = (uint32_t)(i & 1), use = (uint32_t)(i >> 1);
+        if (!mbar_wait(tempty(acc), (use & 1u) ^ 1u, err)) break;
+        const uint32_t d = tmem_base + acc * ACC_STRIDE;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full(stage), phase, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_addr(smem + OFF_A + stage * A_STAGE);
+          const uint32_t b0 = smem_addr(smem + OFF_B + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // A: K-major, 128-byte swizzle, 8-row groups 1024 B apart, 32 B per K step of 16
+            const uint64_t adesc = smem_desc(a0 + 32u * k, 16u, 1024u, kSwizzle128B);
+            // B: N-major, 64-byte swizzle; 32-column boxes B_BOX apart, 8 K-rows 512 B apart,
+            // 16 K-rows (1 KB) per step
+            const uint64_t bdesc = smem_desc(b0 + 1024u * k, (uint32_t)B_BOX, 512u, kSwizzle64B);
+            tc_mma_f16_pair(d, adesc, bdesc, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_both(empty(stage), 3);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull(acc), 3);
+      }
+      tc_commit_pair(done_bar);
+      mbar_wait(done_bar, 0, err);
+    }
+  } else {
+    // ------------------------------------------------ epilogue: 32 rows x 192 columns per warp
+    const int quad = warp & 3;
+    const uint32_t obuf = smem_addr(smem + OFF_OUT + (warp - 2) * OUT_BUFS * OUT_BUF);
+    uint32_t n_stored = 0;
+    bool ok = true;
+    int64_t mp;
+    int nt;
+    for (int64_t i = 0; g2_tile_at(i, n_tiles, n_tn, mp, nt); ++i) {
+      const uint32_t acc = (uint32_t)(i & 1), use = (uint32_t)(i >> 1);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(tfull(acc), use & 1u, err));
+      tc_fence_after();
+      const int64_t row0 = (2 * mp + rank) * BM + 32 * quad;
+      const uint32_t tb = tmem_base + ((uint32_t)(32 * quad) << 16) + acc * ACC_STRIDE;
+      if (ok && row0 < M) {
+#pragma unroll 1
+        for (int c = 0; c < BN / OUT_COLS; ++c) {
+          const int col = nt * BN + OUT_COLS * c;
+          if (col >= N) break;
+          uint32_t v[2][16];
+          tmem_ld16(tb + OUT_COLS * c, v[0]);
+          tmem_ld16(tb + OUT_COLS * c + 16, v[1]);
+          tmem_wait_ld();
+          // row `lane` of the 32 x 32 box: 16-byte chunk j at j ^ (lane & 7) (128-byte swizzle);
+          // the buffer's previous box must have been read by its store first
+          const uint32_t buf = obuf + (n_stored % OUT_BUFS) * OUT_BUF;
+          if (lane == 0 && n_stored >= (uint32_t)OUT_BUFS) {
+            if (OUT_BUFS == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+          }
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t a = buf + lane * 128 + ((j ^ (lane & 7)) << 4);
+            const uint32_t *q = &v[j >> 2][4 * (j & 3)];
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(q[0]), "r"(q[1]), "r"(q[2]),
+                         "r"(q[3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&cmap, col, (int32_t)row0, buf);
+            bulk_commit();
+          }
+          ++n_stored;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(mapa_shared(tempty(acc), 0));
+    }
+    if (lane == 0) bulk_wait<0>();  // stores done before the block's shared memory goes away
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // every MMA into either CTA's TMEM has completed (the even CTA waited above)
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
+// TMA map of a row-major 2-D bf16 / fp32 array [rows x cols] (row stride `ld` elements), in
+// boxes of box_cols x box_rows with the given swizzle.
+cudaError_t make_map(CUtensorMap *map, EncodeTiledFn enc, const void *base, CUtensorMapDataType type, size_t es,
+                     int64_t rows, int64_t cols, int64_t ld, uint32_t box_cols, uint32_t box_rows,
+                     CUtensorMapSwizzle swz) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * (int64_t)es)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(map, type, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   return cudaSuccess;
 }
 
-// Row-major C [M x N] fp32 = A [M x K] (row stride lda) * B [K x N], bf16 inputs, fp32 sums:
-// column-major C^T = B^T A^T for cuBLASLt.
-cudaError_t lt_gemm(cublasLtHandle_t h, const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B,
-                    int N, float *C, void *ws, cudaStream_t stream) {
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  cudaError_t result = cudaErrorUnknown;
-  do {
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
-    // the column-major operands: first B^T [N x K] (ld N), second A^T [K x M] (ld lda)
-    if (cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, N, K, N) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, M, lda) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatrixLayoutCreate(&lc, CUDA_R_32F, N, M, N) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
-    size_t wsb = kLtWorkspace;
-    if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &wsb, sizeof(wsb)) !=
-        CUBLAS_STATUS_SUCCESS)
-      break;
-    cublasLtMatmulHeuristicResult_t heur;
-    int found = 0;
-    if (cublasLtMatmulAlgoGetHeuristic(h, op, lb, la, lc, lc, pref, 1, &heur, &found) != CUBLAS_STATUS_SUCCESS ||
-        found < 1)
-      break;
-    const float alpha = 1.0f, beta = 0.0f;
-    if (cublasLtMatmul(h, op, &alpha, B, lb, A, la, &beta, C, lc, C, lc, &heur.algo, ws, kLtWorkspace, stream) !=
-        CUBLAS_STATUS_SUCCESS)
-      break;
-    result = cudaGetLastError();
-  } while (false);
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return result;
+template <int kBN>
+cudaError_t launch_gemm_bn(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, float *C,
+                           uint32_t *err, int64_t clusters, cudaStream_t stream) {
+  using G = G2<kBN>;
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap amap, bmap, cmap;
+  cudaError_t e;
+  if ((e = make_map(&amap, enc, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, lda, G::BK, G::BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
+      (e = make_map(&bmap, enc, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, N, G::B_BOX_COLS, G::BK,
+                    CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess ||
+      (e = make_map(&cmap, enc, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, N, G::OUT_COLS, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return e;
+  static std::atomic<bool> attr[256];
+  if ((e = set_smem_attr_once(hmlp_gemm_kernel<kBN>, G::SMEM_BYTES, attr)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  cfg.blockDim = dim3(G::THREADS);
+  cfg.dynamicSmemBytes = G::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, hmlp_gemm_kernel<kBN>, amap, bmap, cmap, M, N, K, err);
+}
+
+// Row-major C [M x N] fp32 = A [M x K] (row stride lda) * B [K x N], bf16 inputs, fp32 sums, on
+// hmlp_gemm_kernel (persistent CTA pairs, one per two SMs at most). The tile is 256 x 192 or
+// 256 x 256, whichever finishes its rounds of tiles over the clusters sooner: a 256-column pair
+// MMA takes about 16/15 the time of a 192-column one (measured), so the wider tile wins unless
+// it leaves a nearly empty last round.
+cudaError_t launch_gemm(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, float *C,
+                        uint32_t *err, int num_sms, cudaStream_t stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  if (M > (int64_t)INT32_MAX) return cudaErrorNotSupported;  // TMA row coordinates are 32-bit
+  const int64_t max_clusters = num_sms / 2 > 0 ? num_sms / 2 : 1;
+  const int64_t m_pairs = (M + 255) / 256;
+  auto rounds = [&](int bn, int64_t &clusters) {
+    const int64_t tiles = m_pairs * ((N + bn - 1) / bn);
+    clusters = tiles < max_clusters ? tiles : max_clusters;
+    return (tiles + clusters - 1) / clusters;
+  };
+  int64_t c192, c256;
+  const int64_t r192 = rounds(192, c192), r256 = rounds(256, c256);
+  if (16 * r256 < 15 * r192) return launch_gemm_bn<256>(A, M, K, lda, B, N, C, err, c256, stream);
+  return launch_gemm_bn<192>(A, M, K, lda, B, N, C, err, c192, stream);
 }
 
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct HmlpLayout {
-  size_t a1, h13, h2, f32, lt, w1p, total;
+  size_t a1, h13, h2, f32, w1p, total;
 };
 
 // Stage 1 runs fused (hmlp_stage1_kernel) when d1 is a whole number of 256-column chunks, at
 // most 1536, and the block rows fit the TMA store's 32-bit row coordinate; otherwise as
-// gather + cuBLASLt GEMM + row kernel.
+// gather + this file's GEMM + row kernel.
 bool stage1_fused(int64_t P, const dmel_hmlp_weights &w) {
   return w.d1 % s1::BN == 0 && w.d1 <= s1::MAX_D1 && P * kBlocks <= (int64_t)INT32_MAX;
 }
@@ -635,9 +888,8 @@ HmlpLayout hmlp_layout(int64_t P, const dmel_hmlp_weights &w) {
   if (rows3 * (size_t)w.d3 > f) f = rows3 * (size_t)w.d3;
   if ((size_t)P * (size_t)w.dim > f) f = (size_t)P * (size_t)w.dim;
   L.f32 = r256(f * 4);
-  L.lt = kLtWorkspace;
   L.w1p = r256((size_t)kK1Pad * (size_t)w.d1 * 2);
-  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.lt + L.w1p;
+  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.w1p;
   return L;
 }
 
@@ -664,6 +916,12 @@ cudaError_t launch_gelu_debug(const float *x, float *y, int64_t n, int num_sms, 
   return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_debug(const void *a, int64_t m, int k, int lda, const void *b, int n, float *c, uint32_t *err,
+                              int num_sms, cudaStream_t stream) {
+  return launch_gemm(static_cast<const __nv_bfloat16 *>(a), m, k, lda, static_cast<const __nv_bfloat16 *>(b), n, c,
+                     err, num_sms, stream);
+}
+
 size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w) {
   return n_patches > 0 ? hmlp_layout(n_patches, w).total : 0;
 }
@@ -672,18 +930,15 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
                         void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches) {
   const int64_t P = (int64_t)n * (H / kPatch) * (W / kPatch);
   if (P <= 0) return cudaSuccess;
-  cublasLtHandle_t h;
-  cudaError_t e = lt_handle(&h);
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   const HmlpLayout L = hmlp_layout(P, w);
   uint8_t *base = static_cast<uint8_t *>(workspace);
   auto *A1 = reinterpret_cast<__nv_bfloat16 *>(base);
   auto *H13 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1);
   auto *H2 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13);
   auto *F = reinterpret_cast<float *>(base + L.a1 + L.h13 + L.h2);
-  void *lt_ws = base + L.a1 + L.h13 + L.h2 + L.f32;
   // W1 padded to 80 rows (5 zero rows) so the stage-1 product has a 16-byte aligned K
-  auto *W1 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13 + L.h2 + L.f32 + L.lt);
+  auto *W1 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13 + L.h2 + L.f32);
   if ((e = cudaMemcpyAsync(W1, w.w1, (size_t)kK1 * w.d1 * 2, cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
     return e;
   if ((e = cudaMemsetAsync(W1 + (size_t)kK1 * w.d1, 0, (size_t)(kK1Pad - kK1) * w.d1 * 2, stream)) != cudaSuccess)
@@ -726,19 +981,19 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
     hmlp_gather_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(images), n, H, W, A1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = lt_gemm(h, A1, rows1, kK1Pad, kK1Pad, W1, w.d1, F, lt_ws, stream)) != cudaSuccess) return e;
+    if ((e = launch_gemm(A1, rows1, kK1Pad, kK1Pad, W1, w.d1, F, err, num_sms, stream)) != cudaSuccess) return e;
     if ((e = launch_rows<true>(F, rows1, w.d1, w.b1, w.g1, w.be1, H13, num_sms, stream)) != cudaSuccess) return e;
-    *launches += 2;
+    *launches += 3;
   }
-  if ((e = lt_gemm(h, H13, rows2, 4 * w.d1, 4 * w.d1, W2, w.d2, F, lt_ws, stream)) != cudaSuccess) return e;
+  if ((e = launch_gemm(H13, rows2, 4 * w.d1, 4 * w.d1, W2, w.d2, F, err, num_sms, stream)) != cudaSuccess) return e;
   if ((e = launch_rows<true>(F, rows2, w.d2, w.b2, w.g2, w.be2, H2, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = lt_gemm(h, H2, rows3, 4 * w.d2, 4 * w.d2, W3, w.d3, F, lt_ws, stream)) != cudaSuccess) return e;
+  if ((e = launch_gemm(H2, rows3, 4 * w.d2, 4 * w.d2, W3, w.d3, F, err, num_sms, stream)) != cudaSuccess) return e;
   if ((e = launch_rows<true>(F, rows3, w.d3, w.b3, w.g3, w.be3, H13, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = lt_gemm(h, H13, P, 4 * w.d3, 4 * w.d3, W4, w.dim, F, lt_ws, stream)) != cudaSuccess) return e;
+  if ((e = launch_gemm(H13, P, 4 * w.d3, 4 * w.d3, W4, w.dim, F, err, num_sms, stream)) != cudaSuccess) return e;
   if ((e = launch_rows<false>(F, P, w.dim, w.b4, nullptr, nullptr, static_cast<__nv_bfloat16 *>(out), num_sms,
                               stream)) != cudaSuccess)
     return e;
-  *launches += 3;  // the row kernels of stages 2-4 (their GEMMs are cuBLASLt's)
+  *launches += 6;  // stages 2-4: a GEMM and a row kernel each
   return cudaSuccess;
 }
 

@@ -112,6 +112,8 @@ EncodeTiledFn encode_tiled_fn();
 
 // GELU of n values with the hMLP kernels' formula (diagnostic).
 cudaError_t launch_gelu_debug(const float *x, float *y, int64_t n, int num_sms, cudaStream_t stream);
+cudaError_t launch_gemm_debug(const void *a, int64_t m, int k, int lda, const void *b, int n, float *c, uint32_t *err,
+                              int num_sms, cudaStream_t stream);
 
 // Launches a kernel whose bounded wait cannot be satisfied; *h_returned = 1 once it returned.
 cudaError_t run_wait_timeout_selftest(uint32_t polls, uint32_t *err, int *h_returned);

@@ -114,6 +114,8 @@ def _lib():
         L.dmel_debug_gram.restype = i32
         L.dmel_debug_norm_sumsq_host.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_double)]
         L.dmel_debug_norm_sumsq_host.restype = i32
+        L.dmel_debug_gemm.argtypes = [vp, i64, i32, i32, vp, i32, vp, vp]
+        L.dmel_debug_gemm.restype = i32
         _L = L
     return _L
 
@@ -424,6 +426,16 @@ def dmel_debug_gram(table, gram, stream=None):
     [2, 1280, 1280] (the upper blocks; gram[1] is scratch; diagnostic, see dmel_debug.h)."""
     assert gram.shape == (2, 1280, 1280)
     _check(_lib().dmel_debug_gram(_ptr(table), int(table.shape[1]), _ptr(gram), _stream(stream)), "dmel_debug_gram")
+
+
+def dmel_debug_gemm(a, b, c, stream=None):
+    """c [m, n] fp32 = a [m, k] bf16 @ b [k, n] bf16 on the hMLP stage GEMM (CUDA tensors; a may
+    be a row slice of a wider array: its row stride is passed; diagnostic, see dmel_debug.h)."""
+    m, k = a.shape
+    assert b.shape[0] == k and c.shape == (m, b.shape[1]) and b.is_contiguous() and c.is_contiguous()
+    assert a.stride(1) == 1
+    _check(_lib().dmel_debug_gemm(_ptr(a), int(m), int(k), int(a.stride(0)), _ptr(b), int(b.shape[1]), _ptr(c),
+                                  _stream(stream)), "dmel_debug_gemm")
 
 
 def dmel_debug_norm_sumsq_host(codes80: np.ndarray, gram: np.ndarray) -> float:

@@ -28,8 +28,8 @@
  *     scratch is a fixed array inside the library (see there); dmel_forward_host also creates
  *     two copy streams per device on its first call.
  *   - Calls may come from several host threads at once (each with its own buffers): the
- *     per-device one-time setup (constant tables, kernel attributes, the cuBLASLt handle of
- *     dmel_hmlp) is guarded, and dmel_last_launch_count() reports the calling thread's last call.
+ *     per-device one-time setup (constant tables, kernel attributes) is guarded, and
+ *     dmel_last_launch_count() reports the calling thread's last call.
  *   - Environment (read once per process): DMEL_EMBED_MMA=dense runs the tensor-core embedding
  *     as a dense one-hot product instead of the 2:4-sparse one; DMEL_EMBED_TILE=single runs it
  *     dense on one-CTA tiles instead of CTA pairs; DMEL_COOPERATIVE=0 launches the fused
@@ -322,8 +322,9 @@ size_t dmel_hmlp_workspace_size(int64_t n_patches, const dmel_hmlp_weights *w);
  * out      bf16 [n_images * (height / 40) * (width / 40) x dim], patches in raster order
  * Stage 1 (d1 a multiple of 256, at most 1536; fewer than 2^31 pixel blocks) runs in one
  * tensor-core kernel of the library;
- * otherwise, and for stages 2-4, the products run as dense bf16 GEMMs (cuBLASLt) with the bias,
- * LayerNorm and GELU in the library's kernels. Asynchronous on stream. */
+ * otherwise, and for stages 2-4, the products run on the library's tensor-core GEMM (bf16 x bf16,
+ * fp32 sums, 256 x 192 tiles on CTA pairs) with the bias, LayerNorm and GELU in the library's row
+ * kernel. Asynchronous on stream. */
 dmel_status dmel_hmlp(const void *images, int n_images, int height, int width, const dmel_hmlp_weights *w, void *out,
                       void *workspace, size_t workspace_bytes, dmel_stream_t stream);
 

@@ -63,6 +63,14 @@ dmel_status dmel_debug_forward_host_plan(const int64_t *h_sample_offsets, int n_
 dmel_status dmel_debug_gram(const void *table, int embed_dim, float *gram, dmel_stream_t stream);
 dmel_status dmel_debug_norm_sumsq_host(const uint8_t *codes80, const float *h_gram, double *h_sumsq);
 
+/* The hMLP stage GEMM alone ("Inside Inkling: Audio Design", Part 1 · Modeling: each hMLP stage
+ * is a linear map of the merged features): c [m x n] fp32 = a [m x k] bf16 (row stride lda
+ * elements) times b [k x n] bf16, all row-major device arrays, fp32 sums, on the tcgen05 CTA-pair
+ * kernel dmel_hmlp uses for stages 2-4. m >= 0; n, k and lda positive multiples of 8 with
+ * lda >= k; a, b and c 16-byte aligned; m at most 2^31 - 1. Asynchronous on stream. */
+dmel_status dmel_debug_gemm(const void *a, int64_t m, int k, int lda, const void *b, int n, float *c,
+                            dmel_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -132,3 +132,31 @@ def test_gelu_formula_within_its_error_bound():
     print(f"gelu: worst error / bound {worst:.3f}, max abs error {float(err.max()):.2e}")
     assert worst <= 1.0
     assert float(y[-2]) == 1e4 and float(y[-1]) == 0.0  # saturated tails are exact
+
+
+@pytest.mark.parametrize("m,k,n,lda", [
+    (1, 8, 8, 8),             # one row, one K step (zero-filled past K), one column group
+    (300, 136, 200, 136),     # ragged in every dimension: a half-empty second CTA pair, a partial column tile
+    (4096, 512, 1536, 512),   # 192-column tiles, 16 x 8 = 128 of them: more than one per cluster on 148 SMs
+    (257, 6144, 392, 6200),   # the hMLP's K; A a row slice of a wider array
+    (1600, 256, 6144, 256),   # the last stage's shape: 256-column tiles (fewer rounds of tiles)
+    (25599, 72, 1528, 72),    # 256-column tiles, ragged rows, columns and K, 9 rounds of tiles
+])
+def test_stage_gemm_matches_fp64(m, k, n, lda):
+    """The tcgen05 stage GEMM alone against an fp64 product of the same bf16 inputs: fp32 sums of
+    k products differ from the exact sum by rounding only (bound ~k * 2^-24 of the sum of
+    |a_i b_i|)."""
+    g = torch.Generator(device=DEV).manual_seed(97)
+    a_full = torch.randn((m, lda), device=DEV, generator=g).to(torch.bfloat16)
+    a = a_full[:, :k]
+    b = torch.randn((k, n), device=DEV, generator=g).to(torch.bfloat16)
+    c = torch.full((m, n), float("nan"), device=DEV)
+    dmel.dmel_debug_gemm(a, b, c)
+    torch.cuda.synchronize()
+    assert dmel.dmel_get_device_error(clear=True) == 0
+    ad, bd = a.double().cpu(), b.double().cpu()
+    ref = ad @ bd
+    bound = (ad.abs() @ bd.abs()) * (k * 2.0 ** -24) + 1e-30
+    err = (c.double().cpu() - ref).abs()
+    assert torch.isfinite(c).all()
+    assert (err <= bound).all(), f"worst excess {(err / bound).max().item():.3g}"
