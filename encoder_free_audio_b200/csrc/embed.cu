@@ -1142,8 +1142,9 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         for (int kb = 0; kb < KBLOCKS; ++kb, ++n) {
           if (n >= STAGES_A) sp_issued_sync(sa);  // stage n - 3 (same slot) was issued
           if (lane == 0 && ok) {
+            // the table block is usually long resident: its wait first, the A slot's last
             if (kb == 0) ok = mbar_wait(tempty(acc), acc_phase ^ 1u, err);
-            ok = ok && mbar_wait(full_a(sa), pa, err) && mbar_wait(full_b(sb), pb, err);
+            ok = ok && mbar_wait(full_b(sb), pb, err) && mbar_wait(full_a(sa), pa, err);
           }
           __syncwarp();
           sp_ready_arrive(sa);
@@ -1170,13 +1171,17 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
     bool ok = true;
     int64_t mp;
     int nt;
-    // this row's codes, loaded one tile ahead so a tile boundary does not wait on L2
+    // this row's codes, loaded one tile ahead so a tile boundary does not wait on L2 (volatile
+    // loads: the compiler may not sink them to their first use at the next tile)
     auto load_codes = [&](int64_t mp_, uint4 (&u)[5]) {
       const int64_t f_ = (2 * mp_ + rank) * BM + r;
       if (f_ < F) {
         const uint4 *src = reinterpret_cast<const uint4 *>(codes + f_ * kMel);
 #pragma unroll
-        for (int q = 0; q < 5; ++q) u[q] = __ldg(src + q);
+        for (int q = 0; q < 5; ++q)
+          asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(u[q].x), "=r"(u[q].y), "=r"(u[q].z), "=r"(u[q].w)
+                       : "l"(src + q));
       } else {
 #pragma unroll
         for (int q = 0; q < 5; ++q) u[q] = make_uint4(0u, 0u, 0u, 0u);
@@ -1206,7 +1211,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       const uint32_t one_mask = valid ? 0xFFFFFFFFu : 0u;
 #pragma unroll
       for (int kb = 0; kb < KBLOCKS; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(empty_a(stage), phase ^ 1u, err))) { ok = false; break; }
+        // the stage's one-hot rows and metadata are built before waiting for the slot (the wait
+        // is on the stage three back; building them is off that critical loop)
         const uint32_t wlo = cw[2 * kb], whi = cw[2 * kb + 1];
         // bin j of the stage: stored bf16 8j .. 8j + 7 = columns 4j .. 4j + 3, the 1 in column
         // 4j + (c >> 2), low half when c is even
@@ -1218,7 +1224,6 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
 #pragma unroll
           for (int g = 0; g < 4; ++g) av[4 * j + g] = (c >> 2) == (uint32_t)g ? one : 0u;
         }
-        tmem_st32(lane_base + a_col(stage), av);
         uint32_t m[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -1228,6 +1233,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
           const uint32_t lo = __shfl_sync(0xffffffffu, pk, src_lo), hi = __shfl_sync(0xffffffffu, pk, src_hi);
           m[k] = ((lo >> half_shift) & 0xFFFFu) | (((hi >> half_shift) & 0xFFFFu) << 16);
         }
+        if (!__all_sync(0xffffffffu, mbar_wait(empty_a(stage), phase ^ 1u, err))) { ok = false; break; }
+        tmem_st32(lane_base + a_col(stage), av);
         tmem_st4(lane_base + META_COL + 4u * stage, m[0], m[1], m[2], m[3]);
         tmem_wait_st();
         tc_fence_before();
