@@ -200,19 +200,40 @@ __host__ __device__ inline void dft8(double (&r)[8], double (&i)[8]) {
 
 // Step A, first half, straight from global memory: lane l reads the samples
 // x[800 (t - 1) + 64 j + 2 l] and the next one of frame t (start = 800 (t - 1)), j = 0..24 (the
-// warp reads 64 consecutive samples per j; the previous frame of the warp usually left them in
-// L1). Samples before the clip come from the carried tail (tail points one past its last sample)
-// or are zero. Windowed as in step_a_load.
+// warp reads 64 consecutive samples per j). For the first frame of a clip, samples before the
+// clip come from the carried tail (tail points one past its last sample) or are zero. Windowed
+// as in step_a_load.
 __device__ inline void step_a_load_global(int l, const float *base, const float *tail, int64_t start,
                                           const Tables &T, double (&ar)[25], double (&ai)[25]) {
+  if (start >= 0) {
+    // 8-byte loads from the 8-byte boundary at or below the frame start: when the frame starts
+    // 4 bytes past one (mis = 1), lane l's pair is the high half of its own load and the low half
+    // of lane l + 1's (lane 31: of lane 0's next load; the frame's last sample on its own); one
+    // code path for either alignment
+    const float *p0 = base + start;
+    const uint32_t mis = (uint32_t)(reinterpret_cast<uintptr_t>(p0) >> 2) & 1u;
+    const float2 *q = reinterpret_cast<const float2 *>(p0 - mis) + l;
+    float2 v[25];
+#pragma unroll
+    for (int j = 0; j < 25; ++j) v[j] = __ldg(q + 32 * j);
+    const float last = (mis && l == 31) ? __ldg(p0 + 1599) : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 25; ++j) {
+      const float nx = __shfl_sync(0xffffffffu, v[j].x, (l + 1) & 31);
+      const float wx = __shfl_sync(0xffffffffu, j + 1 < 25 ? v[j + 1].x : last, 0);
+      const float x0 = mis ? v[j].y : v[j].x;
+      const float x1 = mis ? (l == 31 ? (j + 1 < 25 ? wx : last) : nx) : v[j].y;
+      const double2 w = T.hann2[32 * j + l];  // periodic Hann at 64 j + 2 l and the next sample
+      ar[j] = w.x * (double)x0;
+      ai[j] = w.y * (double)x1;
+    }
+    return;
+  }
 #pragma unroll
   for (int j = 0; j < 25; ++j) {
     const int n = 64 * j + 2 * l;  // even: n and n + 1 fall on the same side of sample 800
     float x0, x1;
-    if (start >= 0) {
-      x0 = __ldg(base + start + n);
-      x1 = __ldg(base + start + n + 1);
-    } else if (n >= 800) {  // first frame of a clip (start = -800): the new samples
+    if (n >= 800) {  // first frame of a clip (start = -800): the new samples
       x0 = __ldg(base + (n - 800));
       x1 = __ldg(base + (n - 799));
     } else {  // ... after the carried tail or zeros
@@ -657,11 +678,24 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     lo = lo + (31 - __clz(le));
   }
   int clip = lo;
+  // the clip's bounds stay in registers while the warp walks its frames (four independent loads
+  // when it enters a clip, none per frame)
+  int64_t f_next, f_first, s_first, s_len;
+  auto enter = [&]() {
+    f_next = clip + 1 < n_clips ? foff[clip + 1] : INT64_MAX;
+    f_first = foff[clip];
+    s_first = soff[clip];
+    s_len = soff[clip + 1] - s_first;
+  };
+  enter();
 
   for (int64_t g = g0; g < g1; ++g) {
-    while (clip + 1 < n_clips && foff[clip + 1] <= g) ++clip;
-    const int64_t t = g - foff[clip];
-    const int64_t len = soff[clip + 1] - soff[clip];
+    if (g >= f_next) {  // the next clip with a frame at or before g (clips of no frame skipped)
+      do ++clip; while (clip + 1 < n_clips && foff[clip + 1] <= g);
+      enter();
+    }
+    const int64_t t = g - f_first;
+    const int64_t len = s_len;
     uint8_t *crow = codes + g * kMel;
     if (t < 0 || (int64_t)kHop * (t + 1) > len) {  // offsets do not describe this frame
       if (lane == 0) record_error(err, DMEL_DEVERR_OFFSETS);
@@ -670,11 +704,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     }
     // the next frame of this clip needs samples [800 (t + 1), 800 (t + 2)): start them into L1
     if (g + 1 < g1 && (int64_t)kHop * (t + 2) <= len && lane < 25)
-      asm volatile("prefetch.global.L1 [%0];" ::"l"(wav + soff[clip] + (int64_t)kHop * (t + 1) + 32 * lane));
+      asm volatile("prefetch.global.L1 [%0];" ::"l"(wav + s_first + (int64_t)kHop * (t + 1) + 32 * lane));
     __syncwarp();  // the previous frame's partials are read before this frame's DFT outputs land
     {
       double ar[25], ai[25];
-      step_a_load_global(lane, wav + soff[clip], tails ? tails + (int64_t)clip * kHop + kHop : nullptr,
+      step_a_load_global(lane, wav + s_first, tails ? tails + (int64_t)clip * kHop + kHop : nullptr,
                          (int64_t)kHop * (t - 1), T, ar, ai);
       step_a_dft(lane, T, ar, ai, B);
     }
