@@ -299,7 +299,7 @@ __host__ __device__ inline void step_a_dft(int l, const Tables &T, double (&ar)[
 
 // Step C1, unit u = 4 k1 + l0 (0..99): 8-point DFT over l1 of row k1, columns l0 + 4 l1, times
 // W_32^{l0 k2a}, written back to the same columns (output k2a in column l0 + 4 k2a). Units own
-// disjoint columns, so a lane loads two units before storing either (the loads overlap).
+// disjoint columns, so a lane loads several units before storing any (the loads overlap).
 __host__ __device__ inline void c1_load(int u, const double2 *B, double (&r)[8], double (&i)[8]) {
   const int k1 = u >> 2, l0 = u & 3;
 #pragma unroll
@@ -310,31 +310,34 @@ __host__ __device__ inline void c1_load(int u, const double2 *B, double (&r)[8],
   }
 }
 
-__host__ __device__ inline void c1_finish(int u, const Tables &T, double (&r)[8], double (&i)[8], double2 *B) {
+__host__ __device__ inline void c1_finish(int u, const double2 (&w)[8], double (&r)[8], double (&i)[8], double2 *B) {
   const int k1 = u >> 2, l0 = u & 3;
   dft8(r, i);
 #pragma unroll
   for (int k2a = 0; k2a < 8; ++k2a) {
     double xr = r[k2a], xi = i[k2a];
-    if (l0 * k2a != 0) {
-      const double2 w = tw(T, 50 * l0 * k2a);  // W_32^{l0 k2a}
-      cmul(xr, xi, w.x, w.y);
-    }
+    if (l0 * k2a != 0) cmul(xr, xi, w[k2a].x, w[k2a].y);  // W_32^{l0 k2a}
     B[slot(k1, l0 + 4 * k2a)] = make_double2(xr, xi);
   }
 }
 
-// All C1 units of lane l: u = l, l + 32, l + 64 (and l + 96 for l < 4), two at a time.
+// All C1 units of lane l: u = l, l + 32, l + 64 (loaded together), then l + 96 for l < 4. Every
+// unit of the lane has l0 = l & 3, so its seven twiddles W_32^{l0 k2a} are read once.
 __host__ __device__ inline void step_c1_lane(int l, const Tables &T, double2 *B) {
+  double2 w[8];
 #pragma unroll
-  for (int q = 0; q < 4; q += 2) {
-    const int u0 = l + 32 * q, u1 = l + 32 * (q + 1);
-    double r0[8], i0[8], r1[8], i1[8];
-    const bool has1 = u1 < 100;
-    c1_load(u0, B, r0, i0);
-    if (has1) c1_load(u1, B, r1, i1);
-    c1_finish(u0, T, r0, i0, B);
-    if (has1) c1_finish(u1, T, r1, i1, B);
+  for (int k2a = 0; k2a < 8; ++k2a) w[k2a] = tw(T, 50 * (l & 3) * k2a);
+  {
+    double r[3][8], i[3][8];
+#pragma unroll
+    for (int q = 0; q < 3; ++q) c1_load(l + 32 * q, B, r[q], i[q]);
+#pragma unroll
+    for (int q = 0; q < 3; ++q) c1_finish(l + 32 * q, w, r[q], i[q], B);
+  }
+  if (l < 4) {
+    double r[8], i[8];
+    c1_load(l + 96, B, r, i);
+    c1_finish(l + 96, w, r, i, B);
   }
 }
 
