@@ -43,10 +43,9 @@
 namespace dmel {
 namespace {
 
-// Warps (frames in flight) per block, one block per SM: 12 (168 registers per thread) or 14
-// (the shared-memory limit; the register file then allows 146 per thread and some spill).
+// Warps (frames in flight) per block, one block per SM: 12 (168 registers per thread; 14 fit the
+// shared memory only without the step-D twiddle table and then spill, which measured slower).
 constexpr int kWarpsDefault = 12;
-constexpr int kWarpsMore = 14;
 constexpr int kRunLen = 13;        // bins per lane run (rounds r = 0..12 of step D)
 constexpr int kMaxFlush = 16;      // channel partials one lane writes per run, at most
 constexpr int kMaxSegs = 256;      // channel partials per frame (+ one slot for edge flushes)
@@ -57,20 +56,22 @@ constexpr int kSmW = 0;                                    // double2 [801]: W_1
 constexpr int kSmHann = kSmW + 801 * 16;                   // double2 [800]: (w[2m], w[2m+1])
 constexpr int kSmTwA = kSmHann + 800 * 16;                 // double2 [25 * 32]: W_800^{l k1}
 constexpr int kSmMelW2 = kSmTwA + 800 * 16;                // float2 [2][13][32]: bin weights per lane run
-constexpr int kSmSlot = kSmMelW2 + 2 * kRunLen * 32 * 8;   // ushort [32][2][kMaxFlush]: partial slots
+constexpr int kSmTwD = kSmMelW2 + 2 * kRunLen * 32 * 8;    // double2 [2][13][32]: step-D twiddles per lane run
+constexpr int kSmSlot = kSmTwD + 2 * kRunLen * 32 * 16;    // ushort [32][2][kMaxFlush]: partial slots
 constexpr int kSmFlush = kSmSlot + 32 * 2 * kMaxFlush * 2; // uint [2][32]: run positions of new channels
 constexpr int kSmChanSeg = kSmFlush + 64 * 4;              // int [81]: slot range per channel
 constexpr int kSmTables = (kSmChanSeg + 84 * 4 + 127) / 128 * 128;
 constexpr int kWarpBufBytes = 800 * 16;
 __host__ __device__ constexpr int smem_bytes(int warps) { return kSmTables + warps * kWarpBufBytes; }
 static_assert(kMaxSegs * 4 <= 2 * 32 * 16, "mel partials fit in rows 0 and 1 of the warp's buffer");
-static_assert(smem_bytes(kWarpsMore) <= 227 * 1024, "shared memory budget");
+static_assert(smem_bytes(kWarpsDefault) <= 227 * 1024, "shared memory budget");
 
 // Constant tables, filled once per device from host-computed fp64 values.
 __device__ double2 d_w1600[kBins];
 __device__ double2 d_hann2[800];
 __device__ double2 d_twa[800];
 __device__ float2 d_melw2[2 * kRunLen * 32];
+__device__ double2 d_twd[2 * kRunLen * 32];
 __device__ unsigned short d_slot[32 * 2 * kMaxFlush];
 __device__ unsigned int d_flush[64];
 __device__ int d_chanseg[81];
@@ -82,6 +83,9 @@ struct Tables {
   // mel weights of the bins of lane l's runs, run q (0: ascending, 1: descending) round r, at
   // [(q * 13 + r) * 32 + l]: (weight to the lower channel, weight to the channel above it)
   const float2 *melw2;
+  // W_1600^k of the bin k of lane l's run q at round r, at [(q * 13 + r) * 32 + l] (a copy of the
+  // W table's entry, laid out so the 32 lanes of a round read 32 consecutive entries)
+  const double2 *twd;
   const unsigned short *slot;  // partial slots of lane l's run q, in order, at [(l * 2 + q) * kMaxFlush]
   const unsigned int *flush;   // bit r of [q * 32 + l]: the run enters a new channel at round r
   const int *chanseg;          // channel b adds the partials [chanseg[b], chanseg[b + 1])
@@ -394,12 +398,11 @@ __host__ __device__ inline void step_d_load01(int l, const double2 *B, Pair01 &R
 }
 
 
-// |X_k|^2 of the real 1600-point DFT from a = Z_k and b = Z_{800-k}.
-__host__ __device__ inline double power_bin(const Tables &T, int k, double2 a, double2 b) {
+// |X_k|^2 of the real 1600-point DFT from a = Z_k and b = Z_{800-k}, with w = W_1600^k.
+__host__ __device__ inline double power_bin(double2 w, double2 a, double2 b) {
   const double er = 0.5 * (a.x + b.x), ei = 0.5 * (a.y - b.y);  // (Z_k + conj Z_{800-k}) / 2
   const double dr = a.x - b.x, di = a.y + b.y;                    // Z_k - conj Z_{800-k}
   const double or_ = 0.5 * di, oi = -0.5 * dr;                    // / (2 i)
-  const double2 w = tw(T, k);
   const double xr = er + (or_ * w.x - oi * w.y);
   const double xi = ei + (or_ * w.y + oi * w.x);
   return xr * xr + xi * xi;
@@ -427,13 +430,13 @@ __host__ __device__ inline void step_de_lane(int l, const Tables &T, const Pair0
   const unsigned short *sl[2] = {T.slot + (l * 2) * kMaxFlush, T.slot + (l * 2 + 1) * kMaxFlush};
 #pragma unroll
   for (int r = 0; r < kRunLen; ++r) {
-    const int k = 25 * k2 + r;
     const double2 a = r == 0 ? R.a0 : r == 1 ? R.a1 : B[slot(r, l)];
     const double2 b = r == 0 ? R.b0 : r == 1 ? R.b1 : B[slot(25 - r, 31 - l)];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       if (r == 0 && (q == 0 ? k2 > 16 : k2 > 15)) continue;
-      const float p = q == 0 ? (float)power_bin(T, k, a, b) : (float)power_bin(T, 800 - k, b, a);
+      const double2 w = T.twd[(q * kRunLen + r) * 32 + l];  // W_1600^k (run 0), W_1600^{800-k} (run 1)
+      const float p = q == 0 ? (float)power_bin(w, a, b) : (float)power_bin(w, b, a);
       if ((fl[q] >> r) & 1u) {
         if (q == 0) {
           part[sl[0][nf[0]++]] = lo[0];
@@ -445,9 +448,9 @@ __host__ __device__ inline void step_de_lane(int l, const Tables &T, const Pair0
           lo[1] = 0.0f;
         }
       }
-      const float2 w = T.melw2[(q * kRunLen + r) * 32 + l];
-      lo[q] = fmaf(w.x, p, lo[q]);
-      hi[q] = fmaf(w.y, p, hi[q]);
+      const float2 mw = T.melw2[(q * kRunLen + r) * 32 + l];
+      lo[q] = fmaf(mw.x, p, lo[q]);
+      hi[q] = fmaf(mw.y, p, hi[q]);
     }
   }
 #pragma unroll
@@ -494,11 +497,14 @@ __host__ __device__ inline void step_e_codes(int l, const Tables &T, const float
 struct HostTables {
   std::vector<double2> w, hann2, twa;
   std::vector<float2> melw2;
+  std::vector<double2> twd;
   std::vector<unsigned short> slot;
   std::vector<unsigned int> flush;
   int chanseg[81];
   bool ok = true;  // every check of the mel layout held
-  Tables view() const { return Tables{w.data(), hann2.data(), twa.data(), melw2.data(), slot.data(), flush.data(), chanseg}; }
+  Tables view() const {
+    return Tables{w.data(), hann2.data(), twa.data(), melw2.data(), twd.data(), slot.data(), flush.data(), chanseg};
+  }
 };
 
 void build_host_tables(HostTables &H) {
@@ -540,6 +546,13 @@ void build_host_tables(HostTables &H) {
   // per lane and run: weights, the rounds where the run enters a new channel, the channel of each
   // partial it writes (-1 / 80: outside 0..79, sent to a trash slot)
   H.melw2.assign(2 * kRunLen * 32, make_float2(0.0f, 0.0f));
+  H.twd.assign(2 * kRunLen * 32, make_double2(0.0, 0.0));
+  for (int l = 0; l < 32; ++l)
+    for (int q = 0; q < 2; ++q)
+      for (int r = 0; r < kRunLen; ++r) {
+        const int k = run_bin(l, q, r);  // at most 800: a direct entry of the W table
+        if (k >= 0) H.twd[(q * kRunLen + r) * 32 + l] = H.w[k];
+      }
   H.flush.assign(64, 0u);
   std::vector<int> fch[32][2];
   for (int l = 0; l < 32; ++l)
@@ -603,6 +616,7 @@ cudaError_t ensure_device_tables() {
   if ((e = cudaMemcpyToSymbol(d_hann2, H.hann2.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_twa, H.twa.data(), sizeof(double2) * 800)) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_melw2, H.melw2.data(), sizeof(float2) * H.melw2.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpyToSymbol(d_twd, H.twd.data(), sizeof(double2) * H.twd.size())) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_slot, H.slot.data(), sizeof(unsigned short) * H.slot.size())) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_flush, H.flush.data(), sizeof(unsigned int) * H.flush.size())) != cudaSuccess) return e;
   if ((e = cudaMemcpyToSymbol(d_chanseg, H.chanseg, sizeof(H.chanseg))) != cudaSuccess) return e;
@@ -639,7 +653,11 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
       h2[i] = d_hann2[i];
       ta[i] = d_twa[i];
     }
-    for (int i = threadIdx.x; i < 2 * kRunLen * 32; i += blockDim.x) mw[i] = d_melw2[i];
+    double2 *td = reinterpret_cast<double2 *>(smem + kSmTwD);
+    for (int i = threadIdx.x; i < 2 * kRunLen * 32; i += blockDim.x) {
+      mw[i] = d_melw2[i];
+      td[i] = d_twd[i];
+    }
     for (int i = threadIdx.x; i < 32 * 2 * kMaxFlush; i += blockDim.x) sl[i] = d_slot[i];
     for (int i = threadIdx.x; i < 64; i += blockDim.x) fl[i] = d_flush[i];
     for (int i = threadIdx.x; i < 81; i += blockDim.x) cs[i] = d_chanseg[i];
@@ -647,6 +665,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
   __syncthreads();
   const Tables T{reinterpret_cast<const double2 *>(smem + kSmW), reinterpret_cast<const double2 *>(smem + kSmHann),
                  reinterpret_cast<const double2 *>(smem + kSmTwA), reinterpret_cast<const float2 *>(smem + kSmMelW2),
+                 reinterpret_cast<const double2 *>(smem + kSmTwD),
                  reinterpret_cast<const unsigned short *>(smem + kSmSlot),
                  reinterpret_cast<const unsigned int *>(smem + kSmFlush), reinterpret_cast<const int *>(smem + kSmChanSeg)};
   double2 *B = reinterpret_cast<double2 *>(smem + kSmTables + warp * kWarpBufBytes);
@@ -761,37 +780,19 @@ __global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restric
 
 // ---------------------------------------------------------------- host entry points
 
-// Warps per block of the codes kernel: kWarpsDefault unless the environment sets
-// DMEL_CODES_WARPS=14 (read once per process; for measurement).
-int codes_warps() {
-  static const int w = [] {
-    const char *v = getenv("DMEL_CODES_WARPS");
-    return (v && atoi(v) == kWarpsMore) ? kWarpsMore : kWarpsDefault;
-  }();
-  return w;
-}
-
 cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *foff, int n_clips, int64_t n_frames,
                          const float *tails, float *tails_out, uint8_t *codes, uint32_t *err, int num_sms,
                          cudaStream_t stream, int *launches, Quant q) {
   cudaError_t e = ensure_device_tables();
   if (e != cudaSuccess) return e;
-  static std::atomic<bool> attr12[256], attr14[256];
-  const bool more = codes_warps() == kWarpsMore;
-  if ((e = more ? set_smem_attr_once(codes_kernel_entry<kWarpsMore>, smem_bytes(kWarpsMore), attr14)
-                : set_smem_attr_once(codes_kernel_entry<kWarpsDefault>, smem_bytes(kWarpsDefault), attr12)) !=
-      cudaSuccess)
+  static std::atomic<bool> attr[256];
+  if ((e = set_smem_attr_once(codes_kernel_entry<kWarpsDefault>, smem_bytes(kWarpsDefault), attr)) != cudaSuccess)
     return e;
   if (n_frames > 0) {
-    const int W = more ? kWarpsMore : kWarpsDefault;
-    int64_t blocks = (n_frames + W - 1) / W;
+    int64_t blocks = (n_frames + kWarpsDefault - 1) / kWarpsDefault;
     if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM
-    if (more)
-      codes_kernel_entry<kWarpsMore><<<(unsigned)blocks, kWarpsMore * 32, smem_bytes(kWarpsMore), stream>>>(
-          wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
-    else
-      codes_kernel_entry<kWarpsDefault><<<(unsigned)blocks, kWarpsDefault * 32, smem_bytes(kWarpsDefault), stream>>>(
-          wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
+    codes_kernel_entry<kWarpsDefault><<<(unsigned)blocks, kWarpsDefault * 32, smem_bytes(kWarpsDefault), stream>>>(
+        wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
