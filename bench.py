@@ -64,13 +64,15 @@ def out_bytes(out_es: int) -> int:
     return DIM * out_es
 
 
-# DRAM bytes (read + write) of each stage's kernels, from the ncu capture summarised in
-# profiles/dram_traffic_batch64_10s.md (one 12,800-frame call, cold caches): a fixed part per call
-# and a part per frame, so a launch of F frames moves fixed + F x per_frame. The embedding stage
-# of a call of >= 16,384 frames (the headline's) is gram_kernel (the table once) + norm_partials
-# + embed_sp_kernel<kScaled>. None when a kernel changed since the capture.
-TRAFFIC = {"codes": {"fixed": 0.0, "per_frame": (41083648 + 0) / 12800},
-           "embed": {"fixed": 15749120 + 256, "per_frame": (4639232 + 16945152 + 101312000) / 12800}}
+# DRAM bytes (read + write) of each stage's kernels per launch, from the ncu captures summarised
+# under profiles/: measured on the headline workload itself (318,044 frames: codes_kernel_entry and
+# embed_sp_kernel<kScaled>) where a capture of that size exists, else from the 12,800-frame
+# capture as a fixed part per call plus a part per frame. The embedding stage of a call of >= 16,384 frames is gram_kernel
+# (the table once) + norm_partials_kernel (55 blocks of G + the codes) + embed_sp_kernel<kScaled>.
+TRAFFIC_MEASURED = {318044: {"codes": 1024500480 + 27511296,
+                             "embed": 15749120 + (3604480 + 80 * 318044) + (47177984 + 3850828288)}}
+TRAFFIC = {"codes": {"fixed": 0.0, "per_frame": (41091584 + 0) / 12800},
+           "embed": {"fixed": 15749120 + 3604480 + 15728640, "per_frame": 80 + (16923648 - 15728640 + 101618688) / 12800}}
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144 logical flops, run as a
 # 2:4-sparse product whose peak is twice the dense bf16 peak (nominal 4.5 vs 2.25 PFLOP/s)
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
@@ -225,11 +227,13 @@ def stage_lines(F, codes_ms, embed_ms, out_es, pk) -> dict:
         s = statistics.mean(ms) / 1e3
         achieved = bytes_per_frame * F / s / 1e9
         tr = TRAFFIC.get(name)
+        traffic = None if tr is None else tr["fixed"] + tr["per_frame"] * F
         if name == "embed" and F < 16384:
-            tr = None  # a smaller call takes the exchange form of RMSNorm, not the captured kernels
+            traffic = None  # a smaller call takes the exchange form of RMSNorm, not the captured kernels
+        if F in TRAFFIC_MEASURED:
+            traffic = TRAFFIC_MEASURED[F][name]
         return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"],
-                "traffic": None if tr is None or tr["per_frame"] is None else tr["fixed"] + tr["per_frame"] * F,
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                 "ms": statistics.mean(ms), "kernel": kernel, "peak_source": pk["source"]}
     norm = ("RMSNorm scales from G = T T^T, then the 2:4-sparse one-hot product" if F >= 16384 else
             "2:4-sparse one-hot product, RMSNorm by row-sum exchange")
@@ -492,6 +496,12 @@ def run_profile(args):
     build.build()
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
+    if args.profile in ("shortconv", "hmlp"):
+        fn = shortconv_context if args.profile == "shortconv" else hmlp_context
+        line = fn(torch, dev, dmel, peaks(), 3, steps=args.steps)
+        print(f"profile {args.profile}: {args.steps} calls after 3 warm-ups, device error bits "
+              f"{dmel.dmel_get_device_error(clear=True)}", flush=True)
+        return 0
     wl = load_workload(args.profile)
     fo = dmel.dmel_frame_offsets(wl["off"])
     F = int(fo[-1])
@@ -682,8 +692,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--stream-calls", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=["batch64_10s", "long_20min", "one_clip_2s", "ragged1024"], default=None,
-                    help="run the path's kernels on one workload --steps times, untimed (for profilers)")
+    ap.add_argument("--profile", choices=["batch64_10s", "long_20min", "one_clip_2s", "ragged1024", "shortconv", "hmlp"],
+                    default=None, help="run the path's kernels on one workload --steps times, untimed (for "
+                    "profilers); shortconv / hmlp: the context line's calls, --steps of them after 3 warm-ups")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.profile:
