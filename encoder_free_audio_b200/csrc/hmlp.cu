@@ -12,8 +12,9 @@
 // [rows / 4 x 4 d]: no data moves between stages. Stage 1 runs as one tcgen05 kernel (pixel
 // gather, K = 80 product, LayerNorm and GELU in its epilogue) when d1 is a multiple of 256 up to
 // 1536, else as a gather, this file's GEMM and a row kernel; stages 2-4 run this file's tcgen05
-// GEMM (bf16 x bf16 -> fp32, CTA pairs) followed by its bias / LayerNorm / GELU / rounding row
-// kernel.
+// GEMM (bf16 x bf16 -> fp32, CTA pairs), whose epilogue adds the bias and, for stages 2 and 3,
+// the rows' per-tile statistics for the one-pass LayerNorm / GELU / rounding row kernel that
+// follows; stage 4 rounds to bf16 in the epilogue itself.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -81,47 +82,37 @@ __device__ __forceinline__ float gelu_erf(float u) {
   return fmaf(-fabsf(u), h, fmaxf(u, 0.0f));
 }
 
-// One warp per row of d fp32 sums: + bias, then (kNorm) LayerNorm with gain / shift and the
-// GELU, rounded to bf16. Mean first, then the mean squared deviation (two passes).
-template <bool kNorm>
-__global__ void __launch_bounds__(256) hmlp_row_kernel(const float *__restrict__ in, int64_t rows, int d,
-                                                       const float *__restrict__ bias, const float *__restrict__ g,
-                                                       const float *__restrict__ be, __nv_bfloat16 *__restrict__ out) {
+// One warp per row of d fp32 values that already include the bias, with the row's mean and sum of
+// squared deviations per column tile of bn values from the GEMM epilogue (n_tn tiles, the last
+// one possibly partial): merged in tile order (Chan et al.'s pairwise update), then LayerNorm with
+// gain / shift and GELU, rounded to bf16, in one pass over the row.
+__global__ void __launch_bounds__(256) hmlp_row_kernel(const float *__restrict__ in, const float2 *__restrict__ stats,
+                                                       int n_tn, int bn, int64_t rows, int d,
+                                                       const float *__restrict__ g, const float *__restrict__ be,
+                                                       __nv_bfloat16 *__restrict__ out) {
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const float *x = in + r * d;
     __nv_bfloat16 *y = out + r * d;
-    float mean = 0.0f, rstd = 1.0f;
-    if (kNorm) {
-      float s = 0.0f;
-      for (int j = 4 * lane; j < d; j += 128) {
-        const float4 v = *reinterpret_cast<const float4 *>(x + j), b = *reinterpret_cast<const float4 *>(bias + j);
-        s += (v.x + b.x) + (v.y + b.y) + (v.z + b.z) + (v.w + b.w);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      mean = s / (float)d;
-      float q = 0.0f;
-      for (int j = 4 * lane; j < d; j += 128) {
-        const float4 v = *reinterpret_cast<const float4 *>(x + j), b = *reinterpret_cast<const float4 *>(bias + j);
-        const float e0 = v.x + b.x - mean, e1 = v.y + b.y - mean, e2 = v.z + b.z - mean, e3 = v.w + b.w - mean;
-        q += e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-      rstd = 1.0f / sqrtf(q / (float)d + 1e-6f);
+    float n = 0.0f, mean = 0.0f, m2 = 0.0f;
+    for (int t = 0; t < n_tn; ++t) {
+      const float2 st = stats[r * n_tn + t];
+      const float nb = (float)(d - t * bn < bn ? d - t * bn : bn);
+      const float nn = n + nb, delta = st.x - mean;
+      mean += delta * (nb / nn);
+      m2 += st.y + delta * delta * (n * nb / nn);
+      n = nn;
     }
+    const float rstd = 1.0f / sqrtf(m2 / (float)d + 1e-6f);
     for (int j = 4 * lane; j < d; j += 128) {
-      const float4 v = *reinterpret_cast<const float4 *>(x + j), b = *reinterpret_cast<const float4 *>(bias + j);
-      float t[4] = {v.x + b.x, v.y + b.y, v.z + b.z, v.w + b.w};
-      if (kNorm) {
-        const float4 gg = *reinterpret_cast<const float4 *>(g + j), bb = *reinterpret_cast<const float4 *>(be + j);
-        const float gv[4] = {gg.x, gg.y, gg.z, gg.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+      const float4 v = *reinterpret_cast<const float4 *>(x + j);
+      const float4 gg = *reinterpret_cast<const float4 *>(g + j), bb = *reinterpret_cast<const float4 *>(be + j);
+      const float t[4] = {v.x, v.y, v.z, v.w}, gv[4] = {gg.x, gg.y, gg.z, gg.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+      float o[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) t[k] = gelu_erf((t[k] - mean) * rstd * gv[k] + bv[k]);
-      }
-      __nv_bfloat162 lo = __floats2bfloat162_rn(t[0], t[1]), hi = __floats2bfloat162_rn(t[2], t[3]);
+      for (int k = 0; k < 4; ++k) o[k] = gelu_erf((t[k] - mean) * rstd * gv[k] + bv[k]);
+      __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]), hi = __floats2bfloat162_rn(o[2], o[3]);
       uint2 pk;
       pk.x = *reinterpret_cast<uint32_t *>(&lo);
       pk.y = *reinterpret_cast<uint32_t *>(&hi);
@@ -565,6 +556,12 @@ __global__ void __launch_bounds__(s1::THREADS, 1)
 // fp32 boxes through shared memory and TMA bulk-tensor stores. Rows past M and columns past N
 // (and K past the end) are zero-filled by the loads and clipped by the stores, so any M, N and
 // K that are multiples of 8 work.
+// What the GEMM's epilogue writes: the fp32 product (kEpiF32); the fp32 product plus the bias and,
+// per row and column tile, the mean and sum of squared deviations of those values (kEpiStats: the
+// LayerNorm of the row kernel then reads each value once); bf16(product + bias) (kEpiBiasBf16:
+// the last stage, which has no LayerNorm).
+enum GemmEpi { kEpiF32 = 0, kEpiStats = 1, kEpiBiasBf16 = 2 };
+
 // Tile configuration for pair tiles of 256 x kBN (kBN = 192 or 256): as many K stages as fit
 // beside the output staging (one 4 KB box buffer per epilogue warp, two when that costs no stage).
 template <int kBN>
@@ -609,10 +606,11 @@ __device__ __forceinline__ bool g2_tile_at(int64_t i, int64_t n_tiles, int n_tn,
   return t < n_tiles;
 }
 
-template <int kBN>
+template <int kBN, int kEpi>
 __global__ void __launch_bounds__(G2<kBN>::THREADS, 1)
     hmlp_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-                     const __grid_constant__ CUtensorMap cmap, int64_t M, int N, int K, uint32_t *err) {
+                     const __grid_constant__ CUtensorMap cmap, int64_t M, int N, int K, const float *__restrict__ bias,
+                     float2 *__restrict__ stats, uint32_t *err) {
   using G = G2<kBN>;
   constexpr int BM = G::BM, BN = G::BN, BNH = G::BNH, BK = G::BK, STAGES = G::STAGES;
   constexpr int A_STAGE = G::A_STAGE, B_STAGE = G::B_STAGE, B_BOX = G::B_BOX, B_BOX_COLS = G::B_BOX_COLS;
@@ -745,6 +743,7 @@ __global__ void __launch_bounds__(G2<kBN>::THREADS, 1)
       const int64_t row0 = (2 * mp + rank) * BM + 32 * quad;
       const uint32_t tb = tmem_base + ((uint32_t)(32 * quad) << 16) + acc * ACC_STRIDE;
       if (ok && row0 < M) {
+        float n_run = 0.0f, mean_run = 0.0f, m2_run = 0.0f;  // kEpiStats: this row over the tile
 #pragma unroll 1
         for (int c = 0; c < BN / OUT_COLS; ++c) {
           const int col = nt * BN + OUT_COLS * c;
@@ -753,20 +752,64 @@ __global__ void __launch_bounds__(G2<kBN>::THREADS, 1)
           tmem_ld16(tb + OUT_COLS * c, v[0]);
           tmem_ld16(tb + OUT_COLS * c + 16, v[1]);
           tmem_wait_ld();
-          // row `lane` of the 32 x 32 box: 16-byte chunk j at j ^ (lane & 7) (128-byte swizzle);
+          if (kEpi != kEpiF32) {
+            // + bias (columns past N hold zeros from the zero-filled B and stay zero)
+#pragma unroll
+            for (int k = 0; k < OUT_COLS; ++k) {
+              const float b = col + k < N ? __ldg(bias + col + k) : 0.0f;
+              v[k >> 4][k & 15] = __float_as_uint(__uint_as_float(v[k >> 4][k & 15]) + b);
+            }
+          }
+          if (kEpi == kEpiStats) {
+            // this chunk's mean and sum of squared deviations over its valid columns, merged into
+            // the row's run (Chan et al.'s pairwise update)
+            const int nv = N - col < OUT_COLS ? N - col : OUT_COLS;
+            float sum = 0.0f;
+#pragma unroll
+            for (int k = 0; k < OUT_COLS; ++k) sum += k < nv ? __uint_as_float(v[k >> 4][k & 15]) : 0.0f;
+            const float mb = sum / (float)nv;
+            float q = 0.0f;
+#pragma unroll
+            for (int k = 0; k < OUT_COLS; ++k) {
+              const float dv = __uint_as_float(v[k >> 4][k & 15]) - mb;
+              q = k < nv ? fmaf(dv, dv, q) : q;
+            }
+            const float n_new = n_run + (float)nv, delta = mb - mean_run;
+            mean_run += delta * ((float)nv / n_new);
+            m2_run += q + delta * delta * (n_run * (float)nv / n_new);
+            n_run = n_new;
+          }
           // the buffer's previous box must have been read by its store first
           const uint32_t buf = obuf + (n_stored % OUT_BUFS) * OUT_BUF;
           if (lane == 0 && n_stored >= (uint32_t)OUT_BUFS) {
             if (OUT_BUFS == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
           }
           __syncwarp();
+          if (kEpi == kEpiBiasBf16) {
+            // row `lane` of a 32 x 32 bf16 box: 16-byte chunk j at j ^ ((lane >> 1) & 3) (64-byte swizzle)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t a = buf + lane * 128 + ((j ^ (lane & 7)) << 4);
-            const uint32_t *q = &v[j >> 2][4 * (j & 3)];
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(q[0]), "r"(q[1]), "r"(q[2]),
-                         "r"(q[3])
-                         : "memory");
+            for (int j = 0; j < 4; ++j) {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int k = 8 * j + 2 * h;
+                w[h] = pack_bf16(__uint_as_float(v[k >> 4][k & 15]), __uint_as_float(v[(k + 1) >> 4][(k + 1) & 15]));
+              }
+              const uint32_t a = buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                           "r"(w[3])
+                           : "memory");
+            }
+          } else {
+            // row `lane` of a 32 x 32 fp32 box: 16-byte chunk j at j ^ (lane & 7) (128-byte swizzle)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t a = buf + lane * 128 + ((j ^ (lane & 7)) << 4);
+              const uint32_t *q = &v[j >> 2][4 * (j & 3)];
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(q[0]), "r"(q[1]), "r"(q[2]),
+                           "r"(q[3])
+                           : "memory");
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -776,6 +819,8 @@ __global__ void __launch_bounds__(G2<kBN>::THREADS, 1)
           }
           ++n_stored;
         }
+        if (kEpi == kEpiStats && row0 + lane < M)
+          stats[(row0 + lane) * (int64_t)n_tn + nt] = make_float2(mean_run, m2_run);
       }
       tc_fence_before();
       __syncwarp();
@@ -808,9 +853,9 @@ cudaError_t make_map(CUtensorMap *map, EncodeTiledFn enc, const void *base, CUte
   return cudaSuccess;
 }
 
-template <int kBN>
-cudaError_t launch_gemm_bn(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, float *C,
-                           uint32_t *err, int64_t clusters, cudaStream_t stream) {
+template <int kBN, int kEpi>
+cudaError_t launch_gemm_bn(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, void *C,
+                           const float *bias, float2 *stats, uint32_t *err, int64_t clusters, cudaStream_t stream) {
   using G = G2<kBN>;
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -819,12 +864,17 @@ cudaError_t launch_gemm_bn(const __nv_bfloat16 *A, int64_t M, int K, int lda, co
   if ((e = make_map(&amap, enc, A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, lda, G::BK, G::BM,
                     CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
       (e = make_map(&bmap, enc, B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, N, N, G::B_BOX_COLS, G::BK,
-                    CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess ||
-      (e = make_map(&cmap, enc, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, N, G::OUT_COLS, 32,
-                    CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+                    CU_TENSOR_MAP_SWIZZLE_64B)) != cudaSuccess)
     return e;
+  if (kEpi == kEpiBiasBf16)
+    e = make_map(&cmap, enc, C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, N, G::OUT_COLS, 32,
+                 CU_TENSOR_MAP_SWIZZLE_64B);
+  else
+    e = make_map(&cmap, enc, C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, N, N, G::OUT_COLS, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
   static std::atomic<bool> attr[256];
-  if ((e = set_smem_attr_once(hmlp_gemm_kernel<kBN>, G::SMEM_BYTES, attr)) != cudaSuccess) return e;
+  if ((e = set_smem_attr_once(hmlp_gemm_kernel<kBN, kEpi>, G::SMEM_BYTES, attr)) != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * clusters));
   cfg.blockDim = dim3(G::THREADS);
@@ -837,35 +887,61 @@ cudaError_t launch_gemm_bn(const __nv_bfloat16 *A, int64_t M, int K, int lda, co
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, hmlp_gemm_kernel<kBN>, amap, bmap, cmap, M, N, K, err);
+  return cudaLaunchKernelEx(&cfg, hmlp_gemm_kernel<kBN, kEpi>, amap, bmap, cmap, M, N, K, bias, stats, err);
 }
 
-// Row-major C [M x N] fp32 = A [M x K] (row stride lda) * B [K x N], bf16 inputs, fp32 sums, on
-// hmlp_gemm_kernel (persistent CTA pairs, one per two SMs at most). The tile is 256 x 192 or
-// 256 x 256, whichever finishes its rounds of tiles over the clusters sooner: a 256-column pair
-// MMA takes about 16/15 the time of a 192-column one (measured), so the wider tile wins unless
-// it leaves a nearly empty last round.
-cudaError_t launch_gemm(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, float *C,
-                        uint32_t *err, int num_sms, cudaStream_t stream) {
-  if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
-  if (M > (int64_t)INT32_MAX) return cudaErrorNotSupported;  // TMA row coordinates are 32-bit
+template <int kEpi>
+cudaError_t launch_gemm_epi(int bn, const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N,
+                            void *C, const float *bias, float2 *stats, uint32_t *err, int64_t clusters,
+                            cudaStream_t stream) {
+  return bn == 256 ? launch_gemm_bn<256, kEpi>(A, M, K, lda, B, N, C, bias, stats, err, clusters, stream)
+                   : launch_gemm_bn<192, kEpi>(A, M, K, lda, B, N, C, bias, stats, err, clusters, stream);
+}
+
+// The tile width launch_gemm takes for an M x N product: 192 or 256 columns, whichever finishes
+// its rounds of tiles over the clusters sooner; a 256-column pair MMA takes about 16/15 the time
+// of a 192-column one (measured), so the wider tile wins unless it leaves a nearly empty last
+// round. Also the number of CTA pairs to launch.
+int gemm_tile_width(int64_t M, int N, int num_sms, int64_t *clusters) {
   const int64_t max_clusters = num_sms / 2 > 0 ? num_sms / 2 : 1;
   const int64_t m_pairs = (M + 255) / 256;
-  auto rounds = [&](int bn, int64_t &clusters) {
+  auto rounds = [&](int bn, int64_t &cl) {
     const int64_t tiles = m_pairs * ((N + bn - 1) / bn);
-    clusters = tiles < max_clusters ? tiles : max_clusters;
-    return (tiles + clusters - 1) / clusters;
+    cl = tiles < max_clusters ? tiles : max_clusters;
+    return (tiles + cl - 1) / cl;
   };
   int64_t c192, c256;
   const int64_t r192 = rounds(192, c192), r256 = rounds(256, c256);
-  if (16 * r256 < 15 * r192) return launch_gemm_bn<256>(A, M, K, lda, B, N, C, err, c256, stream);
-  return launch_gemm_bn<192>(A, M, K, lda, B, N, C, err, c192, stream);
+  if (16 * r256 < 15 * r192) {
+    *clusters = c256;
+    return 256;
+  }
+  *clusters = c192;
+  return 192;
+}
+
+// Row-major C [M x N] = A [M x K] (row stride lda) * B [K x N], bf16 inputs, fp32 sums, on
+// hmlp_gemm_kernel (persistent CTA pairs, one per two SMs at most); the epilogue as `epi` says
+// (C fp32 for kEpiF32 and kEpiStats, bf16 for kEpiBiasBf16; stats [M x ceil(N / bn)] for
+// kEpiStats, bn the tile width, returned in *bn_out when given).
+cudaError_t launch_gemm(const __nv_bfloat16 *A, int64_t M, int K, int lda, const __nv_bfloat16 *B, int N, void *C,
+                        int epi, const float *bias, float2 *stats, int *bn_out, uint32_t *err, int num_sms,
+                        cudaStream_t stream) {
+  if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  if (M > (int64_t)INT32_MAX) return cudaErrorNotSupported;  // TMA row coordinates are 32-bit
+  int64_t clusters = 1;
+  const int bn = gemm_tile_width(M, N, num_sms, &clusters);
+  if (bn_out) *bn_out = bn;
+  if (epi == kEpiStats) return launch_gemm_epi<kEpiStats>(bn, A, M, K, lda, B, N, C, bias, stats, err, clusters, stream);
+  if (epi == kEpiBiasBf16)
+    return launch_gemm_epi<kEpiBiasBf16>(bn, A, M, K, lda, B, N, C, bias, stats, err, clusters, stream);
+  return launch_gemm_epi<kEpiF32>(bn, A, M, K, lda, B, N, C, bias, stats, err, clusters, stream);
 }
 
 size_t r256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct HmlpLayout {
-  size_t a1, h13, h2, f32, w1p, total;
+  size_t a1, h13, h2, f32, stats, w1p, total;
 };
 
 // Stage 1 runs fused (hmlp_stage1_kernel) when d1 is a whole number of 256-column chunks, at
@@ -886,10 +962,15 @@ HmlpLayout hmlp_layout(int64_t P, const dmel_hmlp_weights &w) {
   size_t f = fused ? 0 : rows1 * (size_t)w.d1;
   if (rows2 * (size_t)w.d2 > f) f = rows2 * (size_t)w.d2;
   if (rows3 * (size_t)w.d3 > f) f = rows3 * (size_t)w.d3;
-  if ((size_t)P * (size_t)w.dim > f) f = (size_t)P * (size_t)w.dim;
   L.f32 = r256(f * 4);
+  // per row and column tile (192 columns at the narrowest) of the stages with LayerNorm
+  auto tiles = [](int d) { return (size_t)((d + 191) / 192); };
+  size_t st = fused ? 0 : rows1 * tiles(w.d1);
+  if (rows2 * tiles(w.d2) > st) st = rows2 * tiles(w.d2);
+  if (rows3 * tiles(w.d3) > st) st = rows3 * tiles(w.d3);
+  L.stats = r256(st * sizeof(float2));
   L.w1p = r256((size_t)kK1Pad * (size_t)w.d1 * 2);
-  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.w1p;
+  L.total = L.a1 + L.h13 + L.h2 + L.f32 + L.stats + L.w1p;
   return L;
 }
 
@@ -898,13 +979,12 @@ cudaError_t stage1_smem_attr() {
   return set_smem_attr_once(hmlp_stage1_kernel, s1::SMEM_BYTES, done);
 }
 
-template <bool kNorm>
-cudaError_t launch_rows(const float *in, int64_t rows, int d, const float *b, const float *g, const float *be,
-                        __nv_bfloat16 *out, int num_sms, cudaStream_t stream) {
+cudaError_t launch_rows(const float *in, const float2 *stats, int bn, int64_t rows, int d, const float *g,
+                        const float *be, __nv_bfloat16 *out, int num_sms, cudaStream_t stream) {
   const int64_t blocks = (rows + 7) / 8;
   const int64_t cap = (int64_t)num_sms * 16;
   const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
-  hmlp_row_kernel<kNorm><<<grid, 256, 0, stream>>>(in, rows, d, b, g, be, out);
+  hmlp_row_kernel<<<grid, 256, 0, stream>>>(in, stats, (d + bn - 1) / bn, bn, rows, d, g, be, out);
   return cudaGetLastError();
 }
 
@@ -919,7 +999,7 @@ cudaError_t launch_gelu_debug(const float *x, float *y, int64_t n, int num_sms, 
 cudaError_t launch_gemm_debug(const void *a, int64_t m, int k, int lda, const void *b, int n, float *c, uint32_t *err,
                               int num_sms, cudaStream_t stream) {
   return launch_gemm(static_cast<const __nv_bfloat16 *>(a), m, k, lda, static_cast<const __nv_bfloat16 *>(b), n, c,
-                     err, num_sms, stream);
+                     kEpiF32, nullptr, nullptr, nullptr, err, num_sms, stream);
 }
 
 size_t hmlp_workspace_bytes(int64_t n_patches, const dmel_hmlp_weights &w) {
@@ -937,8 +1017,9 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
   auto *H13 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1);
   auto *H2 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13);
   auto *F = reinterpret_cast<float *>(base + L.a1 + L.h13 + L.h2);
+  auto *S = reinterpret_cast<float2 *>(base + L.a1 + L.h13 + L.h2 + L.f32);
   // W1 padded to 80 rows (5 zero rows) so the stage-1 product has a 16-byte aligned K
-  auto *W1 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13 + L.h2 + L.f32);
+  auto *W1 = reinterpret_cast<__nv_bfloat16 *>(base + L.a1 + L.h13 + L.h2 + L.f32 + L.stats);
   if ((e = cudaMemcpyAsync(W1, w.w1, (size_t)kK1 * w.d1 * 2, cudaMemcpyDeviceToDevice, stream)) != cudaSuccess)
     return e;
   if ((e = cudaMemsetAsync(W1 + (size_t)kK1 * w.d1, 0, (size_t)(kK1Pad - kK1) * w.d1 * 2, stream)) != cudaSuccess)
@@ -981,19 +1062,27 @@ cudaError_t launch_hmlp(const void *images, int n, int H, int W, const dmel_hmlp
     hmlp_gather_kernel<<<(unsigned)(blocks < cap ? blocks : cap), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(images), n, H, W, A1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_gemm(A1, rows1, kK1Pad, kK1Pad, W1, w.d1, F, err, num_sms, stream)) != cudaSuccess) return e;
-    if ((e = launch_rows<true>(F, rows1, w.d1, w.b1, w.g1, w.be1, H13, num_sms, stream)) != cudaSuccess) return e;
+    int bn = 0;
+    if ((e = launch_gemm(A1, rows1, kK1Pad, kK1Pad, W1, w.d1, F, kEpiStats, w.b1, S, &bn, err, num_sms, stream)) !=
+        cudaSuccess)
+      return e;
+    if ((e = launch_rows(F, S, bn, rows1, w.d1, w.g1, w.be1, H13, num_sms, stream)) != cudaSuccess) return e;
     *launches += 3;
   }
-  if ((e = launch_gemm(H13, rows2, 4 * w.d1, 4 * w.d1, W2, w.d2, F, err, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = launch_rows<true>(F, rows2, w.d2, w.b2, w.g2, w.be2, H2, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = launch_gemm(H2, rows3, 4 * w.d2, 4 * w.d2, W3, w.d3, F, err, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = launch_rows<true>(F, rows3, w.d3, w.b3, w.g3, w.be3, H13, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = launch_gemm(H13, P, 4 * w.d3, 4 * w.d3, W4, w.dim, F, err, num_sms, stream)) != cudaSuccess) return e;
-  if ((e = launch_rows<false>(F, P, w.dim, w.b4, nullptr, nullptr, static_cast<__nv_bfloat16 *>(out), num_sms,
-                              stream)) != cudaSuccess)
+  int bn = 0;
+  if ((e = launch_gemm(H13, rows2, 4 * w.d1, 4 * w.d1, W2, w.d2, F, kEpiStats, w.b2, S, &bn, err, num_sms, stream)) !=
+      cudaSuccess)
     return e;
-  *launches += 6;  // stages 2-4: a GEMM and a row kernel each
+  if ((e = launch_rows(F, S, bn, rows2, w.d2, w.g2, w.be2, H2, num_sms, stream)) != cudaSuccess) return e;
+  if ((e = launch_gemm(H2, rows3, 4 * w.d2, 4 * w.d2, W3, w.d3, F, kEpiStats, w.b3, S, &bn, err, num_sms, stream)) !=
+      cudaSuccess)
+    return e;
+  if ((e = launch_rows(F, S, bn, rows3, w.d3, w.g3, w.be3, H13, num_sms, stream)) != cudaSuccess) return e;
+  // the last stage has no LayerNorm: bias and rounding in the GEMM's epilogue, straight into out
+  if ((e = launch_gemm(H13, P, 4 * w.d3, 4 * w.d3, W4, w.dim, out, kEpiBiasBf16, w.b4, nullptr, nullptr, err,
+                       num_sms, stream)) != cudaSuccess)
+    return e;
+  *launches += 5;  // stages 2-3: a GEMM and a row kernel each; stage 4: a GEMM
   return cudaSuccess;
 }
 
