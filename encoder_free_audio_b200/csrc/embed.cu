@@ -916,7 +916,10 @@ constexpr int EPI_CHUNK = 32;           // columns staged at a time
 constexpr int OFF_G = OFF_BAR + 256;    // RMSNorm weights of the cluster's column slice
 constexpr int OFF_EPI = OFF_G + BN_EPI * 4;  // row sums [2][128] and scales [128]
 constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;  // staging: 8 warps x 32 rows x up to 128 bytes
-constexpr int SMEM_USED = OFF_STG + EPI_WARPS * 32 * 128;
+constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: tile indices [16], count published
+constexpr int RING = 16;
+constexpr int LOOKAHEAD = 3;  // tiles published ahead of the one the TMA warp starts
+constexpr int SMEM_USED = OFF_RING + (RING + 4) * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int WAITER_WARP = 6 + EPI_WARPS;  // warps: 0 TMA, 1 MMA, 2..5 A, 6..13 epilogue, 14 waits
 constexpr int THREADS = 32 * (WAITER_WARP + 1);
@@ -973,6 +976,25 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const float *p) {
 
 // Number of column tiles of the sparse kernel (the last one may be partial).
 __host__ __device__ constexpr int sp_col_tiles(int D) { return (D + sp::BN - 1) / sp::BN; }
+
+// Shared-memory words of either CTA of the cluster (addresses from mapa_shared), for the tile
+// index ring of the dynamic schedule.
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_release_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cluster_u32(uint32_t local_addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_volatile_shared_u32(uint32_t local_addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local_addr) : "memory");
+  return v;
+}
 
 // Tile i of this cluster: pair frame tile mp, column tile nt. Without RMSNorm the clusters walk
 // one global order (frame tile major); with it, groups of P clusters own fixed column slices
@@ -1041,6 +1063,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       mbar_init(tempty(a), 2 * EPI_WARPS);  // epilogue warps of both CTAs (used in the even CTA)
     }
     mbar_init(done_bar, 1);
+    reinterpret_cast<uint32_t *>(smem + OFF_RING)[RING] = 0u;  // dynamic schedule: nothing published
     mbar_fence_init();
   }
   if (kMode == kFused && threadIdx.x < BN_EPI) {
@@ -1057,6 +1080,31 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
+  // Dynamic schedule (kScaled with a tile counter): the clusters take tiles from one global
+  // counter, so clusters on faster SMs take more; the even CTA's TMA thread fetches the indices
+  // and writes them, in order, into a ring in both CTAs' shared memory, and every role of both
+  // CTAs reads tile i of the cluster from its own copy. The publisher runs at most LOOKAHEAD tiles
+  // ahead of the TMA warp, which the stage barriers keep within a few tiles of the slowest role,
+  // far inside the ring.
+  const bool dyn = kMode == kScaled && counters != nullptr;
+  const int64_t n_tiles_all = n_pm * (int64_t)P;
+  const uint32_t ring_addr = smem_addr(smem + OFF_RING), pub_addr = ring_addr + 4u * RING;
+  auto tile = [&](int64_t i, int64_t &mp_, int &nt_) -> bool {
+    if (!dyn) return sp_tile_at<kMode>(i, n_pm, P, mp_, nt_);
+    uint32_t polls = 0;
+    while ((int64_t)ld_acquire_cluster_u32(pub_addr) <= i) {
+      if (++polls > kMaxPolls) {
+        record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+    const int t = (int)ld_volatile_shared_u32(ring_addr + 4u * (uint32_t)(i & (RING - 1)));
+    if (t < 0 || (int64_t)t >= n_tiles_all) return false;
+    mp_ = t / P;
+    nt_ = t % P;
+    return true;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------ TMA producer: this CTA's half of the table block
     if (lane == 0) {
@@ -1067,7 +1115,23 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       bool ok = true;
       int64_t mp;
       int nt;
-      for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      int64_t n_pub = 0;      // ring entries published (even CTA)
+      bool pub_end = false;   // the entry past the last tile has been published
+      auto publish_upto = [&](int64_t k) {
+        while (dyn && leader && !pub_end && n_pub < k) {
+          const int t = atomicAdd(counters, 1);
+          const uint32_t off = 4u * (uint32_t)(n_pub & (RING - 1));
+          st_cluster_u32(mapa_shared(ring_addr + off, 0), (uint32_t)t);
+          st_cluster_u32(mapa_shared(ring_addr + off, 1), (uint32_t)t);
+          ++n_pub;
+          st_release_cluster_u32(mapa_shared(pub_addr, 0), (uint32_t)n_pub);
+          st_release_cluster_u32(mapa_shared(pub_addr, 1), (uint32_t)n_pub);
+          pub_end = (int64_t)t >= n_tiles_all;
+        }
+      };
+      publish_upto(1 + LOOKAHEAD);
+      for (int64_t i = 0; ok && tile(i, mp, nt); ++i) {
+        publish_upto(i + 1 + LOOKAHEAD);
         const int n0 = nt * BN + (int)rank * BNH;
         for (int kb = 0; kb < KBLOCKS; ++kb) {
           if (!mbar_wait(empty_b(stage), phase ^ 1u, err)) { ok = false; break; }
@@ -1095,7 +1159,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       int sa = 0, sb = 0;
       int64_t mp;
       int nt;
-      for (int64_t i = 0; sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      for (int64_t i = 0; tile(i, mp, nt); ++i) {
         const uint32_t acc = i & 1;
         const uint32_t d_tmem = tmem_base + acc * ACC_STRIDE;
         for (int kb = 0; kb < KBLOCKS; ++kb) {
@@ -1137,7 +1201,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       int64_t n = 0;   // stages announced
       int64_t mp;
       int nt;
-      for (int64_t i = 0; sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+      for (int64_t i = 0; tile(i, mp, nt); ++i) {
         const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
         for (int kb = 0; kb < KBLOCKS; ++kb, ++n) {
           if (n >= STAGES_A) sp_issued_sync(sa);  // stage n - 3 (same slot) was issued
@@ -1188,8 +1252,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       }
     };
     uint4 next[5];
-    if (sp_tile_at<kMode>(0, n_pm, P, mp, nt)) load_codes(mp, next);
-    for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+    if (tile(0, mp, nt)) load_codes(mp, next);
+    for (int64_t i = 0; ok && tile(i, mp, nt); ++i) {
       const int64_t f = (2 * mp + rank) * BM + r;
       const bool valid = f < F;
       uint32_t cw[20];
@@ -1200,7 +1264,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       {
         int64_t mp2;
         int nt2;
-        if (sp_tile_at<kMode>(i + 1, n_pm, P, mp2, nt2)) load_codes(mp2, next);
+        if (tile(i + 1, mp2, nt2)) load_codes(mp2, next);
       }
       if (valid) {
         uint32_t bad = 0;
@@ -1262,7 +1326,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
     bool ok = true;
     int64_t mp;
     int nt;
-    for (int64_t i = 0; ok && sp_tile_at<kMode>(i, n_pm, P, mp, nt); ++i) {
+    for (int64_t i = 0; ok && tile(i, mp, nt); ++i) {
       const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
       if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
       tc_fence_after();
@@ -2012,6 +2076,9 @@ cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
   } else if (resident < 1) {
     return cudaErrorNotSupported;
   }
+  if (kMode == kScaled && sc.counters) {  // the dynamic schedule's tile counter starts at 0
+    if ((e = cudaMemsetAsync(sc.counters, 0, sizeof(int), stream)) != cudaSuccess) return e;
+  }
   return cudaLaunchKernelEx(&cfg, embed_sp_kernel<OT, kMode>, tmap, codes, F, D, out, om, sc.partials, sc.counters, g, eps,
                             err);
 }
@@ -2172,7 +2239,8 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
     if (e == cudaSuccess) {
       const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
       const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
-      e = launch_sp<OT, kScaled>(codes, F, T, D, out, om, TcScratch{scale, nullptr}, g, eps, err, sp_clusters, stream);
+      int *ctr = reinterpret_cast<int *>(ws + gram_bytes() + norm_scale_bytes(F));  // dynamic tile counter
+      e = launch_sp<OT, kScaled>(codes, F, T, D, out, om, TcScratch{scale, ctr}, g, eps, err, sp_clusters, stream);
       if (e == cudaSuccess) {
         *launches += l + 1;
         return e;
@@ -2306,8 +2374,8 @@ size_t embed_exchange_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtyp
 size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_dtype, int with_rmsnorm) {
   const size_t ex = embed_exchange_workspace_bytes(n_frames, embed_dim, table_dtype, with_rmsnorm);
   if (ex == 0) return 0;
-  // or G, the per-frame partial sums of squares and the scales of the G path
-  const size_t gp = gram_bytes() + norm_scale_bytes(n_frames);
+  // or G, the per-frame partial sums of squares and the scales of the G path, and its tile counter
+  const size_t gp = gram_bytes() + norm_scale_bytes(n_frames) + 256;
   return ex > gp ? ex : gp;
 }
 

@@ -54,10 +54,11 @@ def test_workspace_size(lib):
     with_codes = dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True)
     r256 = lambda x: (x + 255) // 256 * 256
     # the larger of: G [1280 x 1280] fp32 and its second partial product + 55 partial sums of
-    # squares per frame + one scale per frame (RMSNorm from the Gram matrix); row sums of squares
+    # squares per frame + one scale per frame + the sparse product's tile counter (RMSNorm from
+    # the Gram matrix, dynamic tile schedule); row sums of squares
     # [frame tiles of 128][column tiles of 192][128] fp32 + one counter per frame tile (the
     # exchange between a row's CTAs)
-    gram = 2 * r256(1280 * 1280 * 4) + r256(55 * F * 4) + r256(F * 4)
+    gram = 2 * r256(1280 * 1280 * 4) + r256(55 * F * 4) + r256(F * 4) + 256
     tiles = (F + 127) // 128
     exchange = r256(tiles * 32 * 128 * 4) + r256(tiles * 4)
     assert with_codes == max(gram, exchange)
