@@ -155,10 +155,20 @@ dmel_status dmel_codes(const float *wav, const int64_t *sample_offsets, const in
   return dmel_codes_q(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, codes, nullptr, stream);
 }
 
-dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
-                            int embed_dim, const void *rms_weight, float eps, void *out, const int64_t *out_rows,
-                            int64_t out_n_rows, dmel_dtype out_dtype, void *workspace, size_t workspace_bytes,
-                            dmel_stream_t stream) {
+namespace {
+// The table's G from dmel_table_prepare, when it applies to this call (RMSNorm on a bf16 table the
+// tensor-core path takes); NULL otherwise. A misaligned pointer is an argument error (*bad).
+const float *prepared_gram(const void *prepared, dmel_dtype table_dtype, int embed_dim, const void *rms_weight,
+                           bool *bad) {
+  *bad = prepared && !aligned(prepared, 256);
+  if (!prepared || *bad || !rms_weight || dmel_table_prepare_size(embed_dim, table_dtype) == 0) return nullptr;
+  return static_cast<const float *>(prepared);
+}
+
+dmel_status embed_rows_impl(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                            int embed_dim, const void *rms_weight, float eps, const void *prepared, void *out,
+                            const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, void *workspace,
+                            size_t workspace_bytes, dmel_stream_t stream) {
   t_last_launches = 0;
   dmel_status st =
       check_embed_args(codes, true, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype);
@@ -167,15 +177,34 @@ dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *
   if (n_frames == 0) return DMEL_OK;
   const size_t need = embed_workspace_bytes(n_frames, embed_dim, table_dtype, rms_weight != nullptr);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DMEL_ERR_INVALID_ARG;
+  bool bad = false;
+  const float *G = prepared_gram(prepared, table_dtype, embed_dim, rms_weight, &bad);
+  if (bad) return DMEL_ERR_INVALID_ARG;
   DeviceInfo d;
   if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
   if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
   int launches = 0;
   cudaError_t e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype,
                                workspace, d.err, d.sms, reinterpret_cast<cudaStream_t>(stream), &launches, out_rows,
-                               out_n_rows);
+                               out_n_rows, true, G);
   t_last_launches = launches;
   return from_cuda(e);
+}
+}  // namespace
+
+dmel_status dmel_embed_rows(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                            int embed_dim, const void *rms_weight, float eps, void *out, const int64_t *out_rows,
+                            int64_t out_n_rows, dmel_dtype out_dtype, void *workspace, size_t workspace_bytes,
+                            dmel_stream_t stream) {
+  return embed_rows_impl(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, nullptr, out, out_rows,
+                         out_n_rows, out_dtype, workspace, workspace_bytes, stream);
+}
+
+dmel_status dmel_embed_prepared(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                                int embed_dim, const void *rms_weight, float eps, const void *prepared, void *out,
+                                dmel_dtype out_dtype, void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
+  return embed_rows_impl(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, prepared, out, nullptr, 0,
+                         out_dtype, workspace, workspace_bytes, stream);
 }
 
 dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype, int embed_dim,
@@ -185,11 +214,13 @@ dmel_status dmel_embed(const uint8_t *codes, int64_t n_frames, const void *table
                          workspace, workspace_bytes, stream);
 }
 
-dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+namespace {
+dmel_status forward_rows_impl(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
                               int n_clips, int64_t n_frames, const float *tails, float *tails_out, const void *table,
-                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
-                              const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, uint8_t *codes_out,
-                              void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps,
+                              const void *prepared, void *out, const int64_t *out_rows, int64_t out_n_rows,
+                              dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
+                              dmel_stream_t stream) {
   t_last_launches = 0;
   if (n_clips < 0 || n_frames < 0 || (n_clips == 0 && n_frames > 0)) return DMEL_ERR_INVALID_ARG;
   if (out_rows && (out_n_rows <= 0 || !aligned(out_rows, 8))) return DMEL_ERR_INVALID_ARG;
@@ -202,6 +233,9 @@ dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, c
   if (n_clips == 0) return DMEL_OK;
   const size_t need = dmel_workspace_size(n_frames, embed_dim, table_dtype, rms_weight != nullptr, codes_out != nullptr);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DMEL_ERR_INVALID_ARG;
+  bool bad = false;
+  const float *G = prepared_gram(prepared, table_dtype, embed_dim, rms_weight, &bad);
+  if (bad) return DMEL_ERR_INVALID_ARG;
   DeviceInfo d;
   if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
   if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
@@ -217,7 +251,51 @@ dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, c
                                d.sms, s, &launches);
   if (e == cudaSuccess)
     e = launch_embed(codes, n_frames, table, table_dtype, embed_dim, rms_weight, eps, out, out_dtype, ws, d.err, d.sms,
-                     s, &launches, out_rows, out_n_rows);
+                     s, &launches, out_rows, out_n_rows, true, G);
+  t_last_launches = launches;
+  return from_cuda(e);
+}
+}  // namespace
+
+dmel_status dmel_forward_rows(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                              int n_clips, int64_t n_frames, const float *tails, float *tails_out, const void *table,
+                              dmel_dtype table_dtype, int embed_dim, const void *rms_weight, float eps, void *out,
+                              const int64_t *out_rows, int64_t out_n_rows, dmel_dtype out_dtype, uint8_t *codes_out,
+                              void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
+  return forward_rows_impl(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, table, table_dtype,
+                           embed_dim, rms_weight, eps, nullptr, out, out_rows, out_n_rows, out_dtype, codes_out,
+                           workspace, workspace_bytes, stream);
+}
+
+dmel_status dmel_forward_prepared(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                                  int n_clips, int64_t n_frames, const float *tails, float *tails_out,
+                                  const void *table, dmel_dtype table_dtype, int embed_dim, const void *rms_weight,
+                                  float eps, const void *prepared, void *out, dmel_dtype out_dtype,
+                                  uint8_t *codes_out, void *workspace, size_t workspace_bytes, dmel_stream_t stream) {
+  return forward_rows_impl(wav, sample_offsets, frame_offsets, n_clips, n_frames, tails, tails_out, table, table_dtype,
+                           embed_dim, rms_weight, eps, prepared, out, nullptr, 0, out_dtype, codes_out, workspace,
+                           workspace_bytes, stream);
+}
+
+size_t dmel_table_prepare_size(int embed_dim, dmel_dtype table_dtype) {
+  // G exists for the tensor-core path's bf16 tables whose width the Gram kernel tiles (128)
+  if (table_dtype != DMEL_BF16 || embed_dim <= 0 || embed_dim % 128 != 0) return 0;
+  if (!embed_uses_tensor_cores(table_dtype, embed_dim)) return 0;
+  return gram_bytes();
+}
+
+dmel_status dmel_table_prepare(const void *table, int embed_dim, dmel_dtype table_dtype, void *prepared,
+                               size_t prepared_bytes, dmel_stream_t stream) {
+  t_last_launches = 0;
+  const size_t need = dmel_table_prepare_size(embed_dim, table_dtype);
+  if (need == 0 || !table || !aligned(table, 16) || !prepared || !aligned(prepared, 256) || prepared_bytes < need)
+    return DMEL_ERR_INVALID_ARG;
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) return DMEL_ERR_CUDA;
+  if (d.major != 10) return DMEL_ERR_UNSUPPORTED;
+  int launches = 0;
+  const cudaError_t e =
+      launch_gram(table, embed_dim, static_cast<float *>(prepared), d.err, reinterpret_cast<cudaStream_t>(stream), &launches);
   t_last_launches = launches;
   return from_cuda(e);
 }

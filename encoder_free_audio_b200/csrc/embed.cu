@@ -913,8 +913,8 @@ constexpr int BN_EPI = BN;              // columns the epilogue walks
 constexpr int EPI_WARPS = 8;            // two per TMEM lane quarter
 constexpr int EPI_COLS = BN / 2;        // columns per epilogue warp
 constexpr int EPI_CHUNK = 32;           // columns staged at a time
-constexpr int OFF_G = OFF_BAR + 256;    // RMSNorm weights of the cluster's column slice
-constexpr int OFF_EPI = OFF_G + BN_EPI * 4;  // row sums [2][128] and scales [128]
+constexpr int OFF_G = OFF_BAR + 256;    // RMSNorm weights of the column tile (kScaled: [2], by accumulator)
+constexpr int OFF_EPI = OFF_G + 2 * BN_EPI * 4;  // row sums [2][128] and scales [128]
 constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;  // staging: 8 warps x 32 rows x up to 128 bytes
 constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: tile indices [16], count published
 constexpr int RING = 16;
@@ -1328,22 +1328,26 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
     int nt;
     for (int64_t i = 0; ok && tile(i, mp, nt); ++i) {
       const uint32_t acc = i & 1, acc_phase = (i >> 1) & 1;
-      if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
-      tc_fence_after();
       const int64_t m = 2 * mp + rank;
       const bool live = m < n_m_tiles;  // uniform over the CTA: the pair's second half may hold no frame
       const int n0 = nt * BN;
       const int ncols = D - n0 < BN ? D - n0 : BN;
-      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + cb;
       float scale = 1.0f;
+      const float *gt = gsm;
       if (kMode == kScaled) {
-        // the column tile changes from tile to tile: its RMSNorm weights, and this row's scale
+        // while the accumulator fills: the column tile's RMSNorm weights, into the buffer of tile
+        // i - 2 (which every epilogue warp finished before the barrier of tile i - 1 let this
+        // warp through), and this row's scale; the barrier below publishes the weights
+        float *gb = gsm + acc * BN_EPI;
         const int t = (warp - 6) * 32 + lane;
-        if (t < BN_EPI) gsm[t] = t < ncols ? __bfloat162float(gw[n0 + t]) : 0.0f;
-        const int64_t f = (2 * mp + rank) * BM + r;
+        if (t < BN_EPI) gb[t] = t < ncols ? __bfloat162float(gw[n0 + t]) : 0.0f;
+        const int64_t f = m * BM + r;
         scale = live && f < F ? __ldg(partials + f) : 0.0f;
-        sp_epi_barrier();
+        gt = gb;
       }
+      if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + cb;
       if (kMode == kFused && live) {
         float ss = 0.0f;
 #pragma unroll
@@ -1413,7 +1417,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
             for (int e = 0; e < E; ++e) {
               const int cc = h * E + e;
               x[e] = __uint_as_float(v[cc >> 4][cc & 15]);
-              if (kMode == kFused || kMode == kScaled) x[e] = gsm[c0 + cc] * (x[e] * scale);
+              if (kMode == kFused || kMode == kScaled) x[e] = gt[c0 + cc] * (x[e] * scale);
             }
             *reinterpret_cast<uint4 *>(slab + lane * RB + (piece(lane, h) << 4)) = pack16<OT>(x);
           }
@@ -2076,9 +2080,7 @@ cudaError_t launch_sp(const uint8_t *codes, int64_t F, const __nv_bfloat16 *tabl
   } else if (resident < 1) {
     return cudaErrorNotSupported;
   }
-  if (kMode == kScaled && sc.counters) {  // the dynamic schedule's tile counter starts at 0
-    if ((e = cudaMemsetAsync(sc.counters, 0, sizeof(int), stream)) != cudaSuccess) return e;
-  }
+  // kScaled: the dynamic schedule's tile counter was set to 0 by the scale kernels before it
   return cudaLaunchKernelEx(&cfg, embed_sp_kernel<OT, kMode>, tmap, codes, F, D, out, om, sc.partials, sc.counters, g, eps,
                             err);
 }
@@ -2186,8 +2188,12 @@ bool stationary_enabled() {
 // RMSNorm scales from G = T T^T for calls of at least kGramMinFrames frames (below that, the
 // fixed cost of G, ~30 us, outweighs what the exchange of row sums costs the embedding kernel),
 // unless the environment sets DMEL_EMBED_NORM=exchange; DMEL_EMBED_NORM=gram takes the G path at
-// every size (read once per process; for comparisons and tests).
+// every size (read once per process; for comparisons and tests). With G prepared for the table
+// beforehand, the G path from kPreparedMinFrames frames: below that, the scale pre-pass and the
+// extra launches cost about what the exchange does (measured: even between 8,000 and 12,800
+// frames, depending on the GPU's MMA rate; 25-35 us gained from 16,384 frames).
 int64_t kGramMinFrames = 16384;
+int64_t kPreparedMinFrames = 12288;
 bool gram_enabled() {
   static const int mode = [] {
     const char *v = getenv("DMEL_EMBED_NORM");
@@ -2195,7 +2201,7 @@ bool gram_enabled() {
     if (v && strcmp(v, "gram") == 0) return 2;
     return 1;
   }();
-  if (mode == 2) kGramMinFrames = 1;
+  if (mode == 2) kGramMinFrames = kPreparedMinFrames = 1;
   return mode != 0;
 }
 
@@ -2205,7 +2211,7 @@ bool gram_enabled() {
 template <typename OT>
 cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int D, OT *out, OutMap om, const __nv_bfloat16 *g,
                    float eps, void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
-                   bool allow_gram) {
+                   bool allow_gram, const float *gram_pre) {
   const int P = D / tc::BN;
   const int64_t tiles = ((F + tc::BM - 1) / tc::BM) * P;
   const int plain_grid = (int)(tiles < num_sms ? tiles : num_sms);
@@ -2225,21 +2231,22 @@ cudaError_t run_tc(const uint8_t *codes, int64_t F, const __nv_bfloat16 *T, int 
     (void)cudaGetLastError();  // refused: the streamed-table kernels below
   }
   const int Psp = sp_col_tiles(D);
-  if (g && allow_gram && gram_enabled() && F >= kGramMinFrames && pairs_enabled() && sparse_enabled() &&
-      max_clusters >= 1) {
-    // RMSNorm scales from the codes and G = T T^T first, then the product on every cluster with
-    // no exchange of row sums
+  const bool use_g = g && gram_enabled() && (gram_pre ? F >= kPreparedMinFrames : allow_gram && F >= kGramMinFrames);
+  if (use_g && pairs_enabled() && sparse_enabled() && max_clusters >= 1) {
+    // RMSNorm scales from the codes and G = T T^T first (G computed here, or prepared for the table
+    // beforehand), then the product on every cluster with no exchange of row sums
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    float *G = reinterpret_cast<float *>(ws);
+    const float *G = gram_pre ? gram_pre : reinterpret_cast<const float *>(ws);
     void *parts = ws + gram_bytes();
     float *scale = reinterpret_cast<float *>(ws + gram_bytes() + norm_scale_bytes(F) - round256((size_t)F * 4));
+    int *ctr = reinterpret_cast<int *>(ws + gram_bytes() + norm_scale_bytes(F));  // dynamic tile counter
     int l = 0;
-    e = launch_gram(T, D, G, err, stream, &l);
-    if (e == cudaSuccess) e = launch_norm_scale(codes, F, D, G, eps, parts, scale, stream, &l);
+    e = gram_pre ? cudaSuccess : launch_gram(T, D, reinterpret_cast<float *>(ws), err, stream, &l);
+    // (the scale kernels zero the tile counter)
+    if (e == cudaSuccess) e = launch_norm_scale(codes, F, D, G, eps, parts, scale, ctr, num_sms, stream, &l);
     if (e == cudaSuccess) {
       const int64_t sp_tiles = ((F + 2 * sp::BM - 1) / (2 * sp::BM)) * Psp;
       const int sp_clusters = (int)(sp_tiles < max_clusters ? sp_tiles : max_clusters);
-      int *ctr = reinterpret_cast<int *>(ws + gram_bytes() + norm_scale_bytes(F));  // dynamic tile counter
       e = launch_sp<OT, kScaled>(codes, F, T, D, out, om, TcScratch{scale, ctr}, g, eps, err, sp_clusters, stream);
       if (e == cudaSuccess) {
         *launches += l + 1;
@@ -2382,7 +2389,7 @@ size_t embed_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtype table_d
 cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dmel_dtype table_dtype, int D,
                          const void *rms_weight, float eps, void *out, dmel_dtype out_dtype, void *workspace,
                          uint32_t *err, int num_sms, cudaStream_t stream, int *launches, const int64_t *out_rows,
-                         int64_t out_n_rows, bool allow_gram) {
+                         int64_t out_n_rows, bool allow_gram, const float *gram) {
   if (F <= 0) return cudaSuccess;
   const OutMap om{out_rows, out_n_rows};
   cudaError_t e;
@@ -2391,9 +2398,9 @@ cudaError_t launch_embed(const uint8_t *codes, int64_t F, const void *table, dme
     const auto *g = static_cast<const __nv_bfloat16 *>(rms_weight);
     if (out_dtype == DMEL_BF16)
       return run_tc(codes, F, T, D, static_cast<__nv_bfloat16 *>(out), om, g, eps, workspace, err, num_sms, stream,
-                    launches, allow_gram);
+                    launches, allow_gram, gram);
     return run_tc(codes, F, T, D, static_cast<float *>(out), om, g, eps, workspace, err, num_sms, stream, launches,
-                  allow_gram);
+                  allow_gram, gram);
   }
   if (table_dtype == DMEL_BF16) {
     const auto *T = static_cast<const __nv_bfloat16 *>(table);

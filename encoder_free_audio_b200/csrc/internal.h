@@ -37,22 +37,24 @@ size_t embed_exchange_workspace_bytes(int64_t n_frames, int embed_dim, dmel_dtyp
 // Embedding of n_frames codes; workspace holds embed_workspace_bytes(...) bytes (with allow_gram
 // false, embed_exchange_workspace_bytes(...)).
 // out_rows: NULL (frame f -> row f of out) or device int64 [n_frames], frame f -> row out_rows[f]
-// of an out with out_n_rows rows.
+// of an out with out_n_rows rows. gram: a table's G prepared beforehand (launch_gram), or NULL; with
+// RMSNorm on a bf16 table it is used at every call size instead of computing G.
 cudaError_t launch_embed(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
                          int embed_dim, const void *rms_weight, float eps, void *out, dmel_dtype out_dtype,
                          void *workspace, uint32_t *err, int num_sms, cudaStream_t stream, int *launches,
-                         const int64_t *out_rows = nullptr, int64_t out_n_rows = 0, bool allow_gram = true);
+                         const int64_t *out_rows = nullptr, int64_t out_n_rows = 0, bool allow_gram = true,
+                         const float *gram = nullptr);
 
 // G = T T^T (fp32 [1280 x 1280], the 55 blocks of 128 x 128 rows with row block <= column block
 // written; gram_bytes() holds it and a second partial product after it) of a bf16 table
 // T [1280 x D], D a multiple of 128; and the RMSNorm scale of each frame,
 // 1 / sqrt(sum_b sum_b' G[r_b, r_b'] / D + eps), from its codes (scratch: norm_scale_bytes(F)
-// minus the F scales at its end).
+// minus the F scales at its end); the scale kernels also set *zero_counter (when given) to 0.
 size_t gram_bytes();
 size_t norm_scale_bytes(int64_t n_frames);
 cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaStream_t stream, int *launches);
 cudaError_t launch_norm_scale(const uint8_t *codes, int64_t n_frames, int D, const float *G, float eps, void *scratch,
-                              float *scale, cudaStream_t stream, int *launches);
+                              float *scale, int *zero_counter, int num_sms, cudaStream_t stream, int *launches);
 double norm_sumsq_host(const uint8_t *codes80, const float *G);
 
 // dmel_forward_host: workspace bytes for this batch (0 when it has no frame) and the pipelined

@@ -18,9 +18,10 @@
 //                   over thousands of products drifts by ~1e-5 relative, and the diagonal carries
 //                   almost all of a frame's sum of squares (80 terms of ~D * var(T) each, against
 //                   off-diagonal terms of either sign ~sqrt(D) times smaller).
-//   norm_partials   per G block and chunk of 4096 frames: the block staged in shared memory once,
-//                   each frame's 64 (on the diagonal 36) terms looked up with eight independent
-//                   accumulators; one partial sum per frame and block.
+//   norm_partials   per G block and chunk of 256 E frames (E = 16, or 4, 2, 1 when that would
+//                   leave SMs idle): the block staged in shared memory once, each frame's 64 (on the
+//                   diagonal 36) terms looked up with eight independent accumulators; one partial
+//                   sum per frame and block.
 //   norm_finalize   scale_f = 1 / sqrt((sum of the 55 partials, in block order) / D + eps).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -211,12 +212,12 @@ __global__ void __launch_bounds__(256) gram_diag_kernel(const __nv_bfloat16 *__r
 // ---------------------------------------------------------------- per-frame sums of squares
 
 namespace nm {
-constexpr int FRAMES = 4096;            // frames per CTA
-constexpr int THREADS = 256;            // 16 frames per thread
+constexpr int THREADS = 256;            // frames per CTA: E of them per thread
+constexpr int CTAS_PER_SM = 3;
 constexpr int LD = gm::BT + 4;          // staged row stride (floats): 528 bytes, spreads the banks
 constexpr int BLK_FLOATS = gm::BT * LD;
 constexpr int SMEM_BYTES = BLK_FLOATS * 4;  // one G block: 67.6 KB, three CTAs per SM
-static_assert(SMEM_BYTES * 3 <= 227 * 1024, "three CTAs per SM");
+static_assert(SMEM_BYTES * CTAS_PER_SM <= 227 * 1024, "three CTAs per SM");
 }  // namespace nm
 
 // Sum of one frame's terms in G block (g, h) (bin groups g <= h, 8 bins each): ci / cj are the
@@ -250,10 +251,12 @@ __host__ __device__ inline float block_terms(const float *blk, const int (&ri)[8
   return s;
 }
 
-// One CTA per (G block q, chunk of 4096 frames): the block is staged once, then each thread
-// takes 16 frames, reads the 16 codes of the block's two bin groups straight from the codes
-// rows (two 8-byte loads) and writes the frame's partial sum for this block.
-__global__ void __launch_bounds__(nm::THREADS, 3)
+// One CTA per (G block q, chunk of THREADS * E frames): the block is staged once, then each
+// thread takes E frames THREADS apart, reads the 16 codes of the block's two bin groups straight
+// from the codes rows (two 8-byte loads) and writes the frame's partial sum for this block. E is
+// a compile-time count, so the loop unrolls and the codes loads run ahead of the lookups.
+template <int E>
+__global__ void __launch_bounds__(nm::THREADS, nm::CTAS_PER_SM)
     norm_partials_kernel(const uint8_t *__restrict__ codes, int64_t F, const float *__restrict__ G,
                          float *__restrict__ partials) {
   using namespace nm;
@@ -262,15 +265,25 @@ __global__ void __launch_bounds__(nm::THREADS, 3)
   int g, h;
   gram_block(q, g, h);
   const float *src = G + (size_t)(g * gm::BT) * kRows + h * gm::BT;
-  for (int i = threadIdx.x; i < gm::BT * (gm::BT / 4); i += THREADS) {
-    const int r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
-    *reinterpret_cast<float4 *>(blk + r * LD + 4 * c4) = __ldg(reinterpret_cast<const float4 *>(src + (size_t)r * kRows) + c4);
+  // the block's 16 float4 per thread, all loads in flight before the first store
+  constexpr int PER = gm::BT * (gm::BT / 4) / THREADS;
+  static_assert(PER * THREADS == gm::BT * (gm::BT / 4), "whole block");
+  float4 v[PER];
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * THREADS, r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
+    v[k] = __ldg(reinterpret_cast<const float4 *>(src + (size_t)r * kRows) + c4);
   }
-  const int64_t f0 = (int64_t)blockIdx.x * FRAMES + threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < PER; ++k) {
+    const int i = threadIdx.x + k * THREADS, r = i / (gm::BT / 4), c4 = i % (gm::BT / 4);
+    *reinterpret_cast<float4 *>(blk + r * LD + 4 * c4) = v[k];
+  }
+  const int64_t f0 = (int64_t)blockIdx.x * (THREADS * E) + threadIdx.x;
   // the codes of this thread's next frame are loaded while the current frame's terms are summed
   auto load = [&](int e, uint2 &ug, uint2 &uh) {
     const int64_t f = f0 + (int64_t)e * THREADS;
-    if (e < FRAMES / THREADS && f < F) {
+    if (e < E && f < F) {
       const uint8_t *row = codes + f * kMel;
       ug = __ldg(reinterpret_cast<const uint2 *>(row + 8 * g));
       uh = __ldg(reinterpret_cast<const uint2 *>(row + 8 * h));
@@ -279,7 +292,8 @@ __global__ void __launch_bounds__(nm::THREADS, 3)
   uint2 ug = make_uint2(0u, 0u), uh = make_uint2(0u, 0u);
   load(0, ug, uh);
   __syncthreads();
-  for (int e = 0; e < FRAMES / THREADS; ++e) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
     const int64_t f = f0 + (int64_t)e * THREADS;
     if (f >= F) break;
     int ri[8], cj[8];
@@ -295,13 +309,19 @@ __global__ void __launch_bounds__(nm::THREADS, 3)
   }
 }
 
-// scale_f = 1 / sqrt((sum over the 55 blocks, in block order) / D + eps)
+// scale_f = 1 / sqrt((sum over the 55 blocks, in block order) / D + eps); the 55 loads of a
+// frame are all issued before the first addition. Also sets *zero (when given) to 0: the tile
+// counter of the product kernel that follows on the stream.
 __global__ void __launch_bounds__(256) norm_finalize_kernel(const float *__restrict__ partials, int64_t F, int D,
-                                                            float eps, float *__restrict__ scale) {
+                                                            float eps, float *__restrict__ scale, int *zero) {
+  if (zero && blockIdx.x == 0 && threadIdx.x == 0) *zero = 0;
   for (int64_t f = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; f < F; f += (int64_t)gridDim.x * blockDim.x) {
+    float v[gm::BLOCKS];
+#pragma unroll
+    for (int q = 0; q < gm::BLOCKS; ++q) v[q] = __ldcs(partials + (size_t)q * F + f);
     float s = 0.0f;
-#pragma unroll 5
-    for (int q = 0; q < gm::BLOCKS; ++q) s += partials[(size_t)q * F + f];
+#pragma unroll
+    for (int q = 0; q < gm::BLOCKS; ++q) s += v[q];
     scale[f] = 1.0f / sqrtf(s / (float)D + eps);
   }
 }
@@ -344,19 +364,32 @@ cudaError_t launch_gram(const void *table, int D, float *G, uint32_t *err, cudaS
   return cudaSuccess;
 }
 
-cudaError_t launch_norm_scale(const uint8_t *codes, int64_t F, int D, const float *G, float eps, void *scratch,
-                              float *scale, cudaStream_t stream, int *launches) {
-  if (F <= 0) return cudaSuccess;
+template <int E>
+cudaError_t launch_partials(const uint8_t *codes, int64_t F, const float *G, float *partials, cudaStream_t stream) {
   static std::atomic<bool> attr[256];
-  cudaError_t e = set_smem_attr_once(norm_partials_kernel, nm::SMEM_BYTES, attr);
+  cudaError_t e = set_smem_attr_once(norm_partials_kernel<E>, nm::SMEM_BYTES, attr);
   if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((F + nm::THREADS * E - 1) / (nm::THREADS * E)), gm::BLOCKS);
+  norm_partials_kernel<E><<<grid, nm::THREADS, nm::SMEM_BYTES, stream>>>(codes, F, G, partials);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_scale(const uint8_t *codes, int64_t F, int D, const float *G, float eps, void *scratch,
+                              float *scale, int *zero, int num_sms, cudaStream_t stream, int *launches) {
+  if (F <= 0) return cudaSuccess;
   float *partials = static_cast<float *>(scratch);
-  const dim3 grid((unsigned)((F + nm::FRAMES - 1) / nm::FRAMES), gm::BLOCKS);
-  norm_partials_kernel<<<grid, nm::THREADS, nm::SMEM_BYTES, stream>>>(codes, F, G, partials);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 16 frames per thread, unless that leaves fewer CTAs than three per SM: then 4, 2 or 1
+  const int64_t slots = (int64_t)nm::CTAS_PER_SM * num_sms;
+  auto ctas = [&](int64_t e) { return (F + nm::THREADS * e - 1) / (nm::THREADS * e) * gm::BLOCKS; };
+  cudaError_t e = ctas(16) >= slots ? launch_partials<16>(codes, F, G, partials, stream)
+                  : ctas(4) >= slots ? launch_partials<4>(codes, F, G, partials, stream)
+                  : ctas(2) >= slots ? launch_partials<2>(codes, F, G, partials, stream)
+                                     : launch_partials<1>(codes, F, G, partials, stream);
+  if (e != cudaSuccess) return e;
   ++*launches;
   const int64_t blocks = (F + 255) / 256;
-  norm_finalize_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(partials, F, D, eps, scale);
+  norm_finalize_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(partials, F, D, eps, scale,
+                                                                                       zero);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ++*launches;
   return cudaSuccess;

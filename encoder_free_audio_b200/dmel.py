@@ -73,6 +73,15 @@ def _lib():
         L.dmel_forward.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, i32, vp, vp,
                                    sz, vp]
         L.dmel_forward.restype = i32
+        L.dmel_table_prepare_size.argtypes = [i32, i32]
+        L.dmel_table_prepare_size.restype = sz
+        L.dmel_table_prepare.argtypes = [vp, i32, i32, vp, sz, vp]
+        L.dmel_table_prepare.restype = i32
+        L.dmel_embed_prepared.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, vp, i32, vp, sz, vp]
+        L.dmel_embed_prepared.restype = i32
+        L.dmel_forward_prepared.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, vp,
+                                            i32, vp, vp, sz, vp]
+        L.dmel_forward_prepared.restype = i32
         L.dmel_embed_rows.argtypes = [vp, i64, vp, i32, i32, vp, ctypes.c_float, vp, vp, i64, i32, vp, sz, vp]
         L.dmel_embed_rows.restype = i32
         L.dmel_forward_rows.argtypes = [vp, vp, vp, i32, i64, vp, vp, vp, i32, i32, vp, ctypes.c_float, vp, vp, i64,
@@ -285,6 +294,40 @@ def dmel_forward(wav, sample_offsets, frame_offsets, n_frames: int, table, out, 
                              _ptr(rms_weight), float(eps), _ptr(out), _dtype_code(out), _ptr(codes_out),
                              _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc, "dmel_forward")
+
+
+def dmel_table_prepare_size(embed_dim: int, table_dtype: int) -> int:
+    """Bytes of a table's prepared data (its Gram matrix), 0 when none applies."""
+    return int(_lib().dmel_table_prepare_size(int(embed_dim), int(table_dtype)))
+
+
+def dmel_table_prepare(table, prepared, stream=None):
+    """G = T T^T of a bf16 CUDA table [1280, D] into the CUDA uint8 tensor prepared (at least
+    dmel_table_prepare_size bytes)."""
+    rc = _lib().dmel_table_prepare(_ptr(table), table.shape[1], _dtype_code(table), _ptr(prepared),
+                                   prepared.numel() * prepared.element_size(), _stream(stream))
+    _check(rc, "dmel_table_prepare")
+
+
+def dmel_embed_prepared(codes, table, out, prepared, rms_weight=None, eps: float = 1e-6, workspace=None, stream=None):
+    """dmel_embed with the table's prepared data (or None)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_embed_prepared(_ptr(codes), int(codes.shape[0]), _ptr(table), _dtype_code(table), table.shape[1],
+                                    _ptr(rms_weight), float(eps), _ptr(prepared), _ptr(out), _dtype_code(out),
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_embed_prepared")
+
+
+def dmel_forward_prepared(wav, sample_offsets, frame_offsets, n_frames: int, table, out, prepared, rms_weight=None,
+                          eps: float = 1e-6, tails=None, tails_out=None, codes_out=None, workspace=None, stream=None):
+    """dmel_forward with the table's prepared data (or None)."""
+    n_clips = sample_offsets.shape[0] - 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib().dmel_forward_prepared(_ptr(wav), _ptr(sample_offsets), _ptr(frame_offsets), n_clips, int(n_frames),
+                                      _ptr(tails), _ptr(tails_out), _ptr(table), _dtype_code(table), table.shape[1],
+                                      _ptr(rms_weight), float(eps), _ptr(prepared), _ptr(out), _dtype_code(out),
+                                      _ptr(codes_out), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "dmel_forward_prepared")
 
 
 def dmel_embed_rows(codes, table, out, out_rows, rms_weight=None, eps: float = 1e-6, workspace=None, stream=None):

@@ -1,7 +1,8 @@
 """Convenience layer over the C ABI for callers that hold torch tensors.
 
 ``FrontEnd`` keeps the embedding table and RMSNorm weight on the device and runs
-``dmel_forward`` on batches of clips. ``plan()`` sizes the per-batch buffers (device offsets,
+``dmel_forward`` on batches of clips; with ``prepare=True`` it computes the table's Gram matrix
+once (``dmel_table_prepare``) and runs ``dmel_forward_prepared``. ``plan()`` sizes the per-batch buffers (device offsets,
 frame offsets, output, workspace) once, so repeated calls allocate nothing new.
 ``forward_host()`` is the end-to-end call: host waveforms in, frame vectors (and codes) back in
 host memory, through ``dmel_forward_host`` (the library overlaps the copies with the kernels).
@@ -37,13 +38,18 @@ class Plan:
 
 class FrontEnd:
     def __init__(self, table: torch.Tensor, rms_weight: torch.Tensor | None = None, eps: float = 1e-6,
-                 out_dtype: torch.dtype = torch.bfloat16):
+                 out_dtype: torch.dtype = torch.bfloat16, prepare: bool = False):
         assert table.is_cuda and table.dim() == 2 and table.shape[0] == dmel.TABLE_ROWS
         self.table = table.contiguous()
         self.rms_weight = None if rms_weight is None else rms_weight.to(table.dtype).contiguous()
         self.eps = float(eps)
         self.out_dtype = out_dtype
         self.dim = int(table.shape[1])
+        self.prepared = None  # the table's Gram matrix, when prepared and used by this configuration
+        n = dmel.dmel_table_prepare_size(self.dim, dmel._dtype_code(self.table)) if prepare else 0
+        if n and self.rms_weight is not None:
+            self.prepared = torch.empty(n, dtype=torch.uint8, device=self.table.device)
+            dmel.dmel_table_prepare(self.table, self.prepared)
 
     def plan(self, sample_offsets_host, chunk_frames: int = 0, host_path: bool = False) -> Plan:
         """Buffers for batches with these clip boundaries; with host_path, also the staging
@@ -76,9 +82,9 @@ class FrontEnd:
     def forward(self, wav: torch.Tensor, plan: Plan, tails=None, tails_out=None, stream=None) -> torch.Tensor:
         """Frame vectors of device waveforms `wav` (fp32 [n_samples]) into plan.out; codes into
         plan.codes."""
-        dmel.dmel_forward(wav, plan.sample_offsets, plan.frame_offsets, plan.n_frames, self.table, plan.out,
-                          rms_weight=self.rms_weight, eps=self.eps, tails=tails, tails_out=tails_out,
-                          codes_out=plan.codes, workspace=plan.workspace, stream=stream)
+        dmel.dmel_forward_prepared(wav, plan.sample_offsets, plan.frame_offsets, plan.n_frames, self.table, plan.out,
+                                   self.prepared, rms_weight=self.rms_weight, eps=self.eps, tails=tails,
+                                   tails_out=tails_out, codes_out=plan.codes, workspace=plan.workspace, stream=stream)
         return plan.out
 
     def forward_host(self, wav_host: torch.Tensor, plan: Plan, out_host: torch.Tensor, codes_host=None, stream=None):

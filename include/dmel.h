@@ -175,6 +175,38 @@ dmel_status dmel_forward(const float *wav, const int64_t *sample_offsets, const 
                          dmel_dtype out_dtype, uint8_t *codes_out, void *workspace, size_t workspace_bytes,
                          dmel_stream_t stream);
 
+/* ---- A table prepared once for many calls. With RMSNorm ("Inside Inkling: Audio Design",
+ * Part 1 · Modeling: the summed embedding, optionally normalised), a frame's sum of squares is
+ * sum_b sum_b' G[r_b, r_b'] with G = T T^T, the table's Gram matrix (T [1280 x embed_dim], r_b the
+ * table row of bin b's level). dmel_embed and dmel_forward compute G inside each call of 16,384
+ * frames or more; a caller with a fixed table computes it once here and passes it to the
+ * _prepared calls, which then take that form of RMSNorm from 12,288 frames per call (below that,
+ * the exchange of row sums inside the product kernel is as fast or faster, and is kept).
+ *
+ * dmel_table_prepare_size: bytes of the prepared data for a table of this width and dtype, or 0
+ *   when no preparation applies (fp32 tables; widths not a multiple of 128).
+ * dmel_table_prepare: computes G of table (bf16 [1280 x embed_dim], device, 16-byte aligned) into
+ *   prepared (device, 256-byte aligned, prepared_bytes >= dmel_table_prepare_size), owned by the
+ *   caller and valid while the table is unchanged. Asynchronous on stream; a size of 0 or a bad
+ *   pointer returns DMEL_ERR_INVALID_ARG.
+ * dmel_embed_prepared / dmel_forward_prepared: as dmel_embed / dmel_forward, plus prepared (from
+ *   dmel_table_prepare for this table, or NULL: then exactly dmel_embed / dmel_forward). It is
+ *   used when rms_weight is given and the table qualifies, and ignored otherwise; the workspace
+ *   is the one dmel_workspace_size reports. A prepared pointer not 256-byte aligned returns
+ *   DMEL_ERR_INVALID_ARG. Results equal the unprepared calls' bit for bit from 16,384 frames
+ *   (both take the G form); from 12,288 to 16,383 frames they differ by float rounding only. */
+size_t dmel_table_prepare_size(int embed_dim, dmel_dtype table_dtype);
+dmel_status dmel_table_prepare(const void *table, int embed_dim, dmel_dtype table_dtype, void *prepared,
+                               size_t prepared_bytes, dmel_stream_t stream);
+dmel_status dmel_embed_prepared(const uint8_t *codes, int64_t n_frames, const void *table, dmel_dtype table_dtype,
+                                int embed_dim, const void *rms_weight, float eps, const void *prepared, void *out,
+                                dmel_dtype out_dtype, void *workspace, size_t workspace_bytes, dmel_stream_t stream);
+dmel_status dmel_forward_prepared(const float *wav, const int64_t *sample_offsets, const int64_t *frame_offsets,
+                                  int n_clips, int64_t n_frames, const float *tails, float *tails_out,
+                                  const void *table, dmel_dtype table_dtype, int embed_dim, const void *rms_weight,
+                                  float eps, const void *prepared, void *out, dmel_dtype out_dtype,
+                                  uint8_t *codes_out, void *workspace, size_t workspace_bytes, dmel_stream_t stream);
+
 /* ---- End to end from host memory: dmel_forward for a batch held in host memory, returning the
  * frame vectors (and optionally the codes) to host memory, with the copies overlapped with the
  * kernels ("Inside Inkling: Audio Design", Part 1 · Modeling for what is computed; Part 3 ·

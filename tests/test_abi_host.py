@@ -279,3 +279,36 @@ def test_hmlp_argument_checks_without_gpu(lib):
     assert nw >= nf + P * 64 * 1792 * 4  # past 1536 columns the fp32 sums are back
     # no image: a no-op
     assert H(None, 0, 40, 40, ctypes.byref(w), None, None, 0, None) == dmel.DMEL_OK
+
+
+def test_table_prepare_size_and_argument_checks_without_gpu(lib):
+    """A prepared table (its Gram matrix G, 1280 x 1280 fp32 and a second partial product) exists
+    for bf16 tables whose width the tensor-core path tiles, and for nothing else; bad pointers and
+    sizes are rejected before any device call."""
+    vp = ctypes.c_void_p
+    a = vp(1 << 20)
+    n = dmel.dmel_table_prepare_size(6144, dmel.DMEL_BF16)
+    assert n >= 2 * 1280 * 1280 * 4
+    assert dmel.dmel_table_prepare_size(256, dmel.DMEL_BF16) == n
+    assert dmel.dmel_table_prepare_size(6144, dmel.DMEL_F32) == 0
+    assert dmel.dmel_table_prepare_size(200, dmel.DMEL_BF16) == 0
+    assert dmel.dmel_table_prepare_size(0, dmel.DMEL_BF16) == 0
+    P = lib.dmel_table_prepare
+    assert P(a, 6144, dmel.DMEL_BF16, a, n - 1, None) == dmel.DMEL_ERR_INVALID_ARG  # too small
+    assert P(a, 6144, dmel.DMEL_BF16, vp((1 << 20) + 16), n, None) == dmel.DMEL_ERR_INVALID_ARG  # misaligned
+    assert P(a, 6144, dmel.DMEL_BF16, None, n, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert P(None, 6144, dmel.DMEL_BF16, a, n, None) == dmel.DMEL_ERR_INVALID_ARG
+    assert P(a, 6144, dmel.DMEL_F32, a, n, None) == dmel.DMEL_ERR_INVALID_ARG  # no G for fp32 tables
+    # a prepared pointer off its 256-byte alignment is an argument error in both calls
+    odd = vp((1 << 20) + 64)
+    ws_n = dmel.dmel_workspace_size(1000, 6144, dmel.DMEL_BF16, True, True)
+    E = lib.dmel_embed_prepared
+    assert E(a, 1000, a, dmel.DMEL_BF16, 6144, a, 1e-6, odd, a, dmel.DMEL_BF16, a, ws_n,
+             None) == dmel.DMEL_ERR_INVALID_ARG
+    ws_f = dmel.dmel_workspace_size(1000, 6144, dmel.DMEL_BF16, True, False)
+    Fw = lib.dmel_forward_prepared
+    assert Fw(a, a, a, 1, 1000, None, None, a, dmel.DMEL_BF16, 6144, a, 1e-6, odd, a, dmel.DMEL_BF16, None, a, ws_f,
+              None) == dmel.DMEL_ERR_INVALID_ARG
+    # and a prepared pointer does not relax the other checks
+    assert E(a, 1000, a, dmel.DMEL_BF16, 6144, a, 1e-6, a, a, dmel.DMEL_BF16, None, 0,
+             None) == dmel.DMEL_ERR_INVALID_ARG

@@ -228,6 +228,83 @@ def test_embed_rmsnorm_from_gram_matches_oracle(table_bf16, rmsw_bf16, oracle_mo
         compare_embed(out[c0:c0 + 4096].cpu().numpy(), ref, 1e-5)
 
 
+def _prepared(T):
+    P = torch.empty(dmel.dmel_table_prepare_size(T.shape[1], dmel.DMEL_BF16), dtype=torch.uint8, device=DEV)
+    dmel.dmel_table_prepare(T, P)
+    return P
+
+
+@pytest.mark.parametrize("out_dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("F", [1, 1000, 12288 + 77])
+def test_embed_prepared_calls_match_oracle(F, out_dt, table_bf16, rmsw_bf16, oracle_mod):
+    """With the table prepared once, calls of 12,288 frames or more take their RMSNorm scales from
+    G (here a ragged last tile); smaller ones (one frame, one ragged tile) exchange row sums as
+    unprepared calls do. Both match the oracle."""
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    P = _prepared(T)
+    codes = synth.random_codes(45 + F, F)
+    out = torch.empty((F, 6144), dtype=out_dt, device=DEV)
+    ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True), dtype=torch.uint8, device=DEV)
+    dmel.dmel_embed_prepared(torch.from_numpy(codes).to(DEV), T, out, P, rms_weight=g, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for c0 in range(0, F, 4096):
+        ref = oracle_mod.embed(codes[c0:c0 + 4096], T64, g64, 1e-6)
+        got = out[c0:c0 + 4096].float().cpu().numpy()
+        worst = max(worst, compare_embed(got, ref, 1e-5 if out_dt == torch.float32 else 1e-2))
+    print(f"prepared embed F={F} out={out_dt}: worst {worst:.2e}")
+
+
+def test_embed_prepared_equals_unprepared_at_gram_sizes(table_bf16, rmsw_bf16):
+    """At 16,384 frames and more an unprepared call computes the same G itself: the outputs are
+    bit-identical. Without RMSNorm the prepared data is ignored."""
+    T, _ = table_bf16
+    g, _ = rmsw_bf16
+    P = _prepared(T)
+    F = 16384 + 333
+    codes = torch.from_numpy(synth.random_codes(46, F)).to(DEV)
+    ws = torch.empty(dmel.dmel_workspace_size(F, 6144, dmel.DMEL_BF16, True, True), dtype=torch.uint8, device=DEV)
+    a = torch.empty((F, 6144), dtype=torch.bfloat16, device=DEV)
+    b = torch.empty_like(a)
+    dmel.dmel_embed(codes, T, a, rms_weight=g, eps=1e-6, workspace=ws)
+    dmel.dmel_embed_prepared(codes, T, b, P, rms_weight=g, eps=1e-6, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    dmel.dmel_embed(codes, T, a, workspace=ws)
+    dmel.dmel_embed_prepared(codes, T, b, P, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_table_prepare_matches_the_gram_matrix(table_bf16):
+    """The prepared data is G = T T^T as the Gram kernel writes it (bit-identical to the debug
+    entry point's first block)."""
+    T, _ = table_bf16
+    P = _prepared(T)
+    G = torch.full((2, 1280, 1280), float("nan"), dtype=torch.float32, device=DEV)
+    dmel.dmel_debug_gram(T, G)
+    torch.cuda.synchronize()
+    got = P[:1280 * 1280 * 4].view(torch.float32).view(1280, 1280)
+    for g in range(10):
+        for h in range(g, 10):
+            blk = (slice(128 * g, 128 * g + 128), slice(128 * h, 128 * h + 128))
+            assert torch.equal(got[blk], G[0][blk]), (g, h)
+
+
+def test_forward_prepared_batch64_10s(table_bf16, rmsw_bf16, oracle_mod):
+    """FrontEnd(prepare=True): dmel_forward_prepared on the 64 x 10 s batch against the oracle."""
+    T, T64 = table_bf16
+    g, g64 = rmsw_bf16
+    wav, off = synth.batch64_10s()
+    fe = FrontEnd(T, g, 1e-6, torch.bfloat16, prepare=True)
+    assert fe.prepared is not None
+    plan = fe.plan(off)
+    fe.forward(torch.from_numpy(wav).to(DEV), plan)
+    torch.cuda.synchronize()
+    _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, label="batch64_10s prepared")
+
+
 # ------------------------------------------------------------- output rows (sentinel splice)
 
 def _rows_case(F, S, seed):
