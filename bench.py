@@ -356,16 +356,18 @@ def streaming_line(torch, dev, dmel, FrontEnd, pk, calls: int, warmup: int, with
     plan = fe.plan(synth.offsets_from_lengths([800] * S.n))
     n_in = min(calls, 64)  # distinct inputs, cycled (13 MB each)
     xs = [torch.from_numpy(S.call(k)).to(dev).reshape(-1) for k in range(n_in)]
-    tails = torch.zeros((S.n, 800), device=dev)
+    # two tail buffers, alternating: call k reads tails[k % 2] and writes tails[(k + 1) % 2] (the
+    # codes kernel writes them; updating one buffer in place takes a copy kernel after it)
+    tails = [torch.zeros((S.n, 800), device=dev), torch.zeros((S.n, 800), device=dev)]
     stream = torch.cuda.current_stream()
     for k in range(warmup):
-        fe.forward(xs[k % n_in], plan, tails=tails, tails_out=tails)
-    tails.zero_()
+        fe.forward(xs[k % n_in], plan, tails=tails[k % 2], tails_out=tails[(k + 1) % 2])
+    tails[0].zero_()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
     for k in range(calls):
         evs[k][0].record(stream)
-        fe.forward(xs[k % n_in], plan, tails=tails, tails_out=tails)
+        fe.forward(xs[k % n_in], plan, tails=tails[k % 2], tails_out=tails[(k + 1) % 2])
         evs[k][1].record(stream)
     torch.cuda.synchronize()
     ms = [a.elapsed_time(b) for a, b in evs]

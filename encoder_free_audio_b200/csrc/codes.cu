@@ -624,6 +624,31 @@ cudaError_t ensure_device_tables() {
   return cudaSuccess;
 }
 
+// Carried tail of clip c into tails_out row c, by threads tid = 0..nt-1 of a warp or block: the
+// last 800 consumed samples of the clip (those ending at sample 800 F), the tail in when the clip
+// has no frame, zeros when there is neither; zeros and an offsets error when the clip is shorter
+// than its frames need.
+__device__ void clip_tail(int c, const float *__restrict__ wav, const int64_t *__restrict__ soff,
+                          const int64_t *__restrict__ foff, const float *tails, float *tails_out, uint32_t *err,
+                          int tid, int nt) {
+  const int64_t F = foff[c + 1] - foff[c];
+  const int64_t len = soff[c + 1] - soff[c];
+  float *dst = tails_out + (int64_t)c * kHop;
+  if (F >= 1 && (int64_t)kHop * F > len) {
+    if (tid == 0) record_error(err, DMEL_DEVERR_OFFSETS);
+    for (int n = tid; n < kHop; n += nt) dst[n] = 0.0f;
+    return;
+  }
+  const float *src = F >= 1 ? wav + soff[c] + (int64_t)kHop * (F - 1) : (tails ? tails + (int64_t)c * kHop : nullptr);
+  if (!src) {
+    for (int n = tid; n < kHop; n += nt) dst[n] = 0.0f;
+  } else if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+    for (int n = tid; n < kHop / 4; n += nt) reinterpret_cast<float4 *>(dst)[n] = reinterpret_cast<const float4 *>(src)[n];
+  } else {
+    for (int n = tid; n < kHop; n += nt) dst[n] = src[n];
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- kernels
@@ -634,6 +659,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
                                                                              const int64_t *__restrict__ foff,
                                                                              int n_clips, int64_t n_frames,
                                                                              const float *__restrict__ tails,
+                                                                             float *__restrict__ tails_out,
                                                                              uint8_t *__restrict__ codes,
                                                                              Quant qz, uint32_t *err) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -673,10 +699,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int64_t gw = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
+  // tails_out (never the tails in): warp gw writes the carried tails of clips gw, gw + warps_total,
+  // ..., after its frames
+  auto tails_after = [&]() {
+    if (tails_out)
+      for (int64_t c = gw; c < n_clips; c += warps_total) clip_tail((int)c, wav, soff, foff, tails, tails_out, err, lane, 32);
+  };
   const int64_t chunk = (n_frames + warps_total - 1) / warps_total;
   const int64_t g0 = gw * chunk;
   const int64_t g1 = g0 + chunk < n_frames ? g0 + chunk : n_frames;
-  if (g0 >= g1) return;
+  if (g0 >= g1) {
+    tails_after();
+    return;
+  }
 
   // last clip with foff[clip] <= g0: a 32-way search, each lane probing one point per round
   int lo = 0, hi = n_clips - 1;
@@ -749,6 +784,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
     step_e_codes(lane, T, part, crow, nullptr, qz);
     __syncwarp();
   }
+  tails_after();
 }
 
 // Carried tails: one block per clip row (800 floats); the source is the last 800 consumed
@@ -757,25 +793,8 @@ __global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restric
                                                           const int64_t *__restrict__ soff,
                                                           const int64_t *__restrict__ foff, int n_clips,
                                                           const float *tails, float *tails_out, uint32_t *err) {
-  for (int c = blockIdx.x; c < n_clips; c += gridDim.x) {
-    const int64_t F = foff[c + 1] - foff[c];
-    const int64_t len = soff[c + 1] - soff[c];
-    float *dst = tails_out + (int64_t)c * kHop;
-    if (F >= 1 && (int64_t)kHop * F > len) {
-      if (threadIdx.x == 0) record_error(err, DMEL_DEVERR_OFFSETS);
-      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = 0.0f;
-      continue;
-    }
-    const float *src = F >= 1 ? wav + soff[c] + (int64_t)kHop * (F - 1) : (tails ? tails + (int64_t)c * kHop : nullptr);
-    if (!src) {
-      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = 0.0f;
-    } else if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-      for (int n = threadIdx.x; n < kHop / 4; n += blockDim.x)
-        reinterpret_cast<float4 *>(dst)[n] = reinterpret_cast<const float4 *>(src)[n];
-    } else {
-      for (int n = threadIdx.x; n < kHop; n += blockDim.x) dst[n] = src[n];
-    }
-  }
+  for (int c = blockIdx.x; c < n_clips; c += gridDim.x)
+    clip_tail(c, wav, soff, foff, tails, tails_out, err, threadIdx.x, blockDim.x);
 }
 
 // ---------------------------------------------------------------- host entry points
@@ -788,15 +807,21 @@ cudaError_t launch_codes(const float *wav, const int64_t *soff, const int64_t *f
   static std::atomic<bool> attr[256];
   if ((e = set_smem_attr_once(codes_kernel_entry<kWarpsDefault>, smem_bytes(kWarpsDefault), attr)) != cudaSuccess)
     return e;
+  // the codes kernel writes the carried tails itself (after its frames) unless tails_out overlaps
+  // the tails in, whose rows other warps may still have to read: then a kernel of its own after it
+  const uintptr_t ti = reinterpret_cast<uintptr_t>(tails), to = reinterpret_cast<uintptr_t>(tails_out);
+  const uintptr_t tb = (uintptr_t)n_clips * kHop * sizeof(float);
+  const bool overlap = tails && tails_out && ti < to + tb && to < ti + tb;
+  const bool fused = tails_out && n_clips > 0 && n_frames > 0 && !overlap;
   if (n_frames > 0) {
     int64_t blocks = (n_frames + kWarpsDefault - 1) / kWarpsDefault;
     if (blocks > num_sms) blocks = num_sms;  // one persistent block per SM
     codes_kernel_entry<kWarpsDefault><<<(unsigned)blocks, kWarpsDefault * 32, smem_bytes(kWarpsDefault), stream>>>(
-        wav, soff, foff, n_clips, n_frames, tails, codes, q, err);
+        wav, soff, foff, n_clips, n_frames, tails, fused ? tails_out : nullptr, codes, q, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
   }
-  if (tails_out && n_clips > 0) {
+  if (tails_out && n_clips > 0 && !fused) {
     int64_t blocks = n_clips;
     if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
     tails_kernel_entry<<<(unsigned)blocks, 256, 0, stream>>>(wav, soff, foff, n_clips, tails, tails_out, err);

@@ -103,8 +103,10 @@ size_t dmel_workspace_size(int64_t n_frames, int embed_dim, dmel_dtype table_dty
  * tails           NULL, or fp32 [n_clips x 800]: the 800 samples that came before each clip
  *                 (streaming); NULL means zeros
  * tails_out       NULL, or fp32 [n_clips x 800]: receives the 800 samples that end at sample
- *                 800*F of each clip (F its frame count), or the tail in when F == 0. May equal
- *                 `tails` (it is written after every frame has been read).
+ *                 800*F of each clip (F its frame count), or the tail in when F == 0. Must not
+ *                 overlap wav. May equal `tails`: it is then written by a kernel of its own after
+ *                 every frame has been read; a tails_out apart from `tails` (two buffers used in
+ *                 turn, for streaming) is written by the codes kernel itself, one launch fewer.
  * codes           uint8 [n_frames x 80], row-major, receives c_b in 0..15 per frame and channel
  *
  * Per frame t of a clip x (causal framing, "Inside Inkling: Audio Design", Part 1 · Modeling:

@@ -73,6 +73,35 @@ def test_codes_edge_lengths_and_tails(oracle_mod):
     np.testing.assert_array_equal(t_out, oracle_mod.tails_out(wav, off, tails))
 
 
+def test_codes_tails_in_place_and_no_frames(oracle_mod):
+    """The carried tails written in place (tails_out = tails: a kernel of their own after the
+    codes) equal those written into another buffer (by the codes kernel itself, after each warp's
+    frames); a batch with no frame at all passes the tails in through."""
+    r = np.random.default_rng(23)
+    lengths = [0, 1, 799, 800, 801, 1599, 1600, 2400, 5 * 800 + 13, 0, 3200] * 300
+    off = synth.offsets_from_lengths(lengths)
+    wav = r.uniform(-0.7, 0.7, int(off[-1])).astype(np.float32)
+    tails = r.uniform(-0.5, 0.5, (len(lengths), 800)).astype(np.float32)
+    g, t_out = _codes_gpu(wav, off, tails=tails, want_tails=True)
+    fo = dmel.dmel_frame_offsets(off)
+    F = int(fo[-1])
+    codes = torch.empty((F, 80), dtype=torch.uint8, device=DEV)
+    t_io = torch.from_numpy(tails).to(DEV)
+    dmel.dmel_codes(torch.from_numpy(wav).to(DEV), torch.from_numpy(off).to(DEV), torch.from_numpy(fo).to(DEV), F,
+                    codes, tails=t_io, tails_out=t_io)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), g)
+    np.testing.assert_array_equal(t_io.cpu().numpy(), t_out)
+    np.testing.assert_array_equal(t_out, oracle_mod.tails_out(wav, off, tails))
+    # no frame in the batch: the codes kernel does not run
+    off0 = synth.offsets_from_lengths([0, 799, 5, 0])
+    w0 = r.uniform(-0.7, 0.7, int(off0[-1])).astype(np.float32)
+    tl0 = r.uniform(-0.5, 0.5, (4, 800)).astype(np.float32)
+    g0, t0 = _codes_gpu(w0, off0, tails=tl0, want_tails=True)
+    assert g0.shape == (0, 80)
+    np.testing.assert_array_equal(t0, oracle_mod.tails_out(w0, off0, tl0))
+
+
 def test_codes_silence_and_full_scale(oracle_mod):
     r = np.random.default_rng(22)
     off = synth.offsets_from_lengths([16000, 16000])
@@ -526,6 +555,25 @@ def test_forward_ragged1024(table_bf16, rmsw_bf16, oracle_mod):
     emb = np.sort(r.choice(frame_ids.shape[0], 768, replace=False))
     _check_forward(wav, off, plan, T64, g64, 1e-2, oracle_mod, frame_ids=frame_ids, embed_ids=emb,
                    label="ragged1024 (sampled)")
+
+
+def test_streaming_two_tail_buffers_equal_in_place(table_bf16, rmsw_bf16):
+    """Streaming calls that alternate two tail buffers (the codes kernel writes the tails) give
+    the same codes, vectors and tails, bit for bit, as calls that update one buffer in place."""
+    T, _ = table_bf16
+    g, _ = rmsw_bf16
+    S = synth.Streams4096()
+    fe = FrontEnd(T, g, 1e-6, torch.bfloat16)
+    pa, pb = fe.plan(synth.offsets_from_lengths([800] * S.n)), fe.plan(synth.offsets_from_lengths([800] * S.n))
+    t_in_place = torch.zeros((S.n, 800), device=DEV)
+    bufs = [torch.zeros((S.n, 800), device=DEV), torch.zeros((S.n, 800), device=DEV)]
+    for k in range(6):
+        x = torch.from_numpy(S.call(k)).to(DEV).reshape(-1)
+        fe.forward(x, pa, tails=t_in_place, tails_out=t_in_place)
+        fe.forward(x, pb, tails=bufs[k % 2], tails_out=bufs[(k + 1) % 2])
+        torch.cuda.synchronize()
+        assert torch.equal(pa.codes, pb.codes) and torch.equal(pa.out, pb.out)
+        assert torch.equal(t_in_place, bufs[(k + 1) % 2])
 
 
 def test_streaming_4096_matches_offline_and_oracle(table_bf16, rmsw_bf16, oracle_mod):
