@@ -624,13 +624,15 @@ cudaError_t ensure_device_tables() {
   return cudaSuccess;
 }
 
-// Carried tail of clip c into tails_out row c, by threads tid = 0..nt-1 of a warp or block: the
+// Carried tail of clip c into tails_out row c, by threads tid = 0..NT-1 of a warp or block: the
 // last 800 consumed samples of the clip (those ending at sample 800 F), the tail in when the clip
 // has no frame, zeros when there is neither; zeros and an offsets error when the clip is shorter
-// than its frames need.
+// than its frames need. The aligned copy issues all of a thread's loads before its stores.
+template <int NT>
 __device__ void clip_tail(int c, const float *__restrict__ wav, const int64_t *__restrict__ soff,
                           const int64_t *__restrict__ foff, const float *tails, float *tails_out, uint32_t *err,
-                          int tid, int nt) {
+                          int tid) {
+  constexpr int nt = NT, PER = (kHop / 4 + NT - 1) / NT;
   const int64_t F = foff[c + 1] - foff[c];
   const int64_t len = soff[c + 1] - soff[c];
   float *dst = tails_out + (int64_t)c * kHop;
@@ -643,7 +645,13 @@ __device__ void clip_tail(int c, const float *__restrict__ wav, const int64_t *_
   if (!src) {
     for (int n = tid; n < kHop; n += nt) dst[n] = 0.0f;
   } else if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-    for (int n = tid; n < kHop / 4; n += nt) reinterpret_cast<float4 *>(dst)[n] = reinterpret_cast<const float4 *>(src)[n];
+    float4 v[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k)
+      if (tid + k * NT < kHop / 4) v[k] = reinterpret_cast<const float4 *>(src)[tid + k * NT];
+#pragma unroll
+    for (int k = 0; k < PER; ++k)
+      if (tid + k * NT < kHop / 4) reinterpret_cast<float4 *>(dst)[tid + k * NT] = v[k];
   } else {
     for (int n = tid; n < kHop; n += nt) dst[n] = src[n];
   }
@@ -699,13 +707,18 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, 1) codes_kernel_entry(con
 
   const int64_t warps_total = (int64_t)gridDim.x * kWarpsPerBlock;
   const int64_t gw = (int64_t)blockIdx.x * kWarpsPerBlock + warp;
-  // tails_out (never the tails in): warp gw writes the carried tails of clips gw, gw + warps_total,
-  // ..., after its frames
-  auto tails_after = [&]() {
-    if (tails_out)
-      for (int64_t c = gw; c < n_clips; c += warps_total) clip_tail((int)c, wav, soff, foff, tails, tails_out, err, lane, 32);
-  };
   const int64_t chunk = (n_frames + warps_total - 1) / warps_total;
+  // tails_out (never the tails in): written after the frames, by the warps that have no frame
+  // when there are enough of them (a tail copy costs a fraction of a frame: at most 4 chunk clips
+  // each), else by every warp, clip c by warp c mod warps_total
+  auto tails_after = [&]() {
+    if (!tails_out) return;
+    const int64_t busy = (n_frames + chunk - 1) / chunk, idle = warps_total - busy;
+    const bool by_idle = idle > 0 && (n_clips + idle - 1) / idle <= 4 * chunk;
+    const int64_t w = by_idle ? gw - busy : gw, nw = by_idle ? idle : warps_total;
+    if (w < 0) return;
+    for (int64_t c = w; c < n_clips; c += nw) clip_tail<32>((int)c, wav, soff, foff, tails, tails_out, err, lane);
+  };
   const int64_t g0 = gw * chunk;
   const int64_t g1 = g0 + chunk < n_frames ? g0 + chunk : n_frames;
   if (g0 >= g1) {
@@ -794,7 +807,7 @@ __global__ void __launch_bounds__(256) tails_kernel_entry(const float *__restric
                                                           const int64_t *__restrict__ foff, int n_clips,
                                                           const float *tails, float *tails_out, uint32_t *err) {
   for (int c = blockIdx.x; c < n_clips; c += gridDim.x)
-    clip_tail(c, wav, soff, foff, tails, tails_out, err, threadIdx.x, blockDim.x);
+    clip_tail<256>(c, wav, soff, foff, tails, tails_out, err, threadIdx.x);
 }
 
 // ---------------------------------------------------------------- host entry points
