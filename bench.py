@@ -64,15 +64,14 @@ def out_bytes(out_es: int) -> int:
     return DIM * out_es
 
 
-# DRAM bytes (read + write) of each stage's kernels per launch, from the ncu captures summarised
-# under profiles/: measured on the headline workload itself (318,044 frames: codes_kernel_entry and
-# embed_sp_kernel<kScaled>) where a capture of that size exists, else from the 12,800-frame
-# capture as a fixed part per call plus a part per frame. The embedding stage of a call of >= 16,384 frames is gram_kernel
-# (the table once) + norm_partials_kernel (55 blocks of G + the codes) + embed_sp_kernel<kScaled>.
-TRAFFIC_MEASURED = {318044: {"codes": 1024500480 + 27511296,
-                             "embed": 15749120 + (3604480 + 80 * 318044) + (47177984 + 3850828288)}}
-TRAFFIC = {"codes": {"fixed": 0.0, "per_frame": (41091584 + 0) / 12800},
-           "embed": {"fixed": 15749120 + 3604480 + 15728640, "per_frame": 80 + (16923648 - 15728640 + 101618688) / 12800}}
+# DRAM bytes (read + write) of each stage's kernels per call, from the ncu capture of the headline
+# workload itself (318,044 frames, profiles/dram_traffic_ragged1024.md, the kernels as they are
+# now): codes_kernel_entry; and the embedding call's six kernels, gram_kernel, gram_combine_kernel,
+# gram_diag_kernel (G), norm_partials_kernel, norm_finalize_kernel (the scales) and
+# embed_sp_kernel<kScaled>. Other frame counts have no capture of the current kernels: null.
+TRAFFIC_MEASURED = {318044: {"codes": 1024452352 + 27800064,
+                             "embed": (15749376 + 7212800 + 15735040) + (29188864 + 21142528) + (69980928 + 23040)
+                             + (43464704 + 3851025408)}}
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144 logical flops, run as a
 # 2:4-sparse product whose peak is twice the dense bf16 peak (nominal 4.5 vs 2.25 PFLOP/s)
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
@@ -226,12 +225,7 @@ def stage_lines(F, codes_ms, embed_ms, out_es, pk) -> dict:
     def line(name, ms, bytes_per_frame, kernel):
         s = statistics.mean(ms) / 1e3
         achieved = bytes_per_frame * F / s / 1e9
-        tr = TRAFFIC.get(name)
-        traffic = None if tr is None else tr["fixed"] + tr["per_frame"] * F
-        if name == "embed" and F < 16384:
-            traffic = None  # a smaller call takes the exchange form of RMSNorm, not the captured kernels
-        if F in TRAFFIC_MEASURED:
-            traffic = TRAFFIC_MEASURED[F][name]
+        traffic = TRAFFIC_MEASURED[F][name] if F in TRAFFIC_MEASURED else None
         return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic,
                 "ms": statistics.mean(ms), "kernel": kernel, "peak_source": pk["source"]}
