@@ -916,10 +916,10 @@ constexpr int EPI_CHUNK = 32;           // columns staged at a time
 constexpr int OFF_G = OFF_BAR + 256;    // RMSNorm weights of the column tile (kScaled: [2], by accumulator)
 constexpr int OFF_EPI = OFF_G + 2 * BN_EPI * 4;  // row sums [2][128] and scales [128]
 constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;  // staging: 8 warps x 32 rows x up to 128 bytes
-constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: tile indices [16], count published
+constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: {tile index, sequence} [16]
 constexpr int RING = 16;
 constexpr int LOOKAHEAD = 3;  // tiles published ahead of the one the TMA warp starts
-constexpr int SMEM_USED = OFF_RING + (RING + 4) * 4;
+constexpr int SMEM_USED = OFF_RING + RING * 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int WAITER_WARP = 6 + EPI_WARPS;  // warps: 0 TMA, 1 MMA, 2..5 A, 6..13 epilogue, 14 waits
 constexpr int THREADS = 32 * (WAITER_WARP + 1);
@@ -977,22 +977,15 @@ __device__ __forceinline__ uint32_t ld_relaxed_u32(const float *p) {
 // Number of column tiles of the sparse kernel (the last one may be partial).
 __host__ __device__ constexpr int sp_col_tiles(int D) { return (D + sp::BN - 1) / sp::BN; }
 
-// Shared-memory words of either CTA of the cluster (addresses from mapa_shared), for the tile
-// index ring of the dynamic schedule.
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+// 8-byte shared-memory slots of either CTA of the cluster (addresses from mapa_shared) for the
+// tile index ring of the dynamic schedule: one aligned 8-byte access is single-copy atomic, so a
+// slot carries its own sequence number and needs no release/acquire pairing with a second word.
+__device__ __forceinline__ void st_relaxed_cluster_u64(uint32_t cluster_addr, unsigned long long v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
 }
-__device__ __forceinline__ void st_release_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.release.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_acquire_cluster_u32(uint32_t local_addr) {
-  uint32_t v;
-  asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local_addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ uint32_t ld_volatile_shared_u32(uint32_t local_addr) {
-  uint32_t v;
-  asm volatile("ld.volatile.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(local_addr) : "memory");
+__device__ __forceinline__ unsigned long long ld_relaxed_cluster_u64(uint32_t local_addr) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.cluster.shared::cta.u64 %0, [%1];" : "=l"(v) : "r"(local_addr) : "memory");
   return v;
 }
 
@@ -1063,7 +1056,9 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       mbar_init(tempty(a), 2 * EPI_WARPS);  // epilogue warps of both CTAs (used in the even CTA)
     }
     mbar_init(done_bar, 1);
-    reinterpret_cast<uint32_t *>(smem + OFF_RING)[RING] = 0u;  // dynamic schedule: nothing published
+    if (kMode == kScaled)
+      for (int q = 0; q < RING; ++q)  // dynamic schedule: nothing published (no sequence number matches)
+        reinterpret_cast<unsigned long long *>(smem + OFF_RING)[q] = ~0ull;
     mbar_fence_init();
   }
   if (kMode == kFused && threadIdx.x < BN_EPI) {
@@ -1083,22 +1078,26 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
   // Dynamic schedule (kScaled with a tile counter): the clusters take tiles from one global
   // counter, so clusters on faster SMs take more; the even CTA's TMA thread fetches the indices
   // and writes them, in order, into a ring in both CTAs' shared memory, and every role of both
-  // CTAs reads tile i of the cluster from its own copy. The publisher runs at most LOOKAHEAD tiles
-  // ahead of the TMA warp, which the stage barriers keep within a few tiles of the slowest role,
-  // far inside the ring.
+  // CTAs reads tile i of the cluster from its own copy: slot i mod RING holds {tile index, i} in
+  // one 8-byte word, so a reader polls that slot until it carries sequence number i (relaxed
+  // loads: no acquire, which cost ~700 cycles per lookup at each tile boundary). The publisher
+  // runs at most LOOKAHEAD tiles ahead of the TMA warp, which the stage barriers keep within a
+  // few tiles of the slowest role, far inside the ring.
   const bool dyn = kMode == kScaled && counters != nullptr;
   const int64_t n_tiles_all = n_pm * (int64_t)P;
-  const uint32_t ring_addr = smem_addr(smem + OFF_RING), pub_addr = ring_addr + 4u * RING;
+  const uint32_t ring_addr = smem_addr(smem + OFF_RING);
   auto tile = [&](int64_t i, int64_t &mp_, int &nt_) -> bool {
     if (!dyn) return sp_tile_at<kMode>(i, n_pm, P, mp_, nt_);
+    const uint32_t slot = ring_addr + 8u * (uint32_t)(i & (RING - 1));
     uint32_t polls = 0;
-    while ((int64_t)ld_acquire_cluster_u32(pub_addr) <= i) {
+    unsigned long long v;
+    while ((uint32_t)((v = ld_relaxed_cluster_u64(slot)) >> 32) != (uint32_t)i) {
       if (++polls > kMaxPolls) {
         record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
         return false;
       }
     }
-    const int t = (int)ld_volatile_shared_u32(ring_addr + 4u * (uint32_t)(i & (RING - 1)));
+    const int t = (int)(uint32_t)v;
     if (t < 0 || (int64_t)t >= n_tiles_all) return false;
     mp_ = t / P;
     nt_ = t % P;
@@ -1120,12 +1119,11 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
       auto publish_upto = [&](int64_t k) {
         while (dyn && leader && !pub_end && n_pub < k) {
           const int t = atomicAdd(counters, 1);
-          const uint32_t off = 4u * (uint32_t)(n_pub & (RING - 1));
-          st_cluster_u32(mapa_shared(ring_addr + off, 0), (uint32_t)t);
-          st_cluster_u32(mapa_shared(ring_addr + off, 1), (uint32_t)t);
+          const unsigned long long v = ((unsigned long long)(uint32_t)n_pub << 32) | (uint32_t)t;
+          const uint32_t off = 8u * (uint32_t)(n_pub & (RING - 1));
+          st_relaxed_cluster_u64(mapa_shared(ring_addr + off, 0), v);
+          st_relaxed_cluster_u64(mapa_shared(ring_addr + off, 1), v);
           ++n_pub;
-          st_release_cluster_u32(mapa_shared(pub_addr, 0), (uint32_t)n_pub);
-          st_release_cluster_u32(mapa_shared(pub_addr, 1), (uint32_t)n_pub);
           pub_end = (int64_t)t >= n_tiles_all;
         }
       };
