@@ -68,6 +68,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
   return false;
 }
 
+// As mbar_wait, sleeping about `ns` nanoseconds between polls: for waits with slack (a warp
+// polling try_wait takes issue slots from the warps that share its scheduler).
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t bar, uint32_t parity, uint32_t *err, uint32_t ns) {
+  for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    __nanosleep(ns);
+  }
+  record_error(err, DMEL_DEVERR_WAIT_TIMEOUT);
+  return false;
+}
+
 // Makes this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor core operand reads, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -930,6 +930,7 @@ __host__ __device__ constexpr uint32_t a_col(int s) { return s == 0 ? 192u : s =
 constexpr uint32_t META_COL = 480;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t kSentinel = 0xFFFFFFFFu;  // a NaN no arithmetic produces: "not yet published"
+constexpr uint32_t kBackoffNs = 256;          // sleep between polls of the waits with slack
 static_assert(KBLOCKS * BKL == kRows, "stages cover the table");
 static_assert(BN % 64 == 0 && BN <= 192, "accumulator columns end where the A slots start");
 static_assert(STAGES_A == 3 && META_COL >= 448 + 32 && META_COL + 4 * STAGES_A <= TMEM_COLS, "TMEM map");
@@ -1132,7 +1133,9 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         publish_upto(i + 1 + LOOKAHEAD);
         const int n0 = nt * BN + (int)rank * BNH;
         for (int kb = 0; kb < KBLOCKS; ++kb) {
-          if (!mbar_wait(empty_b(stage), phase ^ 1u, err)) { ok = false; break; }
+          // the ring runs STAGES_B stages ahead of the MMAs: poll with sleeps, so this thread
+          // leaves the issue slots to the A producers
+          if (!mbar_wait_backoff(empty_b(stage), phase ^ 1u, err, kBackoffNs)) { ok = false; break; }
           const uint32_t fb = in_leader(full_b(stage));
           if (leader) mbar_arrive_expect_tx(full_b(stage), 2 * B_STAGE);  // both CTAs' halves
           const uint32_t dst = smem_addr(smem + OFF_B + stage * B_STAGE);
@@ -1343,7 +1346,9 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         scale = live && f < F ? __ldg(partials + f) : 0.0f;
         gt = gb;
       }
-      if (!sp_epi_barrier_and(mbar_wait(tfull(acc), acc_phase, err))) { ok = false; break; }
+      // a tile's MMAs take several microseconds: the epilogue warps poll with sleeps meanwhile
+      // (polling without them took issue slots from the A producers: 6 % of the kernel's time)
+      if (!sp_epi_barrier_and(mbar_wait_backoff(tfull(acc), acc_phase, err, kBackoffNs))) { ok = false; break; }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_STRIDE + cb;
       if (kMode == kFused && live) {
