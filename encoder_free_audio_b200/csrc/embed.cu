@@ -919,7 +919,8 @@ constexpr int OFF_STG = OFF_EPI + 3 * BM * 4;  // staging: 8 warps x 32 rows x u
 constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: {tile index, sequence} [16]
 constexpr int RING = 16;
 constexpr int LOOKAHEAD = 3;  // tiles published ahead of the one the TMA warp starts
-constexpr int SMEM_USED = OFF_RING + RING * 8;
+constexpr int OFF_ATAB = OFF_RING + RING * 8;  // one bin's 4 stored A words by level, + a zero row
+constexpr int SMEM_USED = OFF_ATAB + 17 * 16;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int WAITER_WARP = 6 + EPI_WARPS;  // warps: 0 TMA, 1 MMA, 2..5 A, 6..13 epilogue, 14 waits
 constexpr int THREADS = 32 * (WAITER_WARP + 1);
@@ -1060,6 +1061,12 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
     if (kMode == kScaled)
       for (int q = 0; q < RING; ++q)  // dynamic schedule: nothing published (no sequence number matches)
         reinterpret_cast<unsigned long long *>(smem + OFF_RING)[q] = ~0ull;
+    // a bin's 8 stored bf16 of A at level c: the 1 in column c >> 2 of the four 32-bit columns,
+    // low half when c is even; row 16 is a frame past the end (no 1)
+    uint32_t *atab = reinterpret_cast<uint32_t *>(smem + OFF_ATAB);
+    for (int c = 0; c < 17; ++c)
+      for (int g = 0; g < 4; ++g)
+        atab[4 * c + g] = c < 16 && (c >> 2) == g ? ((c & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
     mbar_fence_init();
   }
   if (kMode == kFused && threadIdx.x < BN_EPI) {
@@ -1273,21 +1280,23 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         for (int q = 0; q < 20; ++q) bad |= cw[q] & 0xF0F0F0F0u;
         if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
       }
-      const uint32_t one_mask = valid ? 0xFFFFFFFFu : 0u;
+      const uint4 *atab = reinterpret_cast<const uint4 *>(smem + OFF_ATAB);
 #pragma unroll
       for (int kb = 0; kb < KBLOCKS; ++kb) {
         // the stage's one-hot rows and metadata are built before waiting for the slot (the wait
         // is on the stage three back; building them is off that critical loop)
         const uint32_t wlo = cw[2 * kb], whi = cw[2 * kb + 1];
-        // bin j of the stage: stored bf16 8j .. 8j + 7 = columns 4j .. 4j + 3, the 1 in column
-        // 4j + (c >> 2), low half when c is even
+        // bin j of the stage: stored bf16 8j .. 8j + 7 = columns 4j .. 4j + 3, one 16-byte
+        // row of the level table (the 1 in column 4j + (c >> 2), low half when c is even)
         uint32_t av[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t c = ((j < 4 ? wlo : whi) >> (8 * (j & 3))) & 15u;
-          const uint32_t one = ((c & 1u) ? 0x3F800000u : 0x00003F80u) & one_mask;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) av[4 * j + g] = (c >> 2) == (uint32_t)g ? one : 0u;
+          const uint4 w = atab[valid ? c : 16u];
+          av[4 * j] = w.x;
+          av[4 * j + 1] = w.y;
+          av[4 * j + 2] = w.z;
+          av[4 * j + 3] = w.w;
         }
         uint32_t m[4];
 #pragma unroll
