@@ -920,7 +920,8 @@ constexpr int OFF_RING = OFF_STG + EPI_WARPS * 32 * 128;  // dynamic schedule: {
 constexpr int RING = 16;
 constexpr int LOOKAHEAD = 3;  // tiles published ahead of the one the TMA warp starts
 constexpr int OFF_ATAB = OFF_RING + RING * 8;  // one bin's 4 stored A words by level, + a zero row
-constexpr int SMEM_USED = OFF_ATAB + 17 * 16;
+constexpr int OFF_MTAB = OFF_ATAB + 17 * 16;   // metadata of two bins by their levels [256]
+constexpr int SMEM_USED = OFF_MTAB + 256 * 4;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;
 constexpr int WAITER_WARP = 6 + EPI_WARPS;  // warps: 0 TMA, 1 MMA, 2..5 A, 6..13 epilogue, 14 waits
 constexpr int THREADS = 32 * (WAITER_WARP + 1);
@@ -1069,6 +1070,9 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         atab[4 * c + g] = c < 16 && (c >> 2) == g ? ((c & 1) ? 0x3F800000u : 0x00003F80u) : 0u;
     mbar_fence_init();
   }
+  // the metadata of two bins at levels c0 and c1, at index c0 + 16 c1
+  for (int e = threadIdx.x; e < 256; e += blockDim.x)
+    reinterpret_cast<uint32_t *>(smem + OFF_MTAB)[e] = sp_meta_field(e & 15) | (sp_meta_field(e >> 4) << 16);
   if (kMode == kFused && threadIdx.x < BN_EPI) {
     const int c = (int)((blockIdx.x >> 1) % P) * BN + threadIdx.x;
     gsm[threadIdx.x] = c < D ? __bfloat162float(gw[c]) : 0.0f;
@@ -1281,6 +1285,7 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
         if (bad) record_error(err, DMEL_DEVERR_CODE_RANGE);
       }
       const uint4 *atab = reinterpret_cast<const uint4 *>(smem + OFF_ATAB);
+      const uint32_t *mtab = reinterpret_cast<const uint32_t *>(smem + OFF_MTAB);
 #pragma unroll
       for (int kb = 0; kb < KBLOCKS; ++kb) {
         // the stage's one-hot rows and metadata are built before waiting for the slot (the wait
@@ -1302,8 +1307,8 @@ __global__ void __launch_bounds__(sp::THREADS, 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t w = k < 2 ? wlo : whi;
-          const uint32_t c0 = (w >> (16 * (k & 1))) & 15u, c1 = (w >> (16 * (k & 1) + 8)) & 15u;
-          const uint32_t pk = sp_meta_field(c0) | (sp_meta_field(c1) << 16);
+          const uint32_t h = (w >> (16 * (k & 1))) & 0x0F0Fu;  // levels c0 (bits 0-3), c1 (bits 8-11)
+          const uint32_t pk = mtab[(h & 15u) | (h >> 4)];
           const uint32_t lo = __shfl_sync(0xffffffffu, pk, src_lo), hi = __shfl_sync(0xffffffffu, pk, src_hi);
           m[k] = ((lo >> half_shift) & 0xFFFFu) | (((hi >> half_shift) & 0xFFFFu) << 16);
         }
