@@ -69,9 +69,9 @@ def out_bytes(out_es: int) -> int:
 # now): codes_kernel_entry; and the embedding call's six kernels, gram_kernel, gram_combine_kernel,
 # gram_diag_kernel (G), norm_partials_kernel, norm_finalize_kernel (the scales) and
 # embed_sp_kernel<kScaled>. Other frame counts have no capture of the current kernels: null.
-TRAFFIC_MEASURED = {318044: {"codes": 1023952128 + 27933440,
-                             "embed": (15749120 + 7212544 + 15735040) + (29226752 + 21054208) + (69979648 + 20736)
-                             + (42607360 + 3850881536)}}
+TRAFFIC_MEASURED = {318044: {"codes": 1024211456 + 27772160,
+                             "embed": (15749120 + 7212544 + 15735040) + (29174528 + 21165056) + (69979648 + 68096)
+                             + (42732288 + 3851324416)}}
 # the tensor cores' work per frame in the one-hot product: 2 * 1280 * 6144 logical flops, run as a
 # 2:4-sparse product whose peak is twice the dense bf16 peak (nominal 4.5 vs 2.25 PFLOP/s)
 ONEHOT_FLOP_PER_FRAME = 2 * 1280 * DIM
